@@ -1,0 +1,456 @@
+// dec_api.cu -- the C ABI of libdec.so (declared and documented in dec.h):
+// argument checking, the workspace, kernel configuration and launches.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "dec.h"
+#include "dec_internal.h"
+
+using namespace dec;
+
+namespace {
+int g_last_cuda = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda = static_cast<int>(e);
+  return DEC_ERR_CUDA;
+}
+
+size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+}  // namespace
+
+struct dec_handle {
+  dec_shape shape;
+  int device = 0;
+  int sms = 0;
+  int ctas = 0;
+  int smem_optin = 0;
+  int nslot[kMaxBatchSmall + 1] = {0};
+  size_t smem[kMaxBatchSmall + 1] = {0};
+  const uint16_t* embed = nullptr;
+  const uint16_t* lm_head = nullptr;
+  const uint16_t* final_norm = nullptr;
+  LayerPtrs* layers_dev = nullptr;
+  uint8_t* ws = nullptr;
+  WorkspaceLayout wl{};
+  float* logits_dev = nullptr;
+  unsigned long long timeout_ns = 2000000000ull;
+  int stall_cta = -1;
+};
+
+static int check_shape(const dec_shape* s) {
+  if (!s) return DEC_ERR_NULL;
+  if (s->n_layers < 1 || s->n_layers > 255) return DEC_ERR_SHAPE;
+  if (s->hidden < 256 || s->hidden % 256 || s->hidden > 6144) return DEC_ERR_SHAPE;
+  if (s->ffn < 256 || s->ffn % 256 || s->ffn > 6144) return DEC_ERR_SHAPE;
+  if (s->head_dim != 64 && s->head_dim != 128) return DEC_ERR_SHAPE;
+  if (s->n_kv_heads < 1 || s->n_q_heads < s->n_kv_heads || s->n_q_heads % s->n_kv_heads)
+    return DEC_ERR_SHAPE;
+  if (s->n_q_heads / s->n_kv_heads > kMaxRep) return DEC_ERR_SHAPE;
+  const int hqd = s->n_q_heads * s->head_dim;
+  if (hqd % 256 || hqd > 6144) return DEC_ERR_SHAPE;
+  if (s->vocab < 1) return DEC_ERR_SHAPE;
+  if (!(s->rms_eps >= 0.f) || !(s->rope_theta > 0.f)) return DEC_ERR_SHAPE;
+  if (s->max_batch < 1 || s->max_batch > kMaxBatchSmall) return DEC_ERR_BATCH;
+  return DEC_OK;
+}
+
+extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle** out) {
+  if (!shape || !w || !out) return DEC_ERR_NULL;
+  *out = nullptr;
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!w->embed || !w->lm_head || !w->final_norm || !w->layers) return DEC_ERR_NULL;
+  if (!aligned(w->embed, 16) || !aligned(w->lm_head, 16) || !aligned(w->final_norm, 16))
+    return DEC_ERR_ALIGN;
+  const int L = shape->n_layers;
+  for (int i = 0; i < L * DEC_LW_COUNT; ++i) {
+    if (!w->layers[i]) return DEC_ERR_NULL;
+    if (!aligned(w->layers[i], 16)) return DEC_ERR_ALIGN;
+  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (prop.major != 10) return DEC_ERR_DEVICE;
+  if (!prop.cooperativeLaunch) return DEC_ERR_DEVICE;
+
+  dec_handle* h = new (std::nothrow) dec_handle();
+  if (!h) return DEC_ERR_ARG;
+  h->shape = *shape;
+  h->device = dev;
+  h->sms = prop.multiProcessorCount;
+  h->ctas = prop.multiProcessorCount;
+  h->smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
+  const int H = shape->hidden, F = shape->ffn, D = shape->head_dim;
+  const int Hq = shape->n_q_heads, Hkv = shape->n_kv_heads, B = shape->max_batch;
+  const int HqD = Hq * D, rep = Hq / Hkv;
+  if ((H + h->ctas - 1) / h->ctas > 64) {
+    delete h;
+    return DEC_ERR_SHAPE;
+  }
+  const int nchunks = h->ctas + 1;
+  for (int b = 1; b <= B; ++b) {
+    h->nslot[b] = step_max_slots(b, H, F, HqD, D, rep, nchunks, h->smem_optin);
+    if (h->nslot[b] < 2) {
+      delete h;
+      return DEC_ERR_DEVICE;
+    }
+    h->smem[b] = step_smem_bytes(h->nslot[b], b, H, F, HqD, D, rep, nchunks);
+  }
+  h->embed = static_cast<const uint16_t*>(w->embed);
+  h->lm_head = static_cast<const uint16_t*>(w->lm_head);
+  h->final_norm = static_cast<const uint16_t*>(w->final_norm);
+
+  // ---- workspace
+  const int nqkv = (Hq + 2 * Hkv) * D;
+  WorkspaceLayout& wl = h->wl;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o += al256(bytes);
+    return at;
+  };
+  wl.part_chunks = nchunks;
+  wl.x_qkv = take(sizeof(uint64_t) * B * nqkv);
+  wl.x_o = take(sizeof(uint64_t) * B * HqD);
+  wl.x_mid = take(sizeof(uint64_t) * B * H);
+  wl.x_u = take(sizeof(uint64_t) * B * F);
+  wl.x_out = take(sizeof(uint64_t) * B * H);
+  wl.part = take(sizeof(uint64_t) * B * Hq * wl.part_chunks * (D + 2));
+  wl.amax_key = take(sizeof(unsigned long long) * B);
+  wl.exit_cnt = take(sizeof(unsigned));
+  wl.seq = take(sizeof(unsigned));
+  wl.status = take(sizeof(int));
+  wl.abort_flag = take(sizeof(int));
+  wl.inv_freq = take(sizeof(float) * D / 2);
+  wl.tok_dev = take(sizeof(int32_t) * B);
+  wl.pos_dev = take(sizeof(int32_t) * B);
+  wl.out_dev = take(sizeof(int32_t) * B);
+#ifdef DEC_PROFILE
+  wl.prof = take(sizeof(unsigned long long) * h->ctas * (8 * L + 4));
+#endif
+  size_t layers_off = take(sizeof(LayerPtrs) * L);
+  size_t logits_off = take(sizeof(float) * static_cast<size_t>(B) * shape->vocab);
+  wl.total = o;
+  e = cudaMalloc(&h->ws, wl.total);
+  if (e != cudaSuccess) {
+    delete h;
+    return cuda_fail(e);
+  }
+  e = cudaMemset(h->ws, 0, wl.total);
+  // rotary inverse frequencies theta^(-2i/D), rounded once to fp32
+  std::vector<float> inv(D / 2);
+  for (int i = 0; i < D / 2; ++i)
+    inv[i] = static_cast<float>(1.0 / pow(static_cast<double>(shape->rope_theta),
+                                          (2.0 * i) / static_cast<double>(D)));
+  if (e == cudaSuccess)
+    e = cudaMemcpy(h->ws + wl.inv_freq, inv.data(), sizeof(float) * inv.size(),
+                   cudaMemcpyHostToDevice);
+  std::vector<LayerPtrs> lp(L);
+  for (int l = 0; l < L; ++l)
+    for (int j = 0; j < DEC_LW_COUNT; ++j)
+      lp[l].w[j] = static_cast<const uint16_t*>(w->layers[l * DEC_LW_COUNT + j]);
+  h->layers_dev = reinterpret_cast<LayerPtrs*>(h->ws + layers_off);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(h->layers_dev, lp.data(), sizeof(LayerPtrs) * L, cudaMemcpyHostToDevice);
+  h->logits_dev = reinterpret_cast<float*>(h->ws + logits_off);
+  if (e != cudaSuccess) {
+    cudaFree(h->ws);
+    delete h;
+    return cuda_fail(e);
+  }
+  *out = h;
+  return DEC_OK;
+}
+
+extern "C" void dec_free(dec_handle* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  cudaFree(h->ws);
+  delete h;
+}
+
+static size_t kv_code_bytes(const dec_shape& s, int batch, int max_ctx, int elt) {
+  return static_cast<size_t>(s.n_layers) * 2 * batch * s.n_kv_heads * max_ctx * s.head_dim * elt;
+}
+
+extern "C" size_t dec_kv_scale_offset(const dec_handle* h, int batch, int max_ctx, int dtype) {
+  if (!h || batch < 1 || max_ctx < 16 || dtype != DEC_KV_FP8_E4M3) return 0;
+  return al256(kv_code_bytes(h->shape, batch, max_ctx, 1));
+}
+
+extern "C" size_t dec_kv_bytes(const dec_handle* h, int batch, int max_ctx, int dtype) {
+  if (!h || batch < 1 || max_ctx < 16 || max_ctx % 16) return 0;
+  if (dtype == DEC_KV_BF16) return kv_code_bytes(h->shape, batch, max_ctx, 2);
+  if (dtype == DEC_KV_FP8_E4M3)
+    return al256(kv_code_bytes(h->shape, batch, max_ctx, 1)) +
+           static_cast<size_t>(h->shape.n_layers) * 2 * batch * h->shape.n_kv_heads * max_ctx *
+               sizeof(float);
+  return 0;
+}
+
+extern "C" int dec_kv_alloc(dec_handle* h, int batch, int max_ctx, int dtype, void* buf,
+                            size_t buf_bytes, dec_kv* out) {
+  if (!h || !buf || !out) return DEC_ERR_NULL;
+  if (dtype != DEC_KV_BF16 && dtype != DEC_KV_FP8_E4M3) return DEC_ERR_DTYPE;
+  if (batch < 1) return DEC_ERR_BATCH;
+  if (max_ctx < 16 || max_ctx % 16) return DEC_ERR_ARG;
+  if (!aligned(buf, 256)) return DEC_ERR_ALIGN;
+  const size_t need = dec_kv_bytes(h, batch, max_ctx, dtype);
+  if (need == 0) return DEC_ERR_ARG;
+  if (buf_bytes < need) return DEC_ERR_KV_SIZE;
+  out->base = buf;
+  out->bytes = buf_bytes;
+  out->batch = batch;
+  out->max_ctx = max_ctx;
+  out->dtype = dtype;
+  return DEC_OK;
+}
+
+static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* pos,
+                   const dec_kv* kv, int32_t* out_ids, float* logits, float* hidden,
+                   cudaStream_t stream) {
+  if (!h || !kv || !tok || !pos || !out_ids || !kv->base) return DEC_ERR_NULL;
+  if (batch < 1 || batch > h->shape.max_batch || batch > kv->batch) return DEC_ERR_BATCH;
+  if (kv->dtype != DEC_KV_BF16 && kv->dtype != DEC_KV_FP8_E4M3) return DEC_ERR_DTYPE;
+  if (kv->bytes < dec_kv_bytes(h, kv->batch, kv->max_ctx, kv->dtype)) return DEC_ERR_KV_SIZE;
+  const dec_shape& s = h->shape;
+  StepArgs a{};
+  a.L = s.n_layers;
+  a.H = s.hidden;
+  a.Hq = s.n_q_heads;
+  a.Hkv = s.n_kv_heads;
+  a.D = s.head_dim;
+  a.F = s.ffn;
+  a.V = s.vocab;
+  a.B = batch;
+  a.eps = s.rms_eps;
+  a.embed = h->embed;
+  a.lm_head = h->lm_head;
+  a.final_norm = h->final_norm;
+  a.layers = h->layers_dev;
+  a.kv = static_cast<uint8_t*>(kv->base);
+  a.kv_fp8 = kv->dtype == DEC_KV_FP8_E4M3;
+  a.kv_scales = a.kv_fp8 ? reinterpret_cast<float*>(static_cast<uint8_t*>(kv->base) +
+                                                    dec_kv_scale_offset(h, kv->batch, kv->max_ctx,
+                                                                        kv->dtype))
+                         : nullptr;
+  a.kv_batch = kv->batch;
+  a.max_ctx = kv->max_ctx;
+  a.token_ids = tok;
+  a.positions = pos;
+  a.out_ids = out_ids;
+  a.out_logits = logits;
+  a.hidden_out = hidden;
+  const WorkspaceLayout& wl = h->wl;
+  a.x_qkv = reinterpret_cast<uint64_t*>(h->ws + wl.x_qkv);
+  a.x_o = reinterpret_cast<uint64_t*>(h->ws + wl.x_o);
+  a.x_mid = reinterpret_cast<uint64_t*>(h->ws + wl.x_mid);
+  a.x_u = reinterpret_cast<uint64_t*>(h->ws + wl.x_u);
+  a.x_out = reinterpret_cast<uint64_t*>(h->ws + wl.x_out);
+  a.part = reinterpret_cast<uint64_t*>(h->ws + wl.part);
+  a.part_chunks = wl.part_chunks;
+  a.amax_key = reinterpret_cast<unsigned long long*>(h->ws + wl.amax_key);
+  a.exit_cnt = reinterpret_cast<unsigned*>(h->ws + wl.exit_cnt);
+  a.seq = reinterpret_cast<unsigned*>(h->ws + wl.seq);
+  a.status = reinterpret_cast<int*>(h->ws + wl.status);
+  a.abort_flag = reinterpret_cast<int*>(h->ws + wl.abort_flag);
+  a.inv_freq = reinterpret_cast<const float*>(h->ws + wl.inv_freq);
+  a.timeout_ns = h->timeout_ns;
+  a.stall_cta = h->stall_cta;
+  a.nslot = h->nslot[batch];
+#ifdef DEC_PROFILE
+  a.prof = reinterpret_cast<unsigned long long*>(h->ws + wl.prof);
+#else
+  a.prof = nullptr;
+#endif
+  cudaError_t e = launch_step_small(a, h->ctas, h->smem[batch], stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return DEC_OK;
+}
+
+extern "C" int dec_step(dec_handle* h, int batch, const int32_t* token_ids,
+                        const int32_t* positions, const dec_kv* kv, int32_t* out_ids,
+                        float* out_logits, void* stream) {
+  return do_step(h, batch, token_ids, positions, kv, out_ids, out_logits, nullptr,
+                 static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int dec_step_debug(dec_handle* h, int batch, const int32_t* token_ids,
+                              const int32_t* positions, const dec_kv* kv, int32_t* out_ids,
+                              float* out_logits, float* hidden_out, void* stream) {
+  if (!hidden_out) return DEC_ERR_NULL;
+  return do_step(h, batch, token_ids, positions, kv, out_ids, out_logits, hidden_out,
+                 static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int dec_step_host(dec_handle* h, int batch, const int32_t* tok_host,
+                             const int32_t* pos_host, const dec_kv* kv, int32_t* out_host,
+                             float* logits_host, void* stream) {
+  if (!h || !tok_host || !pos_host || !out_host) return DEC_ERR_NULL;
+  if (batch < 1 || batch > h->shape.max_batch) return DEC_ERR_BATCH;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* tok = reinterpret_cast<int32_t*>(h->ws + h->wl.tok_dev);
+  int32_t* pos = reinterpret_cast<int32_t*>(h->ws + h->wl.pos_dev);
+  int32_t* out = reinterpret_cast<int32_t*>(h->ws + h->wl.out_dev);
+  cudaError_t e = cudaMemcpyAsync(tok, tok_host, sizeof(int32_t) * batch, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(pos, pos_host, sizeof(int32_t) * batch, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int rc = do_step(h, batch, tok, pos, kv, out, logits_host ? h->logits_dev : nullptr, nullptr, st);
+  if (rc) return rc;
+  e = cudaMemcpyAsync(out_host, out, sizeof(int32_t) * batch, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess && logits_host)
+    e = cudaMemcpyAsync(logits_host, h->logits_dev,
+                        sizeof(float) * static_cast<size_t>(batch) * h->shape.vocab,
+                        cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return DEC_OK;
+}
+
+extern "C" int dec_check(dec_handle* h, void* stream) {
+  if (!h) return DEC_ERR_NULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int v = 0;
+  e = cudaMemcpy(&v, h->ws + h->wl.status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(h->ws + h->wl.status, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return v;
+}
+
+extern "C" int dec_set_timeout_ns(dec_handle* h, unsigned long long ns) {
+  if (!h) return DEC_ERR_NULL;
+  if (ns < 1000000ull) return DEC_ERR_ARG;
+  h->timeout_ns = ns;
+  return DEC_OK;
+}
+
+extern "C" int dec_set_debug_stall(dec_handle* h, int cta_plus_one) {
+  if (!h) return DEC_ERR_NULL;
+  if (cta_plus_one < 0 || cta_plus_one > h->ctas) return DEC_ERR_ARG;
+  h->stall_cta = cta_plus_one - 1;
+  return DEC_OK;
+}
+
+extern "C" int dec_get_config(const dec_handle* h, int* ctas, int* ring_slots, int* slot_bytes) {
+  if (!h) return DEC_ERR_NULL;
+  if (ctas) *ctas = h->ctas;
+  if (ring_slots) *ring_slots = h->nslot[1];
+  if (slot_bytes) *slot_bytes = kSlotBytes;
+  return DEC_OK;
+}
+
+extern "C" const char* dec_error_string(int code) {
+  switch (code) {
+    case DEC_OK: return "ok";
+    case DEC_ERR_NULL: return "a required pointer is NULL";
+    case DEC_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case DEC_ERR_BATCH: return "batch out of range";
+    case DEC_ERR_KV_SIZE: return "KV buffer too small";
+    case DEC_ERR_DTYPE: return "unsupported KV dtype";
+    case DEC_ERR_ALIGN: return "pointer not aligned";
+    case DEC_ERR_CUDA: return "CUDA runtime error";
+    case DEC_ERR_DEVICE: return "device not supported (needs compute capability 10.0)";
+    case DEC_ERR_ARG: return "invalid argument";
+    default: break;
+  }
+  if (code > 0) {
+    static thread_local char buf[96];
+    buf[0] = 0;
+    if (code & DEC_DEV_BAD_POSITION) strcat(buf, "device: position out of range; ");
+    if (code & DEC_DEV_BAD_TOKEN) strcat(buf, "device: token out of range; ");
+    if (code & DEC_DEV_TIMEOUT) strcat(buf, "device: bounded wait ran out; ");
+    return buf;
+  }
+  return "unknown status";
+}
+
+extern "C" int dec_last_cuda_error(void) { return g_last_cuda; }
+
+// ------------------------------------------------------------ attention
+extern "C" size_t dec_attention_workspace_bytes(int batch, int n_q_heads, int n_kv_heads,
+                                                int head_dim, int max_len) {
+  if (batch < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads || max_len < 1) return 0;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int cr = attention_chunk_rows(batch, n_kv_heads, max_len, sms);
+  const int chunks = (max_len + cr - 1) / cr;
+  return al256(sizeof(float) * static_cast<size_t>(batch) * n_q_heads * chunks * (head_dim + 2)) +
+         al256(sizeof(unsigned) * static_cast<size_t>(batch) * n_kv_heads);
+}
+
+extern "C" int dec_attention(int batch, int n_q_heads, int n_kv_heads, int head_dim,
+                             const void* q, const void* k_cache, const void* v_cache, int max_len,
+                             const int32_t* lengths, float* out, void* workspace,
+                             size_t workspace_bytes, int* status, void* stream) {
+  if (!q || !k_cache || !v_cache || !lengths || !out || !workspace) return DEC_ERR_NULL;
+  if (batch < 1) return DEC_ERR_BATCH;
+  if (head_dim != 64 && head_dim != 128) return DEC_ERR_SHAPE;
+  if (n_kv_heads < 1 || n_q_heads % n_kv_heads || n_q_heads / n_kv_heads > 8) return DEC_ERR_SHAPE;
+  if (max_len < 1) return DEC_ERR_ARG;
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(workspace, 256))
+    return DEC_ERR_ALIGN;
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const size_t need = dec_attention_workspace_bytes(batch, n_q_heads, n_kv_heads, head_dim, max_len);
+  if (workspace_bytes < need) return DEC_ERR_KV_SIZE;
+  AttnArgs a{};
+  a.B = batch;
+  a.Hq = n_q_heads;
+  a.Hkv = n_kv_heads;
+  a.D = head_dim;
+  a.max_len = max_len;
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(k_cache);
+  a.v = static_cast<const uint16_t*>(v_cache);
+  a.lengths = lengths;
+  a.out = out;
+  a.chunk_rows = attention_chunk_rows(batch, n_kv_heads, max_len, sms);
+  a.chunks_max = (max_len + a.chunk_rows - 1) / a.chunk_rows;
+  a.part = static_cast<float*>(workspace);
+  a.cnt = reinterpret_cast<unsigned*>(
+      static_cast<uint8_t*>(workspace) +
+      al256(sizeof(float) * static_cast<size_t>(batch) * n_q_heads * a.chunks_max * (head_dim + 2)));
+  a.status = status;
+  e = launch_attention(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return DEC_OK;
+}
+
+extern "C" int dec_kv_quantize_e4m3(const float* x, int rows, int dim, uint8_t* codes,
+                                    float* scales, void* stream) {
+  if (!x || !codes || !scales) return DEC_ERR_NULL;
+  if (rows < 0) return DEC_ERR_ARG;
+  if (dim != 64 && dim != 128) return DEC_ERR_SHAPE;
+  if (rows == 0) return DEC_OK;
+  cudaError_t e = launch_quantize(x, rows, dim, codes, scales, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return DEC_OK;
+}
+
+#ifdef DEC_PROFILE
+// Profiling builds only (not part of dec.h): copy the per-phase timestamps of
+// the last step, [ctas][8 * n_layers + 4] globaltimer values, to `host`.
+extern "C" int dec_prof_read(dec_handle* h, unsigned long long* host, size_t n) {
+  if (!h || !host) return DEC_ERR_NULL;
+  const size_t need = static_cast<size_t>(h->ctas) * (8 * h->shape.n_layers + 4);
+  if (n < need) return DEC_ERR_ARG;
+  cudaError_t e = cudaMemcpy(host, h->ws + h->wl.prof, need * sizeof(unsigned long long),
+                             cudaMemcpyDeviceToHost);
+  return e == cudaSuccess ? DEC_OK : cuda_fail(e);
+}
+#endif

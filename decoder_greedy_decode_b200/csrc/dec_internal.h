@@ -1,0 +1,93 @@
+// dec_internal.h -- host-side structures shared by the C ABI and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dec {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kStepThreads = kConsumerThreads + 32;  // + one producer warp
+constexpr int kSlotBytes = 24576;                   // ring slot: 12 rows of 1024 bf16
+constexpr int kMaxBatchSmall = 4;                   // batch handled by the GEMV step kernel
+constexpr int kMaxRep = 4;                          // query heads per KV head (step kernel)
+constexpr int kLayerPtrs = 11;
+
+struct LayerPtrs {
+  const uint16_t* w[kLayerPtrs];  // dec_layer_weight order
+};
+
+// Everything one launch of the persistent step kernel reads.
+struct StepArgs {
+  // shape
+  int L, H, Hq, Hkv, D, F, V, B;
+  float eps;
+  // weights
+  const uint16_t* embed;
+  const uint16_t* lm_head;
+  const uint16_t* final_norm;
+  const LayerPtrs* layers;  // device array [L]
+  // KV cache
+  uint8_t* kv;          // values (bf16) or codes (fp8)
+  float* kv_scales;     // fp8 only
+  int kv_batch;         // batch dimension of the cache layout
+  int max_ctx;
+  int kv_fp8;
+  // step inputs / outputs
+  const int32_t* token_ids;
+  const int32_t* positions;
+  int32_t* out_ids;
+  float* out_logits;    // [B, V] or null
+  float* hidden_out;    // [L+1, B, H] or null
+  // workspace
+  uint64_t* x_qkv;      // tagged [B, (Hq+2Hkv)D]
+  uint64_t* x_o;        // tagged [B, Hq D]
+  uint64_t* x_mid;      // tagged [B, H]   residual after o_proj
+  uint64_t* x_u;        // tagged [B, F]
+  uint64_t* x_out;      // tagged [B, H]   residual after the MLP
+  uint64_t* part;       // tagged attention partials [B, Hq, part_chunks, D + 2]
+  int part_chunks;
+  unsigned long long* amax_key;  // [B]
+  unsigned* exit_cnt;
+  unsigned* seq;
+  int* status;
+  int* abort_flag;
+  const float* inv_freq;  // [D/2]
+  unsigned long long timeout_ns;
+  int stall_cta;        // -1: off
+  int nslot;            // ring slots per CTA
+  unsigned long long* prof;  // per-phase timestamps (profiling builds) or null
+};
+
+// Scratch layout inside the library workspace (byte offsets).
+struct WorkspaceLayout {
+  size_t x_qkv, x_o, x_mid, x_u, x_out, part, amax_key, exit_cnt, seq, status, abort_flag,
+      inv_freq, tok_dev, pos_dev, out_dev, prof, total;
+  int part_chunks;
+};
+
+size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep, int nchunks);
+int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int nchunks, int smem_optin);
+cudaError_t launch_step_small(const StepArgs& a, int ctas, size_t smem, cudaStream_t s);
+
+// Isolated split-K decode attention.
+struct AttnArgs {
+  int B, Hq, Hkv, D, max_len;
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const int32_t* lengths;
+  float* out;
+  float* part;          // [B, Hq, chunks_max, D + 2]
+  unsigned* cnt;        // [B * Hkv]
+  int chunk_rows;
+  int chunks_max;
+  int* status;
+};
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+size_t attention_smem_bytes(int D, int rep);
+int attention_chunk_rows(int B, int Hkv, int max_len, int sms);
+cudaError_t launch_quantize(const float* x, int rows, int dim, uint8_t* codes, float* scales,
+                            cudaStream_t s);
+
+}  // namespace dec

@@ -1,0 +1,274 @@
+/*
+ * dec.h -- C ABI of the B200 (sm_100a) greedy decode-step library (libdec.so).
+ *
+ * The library computes one autoregressive greedy decode step of a Qwen3-style
+ * decoder for a batch of sequences: embedding, RMSNorm, QKV projection,
+ * per-head q/k RMSNorm, rotary embedding, KV-cache append, grouped-query
+ * attention over the cached context, o_proj + residual, SwiGLU MLP + residual,
+ * final norm, lm_head and argmax.  The pages this follows:
+ *   - "Qwen3-ASR -- Latency & Bottleneck Analysis", 03 Decode (module list and
+ *     the 18.58 ms/token split), 07 Root causes (q/k/v projections, repeat_kv,
+ *     QK^T, mask, fp32 softmax, AV, o_proj; RMSNorm fp32 up-cast).
+ *   - "Can CTC make Qwen3-ASR faster?", 03 Greedy exactness (emit the argmax)
+ *     and 11 Phase A step 1 (a one-token decode exposing the cache, its
+ *     length and the logits).
+ *   - faster-qwen-asr GB10 benchmark record, notes.configuration (the token,
+ *     mask and position are fed back on the device: out_ids may alias the
+ *     next step's token_ids).
+ *   - Baseten Qwen3-ASR article, "Minimizing host-to-device syncs" (sequence
+ *     lengths are owned by the host; no step reads device data back) and
+ *     "KV cache quantization" (an FP8 cache, attention math in full
+ *     precision).
+ *
+ * Conventions.  Every pointer is a DEVICE pointer unless its comment says
+ * "host".  `stream` is a cudaStream_t (NULL = the legacy default stream).
+ * Calls that take a stream are asynchronous on it unless noted.  Return values
+ * are DEC_OK (0) or a negative dec_status; nothing is written on error.
+ * A handle is not thread-safe: calls on one handle must be serialised (one
+ * stream at a time).  The caller owns every buffer it passes (weights, KV,
+ * token/position/output arrays) and keeps them alive while the handle or an
+ * enqueued step uses them; the library owns only the handle and its
+ * workspace.
+ *
+ * Numerics: bf16 weights and cache, fp32 activations and accumulation, fp32
+ * softmax; RMSNorm eps and rope theta from dec_shape.  Readings of the pages
+ * taken by this library (the pages are silent on them):
+ *   - q/k RMSNorm per head after the projection, before the rotation; one
+ *     gain vector [head_dim] shared by all heads;
+ *   - rotate-half RoPE pairing (i, i + head_dim/2) with
+ *     inv_freq_i = theta^(-2i/head_dim) and angle p * inv_freq_i in fp32
+ *     (for a text decode step the three MRoPE sections share the position);
+ *   - query head h reads KV head floor(h * n_kv_heads / n_q_heads) (each KV
+ *     head serves n_q_heads/n_kv_heads consecutive query heads);
+ *   - attention scale 1/sqrt(head_dim), causal over rows 0..p inclusive (the
+ *     new token attends to itself), no biases, no sliding window;
+ *   - argmax ties go to the lowest token id;
+ *   - FP8 cache: OCP E4M3 codes with one fp32 scale per (layer, K/V, sequence,
+ *     KV head, token): scale = max(amax, 2^-126)/448, code = RNE-satfinite of
+ *     x/scale, both in fp32.
+ */
+#ifndef DEC_H
+#define DEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------------ */
+/* Status codes                                                        */
+/* ------------------------------------------------------------------ */
+typedef enum dec_status {
+  DEC_OK = 0,
+  DEC_ERR_NULL = -1,          /* a required pointer is NULL */
+  DEC_ERR_SHAPE = -2,         /* unsupported or inconsistent shape */
+  DEC_ERR_BATCH = -3,         /* batch < 1 or > max_batch / kv batch */
+  DEC_ERR_KV_SIZE = -4,       /* KV buffer smaller than dec_kv_bytes() */
+  DEC_ERR_DTYPE = -5,         /* unsupported KV dtype */
+  DEC_ERR_ALIGN = -6,         /* pointer not aligned as documented */
+  DEC_ERR_CUDA = -7,          /* a CUDA runtime call failed (dec_last_cuda_error) */
+  DEC_ERR_DEVICE = -8,        /* the current device is not sm_100 or lacks resources */
+  DEC_ERR_ARG = -9,           /* other invalid argument */
+  /* device-detected conditions, returned (OR-ed as a positive bit set) by
+   * dec_check(); the step that saw them wrote -1 to every out_ids entry */
+  DEC_DEV_BAD_POSITION = 1,   /* a position < 0 or >= max_ctx */
+  DEC_DEV_BAD_TOKEN = 2,      /* a token id < 0 or >= vocab */
+  DEC_DEV_TIMEOUT = 4         /* a bounded device wait ran out (see dec_set_timeout_ns) */
+} dec_status;
+
+/* ------------------------------------------------------------------ */
+/* Model description                                                   */
+/* ------------------------------------------------------------------ */
+typedef struct dec_shape {
+  int n_layers;      /* 28 for the 0.6B / 1.7B decoders */
+  int hidden;        /* multiple of 256 */
+  int n_q_heads;     /* multiple of n_kv_heads */
+  int n_kv_heads;
+  int head_dim;      /* 64 or 128 */
+  int ffn;           /* multiple of 256 */
+  int vocab;
+  float rms_eps;     /* 1e-6 */
+  float rope_theta;  /* 1e6 */
+  int max_batch;     /* largest batch dec_step will be called with */
+} dec_shape;
+
+/* Order of the per-layer weight pointers in dec_weights.layers. */
+typedef enum dec_layer_weight {
+  DEC_LW_IN_NORM = 0,  /* bf16 [hidden]                    input RMSNorm gain  */
+  DEC_LW_Q,            /* bf16 [n_q_heads*head_dim, hidden]  row-major, y = W x */
+  DEC_LW_K,            /* bf16 [n_kv_heads*head_dim, hidden]                    */
+  DEC_LW_V,            /* bf16 [n_kv_heads*head_dim, hidden]                    */
+  DEC_LW_Q_NORM,       /* bf16 [head_dim]                  per-head q gain     */
+  DEC_LW_K_NORM,       /* bf16 [head_dim]                  per-head k gain     */
+  DEC_LW_O,            /* bf16 [hidden, n_q_heads*head_dim]                     */
+  DEC_LW_POST_NORM,    /* bf16 [hidden]                    post-attn RMSNorm   */
+  DEC_LW_GATE,         /* bf16 [ffn, hidden]                                    */
+  DEC_LW_UP,           /* bf16 [ffn, hidden]                                    */
+  DEC_LW_DOWN,         /* bf16 [hidden, ffn]                                    */
+  DEC_LW_COUNT
+} dec_layer_weight;
+
+typedef struct dec_weights {
+  const void *embed;        /* bf16 [vocab, hidden] */
+  const void *lm_head;      /* bf16 [vocab, hidden]; may equal embed (tied) */
+  const void *final_norm;   /* bf16 [hidden] */
+  /* HOST array of n_layers * DEC_LW_COUNT device pointers, layer-major in
+   * dec_layer_weight order; copied by dec_init, may be freed afterwards.
+   * Every weight pointer must be 16-byte aligned. */
+  const void *const *layers;
+} dec_weights;
+
+typedef struct dec_handle dec_handle;
+
+/* Create a handle for the current CUDA device.  Validates the shape, copies
+ * the weight pointer table (not the weights: they stay caller-owned and must
+ * stay alive and unchanged), allocates the workspace (activation exchange
+ * buffers, attention partials, counters; a few MB) and picks the kernel
+ * configuration.  Synchronous.  Returns DEC_ERR_SHAPE for unsupported shapes
+ * and DEC_ERR_DEVICE if the device is not compute capability 10.0. */
+int dec_init(const dec_shape *shape, const dec_weights *weights, dec_handle **out);
+
+/* Release the handle and its workspace (synchronises the device first). */
+void dec_free(dec_handle *h);
+
+/* ------------------------------------------------------------------ */
+/* KV cache                                                            */
+/* ------------------------------------------------------------------ */
+typedef enum dec_kv_dtype { DEC_KV_BF16 = 0, DEC_KV_FP8_E4M3 = 1 } dec_kv_dtype;
+
+/* A KV cache bound to a caller buffer.  Layout (fixed, so that a caller can
+ * prefill it):
+ *   bf16: values  [n_layers][2 (K,V)][batch][n_kv_heads][max_ctx][head_dim]
+ *   fp8 : codes   [n_layers][2][batch][n_kv_heads][max_ctx][head_dim] (uint8)
+ *         then, at byte offset dec_kv_scale_offset(), fp32 scales
+ *               [n_layers][2][batch][n_kv_heads][max_ctx]
+ * Row p of (layer, K/V, b, head) holds the key / value of the token at
+ * position p of sequence b (after q/k norm and rotation for K). */
+typedef struct dec_kv {
+  void *base;         /* device, 256-byte aligned */
+  size_t bytes;
+  int batch;
+  int max_ctx;
+  int dtype;          /* dec_kv_dtype */
+} dec_kv;
+
+/* Bytes a cache of this size needs (0 for an invalid request). */
+size_t dec_kv_bytes(const dec_handle *h, int batch, int max_ctx, int dtype);
+
+/* Byte offset of the fp32 scale array inside an fp8 cache (0 for bf16). */
+size_t dec_kv_scale_offset(const dec_handle *h, int batch, int max_ctx, int dtype);
+
+/* Bind a caller-owned device buffer as a KV cache.  Allocates nothing and
+ * does not touch the buffer's contents.  DEC_ERR_KV_SIZE if buf_bytes <
+ * dec_kv_bytes(), DEC_ERR_ALIGN unless buf is 256-byte aligned. */
+int dec_kv_alloc(dec_handle *h, int batch, int max_ctx, int dtype, void *buf,
+                 size_t buf_bytes, dec_kv *out);
+
+/* ------------------------------------------------------------------ */
+/* Decode step                                                         */
+/* ------------------------------------------------------------------ */
+
+/* One greedy decode step for sequences 0..batch-1 of `kv`.
+ *   token_ids  int32 [batch]  the current token of every sequence
+ *   positions  int32 [batch]  p_b: the row the new K/V are written to; the
+ *                             step attends over rows 0..p_b.  The caller
+ *                             (host) owns the lengths: it writes positions
+ *                             every step; the library never reads them back.
+ *   out_ids    int32 [batch]  argmax token of every sequence; may alias
+ *                             token_ids (self-feeding decode).
+ *   out_logits fp32 [batch, vocab] or NULL.
+ * One kernel launch on `stream`; never synchronises.  Invalid positions or
+ * tokens are detected on the device: the step then writes -1 to out_ids,
+ * leaves the cache unchanged and raises a bit that dec_check() returns. */
+int dec_step(dec_handle *h, int batch, const int32_t *token_ids, const int32_t *positions,
+             const dec_kv *kv, int32_t *out_ids, float *out_logits, void *stream);
+
+/* dec_step plus the residual stream after the embedding and after every
+ * layer: hidden_out fp32 [n_layers + 1][batch][hidden] (device). */
+int dec_step_debug(dec_handle *h, int batch, const int32_t *token_ids,
+                   const int32_t *positions, const dec_kv *kv, int32_t *out_ids,
+                   float *out_logits, float *hidden_out, void *stream);
+
+/* dec_step with HOST inputs and outputs: copies token_ids / positions (host,
+ * int32 [batch]) to the device, runs the step, copies out_ids (host) and, if
+ * non-NULL, out_logits (host, fp32 [batch, vocab]) back, and synchronises
+ * `stream` before returning. */
+int dec_step_host(dec_handle *h, int batch, const int32_t *token_ids_host,
+                  const int32_t *positions_host, const dec_kv *kv, int32_t *out_ids_host,
+                  float *out_logits_host, void *stream);
+
+/* Synchronise `stream`, then return and clear the device status bits
+ * (DEC_DEV_*; 0 when every step since the last check was clean), or a
+ * negative dec_status if the synchronisation itself failed. */
+int dec_check(dec_handle *h, void *stream);
+
+/* Bound of every device-side wait, in nanoseconds (default 2e9).  A wait
+ * that runs out sets DEC_DEV_TIMEOUT, the step drains its copies in flight
+ * and returns with out_ids = -1; the context stays usable. */
+int dec_set_timeout_ns(dec_handle *h, unsigned long long ns);
+
+/* Test hook: 0 = normal; k > 0 makes CTA k-1 skip publishing its share of the
+ * first layer's o_proj output, so that every other CTA's bounded wait on it
+ * runs out (exercises the timeout path without any fault). */
+int dec_set_debug_stall(dec_handle *h, int cta_plus_one);
+
+/* Human-readable name of a dec_status value or DEC_DEV_* bit set. */
+const char *dec_error_string(int code);
+
+/* The last CUDA error code a call on any handle saw (cudaError_t as int). */
+int dec_last_cuda_error(void);
+
+/* Kernel configuration chosen by dec_init (for reports): CTAs per step,
+ * ring slots per CTA and slot bytes. */
+int dec_get_config(const dec_handle *h, int *ctas, int *ring_slots, int *slot_bytes);
+
+/* ------------------------------------------------------------------ */
+/* Isolated grouped-query decode attention                             */
+/* ------------------------------------------------------------------ */
+
+/* Split-K (flash-decoding) GQA attention of one query token per sequence over
+ * its cached rows, fp32 softmax ("Latency & Bottleneck Analysis", 07 Root
+ * causes: repeat_kv, QK^T, mask, fp32 softmax, AV in one kernel instead of
+ * ~10 launches per layer):
+ *   out[b, h, :] = sum_j softmax_j(q[b,h,:] . K[b,g,j,:] / sqrt(head_dim)) V[b,g,j,:],
+ *   g = floor(h * n_kv_heads / n_q_heads), j = 0 .. lengths[b]-1.
+ *   q          bf16 [batch, n_q_heads, head_dim]
+ *   k_cache,
+ *   v_cache    bf16 [batch, n_kv_heads, max_len, head_dim] (rows >= lengths[b]
+ *              are not read)
+ *   lengths    int32 [batch] (device), each in [1, max_len]
+ *   out        fp32 [batch, n_q_heads, head_dim]
+ *   workspace  device scratch of dec_attention_workspace_bytes() bytes,
+ *              256-byte aligned, zero-filled by the caller before its first
+ *              use; every completed call leaves it ready for the next one
+ *              (calls sharing one workspace must not overlap on the GPU).
+ * head_dim 64 or 128; n_q_heads/n_kv_heads <= 8.  Lengths outside [1,
+ * max_len] raise DEC_DEV_BAD_POSITION in `status` (device int, may be NULL)
+ * and that sequence's output is left untouched. */
+size_t dec_attention_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int head_dim,
+                                     int max_len);
+int dec_attention(int batch, int n_q_heads, int n_kv_heads, int head_dim, const void *q,
+                  const void *k_cache, const void *v_cache, int max_len,
+                  const int32_t *lengths, float *out, void *workspace,
+                  size_t workspace_bytes, int *status, void *stream);
+
+/* ------------------------------------------------------------------ */
+/* FP8 cache rows                                                      */
+/* ------------------------------------------------------------------ */
+
+/* Quantise `rows` rows of `dim` (64 or 128) fp32 values to OCP E4M3 codes with
+ * one fp32 scale per row, exactly as dec_step stores the rows it appends to an
+ * FP8 cache (Baseten Qwen3-ASR article, KV cache quantization: FP8 storage,
+ * full-precision attention math): scale = max(amax, 2^-126)/448 and
+ * code = RNE-satfinite(x/scale), both divisions in IEEE fp32.  Use it to fill
+ * an FP8 cache from a bf16/fp32 prefill.  x fp32 [rows, dim], codes uint8
+ * [rows, dim], scales fp32 [rows] (all device).  Asynchronous on `stream`. */
+int dec_kv_quantize_e4m3(const float *x, int rows, int dim, uint8_t *codes, float *scales,
+                         void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DEC_H */
