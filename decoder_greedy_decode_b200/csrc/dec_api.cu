@@ -45,7 +45,7 @@ struct dec_handle {
 
 static int check_shape(const dec_shape* s) {
   if (!s) return DEC_ERR_NULL;
-  if (s->n_layers < 1 || s->n_layers > 255) return DEC_ERR_SHAPE;
+  if (s->n_layers < 1 || s->n_layers > 64) return DEC_ERR_SHAPE;
   if (s->hidden < 256 || s->hidden % 256 || s->hidden > 6144) return DEC_ERR_SHAPE;
   if (s->ffn < 256 || s->ffn % 256 || s->ffn > 6144) return DEC_ERR_SHAPE;
   if (s->head_dim != 64 && s->head_dim != 128) return DEC_ERR_SHAPE;
@@ -98,12 +98,12 @@ extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle
   }
   const int nchunks = h->ctas + 1;
   for (int b = 1; b <= B; ++b) {
-    h->nslot[b] = step_max_slots(b, H, F, HqD, D, rep, nchunks, h->smem_optin);
+    h->nslot[b] = step_max_slots(b, H, F, HqD, D, rep, h->smem_optin);
     if (h->nslot[b] < 2) {
       delete h;
       return DEC_ERR_DEVICE;
     }
-    h->smem[b] = step_smem_bytes(h->nslot[b], b, H, F, HqD, D, rep, nchunks);
+    h->smem[b] = step_smem_bytes(h->nslot[b], b, H, F, HqD, D, rep);
   }
   h->embed = static_cast<const uint16_t*>(w->embed);
   h->lm_head = static_cast<const uint16_t*>(w->lm_head);
@@ -135,7 +135,7 @@ extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle
   wl.pos_dev = take(sizeof(int32_t) * B);
   wl.out_dev = take(sizeof(int32_t) * B);
 #ifdef DEC_PROFILE
-  wl.prof = take(sizeof(unsigned long long) * h->ctas * (8 * L + 4));
+  wl.prof = take(sizeof(unsigned long long) * h->ctas * (16 * L + 8));
 #endif
   size_t layers_off = take(sizeof(LayerPtrs) * L);
   size_t logits_off = take(sizeof(float) * static_cast<size_t>(B) * shape->vocab);
@@ -444,10 +444,10 @@ extern "C" int dec_kv_quantize_e4m3(const float* x, int rows, int dim, uint8_t* 
 
 #ifdef DEC_PROFILE
 // Profiling builds only (not part of dec.h): copy the per-phase timestamps of
-// the last step, [ctas][8 * n_layers + 4] globaltimer values, to `host`.
+// the last step, [ctas][16 * n_layers + 8] globaltimer values, to `host`.
 extern "C" int dec_prof_read(dec_handle* h, unsigned long long* host, size_t n) {
   if (!h || !host) return DEC_ERR_NULL;
-  const size_t need = static_cast<size_t>(h->ctas) * (8 * h->shape.n_layers + 4);
+  const size_t need = static_cast<size_t>(h->ctas) * (16 * h->shape.n_layers + 8);
   if (n < need) return DEC_ERR_ARG;
   cudaError_t e = cudaMemcpy(host, h->ws + h->wl.prof, need * sizeof(unsigned long long),
                              cudaMemcpyDeviceToHost);

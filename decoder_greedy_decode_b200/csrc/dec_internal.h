@@ -5,7 +5,7 @@
 
 namespace dec {
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 7;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kStepThreads = kConsumerThreads + 32;  // + one producer warp
 constexpr int kSlotBytes = 24576;                   // ring slot: 12 rows of 1024 bf16
@@ -66,8 +66,8 @@ struct WorkspaceLayout {
   int part_chunks;
 };
 
-size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep, int nchunks);
-int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int nchunks, int smem_optin);
+size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep);
+int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int smem_optin);
 cudaError_t launch_step_small(const StepArgs& a, int ctas, size_t smem, cudaStream_t s);
 
 // Isolated split-K decode attention.

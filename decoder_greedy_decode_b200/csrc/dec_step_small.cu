@@ -42,19 +42,28 @@ constexpr int kMaxHRows = 64;  // hidden rows a CTA may own
 constexpr int kDevTimeout = 4;
 constexpr int kDevBadPos = 1;
 constexpr int kDevBadTok = 2;
+// Tagged words one gather pass stages in shared memory (24 KB).
+constexpr int kStageWords = 3072;
+
+// Stages of one layer; the lm_head runs as stage SQ of layer L (code SLM).
+enum { SQ = 0, SA, SO, SU, SD, kStages, SLM = kStages };
 
 // Optional per-phase timestamps (profiling builds only, -DDEC_PROFILE): thread
 // 0 of every CTA records globaltimer at the phase boundaries of the step into
-// prof[cta][8 * L + 4]: 8l+0 layer start, +1 QKV published, +2 attention
-// inputs gathered and rotated, +3 attention rows consumed and merged, +4
-// attention done, +5 o_proj published, +6 gate/up published, +7 down
-// published; 8L+0 lm_head start, +1 lm_head done, +2 consumer end,
-// +3 consumer start.
+// prof[cta][kStampsPerLayer * L + 8] at the points named by the St* indices
+// below (per layer), then lm_head start / gathered / done, consumer end and
+// consumer start.
+constexpr int kStampsPerLayer = 16;
+enum {
+  StStart = 0, StQGath, StQNorm, StQkv, StAttIn, StAttRows, StAtt, StOGath, StO, StUGath, StUNorm,
+  StU, StDGath, StD
+};
+enum { StLmStart = 0, StLmGath, StLmDone, StEnd, StBegin };
 #ifdef DEC_PROFILE
 #define DEC_STAMP(i)                                                                   \
   do {                                                                                 \
     if (a.prof && tid == 0)                                                            \
-      a.prof[static_cast<size_t>(cta) * (8 * a.L + 4) + (i)] = globaltimer();          \
+      a.prof[static_cast<size_t>(cta) * (kStampsPerLayer * a.L + 8) + (i)] = globaltimer(); \
   } while (0)
 #else
 #define DEC_STAMP(i) \
@@ -66,14 +75,17 @@ __host__ __device__ inline int split_at(int n, int parts, int i) {
   return static_cast<int>((static_cast<long long>(n) * i) / parts);
 }
 
+constexpr int kMaxLayers = 64;  // layer pointer table kept in shared memory
+// Fewer, longer attention chunks keep the combine to one round of loads.
+constexpr int kMinChunkRows = 96;
+
 struct Carve {
-  size_t ring, bars, act, xown, red, bred, ints, total;
+  size_t ring, bars, act, stg, xown, bred, ints, lw, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline Carve carve(int nslot, int B, int kmax, int rmax, int D, int rep,
-                                       int nchunks) {
+__host__ __device__ inline Carve carve(int nslot, int B, int kmax, int D, int rep) {
   Carve c;
   size_t o = 0;
   c.ring = o;
@@ -81,18 +93,19 @@ __host__ __device__ inline Carve carve(int nslot, int B, int kmax, int rmax, int
   c.bars = o;
   o += align_up(2 * nslot * sizeof(uint64_t), 16);
   size_t act_f = static_cast<size_t>(B) * kmax;
-  size_t att_f = static_cast<size_t>(rep + 2) * D + static_cast<size_t>(kCW + rep) * (D + 2) +
-                 static_cast<size_t>(nchunks) * rep * 2;
+  size_t att_f = static_cast<size_t>(rep + 2) * D + static_cast<size_t>(kCW + rep) * (D + 2);
   c.act = o;
   o += align_up((act_f > att_f ? act_f : att_f) * sizeof(float), 16);
+  c.stg = o;
+  o += static_cast<size_t>(kStageWords) * sizeof(uint64_t);
   c.xown = o;
   o += align_up(static_cast<size_t>(kMaxHRows) * B * sizeof(float), 16);
-  c.red = o;
-  o += align_up(2ull * rmax * B * kCW * sizeof(float), 16);
   c.bred = o;
   o += align_up(2ull * kCW * B * sizeof(float) + 2ull * kCW * B * sizeof(int), 16);
   c.ints = o;
   o += 64 * sizeof(int);
+  c.lw = o;
+  o += align_up(sizeof(LayerPtrs) * kMaxLayers, 16);
   c.total = o;
   return c;
 }
@@ -117,6 +130,19 @@ struct Spin {
   }
 };
 
+// sin and cos of an fp32 rotary angle x (0 <= x < 2^16 * 2pi): Cody-Waite
+// reduction by 2pi split into three fp32 parts (c1 has 8 significant bits,
+// so k * c1 is exact for |k| < 2^16), then the fast hardware sin/cos on
+// [-pi, pi], where its absolute error is about 2^-21.
+__device__ __forceinline__ void rope_sincos(float x, float* sn, float* cs) {
+  const float c1 = 6.28125f, c2 = 1.9353071693331003e-3f, c3 = 1.0253376273028358e-11f;
+  const float k = rintf(x * 0.15915493667125702f);
+  float r = fmaf(-k, c1, x);
+  r = fmaf(-k, c2, r);
+  r = fmaf(-k, c3, r);
+  __sincosf(r, sn, cs);
+}
+
 __device__ __forceinline__ float dot8(const uint4 w, const float* x) {
   float s = bf16lo(w.x) * x[0];
   s = fmaf(bf16hi(w.x), x[1], s);
@@ -129,8 +155,95 @@ __device__ __forceinline__ float dot8(const uint4 w, const float* x) {
   return s;
 }
 
-// The per-launch state of one CTA.
-template <int B, int D>
+// Dot products of R weight rows (shared memory, rows row_bytes apart, row i
+// at rows[i]) with the activation rows of B sequences (shared memory, act_stride
+// floats apart), K = 8 * nv columns; lane l takes 16-byte column vectors l,
+// l + 32, ...  Returns the transposed-butterfly reduction: every lane gets the
+// full sum of row (R == 4: lane >> 3; R == 2: lane >> 4; R == 1: 0) for each b.
+// Compiled on its own (not inlined) so that its register allocation and
+// scheduling do not depend on the rest of the persistent kernel.
+template <int R, int B>
+struct GroupSums {
+  float s[B];
+};
+
+template <int R>
+__device__ __forceinline__ float tbfly_lane(float (&p)[R], int lane) {
+  if constexpr (R == 1) {
+    return warp_sum(p[0]);
+  } else if constexpr (R == 2) {
+    const bool hi = lane & 16;
+    float k = hi ? p[1] : p[0];
+    k += __shfl_xor_sync(0xffffffffu, hi ? p[0] : p[1], 16);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+    return k;
+  } else {
+    const bool h16 = lane & 16;
+    float k0 = h16 ? p[2] : p[0], k1 = h16 ? p[3] : p[1];
+    k0 += __shfl_xor_sync(0xffffffffu, h16 ? p[0] : p[2], 16);
+    k1 += __shfl_xor_sync(0xffffffffu, h16 ? p[1] : p[3], 16);
+    const bool h8 = lane & 8;
+    float k = h8 ? k1 : k0;
+    k += __shfl_xor_sync(0xffffffffu, h8 ? k0 : k1, 8);
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+    return k;
+  }
+}
+
+template <int R, int B>
+__device__ __noinline__ GroupSums<R, B> group_dot(const uint32_t* rows, uint32_t act, int act_stride,
+                                                  int nv, int lane) {
+  // two accumulator banks (even / odd column vectors): twice the independent
+  // FMA chains
+  float acc[R][B], acc2[R][B];
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int b = 0; b < B; ++b) acc[i][b] = acc2[i][b] = 0.f;
+#pragma unroll 2
+  for (int v = lane; v < nv; v += 32) {
+    const bool odd = (v >> 5) & 1;
+    float x[B][8];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const uint32_t xa = act + static_cast<uint32_t>(b * act_stride + v * 8) * 4u;
+      asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                   : "=f"(x[b][0]), "=f"(x[b][1]), "=f"(x[b][2]), "=f"(x[b][3]) : "r"(xa));
+      asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                   : "=f"(x[b][4]), "=f"(x[b][5]), "=f"(x[b][6]), "=f"(x[b][7]) : "r"(xa + 16));
+    }
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      uint4 w;
+      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w) : "r"(rows[i] + v * 16));
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const float d = dot8(w, x[b]);
+        if (odd) acc2[i][b] += d;
+        else acc[i][b] += d;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int b = 0; b < B; ++b) acc[i][b] += acc2[i][b];
+  GroupSums<R, B> out;
+#pragma unroll
+  for (int b = 0; b < B; ++b) {
+    float col[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) col[i] = acc[i][b];
+    out.s[b] = tbfly_lane<R>(col, lane);
+  }
+  return out;
+}
+
+// The per-launch state of one CTA.  FP8: the cache holds E4M3 codes + scales.
+template <int B, int D, bool FP8>
 struct Cta {
   static constexpr int DL = D / 32;  // attention dims per lane
   const StepArgs& a;
@@ -139,12 +252,13 @@ struct Cta {
   uint64_t* empty;
   float* act;
   float* xown;
-  float* red;
+  uint64_t* stg;  // gather staging: tagged words
   float* bredf;
   int* bredi;
   int* sints;
+  const LayerPtrs* slw;  // layer pointer table copied to shared memory
   int tid, warp, lane, cta, nc;
-  int kmax, rmax, nqkv;
+  int kmax, nqkv;
   uint32_t seq;
   // per-CTA row ranges
   int q0, q1, h0, h1, f0, f1, v0, v1;
@@ -155,19 +269,19 @@ struct Cta {
   int* tok;     // [B] tokens (shared memory)
   int* nchunk;  // [B] attention chunks per KV head (shared memory)
 
-  __device__ Cta(const StepArgs& args, uint8_t* smem, int kmax_, int rmax_)
-      : a(args), kmax(kmax_), rmax(rmax_) {
+  __device__ Cta(const StepArgs& args, uint8_t* smem, int kmax_) : a(args), kmax(kmax_) {
     const int rep = a.Hq / a.Hkv;
-    Carve c = carve(a.nslot, B, kmax, rmax, D, rep, a.part_chunks);
+    Carve c = carve(a.nslot, B, kmax, D, rep);
     ring = smem + c.ring;
     full = reinterpret_cast<uint64_t*>(smem + c.bars);
     empty = full + a.nslot;
     act = reinterpret_cast<float*>(smem + c.act);
     xown = reinterpret_cast<float*>(smem + c.xown);
-    red = reinterpret_cast<float*>(smem + c.red);
+    stg = reinterpret_cast<uint64_t*>(smem + c.stg);
     bredf = reinterpret_cast<float*>(smem + c.bred);
     bredi = reinterpret_cast<int*>(bredf + 2 * kCW * B);
     sints = reinterpret_cast<int*>(smem + c.ints);
+    slw = reinterpret_cast<const LayerPtrs*>(smem + c.lw);
     pos = sints + 8;
     tok = sints + 16;
     nchunk = sints + 24;
@@ -189,7 +303,7 @@ struct Cta {
     rpt_o = kSlotBytes / (2 * a.Hq * D);
     rpt_u = kSlotBytes / (4 * a.H);
     rpt_d = kSlotBytes / (2 * a.F);
-    if (a.kv_fp8) {
+    if constexpr (FP8) {
       art = (kSlotBytes / (2 * D + 8)) & ~15;
     } else {
       art = kSlotBytes / (4 * D);
@@ -209,7 +323,7 @@ struct Cta {
     if (slots < 1) slots = 1;
     long long cr = (T + slots - 1) / slots;
     cr = (cr + 15) / 16 * 16;
-    if (cr < 16) cr = 16;
+    if (cr < kMinChunkRows) cr = kMinChunkRows;
     crow = static_cast<int>(cr);
     n_items = 0;
     for (int b = 0; b < a.B; ++b) {
@@ -241,27 +355,38 @@ struct Cta {
   }
   __device__ void produce() {
     const uint64_t pol = policy_evict_first();
-    uint32_t n = 0;
+    uint32_t n = 0;     // tiles issued
+    int ps = 0;         // ring slot of tile n
+    uint32_t lap = 0;   // n / nslot
+    uint64_t* fb = full;
     bool dead = false;
     const int ns = a.nslot;
+    // Slot for tile n, once the consumers released its previous use; arms its
+    // full barrier with the tile's byte count.
     auto acquire = [&](uint32_t bytes) -> uint8_t* {
-      const int slot = static_cast<int>(n % ns);
-      if (n >= static_cast<uint32_t>(ns)) {
-        const uint32_t par = ((n / ns) - 1) & 1;
+      if (lap > 0) {
         Spin sp;
-        while (!mbar_test(&empty[slot], par)) {
+        while (!mbar_wait(&empty[ps], (lap - 1) & 1, 20000)) {
           if (sp.tick(a, false)) {
             dead = true;
             return nullptr;
           }
         }
       }
-      mbar_arrive_expect_tx(&full[slot], bytes);
-      return ring + static_cast<size_t>(slot) * kSlotBytes;
+      fb = &full[ps];
+      mbar_arrive_expect_tx(fb, bytes);
+      return ring + static_cast<size_t>(ps) * kSlotBytes;
+    };
+    auto advance = [&]() {
+      ++n;
+      if (++ps == ns) {
+        ps = 0;
+        ++lap;
+      }
     };
     const int H = a.H, HqD = a.Hq * D, HkvD = a.Hkv * D;
     for (int l = 0; l < a.L && !dead; ++l) {
-      const LayerPtrs& lw = a.layers[l];
+      const LayerPtrs& lw = slw[l];
       // ---- QKV rows [q0, q1) of [Wq; Wk; Wv]
       for (int r = q0; r < q1 && !dead; r += rpt_h) {
         const int nr = min(rpt_h, q1 - r);
@@ -279,12 +404,12 @@ struct Cta {
             base = lw.w[3]; lo = rr - HqD - HkvD; cnt = left;
           }
           bulk_g2s(dst, base + static_cast<size_t>(lo) * H, static_cast<uint32_t>(cnt) * H * 2,
-                   &full[n % ns], pol);
+                   fb, pol);
           dst += static_cast<size_t>(cnt) * H * 2;
           rr += cnt;
           left -= cnt;
         }
-        ++n;
+        advance();
       }
       // ---- attention: cached rows [j0, min(j1, p_b)) of every item of this CTA
       for (int it = cta; it < n_items && !dead; it += nc) {
@@ -294,25 +419,25 @@ struct Cta {
         const int jc = min(j0 + crow, pos[b]);
         for (int j = j0; j < jc && !dead; j += art) {
           const int nr = min(art, jc - j);
-          if (!a.kv_fp8) {
+          if constexpr (!FP8) {
             const uint32_t rb = static_cast<uint32_t>(nr) * D * 2;
             uint8_t* dst = acquire(2 * rb);
             if (!dst) break;
             const uint16_t* kvb = reinterpret_cast<const uint16_t*>(a.kv);
-            bulk_g2s(dst, kvb + kv_row(l, 0, b, g, j) * D, rb, &full[n % ns], pol);
-            bulk_g2s(dst + rb, kvb + kv_row(l, 1, b, g, j) * D, rb, &full[n % ns], pol);
+            bulk_g2s(dst, kvb + kv_row(l, 0, b, g, j) * D, rb, fb, pol);
+            bulk_g2s(dst + rb, kvb + kv_row(l, 1, b, g, j) * D, rb, fb, pol);
           } else {
             const uint32_t rb = static_cast<uint32_t>(nr) * D;
             const uint32_t sb = static_cast<uint32_t>((nr + 3) & ~3) * 4;
             uint8_t* dst = acquire(2 * rb + 2 * sb);
             if (!dst) break;
-            bulk_g2s(dst, a.kv + kv_row(l, 0, b, g, j) * D, rb, &full[n % ns], pol);
-            bulk_g2s(dst + rb, a.kv + kv_row(l, 1, b, g, j) * D, rb, &full[n % ns], pol);
-            bulk_g2s(dst + 2 * rb, a.kv_scales + kv_row(l, 0, b, g, j), sb, &full[n % ns], pol);
-            bulk_g2s(dst + 2 * rb + sb, a.kv_scales + kv_row(l, 1, b, g, j), sb, &full[n % ns],
+            bulk_g2s(dst, a.kv + kv_row(l, 0, b, g, j) * D, rb, fb, pol);
+            bulk_g2s(dst + rb, a.kv + kv_row(l, 1, b, g, j) * D, rb, fb, pol);
+            bulk_g2s(dst + 2 * rb, a.kv_scales + kv_row(l, 0, b, g, j), sb, fb, pol);
+            bulk_g2s(dst + 2 * rb + sb, a.kv_scales + kv_row(l, 1, b, g, j), sb, fb,
                      pol);
           }
-          ++n;
+          advance();
         }
       }
       // ---- o_proj rows [h0, h1), K = Hq*D
@@ -321,8 +446,8 @@ struct Cta {
         uint8_t* dst = acquire(static_cast<uint32_t>(nr) * HqD * 2);
         if (!dst) break;
         bulk_g2s(dst, lw.w[6] + static_cast<size_t>(r) * HqD, static_cast<uint32_t>(nr) * HqD * 2,
-                 &full[n % ns], pol);
-        ++n;
+                 fb, pol);
+        advance();
       }
       // ---- gate / up rows [f0, f1): a tile is nr gate rows then nr up rows
       for (int r = f0; r < f1 && !dead; r += rpt_u) {
@@ -330,9 +455,9 @@ struct Cta {
         const uint32_t rb = static_cast<uint32_t>(nr) * H * 2;
         uint8_t* dst = acquire(2 * rb);
         if (!dst) break;
-        bulk_g2s(dst, lw.w[8] + static_cast<size_t>(r) * H, rb, &full[n % ns], pol);
-        bulk_g2s(dst + rb, lw.w[9] + static_cast<size_t>(r) * H, rb, &full[n % ns], pol);
-        ++n;
+        bulk_g2s(dst, lw.w[8] + static_cast<size_t>(r) * H, rb, fb, pol);
+        bulk_g2s(dst + rb, lw.w[9] + static_cast<size_t>(r) * H, rb, fb, pol);
+        advance();
       }
       // ---- down rows [h0, h1), K = F
       for (int r = h0; r < h1 && !dead; r += rpt_d) {
@@ -340,8 +465,8 @@ struct Cta {
         uint8_t* dst = acquire(static_cast<uint32_t>(nr) * a.F * 2);
         if (!dst) break;
         bulk_g2s(dst, lw.w[10] + static_cast<size_t>(r) * a.F,
-                 static_cast<uint32_t>(nr) * a.F * 2, &full[n % ns], pol);
-        ++n;
+                 static_cast<uint32_t>(nr) * a.F * 2, fb, pol);
+        advance();
       }
     }
     // ---- lm_head rows [v0, v1)
@@ -350,8 +475,8 @@ struct Cta {
       uint8_t* dst = acquire(static_cast<uint32_t>(nr) * H * 2);
       if (!dst) break;
       bulk_g2s(dst, a.lm_head + static_cast<size_t>(r) * H, static_cast<uint32_t>(nr) * H * 2,
-               &full[n % ns], pol);
-      ++n;
+               fb, pol);
+      advance();
     }
     // Every copy issued must land before the CTA exits: wait for the last
     // phase armed on each slot (returns at once when consumers already did).
@@ -366,76 +491,143 @@ struct Cta {
   }
 
   // ================================================================ consumers
-  uint32_t rn = 0;         // ring tile counter (consumer side)
+  uint32_t rn = 0;         // ring tiles consumed
+  int rs = 0;              // ring slot of tile rn
+  uint32_t rph = 0;        // full-barrier phase parity of tile rn
   int ab = 0;              // aborted: keep the barrier sequence, compute nothing
   bool ring_dead = false;  // a ring wait ran out: stop waiting on the ring
+  float best_v[B];         // lm_head argmax of this thread, per sequence
+  int best_i[B];
 
   __device__ __forceinline__ void csync() { named_sync(1, kCT); }
 
   // Wait for ring tile rn.  Every consumer thread calls it for every tile, so
-  // the barrier sequence stays uniform even when a wait runs out: the thread
-  // then only stops computing (ab) and stops waiting on the ring.
-  // The outcome is made warp-uniform (__all_sync / __any_sync) so that warp
-  // collectives after it never see a split warp.
+  // the barrier sequence stays uniform even when a wait runs out: the warp
+  // then only stops computing (ab) and stops waiting on the ring.  Lane 0
+  // polls; the outcome is broadcast so that it is warp-uniform.
   __device__ void wait_tile() {
     if (ring_dead) return;
-    const int slot = static_cast<int>(rn % a.nslot);
-    const uint32_t par = (rn / a.nslot) & 1;
-    Spin sp;
-    while (true) {
-      const bool done = mbar_test(&full[slot], par);
-      if (__all_sync(0xffffffffu, done)) break;
-      const bool out = sp.tick(a, false);
-      if (__any_sync(0xffffffffu, out)) {
-        ring_dead = true;
-        ab = 1;
-        return;
+    const int slot = rs;
+    const uint32_t par = rph;
+    int st = 1;
+    if (lane == 0) {
+      Spin sp;
+      while (!mbar_wait(&full[slot], par, 20000)) {
+        if (sp.tick(a, false)) {
+          st = 0;
+          break;
+        }
       }
     }
+    st = __shfl_sync(0xffffffffu, st, 0);
+    if (!st) {
+      ring_dead = true;
+      ab = 1;
+      return;
+    }
+    (void)mbar_test(&full[slot], par);  // every lane observes the completed phase
   }
   __device__ __forceinline__ void release_tile() {
     __syncwarp();
-    if (lane == 0 && !ring_dead) mbar_arrive(&empty[rn % a.nslot]);
+    if (lane == 0 && !ring_dead) mbar_arrive(&empty[rs]);
     ++rn;
+    if (++rs == a.nslot) {
+      rs = 0;
+      rph ^= 1;
+    }
   }
 
-  // Poll `n` tagged words (element i at src[idx(i)]) until their flag is `f`,
-  // store the values to dst[i].  Collective over the consumer threads.
-  // All loads of a round are issued before any is checked, so a gather of up
-  // to 16 words per thread costs one L2 round trip when the data is there.
-  template <class Idx, class Didx>
-  __device__ void gather(const uint64_t* src, int n, uint32_t f, float* dst, Idx idx, Didx didx) {
-    constexpr int kRound = 8;
-    int fail = 0;
+  // Fetch n (even, <= kStageWords) tagged words into stg, word w from
+  // src_of(w) (16-byte aligned for even w), until every flag equals f.  All
+  // copies of a pass are in flight at once (cp.async through L2); a pass
+  // re-fetches only the words that were not ready, so the gather costs one
+  // round trip after the last producer published.  Collective over the
+  // consumer threads; ends with every word visible to every thread.
+  template <class Src>
+  __device__ void gather(int n, uint32_t f, Src src_of) {
+    const int nch = n >> 1;
+    uint32_t pend = 0;
     if (!ab) {
-      for (int base = tid; base < n && !fail; base += kCT * kRound) {
-        uint64_t w[kRound];
-#pragma unroll
-        for (int k = 0; k < kRound; ++k) {
-          const int i = base + k * kCT;
-          if (i < n) w[k] = ld_tagged(src + idx(i));
-        }
-#pragma unroll
-        for (int k = 0; k < kRound; ++k) {
-          const int i = base + k * kCT;
-          if (i < n && !fail) {
-            Spin sp;
-            while (static_cast<uint32_t>(w[k] >> 32) != f) {
-              if (sp.tick(a, true)) {
-                fail = 1;
-                break;
-              }
-              w[k] = ld_tagged(src + idx(i));
-            }
-            dst[didx(i)] = __uint_as_float(static_cast<uint32_t>(w[k]));
-          }
+      int k = 0;
+      for (int c = tid; c < nch; c += kCT, ++k) pend |= 1u << k;
+    }
+    int fail = 0;
+    uint64_t t0 = 0;
+    int more;
+    do {
+      int k = 0;
+      for (int c = tid; c < nch; c += kCT, ++k)
+        if (pend & (1u << k)) cp_async16_cg(stg + 2 * c, src_of(2 * c));
+      cp_async_wait_all();
+      k = 0;
+      for (int c = tid; c < nch; c += kCT, ++k) {
+        if (pend & (1u << k)) {
+          if (static_cast<uint32_t>(stg[2 * c] >> 32) == f &&
+              static_cast<uint32_t>(stg[2 * c + 1] >> 32) == f)
+            pend &= ~(1u << k);
         }
       }
-    }
+      if (pend) {
+        const uint64_t now = globaltimer();
+        if (t0 == 0) t0 = now;
+        if (now - t0 > a.timeout_ns) {
+          atomicOr(a.status, kDevTimeout);
+          atomicExch(a.abort_flag, 1);
+          fail = 1;
+        } else if (ld_relaxed_i32(a.abort_flag)) {
+          fail = 1;
+        }
+        if (fail) pend = 0;
+        else __nanosleep(64);
+      }
+      more = named_sync_or(1, kCT, pend != 0);
+    } while (more);
     ab = named_sync_or(1, kCT, fail | ab);
   }
-  // In-place RMSNorm of rows act[b][0..K) with bf16 gains g.
-  __device__ void rmsnorm_act(int K, const uint16_t* g) {
+
+  // B rows of K tagged words (row stride K) -> act rows (row stride kmax).
+  __device__ void gather_x(const uint64_t* src, int K, uint32_t f) {
+    const int n = a.B * K;
+    for (int w0 = 0; w0 < n; w0 += kStageWords) {
+      const int nw = min(kStageWords, n - w0);
+      gather(nw, f, [=](int w) { return src + w0 + w; });
+      if (!ab)
+        for (int i = tid; i < nw; i += kCT) {
+          const int idx = w0 + i;
+          act[(idx / K) * kmax + idx % K] = __uint_as_float(static_cast<uint32_t>(stg[i]));
+        }
+      csync();
+    }
+  }
+
+  // Layer 0 input: the embedding rows of the step's tokens.
+  __device__ void embed_rows() {
+    const int H = a.H;
+    for (int i = tid; i < a.B * H; i += kCT) {
+      const int b = i / H, k = i % H;
+      act[b * kmax + k] = bf16_to_f(a.embed[static_cast<size_t>(tok[b]) * H + k]);
+    }
+    csync();
+    for (int i = tid; i < (h1 - h0) * a.B; i += kCT) {
+      const int r = i / a.B, b = i % a.B;
+      xown[r * B + b] = act[b * kmax + h0 + r];
+      if (a.hidden_out) a.hidden_out[static_cast<size_t>(b) * H + h0 + r] = xown[r * B + b];
+    }
+  }
+
+  // Gains of an RMSNorm over K (thread tid handles k = tid + kCT * j), loaded
+  // before the gather that precedes the norm so that their latency overlaps it.
+  static constexpr int kGainRegs = 8;
+  __device__ __forceinline__ void load_gains(int K, const uint16_t* g, float (&gr)[kGainRegs]) const {
+#pragma unroll
+    for (int j = 0; j < kGainRegs; ++j) {
+      const int k = tid + kCT * j;
+      gr[j] = k < K ? bf16_to_f(__ldg(g + k)) : 0.f;
+    }
+  }
+  // In-place RMSNorm of rows act[b][0..K) with bf16 gains g (the first
+  // kGainRegs * kCT of them already in gr).
+  __device__ void rmsnorm_act(int K, const uint16_t* g, const float (&gr)[kGainRegs]) {
     if (!ab) {
       float ss[B];
 #pragma unroll
@@ -443,10 +635,8 @@ struct Cta {
       for (int k = tid; k < K; k += kCT) {
 #pragma unroll
         for (int b = 0; b < B; ++b) {
-          if (b < a.B) {
-            const float x = act[b * kmax + k];
-            ss[b] = fmaf(x, x, ss[b]);
-          }
+          const float x = act[b * kmax + k];
+          ss[b] = fmaf(x, x, ss[b]);
         }
       }
 #pragma unroll
@@ -461,18 +651,60 @@ struct Cta {
 #pragma unroll
       for (int b = 0; b < B; ++b) {
         float t = 0.f;
-#pragma unroll
         for (int w = 0; w < kCW; ++w) t += bredf[w * B + b];
         inv[b] = rsqrtf(t / static_cast<float>(K) + a.eps);
       }
-      for (int k = tid; k < K; k += kCT) {
+#pragma unroll
+      for (int j = 0; j < kGainRegs; ++j) {
+        const int k = tid + kCT * j;
+        if (k < K) {
+#pragma unroll
+          for (int b = 0; b < B; ++b) act[b * kmax + k] = act[b * kmax + k] * inv[b] * gr[j];
+        }
+      }
+      for (int k = tid + kCT * kGainRegs; k < K; k += kCT) {
         const float gk = bf16_to_f(g[k]);
 #pragma unroll
-        for (int b = 0; b < B; ++b)
-          if (b < a.B) act[b * kmax + k] = act[b * kmax + k] * inv[b] * gk;
+        for (int b = 0; b < B; ++b) act[b * kmax + k] = act[b * kmax + k] * inv[b] * gk;
       }
     }
     csync();
+  }
+
+  // What each projection does with its output row r of sequence b.
+  __device__ __forceinline__ void epilogue(int sc, int l, int r, int b, float s0, float s1) {
+    switch (sc) {
+      case SQ:
+        st_tagged(a.x_qkv + static_cast<size_t>(b) * nqkv + q0 + r, s0, flag(l));
+        break;
+      case SO: {  // o_proj + residual
+        const float x = xown[r * B + b] + s0;
+        xown[r * B + b] = x;
+        if (!(l == 0 && a.stall_cta == cta))
+          st_tagged(a.x_mid + static_cast<size_t>(b) * a.H + h0 + r, x, flag(l));
+        break;
+      }
+      case SU:  // SiLU(gate) * up
+        st_tagged(a.x_u + static_cast<size_t>(b) * a.F + f0 + r, s0 / (1.0f + __expf(-s0)) * s1,
+                  flag(l));
+        break;
+      case SD: {  // down + residual
+        const float x = xown[r * B + b] + s0;
+        xown[r * B + b] = x;
+        st_tagged(a.x_out + static_cast<size_t>(b) * a.H + h0 + r, x, flag(l));
+        if (a.hidden_out)
+          a.hidden_out[(static_cast<size_t>(l + 1) * a.B + b) * a.H + h0 + r] = x;
+        break;
+      }
+      default: {  // lm_head logit + running argmax (ties: lowest id)
+        const int id = v0 + r;
+        if (a.out_logits) a.out_logits[static_cast<size_t>(b) * a.V + id] = s0;
+        if (s0 > best_v[b] || (s0 == best_v[b] && id < best_i[b])) {
+          best_v[b] = s0;
+          best_i[b] = id;
+        }
+      }
+    }
   }
 
   // Row-group GEMV over ring tiles.  Rows [0, nrows) of the stage arrive
@@ -483,11 +715,9 @@ struct Cta {
   // sums with one transposed butterfly (R = 4: 6 shuffles instead of 20).
   // Groups are dealt to warps round-robin over the whole stage, so there is no
   // CTA barrier per tile.  Every warp waits for every tile (no warp can run a
-  // ring ahead of the others) and releases it.  epi(row, b, s0, s1) is called
-  // once per output row and sequence; s1 is the second matrix's sum in pair
-  // mode.
-  template <int R, class Epi>
-  __device__ void gemv(int K, int nrows, int rpt, bool pair, Epi epi) {
+  // ring ahead of the others) and releases it.
+  template <int R>
+  __device__ void gemv(int K, int nrows, int rpt, bool pair, int sc, int l) {
     const int nv = K >> 3;
     const int per = pair ? R / 2 : R;  // output rows per group
     int gbase = 0;
@@ -496,99 +726,75 @@ struct Cta {
       const int ng = (nr + per - 1) / per;
       wait_tile();
       if (!ab) {
-        const uint8_t* tb = ring + static_cast<size_t>(rn % a.nslot) * kSlotBytes;
+        const uint8_t* tb = ring + static_cast<size_t>(rs) * kSlotBytes;
         int g0 = (warp - gbase) % kCW;
         if (g0 < 0) g0 += kCW;
         for (int gl = g0; gl < ng; gl += kCW) {
-          const uint8_t* rp[R];
-          bool rv[R];
+          uint32_t rows[R];
 #pragma unroll
           for (int i = 0; i < R; ++i) {
             const int j = gl * per + (i % per);
-            rv[i] = j < nr;
             const int trow = (pair && i >= per) ? nr + j : j;
-            rp[i] = tb + static_cast<size_t>(rv[i] ? trow : 0) * K * 2;
+            rows[i] = smem_u32(tb) + static_cast<uint32_t>(j < nr ? trow : 0) * K * 2;
           }
-          float acc[R][B];
-#pragma unroll
-          for (int i = 0; i < R; ++i)
-#pragma unroll
-            for (int b = 0; b < B; ++b) acc[i][b] = 0.f;
-          for (int v = lane; v < nv; v += 32) {
-            float x[B][8];
-#pragma unroll
-            for (int b = 0; b < B; ++b) {
-              const float4* xa = reinterpret_cast<const float4*>(act + b * kmax + v * 8);
-              const float4 x0 = xa[0], x1 = xa[1];
-              x[b][0] = x0.x; x[b][1] = x0.y; x[b][2] = x0.z; x[b][3] = x0.w;
-              x[b][4] = x1.x; x[b][5] = x1.y; x[b][6] = x1.z; x[b][7] = x1.w;
-            }
-#pragma unroll
-            for (int i = 0; i < R; ++i) {
-              if (rv[i]) {
-                const uint4 w = *reinterpret_cast<const uint4*>(rp[i] + v * 16);
-#pragma unroll
-                for (int b = 0; b < B; ++b) acc[i][b] += dot8(w, x[b]);
-              }
-            }
-          }
+          const GroupSums<R, B> gs = group_dot<R, B>(rows, smem_u32(act), kmax, nv, lane);
           const int ri = R == 4 ? (lane >> 3) : (R == 2 ? (lane >> 4) : 0);
           const bool leader = R == 4 ? ((lane & 7) == 0) : (R == 2 ? ((lane & 15) == 0) : lane == 0);
-          float sv[B], su[B];
+          const int j = gl * per + ri;
 #pragma unroll
           for (int b = 0; b < B; ++b) {
-            float col[R];
-#pragma unroll
-            for (int i = 0; i < R; ++i) col[i] = acc[i][b];
-            sv[b] = tbfly<R>(col);
-            su[b] = __shfl_down_sync(0xffffffffu, sv[b], 16);
-          }
-          if (leader && (!pair || ri < per)) {
-            const int j = gl * per + ri;
-            if (j < nr) {
-#pragma unroll
-              for (int b = 0; b < B; ++b)
-                if (b < a.B) epi(r0 + j, b, sv[b], su[b]);
-            }
+            const float sv = gs.s[b];
+            const float su = __shfl_down_sync(0xffffffffu, sv, 16);
+            if (leader && (!pair || ri < per) && j < nr && b < a.B) epilogue(sc, l, r0 + j, b, sv, su);
           }
         }
       }
       gbase += ng;
       release_tile();
     }
-  }
-
-  // Transposed butterfly: lane l holds partial sums p[i] of R rows; returns
-  // the full sum of row (R == 4: l >> 3; R == 2: l >> 4; R == 1: 0).
-  template <int R>
-  __device__ __forceinline__ float tbfly(float (&p)[R]) const {
-    if constexpr (R == 1) {
-      return warp_sum(p[0]);
-    } else if constexpr (R == 2) {
-      const bool hi = lane & 16;
-      float k = hi ? p[1] : p[0];
-      k += __shfl_xor_sync(0xffffffffu, hi ? p[0] : p[1], 16);
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
-      return k;
-    } else {
-      const bool h16 = lane & 16;
-      float k0 = h16 ? p[2] : p[0], k1 = h16 ? p[3] : p[1];
-      k0 += __shfl_xor_sync(0xffffffffu, h16 ? p[0] : p[2], 16);
-      k1 += __shfl_xor_sync(0xffffffffu, h16 ? p[1] : p[3], 16);
-      const bool h8 = lane & 8;
-      float k = h8 ? k1 : k0;
-      k += __shfl_xor_sync(0xffffffffu, h8 ? k0 : k1, 8);
-#pragma unroll
-      for (int o = 4; o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
-      return k;
-    }
+    // the next stage overwrites act: every warp must be done reading it
+    csync();
   }
 
   // ------------------------------------------------------------- attention
-  // Stage buffer (in act): qs[rep][D] (normed, rotated q), kn[D], vn[D] (the
-  // new row as stored), merge[kCW][D + 2], ownb[rep][D + 2] (the
-  // combiner's own partial), mlb[chunks][rep][2] (other chunks' m, l).
+  // One K (or V) row slice of the lane from a ring tile: the lane holds dims
+  // [e8 * DQ, e8 * DQ + DQ) of tile row r (bf16 rows, or E4M3 codes with the
+  // row scales stored after the codes).
+  static constexpr int DQ = D / 8;
+  __device__ __forceinline__ void tile_row(const uint8_t* tb, int nr, int r, int e8, int kvsel,
+                                           float (&o)[DQ]) const {
+    if constexpr (!FP8) {
+      const uint8_t* p = tb + (static_cast<size_t>(kvsel) * nr + r) * D * 2 + e8 * DQ * 2;
+#pragma unroll
+      for (int c = 0; c < DQ / 8; ++c) {
+        const uint4 w = reinterpret_cast<const uint4*>(p)[c];
+        o[8 * c + 0] = bf16lo(w.x); o[8 * c + 1] = bf16hi(w.x);
+        o[8 * c + 2] = bf16lo(w.y); o[8 * c + 3] = bf16hi(w.y);
+        o[8 * c + 4] = bf16lo(w.z); o[8 * c + 5] = bf16hi(w.z);
+        o[8 * c + 6] = bf16lo(w.w); o[8 * c + 7] = bf16hi(w.w);
+      }
+    } else {
+      const uint8_t* p = tb + (static_cast<size_t>(kvsel) * nr + r) * D + e8 * DQ;
+      const int sb = ((nr + 3) & ~3) * 4;
+      const float sc = reinterpret_cast<const float*>(tb + 2 * nr * D + kvsel * sb)[r];
+#pragma unroll
+      for (int c = 0; c < DQ; c += 2) {
+        const float2 f2 = e4m3x2_to_f2(*reinterpret_cast<const uint16_t*>(p + c));
+        o[c] = f2.x * sc;
+        o[c + 1] = f2.y * sc;
+      }
+    }
+  }
+
+  // Split-K attention of one layer.  Item (b, g, chunk): the query heads of KV
+  // head g of sequence b over cached rows [j0, jc) streamed through the ring,
+  // plus the new row p_b (from the gathered q/k/v, rotated and rounded as the
+  // cache stores it; the CTA whose chunk holds p_b writes it to the cache).
+  // Warp w serves query head w % rep; within a warp, lane octet q8 takes every
+  // fourth row and each lane a D/8-wide slice (3-shuffle dot products).  The
+  // CTA of chunk 0 combines the chunks' partial softmax states and publishes
+  // the head outputs; other chunks publish their partial state and move on.
+  // act holds qs[rep][D], kn[D], vn[D], merge[kCW][D + 2], ownb[rep][D + 2].
   __device__ void attention(int l) {
     const int rep = a.Hq / a.Hkv;
     const float qscale = 1.4426950408889634f / sqrtf(static_cast<float>(D));  // log2(e)/sqrt(D)
@@ -597,10 +803,13 @@ struct Cta {
     float* vn = kn + D;
     float* merge = vn + D;
     float* ownb = merge + kCW * (D + 2);
-    float* mlb = ownb + rep * (D + 2);
-    const LayerPtrs& lw = a.layers[l];
+    const LayerPtrs& lw = slw[l];
     const uint32_t f = flag(l);
     const int HqD = a.Hq * D;
+    const int rstep = kCW / rep;
+    const int hw = warp % rep, rw = warp / rep;
+    const bool attw = warp < rstep * rep;
+    const int q8 = lane >> 3, e8 = lane & 7;
     for (int it = cta; it < n_items; it += nc) {
       int b, g, ci;
       item(it, b, g, ci);
@@ -609,17 +818,27 @@ struct Cta {
       const int j1 = min(j0 + crow, p + 1);
       const int jc = min(j1, p);  // cached rows [j0, jc)
       const bool has_new = (p >= j0 && p < j1);
-      // -- gather q heads of the group, k_g and v_g of sequence b
+      // norm gains and rotation frequencies, fetched before the gather
+      float gq[DL], invf[DL / 2];
+      {
+        const uint16_t* gn = warp < rep ? lw.w[4] : lw.w[5];
+#pragma unroll
+        for (int k = 0; k < DL; ++k) gq[k] = warp <= rep ? bf16_to_f(__ldg(gn + lane + 32 * k)) : 0.f;
+#pragma unroll
+        for (int k = 0; k < DL / 2; ++k) invf[k] = __ldg(a.inv_freq + lane + 32 * k);
+      }
+      // -- q heads of the group, k_g and v_g of sequence b -> qs, kn, vn
       {
         const uint64_t* src = a.x_qkv + static_cast<size_t>(b) * nqkv;
         const int qn = rep * D;
         const int qoff = g * rep * D, koff = HqD + g * D, voff = HqD + a.Hkv * D + g * D;
-        gather(
-            src, qn + 2 * D, f, act,
-            [=](int i) {
-              return i < qn ? qoff + i : (i < qn + D ? koff + (i - qn) : voff + (i - qn - D));
-            },
-            [](int i) { return i; });
+        gather(qn + 2 * D, f, [=](int w) {
+          return src + (w < qn ? qoff + w : (w < qn + D ? koff + (w - qn) : voff + (w - qn - D)));
+        });
+        if (!ab)
+          for (int i = tid; i < qn + 2 * D; i += kCT)
+            act[i] = __uint_as_float(static_cast<uint32_t>(stg[i]));
+        csync();
       }
       // -- q/k RMSNorm + RoPE (warp w < rep: q head; rep: k; rep+1: v)
       if (!ab && warp < rep + 2) {
@@ -628,20 +847,18 @@ struct Cta {
 #pragma unroll
         for (int k = 0; k < DL; ++k) v[k] = x[lane + 32 * k];
         if (warp <= rep) {
-          const uint16_t* gn = warp < rep ? lw.w[4] : lw.w[5];
           float ss = 0.f;
 #pragma unroll
           for (int k = 0; k < DL; ++k) ss = fmaf(v[k], v[k], ss);
           ss = warp_sum(ss);
           const float inv = rsqrtf(ss / static_cast<float>(D) + a.eps);
 #pragma unroll
-          for (int k = 0; k < DL; ++k) v[k] = v[k] * inv * bf16_to_f(gn[lane + 32 * k]);
+          for (int k = 0; k < DL; ++k) v[k] = v[k] * inv * gq[k];
 #pragma unroll
           for (int k = 0; k < DL / 2; ++k) {
-            const int i = lane + 32 * k;
-            const float ang = __fmul_rn(static_cast<float>(p), a.inv_freq[i]);
+            const float ang = __fmul_rn(static_cast<float>(p), invf[k]);
             float sn, cs;
-            sincosf(ang, &sn, &cs);
+            rope_sincos(ang, &sn, &cs);
             const float x1 = v[k], x2 = v[k + DL / 2];
             v[k] = x1 * cs - x2 * sn;
             v[k + DL / 2] = x2 * cs + x1 * sn;
@@ -649,9 +866,8 @@ struct Cta {
         }
         if (warp >= rep) {
           // the new K / V row as the cache stores it
-          const int kvsel = warp - rep;
-          const size_t row = kv_row(l, kvsel, b, g, p);
-          if (!a.kv_fp8) {
+          const size_t row = kv_row(l, warp - rep, b, g, p);
+          if constexpr (!FP8) {
             uint16_t* dstp = reinterpret_cast<uint16_t*>(a.kv) + row * D;
 #pragma unroll
             for (int k = 0; k < DL; ++k) {
@@ -662,8 +878,8 @@ struct Cta {
           } else {
             uint8_t code[DL];
             const float sc = quantize_row_e4m3<DL>(v, code);
-            uint8_t* dstp = a.kv + row * D;
             if (has_new) {
+              uint8_t* dstp = a.kv + row * D;
 #pragma unroll
               for (int k = 0; k < DL; ++k) dstp[lane + 32 * k] = code[k];
               if (lane == 0) a.kv_scales[row] = sc;
@@ -674,105 +890,102 @@ struct Cta {
         for (int k = 0; k < DL; ++k) x[lane + 32 * k] = v[k];
       }
       csync();
-      DEC_STAMP(8 * l + 2);
-      // -- partial softmax over this item's rows: warp w serves query head
-      // hw = w % rep of the group on rows rw, rw + rstep, ... (rw = w / rep),
-      // with a warp-level online softmax.
-      const int rstep = kCW / rep;
-      const int hw = warp % rep, rw = warp / rep;
-      const bool attw = warp < rstep * rep;
-      float qv[DL], acc[DL];
+      DEC_STAMP(kStampsPerLayer * l + StAttIn);
+      // -- this chunk's rows: online softmax per lane octet
+      float qv[DQ], acc[DQ];
       float m = -INFINITY, ls = 0.f;
 #pragma unroll
-      for (int k = 0; k < DL; ++k) {
+      for (int k = 0; k < DQ; ++k) {
         acc[k] = 0.f;
-        qv[k] = (attw && !ab) ? qs[hw * D + lane * DL + k] * qscale : 0.f;
+        qv[k] = (attw && !ab) ? qs[hw * D + e8 * DQ + k] * qscale : 0.f;
       }
-      auto consume_row = [&](const float* kr, const float* vr) {
-        float s = 0.f;
-#pragma unroll
-        for (int k = 0; k < DL; ++k) s = fmaf(qv[k], kr[k], s);
-        s = warp_sum(s);
-        const float mn = fmaxf(m, s);
-        const float al = exp2f(m - mn);
-        const float pe = exp2f(s - mn);
-        ls = ls * al + pe;
-#pragma unroll
-        for (int k = 0; k < DL; ++k) acc[k] = fmaf(acc[k], al, pe * vr[k]);
-        m = mn;
-      };
       for (int j = j0; j < jc; j += art) {
         const int nr = min(art, jc - j);
         wait_tile();
-        if (!ab) {
-          const uint8_t* tb = ring + static_cast<size_t>(rn % a.nslot) * kSlotBytes;
-          for (int r = rw; attw && r < nr; r += rstep) {
-            float kr[DL], vr[DL];
-            if (!a.kv_fp8) {
-              const uint8_t* kp = tb + static_cast<size_t>(r) * D * 2 + lane * DL * 2;
-              const uint8_t* vp = kp + static_cast<size_t>(nr) * D * 2;
-              if (DL == 4) {
-                const uint2 kw = *reinterpret_cast<const uint2*>(kp);
-                const uint2 vw = *reinterpret_cast<const uint2*>(vp);
-                kr[0] = bf16lo(kw.x); kr[1] = bf16hi(kw.x);
-                kr[2] = bf16lo(kw.y); kr[3] = bf16hi(kw.y);
-                vr[0] = bf16lo(vw.x); vr[1] = bf16hi(vw.x);
-                vr[2] = bf16lo(vw.y); vr[3] = bf16hi(vw.y);
-              } else {
-                const uint32_t kw = *reinterpret_cast<const uint32_t*>(kp);
-                const uint32_t vw = *reinterpret_cast<const uint32_t*>(vp);
-                kr[0] = bf16lo(kw); kr[1] = bf16hi(kw);
-                vr[0] = bf16lo(vw); vr[1] = bf16hi(vw);
-              }
-            } else {
-              const uint8_t* kp = tb + static_cast<size_t>(r) * D + lane * DL;
-              const uint8_t* vp = kp + static_cast<size_t>(nr) * D;
-              const int sb = ((nr + 3) & ~3) * 4;
-              const float ks = reinterpret_cast<const float*>(tb + 2 * nr * D)[r];
-              const float vs = reinterpret_cast<const float*>(tb + 2 * nr * D + sb)[r];
+        if (!ab && attw) {
+          const uint8_t* tb = ring + static_cast<size_t>(rs) * kSlotBytes;
+          for (int r4 = rw * 4; r4 < nr; r4 += rstep * 4) {
+            const int r = r4 + q8;
+            const bool ok = r < nr;
+            float kr[DQ];
+            tile_row(tb, nr, ok ? r : 0, e8, 0, kr);
+            float s = 0.f;
 #pragma unroll
-              for (int k = 0; k < DL; k += 2) {
-                const float2 kk = e4m3x2_to_f2(*reinterpret_cast<const uint16_t*>(kp + k));
-                const float2 vv = e4m3x2_to_f2(*reinterpret_cast<const uint16_t*>(vp + k));
-                kr[k] = kk.x * ks; kr[k + 1] = kk.y * ks;
-                vr[k] = vv.x * vs; vr[k + 1] = vv.y * vs;
-              }
+            for (int k = 0; k < DQ; ++k) s = fmaf(qv[k], kr[k], s);
+            s += __shfl_xor_sync(0xffffffffu, s, 4);
+            s += __shfl_xor_sync(0xffffffffu, s, 2);
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            if (ok) {
+              float vr[DQ];
+              tile_row(tb, nr, r, e8, 1, vr);
+              const float mn = fmaxf(m, s);
+              const float al = exp2f(m - mn), pe = exp2f(s - mn);
+              ls = ls * al + pe;
+#pragma unroll
+              for (int k = 0; k < DQ; ++k) acc[k] = fmaf(acc[k], al, pe * vr[k]);
+              m = mn;
             }
-            consume_row(kr, vr);
           }
         }
         release_tile();
       }
-      if (!ab && has_new && attw && rw == (jc - j0) % rstep) {
-        float kr[DL], vr[DL];
+      if (!ab && attw && rw == 0 && has_new) {  // the new row, by octet 0
+        float s = 0.f;
 #pragma unroll
-        for (int k = 0; k < DL; ++k) {
-          kr[k] = kn[lane * DL + k];
-          vr[k] = vn[lane * DL + k];
+        for (int k = 0; k < DQ; ++k) s = fmaf(qv[k], kn[e8 * DQ + k], s);
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        if (q8 == 0) {
+          const float mn = fmaxf(m, s);
+          const float al = exp2f(m - mn), pe = exp2f(s - mn);
+          ls = ls * al + pe;
+#pragma unroll
+          for (int k = 0; k < DQ; ++k) acc[k] = fmaf(acc[k], al, pe * vn[e8 * DQ + k]);
+          m = mn;
         }
-        consume_row(kr, vr);
       }
-      // -- merge the warps' states, write this chunk's partial
+      // merge the four octets of the warp, octet 0 writes the warp's state
       if (!ab && attw) {
-        float* mg = merge + static_cast<size_t>(warp) * (D + 2);
 #pragma unroll
-        for (int k = 0; k < DL; ++k) mg[lane * DL + k] = acc[k];
-        if (lane == 0) {
-          mg[D] = m;
-          mg[D + 1] = ls;
+        for (int o = 8; o <= 16; o <<= 1) {
+          const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+          const float lo = __shfl_xor_sync(0xffffffffu, ls, o);
+          const float mn = fmaxf(m, mo);
+          const float e1 = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+          const float e2 = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+          ls = ls * e1 + lo * e2;
+#pragma unroll
+          for (int k = 0; k < DQ; ++k) {
+            const float ao = __shfl_xor_sync(0xffffffffu, acc[k], o);
+            acc[k] = acc[k] * e1 + ao * e2;
+          }
+          m = mn;
+        }
+        if (q8 == 0) {
+          float* mg = merge + static_cast<size_t>(warp) * (D + 2);
+#pragma unroll
+          for (int k = 0; k < DQ; ++k) mg[e8 * DQ + k] = acc[k];
+          if (e8 == 0) {
+            mg[D] = m;
+            mg[D + 1] = ls;
+          }
         }
       }
       csync();
-      // -- this chunk's partial state (m in log2 units, l, unnormalised acc).
-      // Chunk 0's CTA combines (b, g): it keeps its own partial in shared
-      // memory; every other chunk publishes its partial as tagged words and
-      // moves on without waiting.
-      DEC_STAMP(8 * l + 3);
+      DEC_STAMP(kStampsPerLayer * l + StAttRows);
+      // -- this chunk's partial state (m in log2 units, l, unnormalised acc)
       const bool combiner = (ci == 0);
+      const int pc = a.part_chunks;
       const uint64_t* pbase =
-          a.part + (static_cast<size_t>(b) * a.Hq + g * rep) * a.part_chunks * (D + 2);
-      if (!ab) {
-        for (int t = tid; t < rep * D; t += kCT) {
+          a.part + (static_cast<size_t>(b) * a.Hq + g * rep) * pc * (D + 2);
+      float RM[3], RL[3], RA[3];  // (h, d) = t / D, t % D for t = tid + kCT * i
+#pragma unroll
+      for (int i = 0; i < 3; ++i) {
+        const int t = tid + kCT * i;
+        RM[i] = -INFINITY;
+        RL[i] = RA[i] = 0.f;
+        if (!ab && t < rep * D) {
           const int h = t / D, d = t % D;
           float M = -INFINITY;
           for (int w = h; w < rstep * rep; w += rep) M = fmaxf(M, merge[w * (D + 2) + D]);
@@ -784,14 +997,11 @@ struct Cta {
             A += mg[d] * e;
           }
           if (combiner) {
-            ownb[h * (D + 2) + d] = A;
-            if (d == 0) {
-              ownb[h * (D + 2) + D] = M;
-              ownb[h * (D + 2) + D + 1] = Ls;
-            }
+            RM[i] = M;
+            RL[i] = Ls;
+            RA[i] = A;
           } else {
-            uint64_t* pp = a.part + ((static_cast<size_t>(b) * a.Hq + g * rep + h) * a.part_chunks +
-                                     ci) * (D + 2);
+            uint64_t* pp = a.part + ((static_cast<size_t>(b) * a.Hq + g * rep + h) * pc + ci) * (D + 2);
             st_tagged(pp + d, A, f);
             if (d == 0) {
               st_tagged(pp + D, M, f);
@@ -802,53 +1012,46 @@ struct Cta {
       }
       if (combiner) {  // uniform over the CTA: ci is the item's
         const int nc1 = nchunk[b] - 1;
-        const int pc = a.part_chunks;
-        // (m, l) of chunks 1..nc1 -> mlb[(c - 1) * rep * 2 + h * 2 + e]
-        gather(
-            pbase, nc1 * rep * 2, f, mlb,
-            [=](int i) {
-              const int c = i / (rep * 2) + 1, h = (i >> 1) % rep, e = i & 1;
-              return (h * pc + c) * (D + 2) + D + e;
-            },
-            [](int i) { return i; });
-        int fail = 0;
-        if (!ab) {
-          for (int t = tid; t < rep * D; t += kCT) {
-            const int h = t / D, d = t % D;
-            const float* own = ownb + h * (D + 2);
-            float M = own[D];
-            for (int c = 0; c < nc1; ++c) M = fmaxf(M, mlb[(c * rep + h) * 2]);
-            const float e0 = exp2f(own[D] - M);
-            float Ls = own[D + 1] * e0, A = own[d] * e0;
-            const uint64_t* ph = pbase + static_cast<size_t>(h) * pc * (D + 2) + d;
-            for (int c0 = 0; c0 < nc1 && !fail; c0 += 8) {
-              uint64_t wv[8];
+        const int win = kStageWords / (rep * (D + 2));
+        for (int c0 = 1; c0 <= nc1; c0 += win) {
+          const int nw = min(win, nc1 - c0 + 1);
+          gather(nw * rep * (D + 2), f, [=](int w) {
+            const int sg = w / (D + 2), off = w % (D + 2);
+            const int c = c0 + sg / rep, h = sg % rep;
+            return pbase + (static_cast<size_t>(h) * pc + c) * (D + 2) + off;
+          });
+          if (!ab) {
 #pragma unroll
-              for (int k = 0; k < 8; ++k)
-                if (c0 + k < nc1) wv[k] = ld_tagged(ph + static_cast<size_t>(c0 + k + 1) * (D + 2));
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                if (c0 + k < nc1 && !fail) {
-                  Spin sp;
-                  while (static_cast<uint32_t>(wv[k] >> 32) != f) {
-                    if (sp.tick(a, true)) {
-                      fail = 1;
-                      break;
-                    }
-                    wv[k] = ld_tagged(ph + static_cast<size_t>(c0 + k + 1) * (D + 2));
-                  }
-                  const float* ml = mlb + ((c0 + k) * rep + h) * 2;
-                  const float e = exp2f(ml[0] - M);
-                  Ls += ml[1] * e;
-                  A += __uint_as_float(static_cast<uint32_t>(wv[k])) * e;
+            for (int i = 0; i < 3; ++i) {
+              const int t = tid + kCT * i;
+              if (t < rep * D) {
+                const int h = t / D, d = t % D;
+                for (int cc = 0; cc < nw; ++cc) {
+                  const uint64_t* pw = stg + (cc * rep + h) * (D + 2);
+                  const float Mc = __uint_as_float(static_cast<uint32_t>(pw[D]));
+                  const float Lc = __uint_as_float(static_cast<uint32_t>(pw[D + 1]));
+                  const float Ac = __uint_as_float(static_cast<uint32_t>(pw[d]));
+                  const float mn = fmaxf(RM[i], Mc);
+                  const float e1 = exp2f(RM[i] - mn), e2 = exp2f(Mc - mn);
+                  RL[i] = RL[i] * e1 + Lc * e2;
+                  RA[i] = RA[i] * e1 + Ac * e2;
+                  RM[i] = mn;
                 }
               }
             }
-            if (!fail)
-              st_tagged(a.x_o + static_cast<size_t>(b) * HqD + (g * rep + h) * D + d, A / Ls, f);
+          }
+          csync();  // stg is refilled by the next window
+        }
+        if (!ab) {
+#pragma unroll
+          for (int i = 0; i < 3; ++i) {
+            const int t = tid + kCT * i;
+            if (t < rep * D) {
+              const int h = t / D, d = t % D;
+              st_tagged(a.x_o + static_cast<size_t>(b) * HqD + (g * rep + h) * D + d, RA[i] / RL[i], f);
+            }
           }
         }
-        ab = named_sync_or(1, kCT, fail | ab);
       }
       csync();
     }
@@ -857,107 +1060,56 @@ struct Cta {
   // ------------------------------------------------------------- one step
   __device__ void consumer() {
     const int H = a.H, F = a.F, HqD = a.Hq * D;
-    int best_i[B];
-    float best_v[B];
 #pragma unroll
     for (int b = 0; b < B; ++b) {
       best_v[b] = -INFINITY;
       best_i[b] = 0x7fffffff;
     }
-    DEC_STAMP(8 * a.L + 3);
-    for (int l = 0; l < a.L; ++l) {
-      const LayerPtrs& lw = a.layers[l];
-      const uint32_t f = flag(l);
-      DEC_STAMP(8 * l);
-      // ---------------- input RMSNorm + QKV
-      if (l == 0) {
-        for (int i = tid; i < a.B * H; i += kCT) {
-          const int b = i / H, k = i % H;
-          act[b * kmax + k] = bf16_to_f(a.embed[static_cast<size_t>(tok[b]) * H + k]);
+    float gr[kGainRegs];
+    DEC_STAMP(kStampsPerLayer * a.L + StBegin);
+    // Stages of a layer: QKV, attention, o_proj, gate/up, down; the lm_head
+    // runs as stage QKV of layer L.  One copy of each piece of code.
+    for (int l = 0; l <= a.L; ++l) {
+      const bool lm = (l == a.L);
+      for (int st = 0; st < kStages; ++st) {
+        if (lm && st != SQ) break;
+        if (st == SA) {
+          DEC_STAMP(kStampsPerLayer * l + StQkv);
+          attention(l);
+          DEC_STAMP(kStampsPerLayer * l + StAtt);
+          continue;
         }
-        csync();
-        for (int i = tid; i < (h1 - h0) * a.B; i += kCT) {
-          const int r = i / a.B, b = i % a.B;
-          xown[r * B + b] = act[b * kmax + h0 + r];
-          if (a.hidden_out) a.hidden_out[static_cast<size_t>(b) * H + h0 + r] = xown[r * B + b];
+        const uint64_t* src;
+        const uint16_t* gain = nullptr;
+        int K, nrows, rpt, sc;
+        uint32_t fin;
+        bool pair = false;
+        if (st == SQ) {
+          src = a.x_out; K = H; fin = flag(l - 1);
+          gain = lm ? a.final_norm : slw[l].w[0];
+          nrows = lm ? v1 - v0 : q1 - q0; rpt = rpt_h; sc = lm ? SLM : SQ;
+        } else if (st == SO) {
+          src = a.x_o; K = HqD; fin = flag(l); nrows = h1 - h0; rpt = rpt_o; sc = SO;
+        } else if (st == SU) {
+          src = a.x_mid; K = H; fin = flag(l); gain = slw[l].w[7];
+          nrows = f1 - f0; rpt = rpt_u; pair = true; sc = SU;
+        } else {
+          src = a.x_u; K = F; fin = flag(l); nrows = h1 - h0; rpt = rpt_d; sc = SD;
         }
-      } else {
-        gather_x(a.x_out, H, flag(l - 1));
+        if (gain) load_gains(K, gain, gr);
+        if (st == SQ && l == 0) embed_rows();
+        else gather_x(src, K, fin);
+        if (st == SQ) DEC_STAMP(kStampsPerLayer * l + StQGath);
+        if (gain) rmsnorm_act(K, gain, gr);
+        if (st == SQ) DEC_STAMP(kStampsPerLayer * l + StQNorm);
+        if (pair || nrows > 2 * kCW) gemv<4>(K, nrows, rpt, pair, sc, l);
+        else gemv<1>(K, nrows, rpt, pair, sc, l);
+        if (st == SO) DEC_STAMP(kStampsPerLayer * l + StO);
+        if (st == SU) DEC_STAMP(kStampsPerLayer * l + StU);
+        if (st == SD) DEC_STAMP(kStampsPerLayer * l + StD);
       }
-      rmsnorm_act(H, lw.w[0]);
-      {
-        uint64_t* dst = a.x_qkv;
-        const int nq = nqkv, base = q0;
-        gemv<4>(H, q1 - q0, rpt_h, false, [=](int r, int b, float s, float) {
-          st_tagged(dst + static_cast<size_t>(b) * nq + base + r, s, f);
-        });
-      }
-      DEC_STAMP(8 * l + 1);
-      // ---------------- attention
-      attention(l);
-      DEC_STAMP(8 * l + 4);
-      // ---------------- o_proj + residual
-      gather_x(a.x_o, HqD, f);
-      {
-        float* xo = xown;
-        uint64_t* dst = a.x_mid;
-        const int base = h0;
-        const bool stall = (l == 0 && a.stall_cta == cta);
-        gemv<1>(HqD, h1 - h0, rpt_o, false, [=](int r, int b, float s, float) {
-          const float x = xo[r * B + b] + s;
-          xo[r * B + b] = x;
-          if (!stall) st_tagged(dst + static_cast<size_t>(b) * H + base + r, x, f);
-        });
-      }
-      DEC_STAMP(8 * l + 5);
-      // ---------------- post-attention RMSNorm + gate/up + SiLU * up
-      gather_x(a.x_mid, H, f);
-      rmsnorm_act(H, lw.w[7]);
-      {
-        uint64_t* dst = a.x_u;
-        const int base = f0;
-        gemv<4>(H, f1 - f0, rpt_u, true, [=](int r, int b, float gs, float us) {
-          const float u = gs / (1.0f + __expf(-gs)) * us;
-          st_tagged(dst + static_cast<size_t>(b) * F + base + r, u, f);
-        });
-      }
-      DEC_STAMP(8 * l + 6);
-      // ---------------- down + residual
-      gather_x(a.x_u, F, f);
-      {
-        float* xo = xown;
-        uint64_t* dst = a.x_out;
-        const int base = h0;
-        float* hid = a.hidden_out ? a.hidden_out + static_cast<size_t>(l + 1) * a.B * H : nullptr;
-        gemv<1>(F, h1 - h0, rpt_d, false, [=](int r, int b, float s, float) {
-          const float x = xo[r * B + b] + s;
-          xo[r * B + b] = x;
-          st_tagged(dst + static_cast<size_t>(b) * H + base + r, x, f);
-          if (hid) hid[static_cast<size_t>(b) * H + base + r] = x;
-        });
-      }
-      DEC_STAMP(8 * l + 7);
     }
-    DEC_STAMP(8 * a.L);
-    // ---------------- final norm + lm_head + argmax
-    gather_x(a.x_out, H, flag(a.L - 1));
-    rmsnorm_act(H, a.final_norm);
-    {
-      float* lg = a.out_logits;
-      const int base = v0, V = a.V;
-      gemv<4>(H, v1 - v0, rpt_h, false, [&](int r, int b, float s, float) {
-        const int id = base + r;
-        if (lg) lg[static_cast<size_t>(b) * V + id] = s;
-#pragma unroll
-        for (int bb = 0; bb < B; ++bb) {
-          if (bb == b && (s > best_v[bb] || (s == best_v[bb] && id < best_i[bb]))) {
-            best_v[bb] = s;
-            best_i[bb] = id;
-          }
-        }
-      });
-    }
-    DEC_STAMP(8 * a.L + 1);
+    DEC_STAMP(kStampsPerLayer * a.L + StLmDone);
     // CTA argmax -> one 64-bit atomicMax per sequence (ties: lowest id)
 #pragma unroll
     for (int b = 0; b < B; ++b) {
@@ -996,22 +1148,20 @@ struct Cta {
         atomicMax(&a.amax_key[b], key);
       }
     }
-    DEC_STAMP(8 * a.L + 2);
-  }
-
-  // B rows of K tagged words (row stride K) -> act rows (row stride kmax)
-  __device__ void gather_x(const uint64_t* src, int K, uint32_t f) {
-    const int km = kmax;
-    gather(src, a.B * K, f, act, [](int i) { return i; },
-           [K, km](int i) { return (i / K) * km + (i % K); });
+    DEC_STAMP(kStampsPerLayer * a.L + StEnd);
   }
 };
 
-template <int B, int D>
-__global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a, int kmax, int rmax) {
+template <int B, int D, bool FP8>
+__global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a, int kmax) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  Cta<B, D> c(a, smem, kmax, rmax);
-  // ---- set-up: barriers, step inputs, validation
+  Cta<B, D, FP8> c(a, smem, kmax);
+  // ---- set-up: layer pointer table, barriers, step inputs, validation
+  {
+    const uint64_t* src = reinterpret_cast<const uint64_t*>(a.layers);
+    uint64_t* dst = reinterpret_cast<uint64_t*>(const_cast<LayerPtrs*>(c.slw));
+    for (int i = threadIdx.x; i < a.L * kLayerPtrs; i += blockDim.x) dst[i] = src[i];
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.nslot; ++s) {
       mbar_init(&c.full[s], 1);
@@ -1061,15 +1211,15 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
   }
 }
 
-template <int B, int D>
-cudaError_t launch_bd(const StepArgs& a, int ctas, size_t smem, int kmax, int rmax,
+template <int B, int D, bool FP8>
+cudaError_t launch_bd(const StepArgs& a, int ctas, size_t smem, int kmax,
                       cudaStream_t s) {
-  auto k = step_kernel<B, D>;
+  auto k = step_kernel<B, D, FP8>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   StepArgs args = a;
-  void* params[] = {&args, &kmax, &rmax};
+  void* params[] = {&args, &kmax};
   return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k), dim3(ctas),
                                      dim3(kStepThreads), params, smem, s);
 }
@@ -1080,42 +1230,29 @@ static int kmax_of(int H, int F, int HqD) {
   int k = H > F ? H : F;
   return k > HqD ? k : HqD;
 }
-static int rmax_of(int H, int F, int HqD) {
-  int m = H < F ? H : F;
-  m = m < HqD ? m : HqD;
-  return kSlotBytes / (2 * m);
+size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep) {
+  return carve(nslot, B, kmax_of(H, F, HqD), D, rep).total;
 }
 
-size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep, int nchunks) {
-  return carve(nslot, B, kmax_of(H, F, HqD), rmax_of(H, F, HqD), D, rep, nchunks).total;
-}
-
-int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int nchunks, int smem_optin) {
+int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int smem_optin) {
   int best = 0;
   for (int n = 1; n <= 16; ++n)
-    if (step_smem_bytes(n, B, H, F, HqD, D, rep, nchunks) <= static_cast<size_t>(smem_optin))
+    if (step_smem_bytes(n, B, H, F, HqD, D, rep) <= static_cast<size_t>(smem_optin))
       best = n;
   return best;
 }
 
 cudaError_t launch_step_small(const StepArgs& a, int ctas, size_t smem, cudaStream_t s) {
   const int HqD = a.Hq * a.D;
-  const int kmax = kmax_of(a.H, a.F, HqD), rmax = rmax_of(a.H, a.F, HqD);
-  if (a.D == 128) {
-    switch (a.B) {
-      case 1: return launch_bd<1, 128>(a, ctas, smem, kmax, rmax, s);
-      case 2: return launch_bd<2, 128>(a, ctas, smem, kmax, rmax, s);
-      case 3: return launch_bd<3, 128>(a, ctas, smem, kmax, rmax, s);
-      case 4: return launch_bd<4, 128>(a, ctas, smem, kmax, rmax, s);
-    }
-  } else if (a.D == 64) {
-    switch (a.B) {
-      case 1: return launch_bd<1, 64>(a, ctas, smem, kmax, rmax, s);
-      case 2: return launch_bd<2, 64>(a, ctas, smem, kmax, rmax, s);
-      case 3: return launch_bd<3, 64>(a, ctas, smem, kmax, rmax, s);
-      case 4: return launch_bd<4, 64>(a, ctas, smem, kmax, rmax, s);
-    }
-  }
+  const int kmax = kmax_of(a.H, a.F, HqD);
+  const bool f8 = a.kv_fp8 != 0;
+#define DEC_CASE(BB, DD)                                                            \
+  if (a.B == BB && a.D == DD)                                                       \
+    return f8 ? launch_bd<BB, DD, true>(a, ctas, smem, kmax, s)                     \
+              : launch_bd<BB, DD, false>(a, ctas, smem, kmax, s);
+  DEC_CASE(1, 128) DEC_CASE(2, 128) DEC_CASE(3, 128) DEC_CASE(4, 128)
+  DEC_CASE(1, 64) DEC_CASE(2, 64) DEC_CASE(3, 64) DEC_CASE(4, 64)
+#undef DEC_CASE
   return cudaErrorInvalidValue;
 }
 

@@ -82,7 +82,7 @@ typedef enum dec_status {
 /* Model description                                                   */
 /* ------------------------------------------------------------------ */
 typedef struct dec_shape {
-  int n_layers;      /* 28 for the 0.6B / 1.7B decoders */
+  int n_layers;      /* 1..64 (28 for the 0.6B / 1.7B decoders) */
   int hidden;        /* multiple of 256 */
   int n_q_heads;     /* multiple of n_kv_heads */
   int n_kv_heads;
