@@ -276,3 +276,37 @@ def test_0p6b_batch4_ragged(big06):
         assert_id(int(ids[b]), refs[b], f"bs4 seq {b}")
         _check_kv_row(kv, caches[b], b, lengths[b], f"bs4 seq {b}")
     dec.close()
+
+
+# ------------------------------------------------------------ 1.7B shape
+@pytest.fixture(scope="module")
+def big17():
+    s = synth.QWEN3_1_7B
+    w = synth.model_weights(s, seed=17)
+    return s, w, oracle.Model(oracle_shape(s), oracle_weights(w)), to_device(w)
+
+
+@pytest.mark.parametrize("kind,n0", [("bf16", 4095), ("fp8", 2500)])
+def test_1p7b_bs1_long_context(big17, kind, n0):
+    """1.7B shape (hidden 2048, FFN 6144), batch 1, contexts up to 4096, bf16
+    cache and the E4M3 cache read back from the same stored bytes."""
+    s, w, m, wd = big17
+    dec = Decoder(s, wd, 1)
+    kv_host, sc_host = synth.kv_prefill(s, 1, 4096, [n0], seed=18, kind=kind)
+    cache = oracle_cache(kv_host, sc_host, 0)
+    kv = dec.kv_cache(1, 4096, kind)
+    if kind == "bf16":
+        kv.values.copy_(kv_host.cuda())
+    else:
+        kv.codes.copy_(kv_host.cuda())
+        kv.scales.copy_(sc_host.cuda())
+    tok = int(synth.tokens(s.vocab, 1, seed=19)[0])
+    r = m.step(cache, tok, n0, want_hidden=True)
+    ids, logits, hid = _gpu_step(dec, kv, [tok], [n0])
+    assert_close(logits[0], r.logits, f"1.7B {kind} logits")
+    for l in (1, 28):
+        assert_close(hid[l, 0], r.hidden[l], f"1.7B {kind} hidden {l}")
+    assert_id(int(ids[0]), r, f"1.7B {kind}")
+    _check_kv_row(kv, cache, 0, n0, f"1.7B {kind}")
+    del kv
+    dec.close()
