@@ -18,6 +18,7 @@ DEC_KV_FP8_E4M3 = 1
 DEC_DEV_BAD_POSITION = 1
 DEC_DEV_BAD_TOKEN = 2
 DEC_DEV_TIMEOUT = 4
+DEC_ERR_TOO_LARGE = -10
 LW_ORDER = ("in_norm", "q", "k", "v", "q_norm", "k_norm", "o", "post_norm", "gate", "up", "down")
 
 #: every symbol include/dec.h declares
@@ -26,6 +27,7 @@ EXPORTS = (
     "dec_step_debug", "dec_step_host", "dec_check", "dec_set_timeout_ns", "dec_set_debug_stall",
     "dec_error_string", "dec_last_cuda_error", "dec_get_config",
     "dec_attention_workspace_bytes", "dec_attention", "dec_kv_quantize_e4m3",
+    "dec_attention_noalloc",
 )
 
 
@@ -83,6 +85,7 @@ def lib() -> ctypes.CDLL:
             "dec_attention_workspace_bytes": ([I, I, I, I, I], Z),
             "dec_attention": ([I, I, I, I, P, P, P, I, P, P, P, Z, P, P], I),
             "dec_kv_quantize_e4m3": ([P, I, I, P, P, P], I),
+            "dec_attention_noalloc": ([I, I, I, I, P, P, P, I, P, P, P, P], I),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -197,3 +200,10 @@ def dec_attention(batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int, q,
 def dec_kv_quantize_e4m3(x, rows: int, dim: int, codes, scales, stream=None) -> None:
     _ok(lib().dec_kv_quantize_e4m3(_ptr(x), rows, dim, _ptr(codes), _ptr(scales),
                                    _stream(stream)), "dec_kv_quantize_e4m3")
+
+
+def dec_attention_noalloc(batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int, q, k_cache,
+                          v_cache, max_len: int, lengths, out, status=None, stream=None) -> None:
+    _ok(lib().dec_attention_noalloc(batch, n_q_heads, n_kv_heads, head_dim, _ptr(q), _ptr(k_cache),
+                                    _ptr(v_cache), max_len, _ptr(lengths), _ptr(out), _ptr(status),
+                                    _stream(stream)), "dec_attention_noalloc")

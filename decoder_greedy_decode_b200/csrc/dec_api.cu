@@ -363,6 +363,7 @@ extern "C" const char* dec_error_string(int code) {
     case DEC_ERR_CUDA: return "CUDA runtime error";
     case DEC_ERR_DEVICE: return "device not supported (needs compute capability 10.0)";
     case DEC_ERR_ARG: return "invalid argument";
+    case DEC_ERR_TOO_LARGE: return "request exceeds the fixed scratch of dec_attention_noalloc";
     default: break;
   }
   if (code > 0) {

@@ -12,6 +12,9 @@
 // roofline of this kernel is HBM bandwidth over the K/V bytes.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
+#include "dec.h"
 #include "dec_internal.h"
 #include "dec_ptx.cuh"
 #include "dec_quant.cuh"
@@ -261,3 +264,84 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {
 }
 
 }  // namespace dec
+
+// ---------------------------------------------------------------------------
+// dec_attention_noalloc: the same attention with its scratch in a fixed,
+// library-owned device array instead of caller memory.
+//
+// The scratch holds what one call needs between its CTAs: the partial softmax
+// state of every chunk and one arrival counter per (sequence, KV head).  It is
+// a file-scope device array, so every GPU that loads the library holds it
+// until the process exits, and every call on a device shares it.
+using dec::AttnArgs;
+using dec::attention_chunk_rows;
+using dec::launch_attention;
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+std::mutex g_noalloc_mu;
+
+size_t al256n(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" int dec_attention_noalloc(int batch, int n_q_heads, int n_kv_heads, int head_dim,
+                                     const void* q, const void* k_cache, const void* v_cache,
+                                     int max_len, const int32_t* lengths, float* out, int* status,
+                                     void* stream) {
+  if (!q || !k_cache || !v_cache || !lengths || !out) return DEC_ERR_NULL;
+  if (batch < 1) return DEC_ERR_BATCH;
+  if (head_dim != 64 && head_dim != 128) return DEC_ERR_SHAPE;
+  if (n_kv_heads < 1 || n_q_heads % n_kv_heads || n_q_heads / n_kv_heads > 8) return DEC_ERR_SHAPE;
+  if (max_len < 1) return DEC_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15)
+    return DEC_ERR_ALIGN;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DEC_ERR_DEVICE;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return DEC_ERR_DEVICE;
+  const int chunk_rows = attention_chunk_rows(batch, n_kv_heads, max_len, sms);
+  const int chunks = (max_len + chunk_rows - 1) / chunk_rows;
+  const size_t part_bytes =
+      al256n(sizeof(float) * static_cast<size_t>(batch) * n_q_heads * chunks * (head_dim + 2));
+  const size_t cnt_bytes = sizeof(unsigned) * static_cast<size_t>(batch) * n_kv_heads;
+  if (part_bytes + cnt_bytes > kNoAllocScratchBytes) return DEC_ERR_TOO_LARGE;
+  // once per device, with that device current: the device address of the array
+  void* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
+        return DEC_ERR_DEVICE;
+      g_noalloc_ptr[dev] = ptr;
+    }
+    base = g_noalloc_ptr[dev];
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* scratch = static_cast<uint8_t*>(base);
+  // the array keeps the previous call's contents: the counters must start at zero
+  if (cudaMemsetAsync(scratch + part_bytes, 0, cnt_bytes, st) != cudaSuccess) return DEC_ERR_CUDA;
+  AttnArgs a{};
+  a.B = batch;
+  a.Hq = n_q_heads;
+  a.Hkv = n_kv_heads;
+  a.D = head_dim;
+  a.max_len = max_len;
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(k_cache);
+  a.v = static_cast<const uint16_t*>(v_cache);
+  a.lengths = lengths;
+  a.out = out;
+  a.chunk_rows = chunk_rows;
+  a.chunks_max = chunks;
+  a.part = reinterpret_cast<float*>(scratch);
+  a.cnt = reinterpret_cast<unsigned*>(scratch + part_bytes);
+  a.status = status;
+  return launch_attention(a, st) == cudaSuccess ? DEC_OK : DEC_ERR_CUDA;
+}

@@ -71,6 +71,7 @@ typedef enum dec_status {
   DEC_ERR_CUDA = -7,          /* a CUDA runtime call failed (dec_last_cuda_error) */
   DEC_ERR_DEVICE = -8,        /* the current device is not sm_100 or lacks resources */
   DEC_ERR_ARG = -9,           /* other invalid argument */
+  DEC_ERR_TOO_LARGE = -10,    /* problem exceeds dec_attention_noalloc's fixed scratch */
   /* device-detected conditions, returned (OR-ed as a positive bit set) by
    * dec_check(); the step that saw them wrote -1 to every out_ids entry */
   DEC_DEV_BAD_POSITION = 1,   /* a position < 0 or >= max_ctx */
@@ -253,6 +254,29 @@ int dec_attention(int batch, int n_q_heads, int n_kv_heads, int head_dim, const 
                   const void *k_cache, const void *v_cache, int max_len,
                   const int32_t *lengths, float *out, void *workspace,
                   size_t workspace_bytes, int *status, void *stream);
+
+/* dec_attention without a workspace argument: for callers that must not
+ * allocate device memory on their call path -- code running inside another
+ * framework's execute or enqueue callback, where allocating is not permitted;
+ * real-time loops, where cudaMalloc's implicit synchronisation would stall the
+ * device; processes whose device memory is owned by another allocator or fixed
+ * by a budget.  (The pages have no counterpart: this is a deployment variant
+ * of the attention above.)
+ * Same inputs, outputs and numerics as dec_attention.  The scratch (per-chunk
+ * partial softmax states, per-(sequence, KV head) counters) is a fixed 4 MiB
+ * device array inside the library: every GPU that loads the library holds it
+ * until the process exits.  Requests needing more than 4 MiB of it (batch *
+ * n_q_heads * chunks * (head_dim + 2) * 4 bytes, chunks as dec_attention
+ * splits max_len, plus 4 bytes per (sequence, KV head)) return
+ * DEC_ERR_TOO_LARGE; nothing is launched.  Allocates nothing: no cudaMalloc,
+ * no cudaFree.  The first call on a device looks up the array's device address
+ * (with that device current) and should come before any stream capture.  All
+ * calls on a device share the array and each clears its counters first, so
+ * calls that overlap on the GPU (other streams, or other host threads) race:
+ * serialise them. */
+int dec_attention_noalloc(int batch, int n_q_heads, int n_kv_heads, int head_dim, const void *q,
+                          const void *k_cache, const void *v_cache, int max_len,
+                          const int32_t *lengths, float *out, int *status, void *stream);
 
 /* ------------------------------------------------------------------ */
 /* FP8 cache rows                                                      */
