@@ -41,6 +41,7 @@ struct dec_handle {
   float* logits_dev = nullptr;
   unsigned long long timeout_ns = 2000000000ull;
   int stall_cta = -1;
+  BtPlan* bt = nullptr;  // batched path (max_batch > kMaxBatchSmall)
 };
 
 static int check_shape(const dec_shape* s) {
@@ -56,7 +57,7 @@ static int check_shape(const dec_shape* s) {
   if (hqd % 256 || hqd > 6144) return DEC_ERR_SHAPE;
   if (s->vocab < 1) return DEC_ERR_SHAPE;
   if (!(s->rms_eps >= 0.f) || !(s->rope_theta > 0.f)) return DEC_ERR_SHAPE;
-  if (s->max_batch < 1 || s->max_batch > kMaxBatchSmall) return DEC_ERR_BATCH;
+  if (s->max_batch < 1 || s->max_batch > kMaxBatch) return DEC_ERR_BATCH;
   return DEC_OK;
 }
 
@@ -90,7 +91,11 @@ extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle
   h->ctas = prop.multiProcessorCount;
   h->smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
   const int H = shape->hidden, F = shape->ffn, D = shape->head_dim;
-  const int Hq = shape->n_q_heads, Hkv = shape->n_kv_heads, B = shape->max_batch;
+  const int Hq = shape->n_q_heads, Hkv = shape->n_kv_heads;
+  // the persistent kernel serves batches up to kMaxBatchSmall; larger ones
+  // take the batched (tensor-core) path
+  const int B = shape->max_batch < kMaxBatchSmall ? shape->max_batch : kMaxBatchSmall;
+  const int Bfull = shape->max_batch;
   const int HqD = Hq * D, rep = Hq / Hkv;
   if ((H + h->ctas - 1) / h->ctas > 64) {
     delete h;
@@ -131,14 +136,14 @@ extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle
   wl.status = take(sizeof(int));
   wl.abort_flag = take(sizeof(int));
   wl.inv_freq = take(sizeof(float) * D / 2);
-  wl.tok_dev = take(sizeof(int32_t) * B);
-  wl.pos_dev = take(sizeof(int32_t) * B);
-  wl.out_dev = take(sizeof(int32_t) * B);
+  wl.tok_dev = take(sizeof(int32_t) * Bfull);
+  wl.pos_dev = take(sizeof(int32_t) * Bfull);
+  wl.out_dev = take(sizeof(int32_t) * Bfull);
 #ifdef DEC_PROFILE
   wl.prof = take(sizeof(unsigned long long) * h->ctas * (16 * L + 8));
 #endif
   size_t layers_off = take(sizeof(LayerPtrs) * L);
-  size_t logits_off = take(sizeof(float) * static_cast<size_t>(B) * shape->vocab);
+  size_t logits_off = take(sizeof(float) * static_cast<size_t>(Bfull) * shape->vocab);
   wl.total = o;
   e = cudaMalloc(&h->ws, wl.total);
   if (e != cudaSuccess) {
@@ -167,6 +172,18 @@ extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle
     delete h;
     return cuda_fail(e);
   }
+  if (Bfull > kMaxBatchSmall) {
+    const BtShape bs{L, H, Hq, Hkv, D, F, shape->vocab, shape->rms_eps};
+    cudaError_t ce = cudaSuccess;
+    rc = bt_plan_create(bs, h->embed, h->lm_head, h->final_norm, lp.data(),
+                        reinterpret_cast<const float*>(h->ws + wl.inv_freq), h->sms, &h->bt, &ce);
+    if (rc) {
+      cudaFree(h->ws);
+      delete h;
+      if (rc == DEC_ERR_CUDA) g_last_cuda = static_cast<int>(ce);
+      return rc;
+    }
+  }
   *out = h;
   return DEC_OK;
 }
@@ -174,6 +191,7 @@ extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle
 extern "C" void dec_free(dec_handle* h) {
   if (!h) return;
   cudaDeviceSynchronize();
+  bt_plan_destroy(h->bt);
   cudaFree(h->ws);
   delete h;
 }
@@ -223,6 +241,28 @@ static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* 
   if (kv->dtype != DEC_KV_BF16 && kv->dtype != DEC_KV_FP8_E4M3) return DEC_ERR_DTYPE;
   if (kv->bytes < dec_kv_bytes(h, kv->batch, kv->max_ctx, kv->dtype)) return DEC_ERR_KV_SIZE;
   const dec_shape& s = h->shape;
+  if (batch > kMaxBatchSmall) {
+    BtIO io{};
+    io.B = batch;
+    io.tok = tok;
+    io.pos = pos;
+    io.out = out_ids;
+    io.logits = logits;
+    io.hidden = hidden;
+    io.kv = static_cast<uint8_t*>(kv->base);
+    io.kv_fp8 = kv->dtype == DEC_KV_FP8_E4M3;
+    io.kv_scales = io.kv_fp8 ? reinterpret_cast<float*>(
+                                   static_cast<uint8_t*>(kv->base) +
+                                   dec_kv_scale_offset(h, kv->batch, kv->max_ctx, kv->dtype))
+                             : nullptr;
+    io.kv_batch = kv->batch;
+    io.max_ctx = kv->max_ctx;
+    io.status = reinterpret_cast<int*>(h->ws + h->wl.status);
+    io.timeout_ns = h->timeout_ns;
+    cudaError_t e = bt_step(h->bt, io, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return DEC_OK;
+  }
   StepArgs a{};
   a.L = s.n_layers;
   a.H = s.hidden;

@@ -12,6 +12,7 @@ constexpr int kSlotBytes = 24576;                   // ring slot: 12 rows of 102
 constexpr int kMaxBatchSmall = 4;                   // batch handled by the GEMV step kernel
 constexpr int kMaxRep = 4;                          // query heads per KV head (step kernel)
 constexpr int kLayerPtrs = 11;
+constexpr int kMaxBatch = 64;                       // batched step: the N of the tensor-core tiles
 
 struct LayerPtrs {
   const uint16_t* w[kLayerPtrs];  // dec_layer_weight order
@@ -89,5 +90,31 @@ size_t attention_smem_bytes(int D, int rep);
 int attention_chunk_rows(int B, int Hkv, int max_len, int sms);
 cudaError_t launch_quantize(const float* x, int rows, int dim, uint8_t* codes, float* scales,
                             cudaStream_t s);
+
+// ---- batched step (batch > kMaxBatchSmall): tensor-core projections
+struct BtShape {
+  int L, H, Hq, Hkv, D, F, V;
+  float eps;
+};
+struct BtPlan;  // tensor maps, launch configuration and scratch (dec_step_batched.cu)
+// Returns 0, or a DEC_ERR_* code (DEC_ERR_CUDA with *cerr set).
+int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_head,
+                   const uint16_t* final_norm, const LayerPtrs* layers_host,
+                   const float* inv_freq_dev, int sms, BtPlan** out, cudaError_t* cerr);
+void bt_plan_destroy(BtPlan* p);
+struct BtIO {
+  int B;
+  const int32_t* tok;
+  const int32_t* pos;
+  int32_t* out;
+  float* logits;   // [B, V] or null
+  float* hidden;   // [L+1, B, H] or null
+  uint8_t* kv;
+  float* kv_scales;
+  int kv_batch, max_ctx, kv_fp8;
+  int* status;
+  unsigned long long timeout_ns;
+};
+cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t s);
 
 }  // namespace dec

@@ -32,6 +32,7 @@
 #include "dec_internal.h"
 #include "dec_ptx.cuh"
 #include "dec_quant.cuh"
+#include "dec_rope.cuh"
 
 namespace dec {
 namespace {
@@ -129,19 +130,6 @@ struct Spin {
     return false;
   }
 };
-
-// sin and cos of an fp32 rotary angle x (0 <= x < 2^16 * 2pi): Cody-Waite
-// reduction by 2pi split into three fp32 parts (c1 has 8 significant bits,
-// so k * c1 is exact for |k| < 2^16), then the fast hardware sin/cos on
-// [-pi, pi], where its absolute error is about 2^-21.
-__device__ __forceinline__ void rope_sincos(float x, float* sn, float* cs) {
-  const float c1 = 6.28125f, c2 = 1.9353071693331003e-3f, c3 = 1.0253376273028358e-11f;
-  const float k = rintf(x * 0.15915493667125702f);
-  float r = fmaf(-k, c1, x);
-  r = fmaf(-k, c2, r);
-  r = fmaf(-k, c3, r);
-  __sincosf(r, sn, cs);
-}
 
 __device__ __forceinline__ float dot8(const uint4 w, const float* x) {
   float s = bf16lo(w.x) * x[0];

@@ -119,6 +119,29 @@ def kv_prefill(s: ModelShape, batch: int, max_ctx: int, lengths: Sequence[int], 
     raise ValueError(kind)
 
 
+def kv_prefill_seq(s: ModelShape, max_ctx: int, n: int, seed: int, kind: str = "bf16"):
+    """One sequence's cache planes [L, 2, Hkv, max_ctx, D] drawn from its own
+    generator (seed), so that a large batch can be filled one sequence at a
+    time and only the sampled sequences need a host copy.  Same value recipe
+    as kv_prefill: first n rows random, the rest zero."""
+    gen = torch.Generator().manual_seed(int(seed))
+    L, Hkv, D = s.n_layers, s.n_kv_heads, s.head_dim
+    if kind == "bf16":
+        kv = torch.zeros((L, 2, Hkv, max_ctx, D), dtype=torch.bfloat16)
+        if n > 0:
+            kv[:, :, :, :n, :] = torch.randn((L, 2, Hkv, n, D), generator=gen).to(torch.bfloat16)
+        return kv, None
+    if kind == "fp8":
+        codes = torch.zeros((L, 2, Hkv, max_ctx, D), dtype=torch.uint8)
+        scales = torch.zeros((L, 2, Hkv, max_ctx), dtype=torch.float32)
+        if n > 0:
+            z = (torch.randn((L, 2, Hkv, n, D), generator=gen) * 32.0).to(torch.float8_e4m3fn)
+            codes[:, :, :, :n, :] = z.view(torch.uint8)
+            scales[:, :, :, :n] = 0.02 + 0.02 * torch.rand((L, 2, Hkv, n), generator=gen)
+        return codes, scales
+    raise ValueError(kind)
+
+
 def tokens(vocab: int, batch: int, seed: int) -> torch.Tensor:
     """Start tokens uniform in [0, vocab), int32 [batch]."""
     gen = torch.Generator().manual_seed(int(seed))

@@ -67,8 +67,14 @@ def _check_kv_row(kv, cache, b, p, what):
         scales = kv.scales[:, :, b, :, p].cpu().numpy()
         got = oracle.e4m3_decode(codes) * scales[..., None]
         ref = oracle.e4m3_decode(cache.kv[:, :, :, p, :]) * cache.scales[:, :, :, p][..., None]
-        # one E4M3 step is 2^-3 of the value: compare in units of the row scale
-        assert np.max(np.abs(got - ref) / scales[..., None]) <= 32.0 + 1e-6, what
+        # Each side quantises its own k (scale = amax / 448, RNE to E4M3).  An
+        # element near a rounding boundary may land one code apart: at most one
+        # top-binade step, 32 x scale.  When the two amax differ (within the k
+        # tolerance) the same code also decodes to values 448 x |scale gap|
+        # apart.
+        ref_sc = cache.scales[:, :, :, p][..., None]
+        bound = 32.0 * scales[..., None] + 448.0 * np.abs(scales[..., None] - ref_sc)
+        assert np.all(np.abs(got - ref) <= bound * (1 + 1e-6) + 1e-12), what
         assert close_report(got, ref)[1] <= 0.05, what
 
 
