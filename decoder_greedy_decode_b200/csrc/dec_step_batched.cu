@@ -8,20 +8,31 @@
 // activation rows, so the projections are dense [N x K] x [K x B]
 // contractions and run on the tensor cores: tcgen05.mma with bf16 operands
 // staged by TMA (128-byte swizzle) and fp32 accumulators in tensor memory,
-// one 128-row weight tile x 64 sequences per CTA, split along K so that a
-// layer's small matrices still cover every SM.  The split partials meet in
-// L2 and small CUDA-core kernels finish each phase (residual add, RMSNorm,
-// q/k norm, rotation and cache append, SwiGLU).  The Baseten Qwen3-ASR
-// article ("KV cache quantization") notes that at high concurrency the
-// attention over the cache takes the largest share of decode time: it is a
-// split-K kernel over (sequence, KV head, chunk) streaming K/V rows (bf16
-// or E4M3 codes + fp32 row scales) through shared memory.
+// one 128-row weight tile x 64 sequences per CTA.
+//
+// Launches per layer: QKV GEMM, attention, o_proj GEMM, gate/up GEMM, down
+// GEMM.  A GEMM is split along K over the CTAs of a thread-block cluster;
+// the cluster sums the split accumulators through distributed shared memory
+// (in a fixed order: deterministic) and the same launch finishes the phase:
+//   QKV      q/k RMSNorm, rotation, query store, K/V append (bf16 or E4M3)
+//   o_proj   residual add; the next RMSNorm's operand and sums of squares
+//   gate/up  silu(gate) * up (a tile holds 64 gate rows and the same 64 up rows)
+//   down     residual add; the next RMSNorm's operand and sums of squares
+// RMSNorm is applied as a per-sequence scale: the producer of x stores g * x
+// and per-tile sums of x^2, and the consumer GEMM multiplies its accumulator
+// column b by rsqrt(mean x_b^2 + eps) (a column scale commutes with W).
+// Every launch is a programmatic dependent launch: a GEMM's weight tiles
+// (which no earlier kernel writes) stream in while its predecessor finishes.
+//
+// The Baseten Qwen3-ASR article ("KV cache quantization") notes that at high
+// concurrency the attention over the cache takes the largest share of decode
+// time: it is a split-K kernel over (sequence, KV head, chunk) streaming K/V
+// rows (bf16, or E4M3 codes + fp32 row scales) through shared memory.
 //
 // Numerics: weights and the KV cache as stored; the residual stream, norms,
-// softmax and accumulators fp32.  A tensor-core activation operand (the
-// normalised hidden state, the attention output, the SwiGLU output) is held
-// as two bf16 planes, hi = bf16(x) and lo = bf16(x - hi), and every K step
-// issues one MMA per plane: W x = W hi + W lo to about 2^-17 of x, so the
+// softmax and accumulators fp32.  A tensor-core activation operand is held
+// as two bf16 planes, hi = bf16(y) and lo = bf16(y - hi), and every K step
+// issues one MMA per plane: W y = W hi + W lo to about 2^-17 of y, so the
 // batched step keeps the fp32-activation accuracy of the single-sequence
 // kernel (the weights are exactly bf16).  The extra MMAs are free here: the
 // step is bound by HBM, not by the tensor pipe.
@@ -45,26 +56,30 @@ constexpr int kTileM = 128;                       // weight rows per tile (MMA M
 constexpr int kTileN = kMaxBatch;                 // sequences per tile (MMA N)
 constexpr int kChunkK = 64;                       // K columns per pipeline stage
 constexpr int kABytes = kTileM * kChunkK * 2;     // 16 KB
-constexpr int kBRows = 2 * kTileN;               // activation rows: hi plane, then lo plane
+constexpr int kBRows = 2 * kTileN;                // activation rows: hi plane, then lo plane
 constexpr int kBBytes = kBRows * kChunkK * 2;     // 16 KB
 constexpr int kLoOffset = kTileN * kChunkK * 2;   // lo plane inside a B tile (8 KB)
+constexpr int kHalfA = kABytes / 2;               // gate/up tiles: up rows start here
 constexpr int kStageBytes = kABytes + kBBytes;    // 32 KB
 constexpr int kGemmStages = 3;
 constexpr int kGemmThreads = 128;                 // 4 warps = the 4 TMEM sub-partitions
 constexpr uint32_t kTmemCols = 64;                // fp32 accumulator columns (= kTileN)
 constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, kTileN);
-constexpr int kLmStride = kTileM + 4;             // transposed logits tile row (floats)
+constexpr int kTStride = kTileM + 4;              // accumulator tile in smem: T[b][row]
 constexpr size_t kGemmSmem = 1024 + kGemmStages * kStageBytes + 256;
+constexpr int kMaxSplits = 8;                     // cluster size (portable)
 constexpr int kMaxAttnChunks = 32;
-constexpr int kAttWarps = 4;
+constexpr int kAttWarps = 8;
 constexpr int kAttThreads = kAttWarps * 32;
 constexpr int kAttStages = 4;
 constexpr int kAttTileRows = 32;
 constexpr int kAttMaxRep = 8;
 constexpr int kRowThreads = 256;
 
+enum GemmMode { kQKV = 0, kResid = 1, kSwiGLU = 2, kLm = 3 };
+
 static_assert(kTileN == 64 && kTmemCols == 64, "epilogue reads 4 x 16 accumulator columns");
-static_assert(kTileN * kLmStride * 4 <= kGemmStages * kStageBytes, "logits tile fits the ring");
+static_assert(kTileN * kTStride * 4 <= kGemmStages * kStageBytes, "accumulator tile fits the ring");
 
 // Bounded mbarrier wait: the copies and MMAs always complete; the bound only
 // guards the GPU.  Returns false (and raises the timeout status) if it ran
@@ -87,39 +102,76 @@ __device__ bool bt_wait(uint64_t* bar, uint32_t parity, unsigned long long limit
   }
 }
 
+// y as the two bf16 planes of a tensor-core activation buffer [2][64][K]
+__device__ __forceinline__ void put_act(uint16_t* buf, int b, int n, int K, float y) {
+  const uint16_t hi = f_to_bf16(y);
+  buf[static_cast<size_t>(b) * K + n] = hi;
+  buf[static_cast<size_t>(kTileN + b) * K + n] = f_to_bf16(y - bf16_to_f(hi));
+}
+
+// sum over the threads of the CTA (every thread must call it)
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();  // red may still be read from a previous call
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = 0.f;
+  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += red[w];
+  return t;
+}
+
+// rsqrt(mean x_b^2 + eps) from the per-tile sums of squares [n_ssp][64]
+__device__ __forceinline__ float rms_scale(const float* ssp, int n_ssp, int b, int H, float eps) {
+  float ss = 0.f;
+  for (int t = 0; t < n_ssp; ++t) ss += ssp[t * kTileN + b];
+  return rsqrtf(ss / static_cast<float>(H) + eps);
+}
+
 // ===================================================================== GEMM
-// One launch computes, for up to three weight matrices stacked along their
-// output rows, out[b][n] = sum_k W[n][k] * X[b][k] for b < 64 (X is the
-// activation buffer: rows 0..63 the hi plane, 64..127 the lo plane; rows of
-// sequences >= B are ignored).
-// Grid: (stacked 128-row tiles, K splits).  MODE 0 writes the fp32 partial
-// of split s to part[s][b][off + n]; MODE 1 (lm_head, one split) writes the
-// logits (optional) and folds the tile's argmax into a 64-bit atomicMax key
-// per sequence: (order-preserving bits of the logit << 32) | ~id, so equal
-// logits keep the lowest id.
+// out[b][n] = sum_k W[n][k] * Y[b][k] for the 64 sequence columns (Y is the
+// activation buffer: rows 0..63 the hi plane, 64..127 the lo plane; columns
+// of sequences >= B are computed and ignored), followed by the mode's
+// epilogue.  Grid (tiles, splits); cluster (1, splits): the CTAs of a tile.
 struct GemmArgs {
-  int n_mat;
-  int rows[3];   // output rows of each stacked matrix
-  int tiles[3];  // ceil(rows / 128)
-  int off[3];    // first partial column of each matrix
+  int n_mat;     // kQKV: 3 (q, k, v); others 1
+  int rows[3];   // output rows of each matrix (kSwiGLU: F; the tile pairs gate/up)
+  int tiles[3];  // tiles of each matrix
   int k_chunks;  // ceil(K / 64)
   int splits;
-  int ldp;       // partial row length (sum of rows)
-  int B;
-  float* part;   // [splits][64][ldp]
-  unsigned long long* keys;  // MODE 1: [64]
-  float* logits;             // MODE 1: [B][rows[0]] or null
+  int B, H, D, Hq, Hkv, F;
+  float eps;
+  int n_ssp;             // tiles of the residual-producing GEMMs (ceil(H / 128))
+  const float* ssp_in;   // [n_ssp][64] sums of squares of the residual (kQKV, kSwiGLU, kLm)
+  float* ssp_out;        // kResid: [n_ssp][64]
+  float* x;              // kResid: residual [64][H]
+  float* hidden;         // kResid: [B][H] slot or null
+  const uint16_t* gain;  // kResid: the next RMSNorm's gain; kQKV: q-norm gain
+  const uint16_t* gain2; // kQKV: k-norm gain
+  uint16_t* act;         // kResid: act_h; kSwiGLU: act_u
+  float* q;              // kQKV: [64][Hq][D]
+  uint8_t* kv;
+  float* kv_scales;
+  int kv_batch, max_ctx, layer, kv_fp8;
+  const int32_t* pos;
+  const int* bad;
+  const float* inv_freq;
+  unsigned long long* keys;  // kLm: [64]
+  float* logits;             // kLm: [B][V] or null
   int* status;
   unsigned long long timeout_ns;
 };
 
 template <int MODE>
-__global__ void __launch_bounds__(kGemmThreads) gemm_kernel(const __grid_constant__ CUtensorMap w0,
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap w0,
                                                             const __grid_constant__ CUtensorMap w1,
                                                             const __grid_constant__ CUtensorMap w2,
                                                             const __grid_constant__ CUtensorMap xm,
                                                             const GemmArgs g) {
   extern __shared__ uint8_t dsm[];
+  __shared__ float s_red[8];
+  __shared__ float s_e[kTileM];
+  __shared__ float s_inv[kTileN];
   const uint32_t raw = smem_u32(dsm);
   uint8_t* sm = dsm + (((raw + 1023u) & ~1023u) - raw);  // swizzle atoms need 1024-B alignment
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + kGemmStages * kStageBytes);
@@ -141,7 +193,6 @@ __global__ void __launch_bounds__(kGemmThreads) gemm_kernel(const __grid_constan
   }
   const CUtensorMap* wm = mat == 0 ? &w0 : (mat == 1 ? &w1 : &w2);
   const int mrows = mat == 0 ? g.rows[0] : (mat == 1 ? g.rows[1] : g.rows[2]);
-  const int moff = mat == 0 ? g.off[0] : (mat == 1 ? g.off[1] : g.off[2]);
   const int split = blockIdx.y;
   const int c0 = split * g.k_chunks / g.splits;
   const int nch = (split + 1) * g.k_chunks / g.splits - c0;
@@ -161,25 +212,45 @@ __global__ void __launch_bounds__(kGemmThreads) gemm_kernel(const __grid_constan
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (tid == 0) pdl_trigger();
   const uint32_t tmem = *tslot;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---- producer: weight tile (streamed once: evict first) + activations
+      // ---- producer.  Weight tiles (streamed once: evict first) do not
+      // depend on earlier kernels: the first stages load before pdl_wait().
       tma_prefetch_map(wm);
       tma_prefetch_map(&xm);
       const uint64_t pw = policy_evict_first();
       const uint64_t px = policy_evict_last();
-      int issued = 0;
-      for (int i = 0; i < nch; ++i) {
-        const int s = i % kGemmStages;
-        if (i >= kGemmStages &&
-            !bt_wait(&empty[s], ((i / kGemmStages) - 1) & 1, g.timeout_ns, g.status))
-          break;
+      auto load_a = [&](int i, int s) {
         const uint32_t st = smem_u32(sm + s * kStageBytes);
-        mbar_arrive_expect_tx(&full[s], kStageBytes);
-        tma_load_2d(st, wm, (c0 + i) * kChunkK, tile * kTileM, smem_u32(&full[s]), pw);
+        const int x = (c0 + i) * kChunkK;
+        if constexpr (MODE == kSwiGLU) {
+          tma_load_2d(st, &w0, x, tile * (kTileM / 2), smem_u32(&full[s]), pw);
+          tma_load_2d(st + kHalfA, &w1, x, tile * (kTileM / 2), smem_u32(&full[s]), pw);
+        } else {
+          tma_load_2d(st, wm, x, tile * kTileM, smem_u32(&full[s]), pw);
+        }
+      };
+      auto load_b = [&](int i, int s) {
+        const uint32_t st = smem_u32(sm + s * kStageBytes);
         tma_load_2d(st + kABytes, &xm, (c0 + i) * kChunkK, 0, smem_u32(&full[s]), px);
+      };
+      const int pre = nch < kGemmStages ? nch : kGemmStages;
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&full[i], kStageBytes);
+        load_a(i, i);
+      }
+      pdl_wait();
+      for (int i = 0; i < pre; ++i) load_b(i, i);
+      int issued = pre;
+      for (int i = pre; i < nch; ++i) {
+        const int s = i % kGemmStages;
+        if (!bt_wait(&empty[s], ((i / kGemmStages) - 1) & 1, g.timeout_ns, g.status)) break;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        load_a(i, s);
+        load_b(i, s);
         ++issued;
       }
       // drain: every issued copy has landed before the CTA may exit
@@ -191,7 +262,7 @@ __global__ void __launch_bounds__(kGemmThreads) gemm_kernel(const __grid_constan
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---- MMA issuer: 4 x (128 x 64 x 16) per stage, accumulating in TMEM
+      // ---- MMA issuer: per stage 4 K-steps x (hi, lo) of 128 x 64 x 16
       for (int i = 0; i < nch; ++i) {
         const int s = i % kGemmStages;
         if (!bt_wait(&full[s], (i / kGemmStages) & 1, g.timeout_ns, g.status)) break;
@@ -211,7 +282,7 @@ __global__ void __launch_bounds__(kGemmThreads) gemm_kernel(const __grid_constan
     __syncwarp();
   }
 
-  // ---- epilogue: TMEM lane = weight row (warp w: rows 32w..32w+31), column = sequence
+  // ---- accumulator: TMEM lane = tile row (warp w: rows 32w..32w+31), column = sequence
   bt_wait(done, 0, g.timeout_ns, g.status);
   tc_fence_after();
   float v[kTileN];
@@ -220,34 +291,31 @@ __global__ void __launch_bounds__(kGemmThreads) gemm_kernel(const __grid_constan
   for (int c = 0; c < kTileN; c += 16) tc_ld16(tl + c, v + c);
   tc_wait_ld();
   const int m = warp * 32 + lane;
-  const int row = tile * kTileM + m;
-  const bool valid = row < mrows;
+  pdl_wait();  // everything below reads or writes what earlier kernels use
 
-  if constexpr (MODE == 0) {
-    if (valid) {
-      float* dst = g.part + static_cast<size_t>(split) * kTileN * g.ldp + moff + row;
+  if constexpr (MODE == kLm) {
+    // logits = rsqrt(mean x^2 + eps) * (W (g x)); argmax per sequence
+    if (tid < kTileN) s_inv[tid] = rms_scale(g.ssp_in, g.n_ssp, tid, g.H, g.eps);
+    __syncthreads();
 #pragma unroll
-      for (int b = 0; b < kTileN; ++b)
-        if (b < g.B) dst[static_cast<size_t>(b) * g.ldp] = v[b];
-    }
-  } else {
+    for (int b = 0; b < kTileN; ++b) v[b] *= s_inv[b];
     const int V = g.rows[0];
-    if (g.logits && valid) {
+    const int row = tile * kTileM + m;
+    if (g.logits && row < V) {
 #pragma unroll
       for (int b = 0; b < kTileN; ++b)
         if (b < g.B) g.logits[static_cast<size_t>(b) * V + row] = v[b];
     }
-    // transpose through the (now idle) stage buffers: T[b][m]
-    float* T = reinterpret_cast<float*>(sm);
+    float* T = reinterpret_cast<float*>(sm);  // the (idle) ring: T[b][row]
 #pragma unroll
-    for (int b = 0; b < kTileN; ++b) T[b * kLmStride + m] = v[b];
+    for (int b = 0; b < kTileN; ++b) T[b * kTStride + m] = v[b];
     __syncthreads();
     // thread (b = tid / 2, half = tid % 2) scans rows half*64 .. half*64+63 of sequence b
     const int b = tid >> 1, half = tid & 1;
     float best = -INFINITY;
     int bi = 0x7fffffff;
     if (b < g.B) {
-      const float4* t4 = reinterpret_cast<const float4*>(T + b * kLmStride + half * 64);
+      const float4* t4 = reinterpret_cast<const float4*>(T + b * kTStride + half * 64);
       for (int j = 0; j < 16; ++j) {
         const float4 x = t4[j];
         const float xs[4] = {x.x, x.y, x.z, x.w};
@@ -270,6 +338,97 @@ __global__ void __launch_bounds__(kGemmThreads) gemm_kernel(const __grid_constan
     if (half == 0 && b < g.B && bi != 0x7fffffff)
       atomicMax(&g.keys[b], (static_cast<unsigned long long>(order_key(best)) << 32) |
                                 static_cast<uint32_t>(~bi));
+  } else {
+    // ---- split-K reduction across the cluster, then the phase's epilogue
+    float* T = reinterpret_cast<float*>(sm);
+#pragma unroll
+    for (int b = 0; b < kTileN; ++b) T[b * kTStride + m] = v[b];
+    cluster_sync();  // every split's tile is in its CTA's shared memory
+    const uint32_t S = static_cast<uint32_t>(g.splits);
+    const uint32_t rank = cluster_rank();
+    const uint32_t t_addr = smem_u32(T);
+    const int D = g.D;
+    for (int b = static_cast<int>(rank); b < g.B; b += static_cast<int>(S)) {
+      float val = 0.f;
+      for (uint32_t s = 0; s < S; ++s)  // fixed order: deterministic
+        val += ld_dsmem(map_rank(t_addr + 4u * static_cast<uint32_t>(b * kTStride + m), s));
+      if constexpr (MODE == kQKV) {
+        const int row = tile * kTileM + m;  // row within q, k or v
+        const int head = row / D, d = row - head * D;
+        val *= rms_scale(g.ssp_in, g.n_ssp, b, g.H, g.eps);
+        const int p = g.pos[b];
+        if (mat < 2) {
+          // RMSNorm over the head (D / 32 warps), gain, rotate pairs (i, i + D/2)
+          const float ss = warp_sum(val * val);
+          if (lane == 0) s_red[warp] = ss;
+          __syncthreads();
+          const int wh = (m / D) * (D / 32);
+          float hs = 0.f;
+          for (int w = 0; w < D / 32; ++w) hs += s_red[wh + w];
+          const uint16_t* gn = mat == 0 ? g.gain : g.gain2;
+          val = val * rsqrtf(hs / static_cast<float>(D) + g.eps) * bf16_to_f(gn[d]);
+          s_e[m] = val;
+          __syncthreads();
+          const int half = D / 2;
+          const int i = d < half ? d : d - half;
+          const float partner = s_e[m ^ half];
+          const float ang = __fmul_rn(static_cast<float>(p), g.inv_freq[i]);
+          float sn, cs;
+          rope_sincos(ang, &sn, &cs);
+          val = d < half ? val * cs - partner * sn : val * cs + partner * sn;
+        }
+        if (mat == 0) {
+          g.q[(static_cast<size_t>(b) * g.Hq + head) * D + d] = val;
+        } else if (!*g.bad) {  // an invalid step leaves the cache unchanged
+          const int kvsel = mat - 1;
+          const size_t plane =
+              ((static_cast<size_t>(g.layer) * 2 + kvsel) * g.kv_batch + b) * g.Hkv + head;
+          const size_t crow = plane * g.max_ctx + p;
+          if (!g.kv_fp8) {
+            reinterpret_cast<uint16_t*>(g.kv)[crow * D + d] = f_to_bf16(val);
+          } else {
+            // E4M3 with one fp32 scale per row: scale = max(amax, 2^-126) / 448
+            const float am = warp_max(fabsf(val));
+            __syncthreads();  // s_red may still hold the norm sums
+            if (lane == 0) s_red[warp] = am;
+            __syncthreads();
+            const int wh = (m / D) * (D / 32);
+            float hm = 0.f;
+            for (int w = 0; w < D / 32; ++w) hm = fmaxf(hm, s_red[wh + w]);
+            hm = fmaxf(hm, 1.17549435e-38f);
+            const float sc = __fdiv_rn(hm, 448.0f);
+            g.kv[crow * D + d] =
+                static_cast<uint8_t>(f2_to_e4m3x2(__fdiv_rn(val, sc), 0.f) & 0xFF);
+            if (d == 0) g.kv_scales[crow] = sc;
+          }
+        }
+        __syncthreads();  // s_red / s_e are reused by the next sequence
+      } else if constexpr (MODE == kResid) {
+        const int row = tile * kTileM + m;
+        float sq = 0.f;
+        if (row < mrows) {
+          float* xp = g.x + static_cast<size_t>(b) * g.H + row;
+          const float xn = *xp + val;
+          *xp = xn;
+          if (g.hidden) g.hidden[static_cast<size_t>(b) * g.H + row] = xn;
+          put_act(g.act, b, row, g.H, xn * bf16_to_f(g.gain[row]));
+          sq = xn * xn;
+        }
+        const float ss = block_sum(sq, s_red);
+        if (tid == 0) g.ssp_out[tile * kTileN + b] = ss;
+      } else {  // kSwiGLU: rows 0..63 gate, 64..127 up, of columns tile*64 ..
+        val *= rms_scale(g.ssp_in, g.n_ssp, b, g.H, g.eps);
+        s_e[m] = val;
+        __syncthreads();
+        const int n = tile * (kTileM / 2) + m;
+        if (m < kTileM / 2 && n < g.F) {
+          const float up = s_e[m + kTileM / 2];
+          put_act(g.act, b, n, g.F, val / (1.0f + __expf(-val)) * up);
+        }
+        __syncthreads();
+      }
+    }
+    cluster_sync();  // no CTA leaves while another may still read its tile
   }
   tc_fence_before();
   __syncthreads();
@@ -279,55 +438,35 @@ __global__ void __launch_bounds__(kGemmThreads) gemm_kernel(const __grid_constan
   }
 }
 
-// ================================================================ row kernels
+// ================================================================ small kernels
 struct StepArgs2 {
-  int B, L, H, Hq, Hkv, D, F, V;
-  float eps;
+  int B, H, V, n_ssp, max_ctx;
   const int32_t* tok;
   const int32_t* pos;
   int32_t* out;
   const uint16_t* embed;
-  float* x;           // residual stream [64][H] fp32
-  uint16_t* act_h;    // [2][64][H]   normalised hidden state (GEMM operand, hi/lo planes)
-  uint16_t* act_o;    // [2][64][HqD] attention output
-  uint16_t* act_u;    // [2][64][F]   SwiGLU output
-  float* q;           // [64][Hq][D] fp32 rotated queries
-  float* part;        // GEMM split partials
-  unsigned long long* keys;  // [64]
-  int* bad;           // this step's input-validation bits
+  const uint16_t* g_in;   // layer 0 input RMSNorm gain
+  float* x;               // residual stream [64][H] fp32
+  uint16_t* act_h;        // [2][64][H]
+  float* ssp;             // [n_ssp][64]
+  unsigned long long* keys;
+  int* bad;
   int* status;
-  const float* inv_freq;
-  float* hidden;      // [L+1][B][H] or null
-  uint8_t* kv;
-  float* kv_scales;
-  int kv_batch, max_ctx;
+  float* hidden;          // [B][H] slot 0 or null
 };
 
-// x as the two bf16 planes of a tensor-core activation buffer [2][64][K]
-__device__ __forceinline__ void put_act(uint16_t* buf, int b, int n, int K, float x) {
-  const uint16_t hi = f_to_bf16(x);
-  buf[static_cast<size_t>(b) * K + n] = hi;
-  buf[static_cast<size_t>(kTileN + b) * K + n] = f_to_bf16(x - bf16_to_f(hi));
-}
-
-__device__ float block_sum(float v, float* red) {
-  v = warp_sum(v);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __syncthreads();  // red may still be read from a previous call
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  float t = 0.f;
-  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += red[w];
-  return t;
-}
-
 // Validation of every sequence's token and position (all CTAs reach the same
-// answer), the embedding row, the first input RMSNorm.  Grid: B.
-__global__ void __launch_bounds__(kRowThreads) embed_kernel(const StepArgs2 a, const uint16_t* g_in) {
+// answer), the embedding row, the first RMSNorm's operand g * x and sum of
+// squares.  Grid: B.
+__global__ void __launch_bounds__(kRowThreads) embed_kernel(const StepArgs2 a) {
   __shared__ float red[kRowThreads / 32];
   __shared__ int s_bad;
   const int b = blockIdx.x, tid = threadIdx.x;
-  if (tid == 0) s_bad = 0;
+  if (tid == 0) {
+    pdl_trigger();
+    s_bad = 0;
+  }
+  pdl_wait();
   __syncthreads();
   for (int i = tid; i < a.B; i += blockDim.x) {
     const int t = a.tok[i], p = a.pos[i];
@@ -350,121 +489,29 @@ __global__ void __launch_bounds__(kRowThreads) embed_kernel(const StepArgs2 a, c
     const float xv = bf16_to_f(e[n]);
     x[n] = xv;
     if (a.hidden) a.hidden[static_cast<size_t>(b) * a.H + n] = xv;
+    put_act(a.act_h, b, n, a.H, xv * bf16_to_f(a.g_in[n]));
     ss = fmaf(xv, xv, ss);
   }
   ss = block_sum(ss, red);
-  const float inv = rsqrtf(ss / static_cast<float>(a.H) + a.eps);
-  for (int n = tid; n < a.H; n += blockDim.x)
-    put_act(a.act_h, b, n, a.H, x[n] * inv * bf16_to_f(g_in[n]));
+  if (tid < a.n_ssp) a.ssp[tid * kTileN + b] = tid == 0 ? ss : 0.f;
 }
 
-// x += sum of the GEMM split partials; optionally record x; act = bf16(RMSNorm(x) * g).
-// Grid: B.
-__global__ void __launch_bounds__(kRowThreads) resid_norm_kernel(const StepArgs2 a, int splits,
-                                                                 const uint16_t* gain,
-                                                                 float* hidden_slot) {
-  __shared__ float red[kRowThreads / 32];
-  const int b = blockIdx.x, tid = threadIdx.x, H = a.H;
-  float* x = a.x + static_cast<size_t>(b) * H;
-  float ss = 0.f;
-  for (int n = tid; n < H; n += blockDim.x) {
-    float xv = x[n];
-    for (int s = 0; s < splits; ++s) xv += a.part[(static_cast<size_t>(s) * kTileN + b) * H + n];
-    x[n] = xv;
-    if (hidden_slot) hidden_slot[static_cast<size_t>(b) * H + n] = xv;
-    ss = fmaf(xv, xv, ss);
-  }
-  ss = block_sum(ss, red);
-  const float inv = rsqrtf(ss / static_cast<float>(H) + a.eps);
-  for (int n = tid; n < H; n += blockDim.x) put_act(a.act_h, b, n, H, x[n] * inv * bf16_to_f(gain[n]));
-}
-
-// u = silu(gate) * up from the split partials [s][b][gate F | up F].  Grid: (ceil(F/256), B).
-__global__ void __launch_bounds__(kRowThreads) swiglu_kernel(const StepArgs2 a, int splits) {
-  const int b = blockIdx.y, n = blockIdx.x * blockDim.x + threadIdx.x, F = a.F;
-  if (n >= F) return;
-  float gs = 0.f, us = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float* pr = a.part + (static_cast<size_t>(s) * kTileN + b) * (2 * F);
-    gs += pr[n];
-    us += pr[F + n];
-  }
-  put_act(a.act_u, b, n, F, gs / (1.0f + __expf(-gs)) * us);
-}
-
-// Per (sequence, head) of the stacked QKV output: sum the split partials,
-// RMSNorm + rotate q and k heads, store the rotated query, append the new K
-// and V rows to the cache (bf16, or E4M3 codes + row scale).  One warp per
-// head; lane holds elements lane + 32 k, so rotation pairs (i, i + D/2) sit
-// in the same lane.  Grid: (ceil((Hq + 2 Hkv) / 4), B).
-template <int D, bool FP8>
-__global__ void __launch_bounds__(128) qkv_post_kernel(const StepArgs2 a, int splits, int l,
-                                                       const uint16_t* gq, const uint16_t* gk) {
-  constexpr int DL = D / 32;
-  const int b = blockIdx.y, lane = threadIdx.x & 31;
-  const int head = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int nh = a.Hq + 2 * a.Hkv;
-  if (head >= nh) return;
-  const int ldp = nh * D;
-  float v[DL];
-#pragma unroll
-  for (int k = 0; k < DL; ++k) {
-    const int n = head * D + lane + 32 * k;
-    float s = 0.f;
-    for (int sp = 0; sp < splits; ++sp) s += a.part[(static_cast<size_t>(sp) * kTileN + b) * ldp + n];
-    v[k] = s;
-  }
-  const int p = a.pos[b];
-  if (head < a.Hq + a.Hkv) {
-    const uint16_t* gn = head < a.Hq ? gq : gk;
-    float ss = 0.f;
-#pragma unroll
-    for (int k = 0; k < DL; ++k) ss = fmaf(v[k], v[k], ss);
-    ss = warp_sum(ss);
-    const float inv = rsqrtf(ss / static_cast<float>(D) + a.eps);
-#pragma unroll
-    for (int k = 0; k < DL; ++k) v[k] = v[k] * inv * bf16_to_f(gn[lane + 32 * k]);
-#pragma unroll
-    for (int k = 0; k < DL / 2; ++k) {
-      const float ang = __fmul_rn(static_cast<float>(p), a.inv_freq[lane + 32 * k]);
-      float sn, cs;
-      rope_sincos(ang, &sn, &cs);
-      const float x1 = v[k], x2 = v[k + DL / 2];
-      v[k] = x1 * cs - x2 * sn;
-      v[k + DL / 2] = x2 * cs + x1 * sn;
-    }
-  }
-  if (head < a.Hq) {
-    float* qd = a.q + (static_cast<size_t>(b) * a.Hq + head) * D;
-#pragma unroll
-    for (int k = 0; k < DL; ++k) qd[lane + 32 * k] = v[k];
-    return;
-  }
-  if (*a.bad) return;  // an invalid step leaves the cache unchanged
-  const int kvsel = head < a.Hq + a.Hkv ? 0 : 1;
-  const int g = head - a.Hq - kvsel * a.Hkv;
-  const size_t plane = ((static_cast<size_t>(l) * 2 + kvsel) * a.kv_batch + b) * a.Hkv + g;
-  const size_t row = plane * a.max_ctx + p;
-  if constexpr (!FP8) {
-    uint16_t* dst = reinterpret_cast<uint16_t*>(a.kv) + row * D;
-#pragma unroll
-    for (int k = 0; k < DL; ++k) dst[lane + 32 * k] = f_to_bf16(v[k]);
-  } else {
-    uint8_t code[DL];
-    const float sc = quantize_row_e4m3<DL>(v, code);
-    uint8_t* dst = a.kv + row * D;
-#pragma unroll
-    for (int k = 0; k < DL; ++k) dst[lane + 32 * k] = code[k];
-    if (lane == 0) a.kv_scales[row] = sc;
-  }
+// out_ids from the argmax keys (-1 for every sequence of an invalid step).
+__global__ void finish_kernel(const StepArgs2 a) {
+  pdl_wait();
+  const int b = threadIdx.x;
+  if (b >= a.B) return;
+  const unsigned long long key = a.keys[b];
+  a.out[b] = (*a.bad || key == 0ull) ? -1 : static_cast<int32_t>(~static_cast<uint32_t>(key));
 }
 
 // ================================================================ attention
 // Split-K GQA decode attention over the step's cache: CTA = (sequence b, KV
 // head g, chunk of chunk_rows rows of 0..p_b).  K and V rows of 32-row tiles
-// arrive by 1-D bulk copies into a 4-stage ring; each warp keeps an fp32
-// online softmax (base-2 exponent) per query head of the group; the last
-// CTA of (b, g) merges the chunks and writes the bf16 o_proj operand.
+// arrive by 1-D bulk copies into a 4-stage ring; each warp takes two rows at
+// a time (two independent dot-product chains) and keeps an fp32 online
+// softmax (base-2 exponent) per query head of the group; the last CTA of
+// (b, g) merges the chunks and writes the o_proj operand planes.
 struct AttnArgs2 {
   int B, Hq, Hkv, max_ctx, kv_batch, l;
   const uint8_t* kv;
@@ -478,6 +525,41 @@ struct AttnArgs2 {
   int chunk_rows, chunks;
 };
 
+__device__ __forceinline__ void warp_sum2(float& a, float& b) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+}
+
+template <int D, bool FP8>
+__device__ __forceinline__ void load_kv_row(const uint8_t* kp, const uint8_t* vp, float ks,
+                                            float vs, float (&kr)[D / 32], float (&vr)[D / 32]) {
+  constexpr int DL = D / 32;
+  if constexpr (!FP8) {
+    if constexpr (DL == 4) {
+      const uint2 kw = *reinterpret_cast<const uint2*>(kp);
+      const uint2 vw = *reinterpret_cast<const uint2*>(vp);
+      kr[0] = bf16lo(kw.x); kr[1] = bf16hi(kw.x); kr[2] = bf16lo(kw.y); kr[3] = bf16hi(kw.y);
+      vr[0] = bf16lo(vw.x); vr[1] = bf16hi(vw.x); vr[2] = bf16lo(vw.y); vr[3] = bf16hi(vw.y);
+    } else {
+      const uint32_t kw = *reinterpret_cast<const uint32_t*>(kp);
+      const uint32_t vw = *reinterpret_cast<const uint32_t*>(vp);
+      kr[0] = bf16lo(kw); kr[1] = bf16hi(kw);
+      vr[0] = bf16lo(vw); vr[1] = bf16hi(vw);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < DL; k += 2) {
+      const float2 kf = e4m3x2_to_f2(*reinterpret_cast<const uint16_t*>(kp + k));
+      const float2 vf = e4m3x2_to_f2(*reinterpret_cast<const uint16_t*>(vp + k));
+      kr[k] = kf.x * ks; kr[k + 1] = kf.y * ks;
+      vr[k] = vf.x * vs; vr[k + 1] = vf.y * vs;
+    }
+  }
+}
+
 template <int D, bool FP8>
 __global__ void __launch_bounds__(kAttThreads) attn_kernel(const AttnArgs2 a) {
   constexpr int DL = D / 32;
@@ -490,6 +572,8 @@ __global__ void __launch_bounds__(kAttThreads) attn_kernel(const AttnArgs2 a) {
   float* merge = reinterpret_cast<float*>(full + kAttStages);  // [warps][rep][D + 2]
   __shared__ int s_last;
 
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
   if (*a.bad) return;
   const int rep = a.Hq / a.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -551,45 +635,35 @@ __global__ void __launch_bounds__(kAttThreads) attn_kernel(const AttnArgs2 a) {
         if (sp.expired()) break;
     }
     const uint8_t* tb = ring + (t % kAttStages) * kTile;
-    for (int r = warp; r < nr; r += kAttWarps) {
-      float kr[DL], vr[DL];
-      const uint8_t* kp = tb + static_cast<size_t>(r) * D * E + lane * DL * E;
-      const uint8_t* vp = kp + kHalf;
-      if constexpr (!FP8) {
-        if constexpr (DL == 4) {
-          const uint2 kw = *reinterpret_cast<const uint2*>(kp);
-          const uint2 vw = *reinterpret_cast<const uint2*>(vp);
-          kr[0] = bf16lo(kw.x); kr[1] = bf16hi(kw.x); kr[2] = bf16lo(kw.y); kr[3] = bf16hi(kw.y);
-          vr[0] = bf16lo(vw.x); vr[1] = bf16hi(vw.x); vr[2] = bf16lo(vw.y); vr[3] = bf16hi(vw.y);
-        } else {
-          const uint32_t kw = *reinterpret_cast<const uint32_t*>(kp);
-          const uint32_t vw = *reinterpret_cast<const uint32_t*>(vp);
-          kr[0] = bf16lo(kw); kr[1] = bf16hi(kw);
-          vr[0] = bf16lo(vw); vr[1] = bf16hi(vw);
-        }
-      } else {
-        const float ks = ksc[j + r], vs = vsc[j + r];
-#pragma unroll
-        for (int k = 0; k < DL; k += 2) {
-          const float2 kf = e4m3x2_to_f2(*reinterpret_cast<const uint16_t*>(kp + k));
-          const float2 vf = e4m3x2_to_f2(*reinterpret_cast<const uint16_t*>(vp + k));
-          kr[k] = kf.x * ks; kr[k + 1] = kf.y * ks;
-          vr[k] = vf.x * vs; vr[k + 1] = vf.y * vs;
-        }
-      }
+    for (int r = warp; r < nr; r += 2 * kAttWarps) {
+      const int r2 = r + kAttWarps;
+      const bool two = r2 < nr;  // warp-uniform
+      const int rr = two ? r2 : r;
+      float k1[DL], v1[DL], k2[DL], v2[DL];
+      load_kv_row<D, FP8>(tb + static_cast<size_t>(r) * D * E + lane * DL * E,
+                          tb + kHalf + static_cast<size_t>(r) * D * E + lane * DL * E,
+                          FP8 ? ksc[j + r] : 1.f, FP8 ? vsc[j + r] : 1.f, k1, v1);
+      load_kv_row<D, FP8>(tb + static_cast<size_t>(rr) * D * E + lane * DL * E,
+                          tb + kHalf + static_cast<size_t>(rr) * D * E + lane * DL * E,
+                          FP8 ? ksc[j + rr] : 1.f, FP8 ? vsc[j + rr] : 1.f, k2, v2);
 #pragma unroll
       for (int h = 0; h < kAttMaxRep; ++h) {
         if (h < rep) {
-          float s = 0.f;
+          float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-          for (int k = 0; k < DL; ++k) s = fmaf(qv[h][k], kr[k], s);
-          s = warp_sum(s);
-          const float mn = fmaxf(m[h], s);
+          for (int k = 0; k < DL; ++k) {
+            s1 = fmaf(qv[h][k], k1[k], s1);
+            s2 = fmaf(qv[h][k], k2[k], s2);
+          }
+          warp_sum2(s1, s2);
+          if (!two) s2 = -INFINITY;
+          const float mn = fmaxf(m[h], fmaxf(s1, s2));
           const float al = exp2f(m[h] - mn);
-          const float pe = exp2f(s - mn);
-          ls[h] = ls[h] * al + pe;
+          const float p1 = exp2f(s1 - mn);
+          const float p2 = exp2f(s2 - mn);
+          ls[h] = ls[h] * al + p1 + p2;
 #pragma unroll
-          for (int k = 0; k < DL; ++k) acc[h][k] = fmaf(acc[h][k], al, pe * vr[k]);
+          for (int k = 0; k < DL; ++k) acc[h][k] = fmaf(acc[h][k], al, fmaf(p1, v1[k], p2 * v2[k]));
           m[h] = mn;
         }
       }
@@ -657,14 +731,6 @@ __global__ void __launch_bounds__(kAttThreads) attn_kernel(const AttnArgs2 a) {
   }
 }
 
-// out_ids from the argmax keys (-1 for every sequence of an invalid step).
-__global__ void finish_kernel(const StepArgs2 a) {
-  const int b = threadIdx.x;
-  if (b >= a.B) return;
-  const unsigned long long key = a.keys[b];
-  a.out[b] = (*a.bad || key == 0ull) ? -1 : static_cast<int32_t>(~static_cast<uint32_t>(key));
-}
-
 size_t attn_smem(int D, int rep, bool fp8) {
   return static_cast<size_t>(kAttStages) * kAttTileRows * D * (fp8 ? 1 : 2) * 2 +
          kAttStages * sizeof(uint64_t) + static_cast<size_t>(kAttWarps) * rep * (D + 2) * sizeof(float);
@@ -676,6 +742,33 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// Launch with the programmatic-dependent-launch attribute and, for split-K
+// GEMMs, a (1, cluster_y, 1) cluster.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, unsigned cluster_y, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  int n = 0;
+  at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_y > 1) {
+    at[n].id = cudaLaunchAttributeClusterDimension;
+    at[n].val.clusterDim.x = 1;
+    at[n].val.clusterDim.y = cluster_y;
+    at[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 }  // namespace
 
@@ -690,6 +783,7 @@ struct GemmPlan {
 struct BtPlan {
   BtShape s;
   int sms = 0;
+  int n_ssp = 0;
   const uint16_t* embed = nullptr;
   const uint16_t* final_norm = nullptr;
   std::vector<LayerPtrs> layers;
@@ -701,7 +795,7 @@ struct BtPlan {
   float* x = nullptr;
   uint16_t *act_h = nullptr, *act_o = nullptr, *act_u = nullptr;
   float* q = nullptr;
-  float* part = nullptr;
+  float* ssp = nullptr;
   float* att_part = nullptr;
   unsigned* att_cnt = nullptr;
   unsigned long long* keys = nullptr;
@@ -721,59 +815,55 @@ bool encode_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t co
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Split count so that tiles x splits covers the SMs about once.
+// K splits (= cluster size) so that tiles x splits covers the SMs about once.
 int pick_splits(int tiles, int k_chunks, int sms) {
   int s = (sms + tiles / 2) / tiles;
   if (s < 1) s = 1;
+  if (s > kMaxSplits) s = kMaxSplits;
   if (s > k_chunks) s = k_chunks;
   return s;
 }
 
+// n_mat matrices stacked along their rows; box_rows = 128 (one matrix per
+// tile) or 64 (gate/up pairs: 64 rows of each per tile).
 bool make_gemm(EncodeTiledFn enc, GemmPlan& gp, int n_mat, const uint16_t* const* w,
-               const int* rows, int K, const CUtensorMap* xmap, int sms, bool lm) {
+               const int* rows, int K, uint32_t box_rows, const CUtensorMap* xmap, int sms,
+               bool one_split) {
   GemmArgs& g = gp.args;
   g = GemmArgs{};
-  g.n_mat = n_mat;
-  int tiles = 0, off = 0;
+  g.n_mat = box_rows == kTileM ? n_mat : 1;
+  int tiles = 0;
   for (int i = 0; i < 3; ++i) {
     if (i < n_mat) {
       g.rows[i] = rows[i];
-      g.tiles[i] = (rows[i] + kTileM - 1) / kTileM;
-      g.off[i] = off;
-      off += rows[i];
-      tiles += g.tiles[i];
-      if (!encode_map(enc, &gp.w[i], w[i], K, rows[i], kTileM)) return false;
+      g.tiles[i] = (rows[i] + static_cast<int>(box_rows) - 1) / static_cast<int>(box_rows);
+      if (box_rows == kTileM || i == 0) tiles += g.tiles[i];
+      if (!encode_map(enc, &gp.w[i], w[i], K, rows[i], box_rows)) return false;
     } else {
       gp.w[i] = gp.w[0];
     }
   }
-  g.ldp = off;
   g.k_chunks = (K + kChunkK - 1) / kChunkK;
-  g.splits = lm ? 1 : pick_splits(tiles, g.k_chunks, sms);
+  g.splits = one_split ? 1 : pick_splits(tiles, g.k_chunks, sms);
   gp.x = xmap;
   gp.grid = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(g.splits));
   return true;
 }
 
-size_t part_floats(const GemmPlan& gp) {
-  return static_cast<size_t>(gp.args.splits) * kTileN * gp.args.ldp;
+template <int MODE>
+cudaError_t launch_gemm(const GemmPlan& gp, const GemmArgs& g, cudaStream_t st) {
+  return launch_pdl(gemm_kernel<MODE>, gp.grid, dim3(kGemmThreads), kGemmSmem, st,
+                    static_cast<unsigned>(g.splits), gp.w[0], gp.w[1], gp.w[2], *gp.x, g);
 }
 
-cudaError_t launch_gemm(const GemmPlan& gp, int mode, int B, float* part,
-                        unsigned long long* keys, float* logits, int* status,
-                        unsigned long long timeout, cudaStream_t st) {
-  GemmArgs g = gp.args;
-  g.B = B;
-  g.part = part;
-  g.keys = keys;
-  g.logits = logits;
-  g.status = status;
-  g.timeout_ns = timeout;
-  if (mode == 0)
-    gemm_kernel<0><<<gp.grid, kGemmThreads, kGemmSmem, st>>>(gp.w[0], gp.w[1], gp.w[2], *gp.x, g);
-  else
-    gemm_kernel<1><<<gp.grid, kGemmThreads, kGemmSmem, st>>>(gp.w[0], gp.w[1], gp.w[2], *gp.x, g);
-  return cudaGetLastError();
+template <int D>
+cudaError_t launch_attn(const AttnArgs2& a, int rep, bool fp8, cudaStream_t st) {
+  const dim3 grid(static_cast<unsigned>(a.B) * a.Hkv * a.chunks);
+  if (fp8)
+    return launch_pdl(attn_kernel<D, true>, grid, dim3(kAttThreads), attn_smem(D, rep, true), st,
+                      1u, a);
+  return launch_pdl(attn_kernel<D, false>, grid, dim3(kAttThreads), attn_smem(D, rep, false), st,
+                    1u, a);
 }
 
 }  // namespace
@@ -783,7 +873,9 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_h
                    const float* inv_freq_dev, int sms, BtPlan** out, cudaError_t* cerr) {
   *out = nullptr;
   *cerr = cudaSuccess;
-  if (s.H % kChunkK || (s.Hq * s.D) % kChunkK || s.F % kChunkK) return DEC_ERR_SHAPE;
+  const int HqD = s.Hq * s.D, HkvD = s.Hkv * s.D;
+  // tiles of 128 q / k / v rows hold whole heads; gate/up tiles pair 64 rows
+  if (s.H % kChunkK || HqD % kTileM || HkvD % kTileM || s.F % (kTileM / 2)) return DEC_ERR_SHAPE;
   if (s.Hq / s.Hkv > kAttMaxRep) return DEC_ERR_SHAPE;
   void* fn = nullptr;
   cudaDriverEntryPointQueryResult q;
@@ -797,11 +889,11 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_h
   if (!p) return DEC_ERR_ARG;
   p->s = s;
   p->sms = sms;
+  p->n_ssp = (s.H + kTileM - 1) / kTileM;
   p->embed = embed;
   p->final_norm = final_norm;
   p->inv_freq = inv_freq_dev;
   p->layers.assign(layers_host, layers_host + s.L);
-  const int HqD = s.Hq * s.D, HkvD = s.Hkv * s.D;
 
   // ---- scratch
   size_t o = 0;
@@ -815,25 +907,11 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_h
   const size_t ao_off = take(2ull * kBRows * HqD);
   const size_t au_off = take(2ull * kBRows * s.F);
   const size_t q_off = take(sizeof(float) * kTileN * HqD);
+  const size_t ssp_off = take(sizeof(float) * kTileN * p->n_ssp);
   const size_t ap_off = take(sizeof(float) * kTileN * s.Hq * kMaxAttnChunks * (s.D + 2));
   const size_t ac_off = take(sizeof(unsigned) * kTileN * s.Hkv);
   const size_t keys_off = take(sizeof(unsigned long long) * kTileN);
   const size_t bad_off = take(sizeof(int));
-  // the activation maps need the buffers' addresses: allocate after sizing the partials,
-  // which depend only on the shape (not on addresses), so plan the GEMMs twice
-  size_t part_max = 0;
-  {
-    const int tiles_qkv = (HqD + kTileM - 1) / kTileM + 2 * ((HkvD + kTileM - 1) / kTileM);
-    const int tiles_o = (s.H + kTileM - 1) / kTileM, tiles_gu = 2 * ((s.F + kTileM - 1) / kTileM);
-    const size_t c[4] = {
-        static_cast<size_t>(pick_splits(tiles_qkv, (s.H + 63) / 64, sms)) * (HqD + 2 * HkvD),
-        static_cast<size_t>(pick_splits(tiles_o, (HqD + 63) / 64, sms)) * s.H,
-        static_cast<size_t>(pick_splits(tiles_gu, (s.H + 63) / 64, sms)) * 2 * s.F,
-        static_cast<size_t>(pick_splits(tiles_o, (s.F + 63) / 64, sms)) * s.H};
-    for (size_t v : c) part_max = v > part_max ? v : part_max;
-    part_max *= kTileN;
-  }
-  const size_t part_off = take(sizeof(float) * part_max);
   e = cudaMalloc(&p->ws, o);
   if (e == cudaSuccess) e = cudaMemset(p->ws, 0, o);
   if (e != cudaSuccess) {
@@ -847,11 +925,11 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_h
   p->act_o = reinterpret_cast<uint16_t*>(p->ws + ao_off);
   p->act_u = reinterpret_cast<uint16_t*>(p->ws + au_off);
   p->q = reinterpret_cast<float*>(p->ws + q_off);
+  p->ssp = reinterpret_cast<float*>(p->ws + ssp_off);
   p->att_part = reinterpret_cast<float*>(p->ws + ap_off);
   p->att_cnt = reinterpret_cast<unsigned*>(p->ws + ac_off);
   p->keys = reinterpret_cast<unsigned long long*>(p->ws + keys_off);
   p->bad = reinterpret_cast<int*>(p->ws + bad_off);
-  p->part = reinterpret_cast<float*>(p->ws + part_off);
 
   // ---- tensor maps and GEMM plans
   bool ok = encode_map(enc, &p->map_h, p->act_h, s.H, kBRows, kBRows) &&
@@ -870,24 +948,38 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_h
     const uint16_t* wgu[2] = {lp.w[DEC_LW_GATE], lp.w[DEC_LW_UP]};
     const int rgu[2] = {s.F, s.F};
     const uint16_t* wd[1] = {lp.w[DEC_LW_DOWN]};
-    ok = make_gemm(enc, p->qkv[l], 3, wqkv, rqkv, s.H, &p->map_h, sms, false) &&
-         make_gemm(enc, p->o[l], 1, wo, ro, HqD, &p->map_o, sms, false) &&
-         make_gemm(enc, p->gu[l], 2, wgu, rgu, s.H, &p->map_h, sms, false) &&
-         make_gemm(enc, p->down[l], 1, wd, ro, s.F, &p->map_u, sms, false);
-    ok = ok && part_floats(p->qkv[l]) <= part_max && part_floats(p->o[l]) <= part_max &&
-         part_floats(p->gu[l]) <= part_max && part_floats(p->down[l]) <= part_max;
+    ok = make_gemm(enc, p->qkv[l], 3, wqkv, rqkv, s.H, kTileM, &p->map_h, sms, false) &&
+         make_gemm(enc, p->o[l], 1, wo, ro, HqD, kTileM, &p->map_o, sms, false) &&
+         make_gemm(enc, p->gu[l], 2, wgu, rgu, s.H, kTileM / 2, &p->map_h, sms, false) &&
+         make_gemm(enc, p->down[l], 1, wd, ro, s.F, kTileM, &p->map_u, sms, false);
   }
   if (ok) {
     const uint16_t* wl[1] = {lm_head};
     const int rl[1] = {s.V};
-    ok = make_gemm(enc, p->lm, 1, wl, rl, s.H, &p->map_h, sms, true);
+    ok = make_gemm(enc, p->lm, 1, wl, rl, s.H, kTileM, &p->map_h, sms, true);
   }
-  if (ok) {
-    e = cudaFuncSetAttribute(gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kGemmSmem));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kGemmSmem));
+  // kernel attributes, once
+  const int smem = static_cast<int>(kGemmSmem);
+  const cudaFuncAttribute dyn = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  if (ok) e = cudaFuncSetAttribute(gemm_kernel<kQKV>, dyn, smem);
+  if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kResid>, dyn, smem);
+  if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kSwiGLU>, dyn, smem);
+  if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kLm>, dyn, smem);
+  const int rep = s.Hq / s.Hkv;
+  if (ok && e == cudaSuccess) {
+    if (s.D == 128) {
+      e = cudaFuncSetAttribute(attn_kernel<128, false>, dyn,
+                               static_cast<int>(attn_smem(128, rep, false)));
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(attn_kernel<128, true>, dyn,
+                                 static_cast<int>(attn_smem(128, rep, true)));
+    } else {
+      e = cudaFuncSetAttribute(attn_kernel<64, false>, dyn,
+                               static_cast<int>(attn_smem(64, rep, false)));
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(attn_kernel<64, true>, dyn,
+                                 static_cast<int>(attn_smem(64, rep, true)));
+    }
   }
   if (!ok || e != cudaSuccess) {
     *cerr = e;
@@ -905,61 +997,44 @@ void bt_plan_destroy(BtPlan* p) {
   delete p;
 }
 
-namespace {
-
-template <int D, bool FP8>
-cudaError_t launch_attn(const AttnArgs2& a, int rep, cudaStream_t st) {
-  const size_t smem = attn_smem(D, rep, FP8);
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, FP8>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  attn_kernel<D, FP8><<<static_cast<unsigned>(a.B) * a.Hkv * a.chunks, kAttThreads, smem, st>>>(a);
-  return cudaGetLastError();
-}
-
-template <int D, bool FP8>
-cudaError_t launch_qkv_post(const StepArgs2& a, int splits, int l, const LayerPtrs& lp,
-                            cudaStream_t st) {
-  const dim3 grid((a.Hq + 2 * a.Hkv + 3) / 4, a.B);
-  qkv_post_kernel<D, FP8><<<grid, 128, 0, st>>>(a, splits, l, lp.w[DEC_LW_Q_NORM],
-                                                lp.w[DEC_LW_K_NORM]);
-  return cudaGetLastError();
-}
-
-}  // namespace
-
 cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
   const BtShape& s = p->s;
-  StepArgs2 a{};
-  a.B = io.B;
-  a.L = s.L;
-  a.H = s.H;
-  a.Hq = s.Hq;
-  a.Hkv = s.Hkv;
-  a.D = s.D;
-  a.F = s.F;
-  a.V = s.V;
-  a.eps = s.eps;
-  a.tok = io.tok;
-  a.pos = io.pos;
-  a.out = io.out;
-  a.embed = p->embed;
-  a.x = p->x;
-  a.act_h = p->act_h;
-  a.act_o = p->act_o;
-  a.act_u = p->act_u;
-  a.q = p->q;
-  a.part = p->part;
-  a.keys = p->keys;
-  a.bad = p->bad;
-  a.status = io.status;
-  a.inv_freq = p->inv_freq;
-  a.hidden = io.hidden;
-  a.kv = io.kv;
-  a.kv_scales = io.kv_scales;
-  a.kv_batch = io.kv_batch;
-  a.max_ctx = io.max_ctx;
+  // fields every GEMM launch shares
+  GemmArgs base{};
+  base.B = io.B;
+  base.H = s.H;
+  base.D = s.D;
+  base.Hq = s.Hq;
+  base.Hkv = s.Hkv;
+  base.F = s.F;
+  base.eps = s.eps;
+  base.n_ssp = p->n_ssp;
+  base.ssp_in = p->ssp;
+  base.ssp_out = p->ssp;
+  base.x = p->x;
+  base.q = p->q;
+  base.kv = io.kv;
+  base.kv_scales = io.kv_scales;
+  base.kv_batch = io.kv_batch;
+  base.max_ctx = io.max_ctx;
+  base.kv_fp8 = io.kv_fp8;
+  base.pos = io.pos;
+  base.bad = p->bad;
+  base.inv_freq = p->inv_freq;
+  base.keys = p->keys;
+  base.status = io.status;
+  base.timeout_ns = io.timeout_ns;
+  auto args_of = [&](const GemmPlan& gp) {
+    GemmArgs g = base;
+    g.n_mat = gp.args.n_mat;
+    for (int i = 0; i < 3; ++i) {
+      g.rows[i] = gp.args.rows[i];
+      g.tiles[i] = gp.args.tiles[i];
+    }
+    g.k_chunks = gp.args.k_chunks;
+    g.splits = gp.args.splits;
+    return g;
+  };
 
   // attention chunking: about 4 CTAs per SM over the cache capacity, at most
   // kMaxAttnChunks chunks per (sequence, KV head)
@@ -984,48 +1059,57 @@ cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
   at.chunk_rows = cr;
   at.chunks = (io.max_ctx + cr - 1) / cr;
   const int rep = s.Hq / s.Hkv;
-  const unsigned long long to = io.timeout_ns;
 
-  cudaError_t e;
-  embed_kernel<<<io.B, kRowThreads, 0, st>>>(a, p->layers[0].w[DEC_LW_IN_NORM]);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  StepArgs2 sa{};
+  sa.B = io.B;
+  sa.H = s.H;
+  sa.V = s.V;
+  sa.n_ssp = p->n_ssp;
+  sa.max_ctx = io.max_ctx;
+  sa.tok = io.tok;
+  sa.pos = io.pos;
+  sa.out = io.out;
+  sa.embed = p->embed;
+  sa.g_in = p->layers[0].w[DEC_LW_IN_NORM];
+  sa.x = p->x;
+  sa.act_h = p->act_h;
+  sa.ssp = p->ssp;
+  sa.keys = p->keys;
+  sa.bad = p->bad;
+  sa.status = io.status;
+  sa.hidden = io.hidden;
+
+  cudaError_t e = launch_pdl(embed_kernel, dim3(io.B), dim3(kRowThreads), 0, st, 1u, sa);
+  if (e != cudaSuccess) return e;
   for (int l = 0; l < s.L; ++l) {
     const LayerPtrs& lp = p->layers[l];
-    if ((e = launch_gemm(p->qkv[l], 0, io.B, p->part, nullptr, nullptr, io.status, to, st)))
-      return e;
-    const int sq = p->qkv[l].args.splits;
-    if (s.D == 128)
-      e = io.kv_fp8 ? launch_qkv_post<128, true>(a, sq, l, lp, st)
-                    : launch_qkv_post<128, false>(a, sq, l, lp, st);
-    else
-      e = io.kv_fp8 ? launch_qkv_post<64, true>(a, sq, l, lp, st)
-                    : launch_qkv_post<64, false>(a, sq, l, lp, st);
-    if (e) return e;
+    GemmArgs g = args_of(p->qkv[l]);
+    g.layer = l;
+    g.gain = lp.w[DEC_LW_Q_NORM];
+    g.gain2 = lp.w[DEC_LW_K_NORM];
+    if ((e = launch_gemm<kQKV>(p->qkv[l], g, st)) != cudaSuccess) return e;
     at.l = l;
-    if (s.D == 128)
-      e = io.kv_fp8 ? launch_attn<128, true>(at, rep, st) : launch_attn<128, false>(at, rep, st);
-    else
-      e = io.kv_fp8 ? launch_attn<64, true>(at, rep, st) : launch_attn<64, false>(at, rep, st);
-    if (e) return e;
-    if ((e = launch_gemm(p->o[l], 0, io.B, p->part, nullptr, nullptr, io.status, to, st))) return e;
-    resid_norm_kernel<<<io.B, kRowThreads, 0, st>>>(a, p->o[l].args.splits,
-                                                    lp.w[DEC_LW_POST_NORM], nullptr);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = launch_gemm(p->gu[l], 0, io.B, p->part, nullptr, nullptr, io.status, to, st)))
-      return e;
-    swiglu_kernel<<<dim3((s.F + kRowThreads - 1) / kRowThreads, io.B), kRowThreads, 0, st>>>(
-        a, p->gu[l].args.splits);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = launch_gemm(p->down[l], 0, io.B, p->part, nullptr, nullptr, io.status, to, st)))
-      return e;
-    const uint16_t* next_gain = l + 1 < s.L ? p->layers[l + 1].w[DEC_LW_IN_NORM] : p->final_norm;
-    float* hs = io.hidden ? io.hidden + static_cast<size_t>(l + 1) * io.B * s.H : nullptr;
-    resid_norm_kernel<<<io.B, kRowThreads, 0, st>>>(a, p->down[l].args.splits, next_gain, hs);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = s.D == 128 ? launch_attn<128>(at, rep, io.kv_fp8 != 0, st)
+                   : launch_attn<64>(at, rep, io.kv_fp8 != 0, st);
+    if (e != cudaSuccess) return e;
+    g = args_of(p->o[l]);
+    g.gain = lp.w[DEC_LW_POST_NORM];
+    g.act = p->act_h;
+    g.hidden = nullptr;
+    if ((e = launch_gemm<kResid>(p->o[l], g, st)) != cudaSuccess) return e;
+    g = args_of(p->gu[l]);
+    g.act = p->act_u;
+    if ((e = launch_gemm<kSwiGLU>(p->gu[l], g, st)) != cudaSuccess) return e;
+    g = args_of(p->down[l]);
+    g.gain = l + 1 < s.L ? p->layers[l + 1].w[DEC_LW_IN_NORM] : p->final_norm;
+    g.act = p->act_h;
+    g.hidden = io.hidden ? io.hidden + static_cast<size_t>(l + 1) * io.B * s.H : nullptr;
+    if ((e = launch_gemm<kResid>(p->down[l], g, st)) != cudaSuccess) return e;
   }
-  if ((e = launch_gemm(p->lm, 1, io.B, nullptr, p->keys, io.logits, io.status, to, st))) return e;
-  finish_kernel<<<1, kTileN, 0, st>>>(a);
-  return cudaGetLastError();
+  GemmArgs g = args_of(p->lm);
+  g.logits = io.logits;
+  if ((e = launch_gemm<kLm>(p->lm, g, st)) != cudaSuccess) return e;
+  return launch_pdl(finish_kernel, dim3(1), dim3(kTileN), 0, st, 1u, sa);
 }
 
 }  // namespace dec
