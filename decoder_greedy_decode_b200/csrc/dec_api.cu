@@ -484,6 +484,16 @@ extern "C" int dec_kv_quantize_e4m3(const float* x, int rows, int dim, uint8_t* 
 }
 
 #ifdef DEC_PROFILE
+namespace dec {
+int bt_prof_read(BtPlan* p, unsigned long long* host, size_t n);
+}
+// Profiling builds only (not part of dec.h): GEMM phase timestamps of the
+// batched step, [4 modes][2048 CTAs][16] globaltimer values.
+extern "C" int dec_bt_prof_read(dec_handle* h, unsigned long long* host, size_t n) {
+  if (!h || !h->bt || !host) return DEC_ERR_NULL;
+  return dec::bt_prof_read(h->bt, host, n) == 0 ? DEC_OK : DEC_ERR_ARG;
+}
+
 // Profiling builds only (not part of dec.h): copy the per-phase timestamps of
 // the last step, [ctas][16 * n_layers + 8] globaltimer values, to `host`.
 extern "C" int dec_prof_read(dec_handle* h, unsigned long long* host, size_t n) {

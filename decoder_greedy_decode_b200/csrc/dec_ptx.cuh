@@ -57,6 +57,12 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Suspend-time hint (ns) of the blocking mbarrier waits below.
+#ifndef DEC_WAIT_HINT_NS
+#define DEC_WAIT_HINT_NS 20000
+#endif
+constexpr uint32_t kWaitHintNs = DEC_WAIT_HINT_NS;
+
 // Like mbar_test, but the thread may be suspended (it issues nothing) until
 // the phase completes or about hint_ns nanoseconds pass: waiting warps then
 // leave the issue slots to the warps that compute.

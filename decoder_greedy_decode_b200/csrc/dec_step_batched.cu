@@ -62,10 +62,12 @@ constexpr int kLoOffset = kTileN * kChunkK * 2;   // lo plane inside a B tile (8
 constexpr int kHalfA = kABytes / 2;               // gate/up tiles: up rows start here
 constexpr int kStageBytes = kABytes + kBBytes;    // 32 KB
 constexpr int kGemmStages = 3;
-constexpr int kGemmThreads = 128;                 // 4 warps = the 4 TMEM sub-partitions
+constexpr int kGemmThreads = 256;                 // 8 warps: 2 per TMEM sub-partition
+constexpr int kHalfN = kTileN / 2;                // accumulator columns read per warp
 constexpr uint32_t kTmemCols = 64;                // fp32 accumulator columns (= kTileN)
 constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, kTileN);
 constexpr int kTStride = kTileM + 4;              // accumulator tile in smem: T[b][row]
+constexpr int kWOffset = 40 * 1024;               // reduced rows of this CTA's sequences
 constexpr size_t kGemmSmem = 1024 + kGemmStages * kStageBytes + 256;
 constexpr int kMaxSplits = 8;                     // cluster size (portable)
 constexpr int kMaxAttnChunks = 32;
@@ -73,13 +75,16 @@ constexpr int kAttWarps = 8;
 constexpr int kAttThreads = kAttWarps * 32;
 constexpr int kAttStages = 4;
 constexpr int kAttTileRows = 32;
-constexpr int kAttMaxRep = 8;
+constexpr int kAttMaxRep = 4;  // query heads per KV head (attention template)
 constexpr int kRowThreads = 256;
+constexpr int kProfCtas = 2048;                   // GEMM CTAs with timestamps (profiling builds)
 
 enum GemmMode { kQKV = 0, kResid = 1, kSwiGLU = 2, kLm = 3 };
 
 static_assert(kTileN == 64 && kTmemCols == 64, "epilogue reads 4 x 16 accumulator columns");
-static_assert(kTileN * kTStride * 4 <= kGemmStages * kStageBytes, "accumulator tile fits the ring");
+static_assert(kTileN * kTStride * 4 <= kWOffset, "accumulator tile below the reduced rows");
+static_assert((kTileN + kMaxSplits) * kTileM * 4 <= kWOffset, "split receive rows below them");
+static_assert(kWOffset + kTileN * kTileM * 4 <= kGemmStages * kStageBytes, "both fit the ring");
 
 // Bounded mbarrier wait: the copies and MMAs always complete; the bound only
 // guards the GPU.  Returns false (and raises the timeout status) if it ran
@@ -89,7 +94,7 @@ __device__ bool bt_wait(uint64_t* bar, uint32_t parity, unsigned long long limit
                         bool give_up = true) {
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
-    if (mbar_wait(bar, parity, 20000)) return true;
+    if (mbar_wait(bar, parity, kWaitHintNs)) return true;
     if (it == 0) {
       t0 = globaltimer();
     } else {
@@ -160,7 +165,22 @@ struct GemmArgs {
   float* logits;             // kLm: [B][V] or null
   int* status;
   unsigned long long timeout_ns;
+  unsigned long long* prof;  // profiling builds: [4 modes][kProfCtas][16] timestamps, else null
 };
+
+// Phase timestamps of one GEMM CTA (profiling builds only).
+#ifdef DEC_PROFILE
+#define BT_STAMP(k)                                                                      \
+  do {                                                                                   \
+    if (g.prof && blockIdx.y * gridDim.x + blockIdx.x < kProfCtas)                       \
+      g.prof[((MODE * kProfCtas) + blockIdx.y * gridDim.x + blockIdx.x) * 16 + (k)] =    \
+          globaltimer();                                                                 \
+  } while (0)
+#else
+#define BT_STAMP(k) \
+  do {              \
+  } while (0)
+#endif
 
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap w0,
@@ -169,9 +189,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                                                             const __grid_constant__ CUtensorMap xm,
                                                             const GemmArgs g) {
   extern __shared__ uint8_t dsm[];
-  __shared__ float s_red[8];
-  __shared__ float s_e[kTileM];
-  __shared__ float s_inv[kTileN];
+  __shared__ float s_red[kGemmThreads / 32][kTileN];  // per-warp partial sums, per slot
+  __shared__ float s_inv[kTileN];      // rsqrt(mean x^2 + eps) per sequence
+  __shared__ int s_pos[kTileN];
   const uint32_t raw = smem_u32(dsm);
   uint8_t* sm = dsm + (((raw + 1023u) & ~1023u) - raw);  // swizzle atoms need 1024-B alignment
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + kGemmStages * kStageBytes);
@@ -180,6 +200,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) BT_STAMP(0);
   // stacked tile -> (matrix, tile); selects rather than indexing keep the
   // parameter arrays out of local memory
   int mat = 0, tile = blockIdx.x;
@@ -212,8 +233,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid == 0) pdl_trigger();
+  if (tid == 0) {
+    pdl_trigger();
+    BT_STAMP(1);
+  }
   const uint32_t tmem = *tslot;
+  // per-row constants of the epilogue (weights: no earlier kernel writes them)
+  float row_gain = 1.f, row_invf = 0.f;
+  {
+    const int r = tile * kTileM + (warp & 3) * 32 + lane;
+    if constexpr (MODE == kQKV) {
+      const int d = r % g.D;
+      if (mat < 2) row_gain = bf16_to_f((mat == 0 ? g.gain : g.gain2)[d]);
+      row_invf = g.inv_freq[d < g.D / 2 ? d : d - g.D / 2];
+    } else if constexpr (MODE == kResid) {
+      if (r < mrows) row_gain = bf16_to_f(g.gain[r]);
+    }
+  }
 
   if (warp == 0) {
     if (lane == 0) {
@@ -242,7 +278,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         mbar_arrive_expect_tx(&full[i], kStageBytes);
         load_a(i, i);
       }
+      BT_STAMP(2);
       pdl_wait();
+      BT_STAMP(3);
       for (int i = 0; i < pre; ++i) load_b(i, i);
       int issued = pre;
       for (int i = pre; i < nch; ++i) {
@@ -266,6 +304,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       for (int i = 0; i < nch; ++i) {
         const int s = i % kGemmStages;
         if (!bt_wait(&full[s], (i / kGemmStages) & 1, g.timeout_ns, g.status)) break;
+        if (i == 0) BT_STAMP(4);
         tc_fence_after();
         const uint32_t a_addr = smem_u32(sm + s * kStageBytes);
         const uint64_t ad = sw128_desc(a_addr), bh = sw128_desc(a_addr + kABytes),
@@ -277,51 +316,59 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         }
         tc_commit(smem_u32(&empty[s]));  // stage s is free once these MMAs are done
       }
+      BT_STAMP(5);
       tc_commit(smem_u32(done));
     }
     __syncwarp();
   }
 
-  // ---- accumulator: TMEM lane = tile row (warp w: rows 32w..32w+31), column = sequence
+  // ---- accumulator: TMEM lane = tile row, column = sequence.  Warp w reads
+  // the rows of its sub-partition (w % 4) and the 32 columns of half w / 4.
   bt_wait(done, 0, g.timeout_ns, g.status);
+  if (tid == 0) BT_STAMP(6);
   tc_fence_after();
-  float v[kTileN];
-  const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-#pragma unroll
-  for (int c = 0; c < kTileN; c += 16) tc_ld16(tl + c, v + c);
+  const int quad = warp & 3, hg = warp >> 2;
+  float v[kHalfN];  // v[c]: sequence hg * 32 + c
+  const uint32_t tl =
+      tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(hg * kHalfN);
+  tc_ld16(tl, v);
+  tc_ld16(tl + 16, v + 16);
   tc_wait_ld();
-  const int m = warp * 32 + lane;
+  const int m = quad * 32 + lane;
+  if (tid == 0) BT_STAMP(7);
   pdl_wait();  // everything below reads or writes what earlier kernels use
+  if (tid == 0) BT_STAMP(8);
 
   if constexpr (MODE == kLm) {
     // logits = rsqrt(mean x^2 + eps) * (W (g x)); argmax per sequence
     if (tid < kTileN) s_inv[tid] = rms_scale(g.ssp_in, g.n_ssp, tid, g.H, g.eps);
     __syncthreads();
 #pragma unroll
-    for (int b = 0; b < kTileN; ++b) v[b] *= s_inv[b];
+    for (int c = 0; c < kHalfN; ++c) v[c] *= s_inv[hg * kHalfN + c];
     const int V = g.rows[0];
     const int row = tile * kTileM + m;
     if (g.logits && row < V) {
 #pragma unroll
-      for (int b = 0; b < kTileN; ++b)
-        if (b < g.B) g.logits[static_cast<size_t>(b) * V + row] = v[b];
+      for (int c = 0; c < kHalfN; ++c)
+        if (hg * kHalfN + c < g.B) g.logits[static_cast<size_t>(hg * kHalfN + c) * V + row] = v[c];
     }
     float* T = reinterpret_cast<float*>(sm);  // the (idle) ring: T[b][row]
 #pragma unroll
-    for (int b = 0; b < kTileN; ++b) T[b * kTStride + m] = v[b];
+    for (int c = 0; c < kHalfN; ++c) T[(hg * kHalfN + c) * kTStride + m] = v[c];
     __syncthreads();
-    // thread (b = tid / 2, half = tid % 2) scans rows half*64 .. half*64+63 of sequence b
-    const int b = tid >> 1, half = tid & 1;
+    // thread (b = tid / 4, q = tid % 4) scans rows 32q .. 32q+31 of sequence b
+    const int b = tid >> 2, q = tid & 3;
     float best = -INFINITY;
     int bi = 0x7fffffff;
     if (b < g.B) {
-      const float4* t4 = reinterpret_cast<const float4*>(T + b * kTStride + half * 64);
-      for (int j = 0; j < 16; ++j) {
+      const float4* t4 = reinterpret_cast<const float4*>(T + b * kTStride + q * 32);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
         const float4 x = t4[j];
         const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int id = tile * kTileM + half * 64 + 4 * j + e;
+          const int id = tile * kTileM + q * 32 + 4 * j + e;
           if (id < V && xs[e] > best) {  // ascending ids: strict > keeps the lowest on ties
             best = xs[e];
             bi = id;
@@ -329,106 +376,194 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         }
       }
     }
-    const float ob = __shfl_xor_sync(0xffffffffu, best, 1);
-    const int oi = __shfl_xor_sync(0xffffffffu, bi, 1);
-    if (ob > best || (ob == best && oi < bi)) {
-      best = ob;
-      bi = oi;
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob > best || (ob == best && oi < bi)) {
+        best = ob;
+        bi = oi;
+      }
     }
-    if (half == 0 && b < g.B && bi != 0x7fffffff)
+    if (q == 0 && b < g.B && bi != 0x7fffffff)
       atomicMax(&g.keys[b], (static_cast<unsigned long long>(order_key(best)) << 32) |
                                 static_cast<uint32_t>(~bi));
   } else {
-    // ---- split-K reduction across the cluster, then the phase's epilogue
-    float* T = reinterpret_cast<float*>(sm);
+    // ---- split-K reduction across the cluster, then the phase's epilogue.
+    // CTA `rank` of the cluster finishes sequences b = rank, rank + S, ...
+    // (slot bi = b / S).  Every CTA pushes its partial rows into the owner's
+    // receive rows R[split][bi][row] with remote stores; after one cluster
+    // barrier each owner sums them locally.  Thread (row m, half hg) then
+    // finishes the slots bi = hg, hg + 2, ...
+    const int S = g.splits;
+    const int rank = static_cast<int>(cluster_rank());
+    const int nbmax = (kTileN + S - 1) / S;
+    const int nb = g.B > rank ? (g.B - rank + S - 1) / S : 0;
+    float* R = reinterpret_cast<float*>(sm);                         // [S][nbmax][128]
+    float* W = reinterpret_cast<float*>(sm + kWOffset);              // [nb][128]
+    // R overlays the operand ring: wait until every CTA of the cluster is
+    // past its MMAs before writing into another CTA's ring
+    cluster_arrive();
+    if (tid < kTileN) {
+      if constexpr (MODE != kResid) s_inv[tid] = tid < g.B ? rms_scale(g.ssp_in, g.n_ssp, tid, g.H, g.eps) : 0.f;
+      if constexpr (MODE == kQKV) s_pos[tid] = tid < g.B ? g.pos[tid] : 0;
+    }
+    const bool bad = MODE == kQKV ? (*g.bad != 0) : false;
+    cluster_wait();
+    const uint32_t r_addr = smem_u32(R) + 4u * static_cast<uint32_t>(rank * nbmax * kTileM + m);
+    {
+      int dst = (hg * kHalfN) % S, slot = (hg * kHalfN) / S;  // owner and slot of sequence b
 #pragma unroll
-    for (int b = 0; b < kTileN; ++b) T[b * kTStride + m] = v[b];
-    cluster_sync();  // every split's tile is in its CTA's shared memory
-    const uint32_t S = static_cast<uint32_t>(g.splits);
-    const uint32_t rank = cluster_rank();
-    const uint32_t t_addr = smem_u32(T);
-    const int D = g.D;
-    for (int b = static_cast<int>(rank); b < g.B; b += static_cast<int>(S)) {
-      float val = 0.f;
-      for (uint32_t s = 0; s < S; ++s)  // fixed order: deterministic
-        val += ld_dsmem(map_rank(t_addr + 4u * static_cast<uint32_t>(b * kTStride + m), s));
-      if constexpr (MODE == kQKV) {
-        const int row = tile * kTileM + m;  // row within q, k or v
-        const int head = row / D, d = row - head * D;
-        val *= rms_scale(g.ssp_in, g.n_ssp, b, g.H, g.eps);
-        const int p = g.pos[b];
-        if (mat < 2) {
-          // RMSNorm over the head (D / 32 warps), gain, rotate pairs (i, i + D/2)
-          const float ss = warp_sum(val * val);
-          if (lane == 0) s_red[warp] = ss;
-          __syncthreads();
-          const int wh = (m / D) * (D / 32);
-          float hs = 0.f;
-          for (int w = 0; w < D / 32; ++w) hs += s_red[wh + w];
-          const uint16_t* gn = mat == 0 ? g.gain : g.gain2;
-          val = val * rsqrtf(hs / static_cast<float>(D) + g.eps) * bf16_to_f(gn[d]);
-          s_e[m] = val;
-          __syncthreads();
-          const int half = D / 2;
-          const int i = d < half ? d : d - half;
-          const float partner = s_e[m ^ half];
-          const float ang = __fmul_rn(static_cast<float>(p), g.inv_freq[i]);
-          float sn, cs;
-          rope_sincos(ang, &sn, &cs);
-          val = d < half ? val * cs - partner * sn : val * cs + partner * sn;
+      for (int c = 0; c < kHalfN; ++c) {
+        if (hg * kHalfN + c < g.B)
+          st_dsmem(map_rank(r_addr + 4u * static_cast<uint32_t>(slot * kTileM),
+                            static_cast<uint32_t>(dst)),
+                   v[c]);
+        if (++dst == S) {
+          dst = 0;
+          ++slot;
         }
-        if (mat == 0) {
-          g.q[(static_cast<size_t>(b) * g.Hq + head) * D + d] = val;
-        } else if (!*g.bad) {  // an invalid step leaves the cache unchanged
-          const int kvsel = mat - 1;
-          const size_t plane =
-              ((static_cast<size_t>(g.layer) * 2 + kvsel) * g.kv_batch + b) * g.Hkv + head;
-          const size_t crow = plane * g.max_ctx + p;
-          if (!g.kv_fp8) {
-            reinterpret_cast<uint16_t*>(g.kv)[crow * D + d] = f_to_bf16(val);
-          } else {
-            // E4M3 with one fp32 scale per row: scale = max(amax, 2^-126) / 448
-            const float am = warp_max(fabsf(val));
-            __syncthreads();  // s_red may still hold the norm sums
-            if (lane == 0) s_red[warp] = am;
-            __syncthreads();
-            const int wh = (m / D) * (D / 32);
-            float hm = 0.f;
-            for (int w = 0; w < D / 32; ++w) hm = fmaxf(hm, s_red[wh + w]);
-            hm = fmaxf(hm, 1.17549435e-38f);
-            const float sc = __fdiv_rn(hm, 448.0f);
-            g.kv[crow * D + d] =
-                static_cast<uint8_t>(f2_to_e4m3x2(__fdiv_rn(val, sc), 0.f) & 0xFF);
-            if (d == 0) g.kv_scales[crow] = sc;
-          }
+      }
+    }
+    cluster_sync();  // every split's rows have arrived
+    if (tid == 0) BT_STAMP(9);
+#pragma unroll 2
+    for (int bi = hg; bi < nb; bi += 2) {
+      float acc = 0.f;
+      for (int sp = 0; sp < S; ++sp) acc += R[(sp * nbmax + bi) * kTileM + m];  // fixed order
+      W[bi * kTileM + m] = acc;
+    }
+    if (tid == 0) BT_STAMP(10);
+    const int row = tile * kTileM + m;  // row within the (first) matrix of this tile
+    if constexpr (MODE == kQKV) {
+      const int D = g.D, half = D / 2;
+      const int head = row / D, d = row - head * D;
+      const int wh = hg * 4 + (m / D) * (D / 32);  // first warp of this thread's head
+#pragma unroll 4
+      for (int bi = hg; bi < nb; bi += 2) W[bi * kTileM + m] *= s_inv[rank + S * bi];
+      if (mat < 2) {
+        // RMSNorm over the head (D / 32 warps of this half) and gain
+#pragma unroll 4
+        for (int bi = hg; bi < nb; bi += 2) {
+          const float x = W[bi * kTileM + m];
+          const float ss = warp_sum(x * x);
+          if (lane == 0) s_red[warp][bi] = ss;
         }
-        __syncthreads();  // s_red / s_e are reused by the next sequence
-      } else if constexpr (MODE == kResid) {
-        const int row = tile * kTileM + m;
-        float sq = 0.f;
-        if (row < mrows) {
-          float* xp = g.x + static_cast<size_t>(b) * g.H + row;
-          const float xn = *xp + val;
-          *xp = xn;
-          if (g.hidden) g.hidden[static_cast<size_t>(b) * g.H + row] = xn;
-          put_act(g.act, b, row, g.H, xn * bf16_to_f(g.gain[row]));
-          sq = xn * xn;
-        }
-        const float ss = block_sum(sq, s_red);
-        if (tid == 0) g.ssp_out[tile * kTileN + b] = ss;
-      } else {  // kSwiGLU: rows 0..63 gate, 64..127 up, of columns tile*64 ..
-        val *= rms_scale(g.ssp_in, g.n_ssp, b, g.H, g.eps);
-        s_e[m] = val;
         __syncthreads();
-        const int n = tile * (kTileM / 2) + m;
-        if (m < kTileM / 2 && n < g.F) {
-          const float up = s_e[m + kTileM / 2];
-          put_act(g.act, b, n, g.F, val / (1.0f + __expf(-val)) * up);
+        const float gn = row_gain;
+#pragma unroll 4
+        for (int bi = hg; bi < nb; bi += 2) {
+          float hs = 0.f;
+          for (int w = 0; w < D / 32; ++w) hs += s_red[wh + w][bi];
+          W[bi * kTileM + m] *= rsqrtf(hs / static_cast<float>(D) + g.eps) * gn;
         }
         __syncthreads();
       }
+      // the rotated (q, k) or plain (v) value of slot bi
+      const float invf = row_invf;
+      auto value = [&](int bi) {
+        const float x = W[bi * kTileM + m];
+        if (mat == 2) return x;
+        const float partner = W[bi * kTileM + (m ^ half)];
+        const float ang = __fmul_rn(static_cast<float>(s_pos[rank + S * bi]), invf);
+        float sn, cs;
+        rope_sincos(ang, &sn, &cs);
+        return d < half ? x * cs - partner * sn : x * cs + partner * sn;
+      };
+      if (mat == 0) {
+#pragma unroll 4
+        for (int bi = hg; bi < nb; bi += 2) {
+          const int b = rank + S * bi;
+          g.q[(static_cast<size_t>(b) * g.Hq + head) * D + d] = value(bi);
+        }
+      } else if (!bad) {  // an invalid step leaves the cache unchanged
+        const int kvsel = mat - 1;
+        auto crow_of = [&](int b) {
+          const size_t plane =
+              ((static_cast<size_t>(g.layer) * 2 + kvsel) * g.kv_batch + b) * g.Hkv + head;
+          return plane * g.max_ctx + s_pos[b];
+        };
+        if (!g.kv_fp8) {
+#pragma unroll 4
+          for (int bi = hg; bi < nb; bi += 2) {
+            const int b = rank + S * bi;
+            reinterpret_cast<uint16_t*>(g.kv)[crow_of(b) * D + d] = f_to_bf16(value(bi));
+          }
+        } else {
+          // E4M3 with one fp32 scale per row: scale = max(amax, 2^-126) / 448
+#pragma unroll 4
+          for (int bi = hg; bi < nb; bi += 2) {
+            const float am = warp_max(fabsf(value(bi)));
+            if (lane == 0) s_red[warp][bi] = am;
+          }
+          __syncthreads();
+#pragma unroll 4
+          for (int bi = hg; bi < nb; bi += 2) {
+            const int b = rank + S * bi;
+            float hm = 0.f;
+            for (int w = 0; w < D / 32; ++w) hm = fmaxf(hm, s_red[wh + w][bi]);
+            hm = fmaxf(hm, 1.17549435e-38f);
+            const float sc = __fdiv_rn(hm, 448.0f);
+            const size_t cr = crow_of(b);
+            g.kv[cr * D + d] =
+                static_cast<uint8_t>(f2_to_e4m3x2(__fdiv_rn(value(bi), sc), 0.f) & 0xFF);
+            if (d == 0) g.kv_scales[cr] = sc;
+          }
+        }
+      }
+    } else if constexpr (MODE == kResid) {
+      const bool ok = row < mrows;
+      const float gn = row_gain;
+      for (int bi0 = hg; bi0 < nb; bi0 += 16) {
+        // the residual loads of the batch before any store (the stores may alias)
+        float xv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          xv[j] = (ok && bi0 + 2 * j < nb)
+                      ? g.x[static_cast<size_t>(rank + S * (bi0 + 2 * j)) * g.H + row] +
+                            W[(bi0 + 2 * j) * kTileM + m]
+                      : 0.f;
+        float sq[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          sq[j] = xv[j] * xv[j];
+          if (ok && bi0 + 2 * j < nb) {
+            const int b = rank + S * (bi0 + 2 * j);
+            g.x[static_cast<size_t>(b) * g.H + row] = xv[j];
+            if (g.hidden) g.hidden[static_cast<size_t>(b) * g.H + row] = xv[j];
+            put_act(g.act, b, row, g.H, xv[j] * gn);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sq[j] += __shfl_xor_sync(0xffffffffu, sq[j], o);
+        if (lane == 0) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (bi0 + 2 * j < nb) s_red[warp][bi0 + 2 * j] = sq[j];
+        }
+      }
+      __syncthreads();
+      if (tid < nb) {
+        const int w0 = (tid & 1) * 4;  // the half that finished slot tid
+        g.ssp_out[tile * kTileN + rank + S * tid] =
+            s_red[w0][tid] + s_red[w0 + 1][tid] + s_red[w0 + 2][tid] + s_red[w0 + 3][tid];
+      }
+    } else {  // kSwiGLU: rows 0..63 gate, 64..127 up, of columns tile*64 ..
+#pragma unroll 4
+      for (int bi = hg; bi < nb; bi += 2) W[bi * kTileM + m] *= s_inv[rank + S * bi];
+      __syncthreads();
+      const int n = tile * (kTileM / 2) + m;
+      if (m < kTileM / 2 && n < g.F) {
+#pragma unroll 4
+        for (int bi = hg; bi < nb; bi += 2) {
+          const float gt = W[bi * kTileM + m], up = W[bi * kTileM + m + kTileM / 2];
+          put_act(g.act, rank + S * bi, n, g.F, gt / (1.0f + __expf(-gt)) * up);
+        }
+      }
     }
-    cluster_sync();  // no CTA leaves while another may still read its tile
+    if (tid == 0) BT_STAMP(11);
   }
   tc_fence_before();
   __syncthreads();
@@ -436,6 +571,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  if (tid == 0) BT_STAMP(13);
 }
 
 // ================================================================ small kernels
@@ -560,8 +696,8 @@ __device__ __forceinline__ void load_kv_row(const uint8_t* kp, const uint8_t* vp
   }
 }
 
-template <int D, bool FP8>
-__global__ void __launch_bounds__(kAttThreads) attn_kernel(const AttnArgs2 a) {
+template <int D, bool FP8, int REP>
+__global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const AttnArgs2 a) {
   constexpr int DL = D / 32;
   constexpr int E = FP8 ? 1 : 2;                      // bytes per element
   constexpr int kHalf = kAttTileRows * D * E;          // K (or V) rows of one tile
@@ -575,7 +711,7 @@ __global__ void __launch_bounds__(kAttThreads) attn_kernel(const AttnArgs2 a) {
   if (threadIdx.x == 0) pdl_trigger();
   pdl_wait();
   if (*a.bad) return;
-  const int rep = a.Hq / a.Hkv;
+  constexpr int rep = REP;  // query heads per KV head
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ci = blockIdx.x % a.chunks;
   const int bg = blockIdx.x / a.chunks;
@@ -613,17 +749,15 @@ __global__ void __launch_bounds__(kAttThreads) attn_kernel(const AttnArgs2 a) {
     for (int t = 0; t < ntiles && t < kAttStages; ++t) issue(t);
 
   const float qscale = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-  float qv[kAttMaxRep][DL], acc[kAttMaxRep][DL], m[kAttMaxRep], ls[kAttMaxRep];
+  float qv[REP][DL], acc[REP][DL], m[REP], ls[REP];
 #pragma unroll
-  for (int h = 0; h < kAttMaxRep; ++h) {
+  for (int h = 0; h < REP; ++h) {
     m[h] = -INFINITY;
     ls[h] = 0.f;
 #pragma unroll
     for (int k = 0; k < DL; ++k) {
       acc[h][k] = 0.f;
-      qv[h][k] = h < rep ? a.q[(static_cast<size_t>(b) * a.Hq + g * rep + h) * D + lane * DL + k] *
-                               qscale
-                         : 0.f;
+      qv[h][k] = a.q[(static_cast<size_t>(b) * a.Hq + g * rep + h) * D + lane * DL + k] * qscale;
     }
   }
   for (int t = 0; t < ntiles; ++t) {
@@ -647,8 +781,8 @@ __global__ void __launch_bounds__(kAttThreads) attn_kernel(const AttnArgs2 a) {
                           tb + kHalf + static_cast<size_t>(rr) * D * E + lane * DL * E,
                           FP8 ? ksc[j + rr] : 1.f, FP8 ? vsc[j + rr] : 1.f, k2, v2);
 #pragma unroll
-      for (int h = 0; h < kAttMaxRep; ++h) {
-        if (h < rep) {
+      for (int h = 0; h < REP; ++h) {
+        {
           float s1 = 0.f, s2 = 0.f;
 #pragma unroll
           for (int k = 0; k < DL; ++k) {
@@ -673,8 +807,8 @@ __global__ void __launch_bounds__(kAttThreads) attn_kernel(const AttnArgs2 a) {
   }
   // merge the warps -> this chunk's partial (m in log2 units, l, unnormalised acc)
 #pragma unroll
-  for (int h = 0; h < kAttMaxRep; ++h) {
-    if (h < rep) {
+  for (int h = 0; h < REP; ++h) {
+    {
       float* mg = merge + (static_cast<size_t>(warp) * rep + h) * (D + 2);
 #pragma unroll
       for (int k = 0; k < DL; ++k) mg[lane * DL + k] = acc[h][k];
@@ -800,6 +934,7 @@ struct BtPlan {
   unsigned* att_cnt = nullptr;
   unsigned long long* keys = nullptr;
   int* bad = nullptr;
+  unsigned long long* prof = nullptr;  // profiling builds: GEMM phase timestamps
 };
 
 namespace {
@@ -856,14 +991,47 @@ cudaError_t launch_gemm(const GemmPlan& gp, const GemmArgs& g, cudaStream_t st) 
                     static_cast<unsigned>(g.splits), gp.w[0], gp.w[1], gp.w[2], *gp.x, g);
 }
 
-template <int D>
-cudaError_t launch_attn(const AttnArgs2& a, int rep, bool fp8, cudaStream_t st) {
+template <int D, int REP>
+cudaError_t launch_attn_rep(const AttnArgs2& a, bool fp8, cudaStream_t st) {
   const dim3 grid(static_cast<unsigned>(a.B) * a.Hkv * a.chunks);
   if (fp8)
-    return launch_pdl(attn_kernel<D, true>, grid, dim3(kAttThreads), attn_smem(D, rep, true), st,
-                      1u, a);
-  return launch_pdl(attn_kernel<D, false>, grid, dim3(kAttThreads), attn_smem(D, rep, false), st,
-                    1u, a);
+    return launch_pdl(attn_kernel<D, true, REP>, grid, dim3(kAttThreads), attn_smem(D, REP, true),
+                      st, 1u, a);
+  return launch_pdl(attn_kernel<D, false, REP>, grid, dim3(kAttThreads), attn_smem(D, REP, false),
+                    st, 1u, a);
+}
+
+template <int D>
+cudaError_t launch_attn(const AttnArgs2& a, int rep, bool fp8, cudaStream_t st) {
+  switch (rep) {
+    case 1: return launch_attn_rep<D, 1>(a, fp8, st);
+    case 2: return launch_attn_rep<D, 2>(a, fp8, st);
+    case 3: return launch_attn_rep<D, 3>(a, fp8, st);
+    case 4: return launch_attn_rep<D, 4>(a, fp8, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int D, int REP>
+cudaError_t attn_attrs() {
+  const cudaFuncAttribute dyn = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, false, REP>, dyn,
+                                       static_cast<int>(attn_smem(D, REP, false)));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_kernel<D, true, REP>, dyn,
+                             static_cast<int>(attn_smem(D, REP, true)));
+  return e;
+}
+
+template <int D>
+cudaError_t attn_attrs_for(int rep) {
+  switch (rep) {
+    case 1: return attn_attrs<D, 1>();
+    case 2: return attn_attrs<D, 2>();
+    case 3: return attn_attrs<D, 3>();
+    case 4: return attn_attrs<D, 4>();
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
@@ -912,6 +1080,9 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_h
   const size_t ac_off = take(sizeof(unsigned) * kTileN * s.Hkv);
   const size_t keys_off = take(sizeof(unsigned long long) * kTileN);
   const size_t bad_off = take(sizeof(int));
+#ifdef DEC_PROFILE
+  const size_t prof_off = take(sizeof(unsigned long long) * 4 * kProfCtas * 16);
+#endif
   e = cudaMalloc(&p->ws, o);
   if (e == cudaSuccess) e = cudaMemset(p->ws, 0, o);
   if (e != cudaSuccess) {
@@ -930,6 +1101,9 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_h
   p->att_cnt = reinterpret_cast<unsigned*>(p->ws + ac_off);
   p->keys = reinterpret_cast<unsigned long long*>(p->ws + keys_off);
   p->bad = reinterpret_cast<int*>(p->ws + bad_off);
+#ifdef DEC_PROFILE
+  p->prof = reinterpret_cast<unsigned long long*>(p->ws + prof_off);
+#endif
 
   // ---- tensor maps and GEMM plans
   bool ok = encode_map(enc, &p->map_h, p->act_h, s.H, kBRows, kBRows) &&
@@ -966,21 +1140,7 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_h
   if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kSwiGLU>, dyn, smem);
   if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kLm>, dyn, smem);
   const int rep = s.Hq / s.Hkv;
-  if (ok && e == cudaSuccess) {
-    if (s.D == 128) {
-      e = cudaFuncSetAttribute(attn_kernel<128, false>, dyn,
-                               static_cast<int>(attn_smem(128, rep, false)));
-      if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(attn_kernel<128, true>, dyn,
-                                 static_cast<int>(attn_smem(128, rep, true)));
-    } else {
-      e = cudaFuncSetAttribute(attn_kernel<64, false>, dyn,
-                               static_cast<int>(attn_smem(64, rep, false)));
-      if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(attn_kernel<64, true>, dyn,
-                                 static_cast<int>(attn_smem(64, rep, true)));
-    }
-  }
+  if (ok && e == cudaSuccess) e = s.D == 128 ? attn_attrs_for<128>(rep) : attn_attrs_for<64>(rep);
   if (!ok || e != cudaSuccess) {
     *cerr = e;
     cudaFree(p->ws);
@@ -1024,6 +1184,7 @@ cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
   base.keys = p->keys;
   base.status = io.status;
   base.timeout_ns = io.timeout_ns;
+  base.prof = p->prof;
   auto args_of = [&](const GemmPlan& gp) {
     GemmArgs g = base;
     g.n_mat = gp.args.n_mat;
@@ -1113,3 +1274,17 @@ cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
 }
 
 }  // namespace dec
+
+#ifdef DEC_PROFILE
+namespace dec {
+// Profiling builds: the GEMM phase timestamps of the last launch of each mode.
+int bt_prof_read(BtPlan* p, unsigned long long* host, size_t n) {
+  const size_t need = 4ull * kProfCtas * 16;
+  if (!p || !p->prof || n < need) return -1;
+  return cudaMemcpy(host, p->prof, need * sizeof(unsigned long long), cudaMemcpyDeviceToHost) ==
+                 cudaSuccess
+             ? 0
+             : -1;
+}
+}  // namespace dec
+#endif

@@ -354,7 +354,7 @@ struct Cta {
     auto acquire = [&](uint32_t bytes) -> uint8_t* {
       if (lap > 0) {
         Spin sp;
-        while (!mbar_wait(&empty[ps], (lap - 1) & 1, 20000)) {
+        while (!mbar_wait(&empty[ps], (lap - 1) & 1, kWaitHintNs)) {
           if (sp.tick(a, false)) {
             dead = true;
             return nullptr;
@@ -500,7 +500,7 @@ struct Cta {
     int st = 1;
     if (lane == 0) {
       Spin sp;
-      while (!mbar_wait(&full[slot], par, 20000)) {
+      while (!mbar_wait(&full[slot], par, kWaitHintNs)) {
         if (sp.tick(a, false)) {
           st = 0;
           break;
