@@ -92,7 +92,13 @@ typedef struct dec_shape {
   int vocab;
   float rms_eps;     /* 1e-6 */
   float rope_theta;  /* 1e6 */
-  int max_batch;     /* largest batch dec_step will be called with */
+  int max_batch;     /* largest batch dec_step will be called with, 1..64.
+                      * Batches of 1..4 run the single persistent kernel; a
+                      * handle with max_batch > 4 also plans the batched
+                      * (tensor-core) step for batches of 5..max_batch, which
+                      * needs n_q_heads*head_dim and n_kv_heads*head_dim to be
+                      * multiples of 128, ffn a multiple of 64 and at most 4
+                      * query heads per KV head (else DEC_ERR_SHAPE) */
 } dec_shape;
 
 /* Order of the per-layer weight pointers in dec_weights.layers. */
@@ -180,7 +186,10 @@ int dec_kv_alloc(dec_handle *h, int batch, int max_ctx, int dtype, void *buf,
  *   out_ids    int32 [batch]  argmax token of every sequence; may alias
  *                             token_ids (self-feeding decode).
  *   out_logits fp32 [batch, vocab] or NULL.
- * One kernel launch on `stream`; never synchronises.  Invalid positions or
+ * Asynchronous on `stream`; never synchronises.  Batches of 1..4: one
+ * kernel launch.  Batches of 5..64: 5 launches per layer + 3 (programmatic
+ * dependent launches, so the caller's stream must not be shared with work
+ * that expects the step to be a single kernel).  Invalid positions or
  * tokens are detected on the device: the step then writes -1 to out_ids,
  * leaves the cache unchanged and raises a bit that dec_check() returns. */
 int dec_step(dec_handle *h, int batch, const int32_t *token_ids, const int32_t *positions,
