@@ -74,7 +74,7 @@ constexpr int kMaxAttnChunks = 32;
 constexpr int kAttWarps = 8;
 constexpr int kAttThreads = kAttWarps * 32;
 constexpr int kAttStages = 4;
-constexpr int kAttTileRows = 32;
+constexpr int kAttTileRows = 32;                // = kAttWarps x 4 rows (lane octets)
 constexpr int kAttMaxRep = 4;  // query heads per KV head (attention template)
 constexpr int kRowThreads = 256;
 constexpr int kProfCtas = 2048;                   // GEMM CTAs with timestamps (profiling builds)
@@ -82,6 +82,7 @@ constexpr int kProfCtas = 2048;                   // GEMM CTAs with timestamps (
 enum GemmMode { kQKV = 0, kResid = 1, kSwiGLU = 2, kLm = 3 };
 
 static_assert(kTileN == 64 && kTmemCols == 64, "epilogue reads 4 x 16 accumulator columns");
+static_assert(kAttWarps * 4 == kAttTileRows, "a tile is one row per octet");
 static_assert(kTileN * kTStride * 4 <= kWOffset, "accumulator tile below the reduced rows");
 static_assert((kTileN + kMaxSplits) * kTileM * 4 <= kWOffset, "split receive rows below them");
 static_assert(kWOffset + kTileN * kTileM * 4 <= kGemmStages * kStageBytes, "both fit the ring");
@@ -644,10 +645,14 @@ __global__ void finish_kernel(const StepArgs2 a) {
 // ================================================================ attention
 // Split-K GQA decode attention over the step's cache: CTA = (sequence b, KV
 // head g, chunk of chunk_rows rows of 0..p_b).  K and V rows of 32-row tiles
-// arrive by 1-D bulk copies into a 4-stage ring; each warp takes two rows at
-// a time (two independent dot-product chains) and keeps an fp32 online
-// softmax (base-2 exponent) per query head of the group; the last CTA of
-// (b, g) merges the chunks and writes the o_proj operand planes.
+// arrive by 1-D bulk copies into a ring.  Lane octets: each warp takes 4 rows
+// of a tile at once, 8 lanes per row; lane o of an octet holds elements
+// [o*D/16, (o+1)*D/16) and the same span of the second half of the row (so
+// the 8 lanes of a row read 8 consecutive 16-byte pieces: no bank conflicts),
+// a dot product is 3 shuffles, and every octet keeps its own fp32 online
+// softmax (base-2 exponent) per query head.  The octets and warps merge at
+// the end; a CTA that holds the whole context writes the o_proj operand
+// planes, otherwise the last chunk CTA of (b, g) merges the chunks.
 struct AttnArgs2 {
   int B, Hq, Hkv, max_ctx, kv_batch, l;
   const uint8_t* kv;
@@ -661,58 +666,61 @@ struct AttnArgs2 {
   int chunk_rows, chunks;
 };
 
-__device__ __forceinline__ void warp_sum2(float& a, float& b) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    a += __shfl_xor_sync(0xffffffffu, a, o);
-    b += __shfl_xor_sync(0xffffffffu, b, o);
-  }
-}
-
+// Elements [i*HALF, i*HALF + HALF) (i = 0, 1) of this lane's two spans of a
+// K or V row as fp32: bf16 values, or E4M3 code values (the caller applies
+// the row scale once per row).
 template <int D, bool FP8>
-__device__ __forceinline__ void load_kv_row(const uint8_t* kp, const uint8_t* vp, float ks,
-                                            float vs, float (&kr)[D / 32], float (&vr)[D / 32]) {
-  constexpr int DL = D / 32;
+__device__ __forceinline__ void load_span(const uint8_t* row, int o, int i, float (&x)[D / 16]) {
+  constexpr int HALF = D / 16;
+  const int e0 = i * (D / 2) + o * HALF;
   if constexpr (!FP8) {
-    if constexpr (DL == 4) {
-      const uint2 kw = *reinterpret_cast<const uint2*>(kp);
-      const uint2 vw = *reinterpret_cast<const uint2*>(vp);
-      kr[0] = bf16lo(kw.x); kr[1] = bf16hi(kw.x); kr[2] = bf16lo(kw.y); kr[3] = bf16hi(kw.y);
-      vr[0] = bf16lo(vw.x); vr[1] = bf16hi(vw.x); vr[2] = bf16lo(vw.y); vr[3] = bf16hi(vw.y);
+    if constexpr (HALF == 8) {
+      const uint4 w = *reinterpret_cast<const uint4*>(row + 2 * e0);
+      x[0] = bf16lo(w.x); x[1] = bf16hi(w.x); x[2] = bf16lo(w.y); x[3] = bf16hi(w.y);
+      x[4] = bf16lo(w.z); x[5] = bf16hi(w.z); x[6] = bf16lo(w.w); x[7] = bf16hi(w.w);
     } else {
-      const uint32_t kw = *reinterpret_cast<const uint32_t*>(kp);
-      const uint32_t vw = *reinterpret_cast<const uint32_t*>(vp);
-      kr[0] = bf16lo(kw); kr[1] = bf16hi(kw);
-      vr[0] = bf16lo(vw); vr[1] = bf16hi(vw);
+      const uint2 w = *reinterpret_cast<const uint2*>(row + 2 * e0);
+      x[0] = bf16lo(w.x); x[1] = bf16hi(w.x); x[2] = bf16lo(w.y); x[3] = bf16hi(w.y);
     }
   } else {
+    if constexpr (HALF == 8) {
+      const uint2 w = *reinterpret_cast<const uint2*>(row + e0);
+      const uint32_t ws[2] = {w.x, w.y};
 #pragma unroll
-    for (int k = 0; k < DL; k += 2) {
-      const float2 kf = e4m3x2_to_f2(*reinterpret_cast<const uint16_t*>(kp + k));
-      const float2 vf = e4m3x2_to_f2(*reinterpret_cast<const uint16_t*>(vp + k));
-      kr[k] = kf.x * ks; kr[k + 1] = kf.y * ks;
-      vr[k] = vf.x * vs; vr[k + 1] = vf.y * vs;
+      for (int j = 0; j < 2; ++j) {
+        const float2 a0 = e4m3x2_to_f2(static_cast<uint16_t>(ws[j] & 0xFFFF));
+        const float2 a1 = e4m3x2_to_f2(static_cast<uint16_t>(ws[j] >> 16));
+        x[4 * j + 0] = a0.x; x[4 * j + 1] = a0.y;
+        x[4 * j + 2] = a1.x; x[4 * j + 3] = a1.y;
+      }
+    } else {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(row + e0);
+      const float2 a0 = e4m3x2_to_f2(static_cast<uint16_t>(w & 0xFFFF));
+      const float2 a1 = e4m3x2_to_f2(static_cast<uint16_t>(w >> 16));
+      x[0] = a0.x; x[1] = a0.y; x[2] = a1.x; x[3] = a1.y;
     }
   }
 }
 
 template <int D, bool FP8, int REP>
 __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const AttnArgs2 a) {
-  constexpr int DL = D / 32;
   constexpr int E = FP8 ? 1 : 2;                      // bytes per element
-  constexpr int kHalf = kAttTileRows * D * E;          // K (or V) rows of one tile
-  constexpr int kTile = 2 * kHalf;
+  constexpr int HALF = D / 16;                        // elements per span
+  constexpr int RB = D * E;                           // bytes per row
+  constexpr int kHalf = kAttTileRows * RB;            // K (or V) rows of one tile
+  // a tile: K rows, V rows, then (E4M3) the K and V row scales
+  constexpr int kTile = 2 * kHalf + (FP8 ? 2 * kAttTileRows * 4 : 0);
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kAttStages * kTile);
-  float* merge = reinterpret_cast<float*>(full + kAttStages);  // [warps][rep][D + 2]
+  float* merge = reinterpret_cast<float*>(full + kAttStages);  // [warps][REP][D + 2]
   __shared__ int s_last;
 
   if (threadIdx.x == 0) pdl_trigger();
   pdl_wait();
   if (*a.bad) return;
-  constexpr int rep = REP;  // query heads per KV head
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int oct = lane >> 3, o = lane & 7;            // row of the warp's 4, lane in the octet
   const int ci = blockIdx.x % a.chunks;
   const int bg = blockIdx.x / a.chunks;
   const int b = bg / a.Hkv, g = bg % a.Hkv;
@@ -724,8 +732,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const AttnArgs2 a)
   const int ntiles = (j1 - j0 + kAttTileRows - 1) / kAttTileRows;
   const size_t kplane = ((static_cast<size_t>(a.l) * 2 + 0) * a.kv_batch + b) * a.Hkv + g;
   const size_t vplane = ((static_cast<size_t>(a.l) * 2 + 1) * a.kv_batch + b) * a.Hkv + g;
-  const uint8_t* kbase = a.kv + kplane * a.max_ctx * D * E;
-  const uint8_t* vbase = a.kv + vplane * a.max_ctx * D * E;
+  const uint8_t* kbase = a.kv + kplane * a.max_ctx * RB;
+  const uint8_t* vbase = a.kv + vplane * a.max_ctx * RB;
   const float* ksc = FP8 ? a.kv_scales + kplane * a.max_ctx : nullptr;
   const float* vsc = FP8 ? a.kv_scales + vplane * a.max_ctx : nullptr;
 
@@ -738,27 +746,38 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const AttnArgs2 a)
   auto issue = [&](int t) {
     const int j = j0 + t * kAttTileRows;
     const int nr = min(kAttTileRows, j1 - j);
-    const uint32_t rb = static_cast<uint32_t>(nr) * D * E;
+    const uint32_t rb = static_cast<uint32_t>(nr) * RB;
     uint64_t* bar = &full[t % kAttStages];
     uint8_t* dst = ring + (t % kAttStages) * kTile;
-    mbar_arrive_expect_tx(bar, 2 * rb);
-    bulk_g2s(dst, kbase + static_cast<size_t>(j) * D * E, rb, bar, pol);
-    bulk_g2s(dst + kHalf, vbase + static_cast<size_t>(j) * D * E, rb, bar, pol);
+    // scales: rows j .. j + nr rounded up to 4 (16 bytes; stays inside max_ctx,
+    // a multiple of 16, since j is a multiple of 32)
+    const uint32_t sb = FP8 ? static_cast<uint32_t>((nr + 3) & ~3) * 4u : 0u;
+    mbar_arrive_expect_tx(bar, 2 * rb + 2 * sb);
+    bulk_g2s(dst, kbase + static_cast<size_t>(j) * RB, rb, bar, pol);
+    bulk_g2s(dst + kHalf, vbase + static_cast<size_t>(j) * RB, rb, bar, pol);
+    if (FP8) {
+      bulk_g2s(dst + 2 * kHalf, ksc + j, sb, bar, pol);
+      bulk_g2s(dst + 2 * kHalf + kAttTileRows * 4, vsc + j, sb, bar, pol);
+    }
   };
   if (tid == 0)
     for (int t = 0; t < ntiles && t < kAttStages; ++t) issue(t);
 
+  // this lane's elements of the query heads of the group, scaled to base 2
   const float qscale = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-  float qv[REP][DL], acc[REP][DL], m[REP], ls[REP];
+  float qv[REP][2][HALF], acc[REP][2][HALF], m[REP], ls[REP];
 #pragma unroll
   for (int h = 0; h < REP; ++h) {
     m[h] = -INFINITY;
     ls[h] = 0.f;
+    const float* qh = a.q + (static_cast<size_t>(b) * a.Hq + g * REP + h) * D;
 #pragma unroll
-    for (int k = 0; k < DL; ++k) {
-      acc[h][k] = 0.f;
-      qv[h][k] = a.q[(static_cast<size_t>(b) * a.Hq + g * rep + h) * D + lane * DL + k] * qscale;
-    }
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int e = 0; e < HALF; ++e) {
+        acc[h][i][e] = 0.f;
+        qv[h][i][e] = qh[i * (D / 2) + o * HALF + e] * qscale;
+      }
   }
   for (int t = 0; t < ntiles; ++t) {
     const int j = j0 + t * kAttTileRows;
@@ -769,74 +788,126 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const AttnArgs2 a)
         if (sp.expired()) break;
     }
     const uint8_t* tb = ring + (t % kAttStages) * kTile;
-    for (int r = warp; r < nr; r += 2 * kAttWarps) {
-      const int r2 = r + kAttWarps;
-      const bool two = r2 < nr;  // warp-uniform
-      const int rr = two ? r2 : r;
-      float k1[DL], v1[DL], k2[DL], v2[DL];
-      load_kv_row<D, FP8>(tb + static_cast<size_t>(r) * D * E + lane * DL * E,
-                          tb + kHalf + static_cast<size_t>(r) * D * E + lane * DL * E,
-                          FP8 ? ksc[j + r] : 1.f, FP8 ? vsc[j + r] : 1.f, k1, v1);
-      load_kv_row<D, FP8>(tb + static_cast<size_t>(rr) * D * E + lane * DL * E,
-                          tb + kHalf + static_cast<size_t>(rr) * D * E + lane * DL * E,
-                          FP8 ? ksc[j + rr] : 1.f, FP8 ? vsc[j + rr] : 1.f, k2, v2);
+    // 8 warps x 4 rows = the 32 rows of a tile; every lane takes part in the
+    // shuffles, rows past nr are masked out of the softmax
+    const int r = warp * 4 + oct;
+    const bool valid = r < nr;
+    const int rr = valid ? r : 0;
+    const uint8_t* krow = tb + static_cast<size_t>(rr) * RB;
+    const uint8_t* vrow = krow + kHalf;
+    const float* tsc = reinterpret_cast<const float*>(tb + 2 * kHalf);
+    const float ks = FP8 ? tsc[rr] : 1.f;
+    float s[REP];
+#pragma unroll
+    for (int h = 0; h < REP; ++h) s[h] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      float kx[HALF];
+      load_span<D, FP8>(krow, o, i, kx);
+#pragma unroll
+      for (int h = 0; h < REP; ++h)
+#pragma unroll
+        for (int e = 0; e < HALF; ++e) s[h] = fmaf(qv[h][i][e], kx[e], s[h]);
+    }
+#pragma unroll
+    for (int sh = 4; sh > 0; sh >>= 1)
+#pragma unroll
+      for (int h = 0; h < REP; ++h) s[h] += __shfl_xor_sync(0xffffffffu, s[h], sh);
+    if (FP8) {
+#pragma unroll
+      for (int h = 0; h < REP; ++h) s[h] *= ks;  // q . (code x scale) = scale x (q . code)
+    }
+    if (valid) {
+      float al[REP], p[REP];
 #pragma unroll
       for (int h = 0; h < REP; ++h) {
-        {
-          float s1 = 0.f, s2 = 0.f;
+        const float mn = fmaxf(m[h], s[h]);
+        al[h] = exp2f(m[h] - mn);
+        p[h] = exp2f(s[h] - mn);
+        ls[h] = ls[h] * al[h] + p[h];
+        m[h] = mn;
+      }
+      if (FP8) {
+        const float vs = tsc[kAttTileRows + rr];
 #pragma unroll
-          for (int k = 0; k < DL; ++k) {
-            s1 = fmaf(qv[h][k], k1[k], s1);
-            s2 = fmaf(qv[h][k], k2[k], s2);
-          }
-          warp_sum2(s1, s2);
-          if (!two) s2 = -INFINITY;
-          const float mn = fmaxf(m[h], fmaxf(s1, s2));
-          const float al = exp2f(m[h] - mn);
-          const float p1 = exp2f(s1 - mn);
-          const float p2 = exp2f(s2 - mn);
-          ls[h] = ls[h] * al + p1 + p2;
+        for (int h = 0; h < REP; ++h) p[h] *= vs;  // p (code x scale) = (p scale) code
+      }
 #pragma unroll
-          for (int k = 0; k < DL; ++k) acc[h][k] = fmaf(acc[h][k], al, fmaf(p1, v1[k], p2 * v2[k]));
-          m[h] = mn;
-        }
+      for (int i = 0; i < 2; ++i) {
+        float vx[HALF];
+        load_span<D, FP8>(vrow, o, i, vx);
+#pragma unroll
+        for (int h = 0; h < REP; ++h)
+#pragma unroll
+          for (int e = 0; e < HALF; ++e) acc[h][i][e] = fmaf(acc[h][i][e], al[h], p[h] * vx[e]);
       }
     }
     __syncthreads();  // slot t % stages fully read
     if (tid == 0 && t + kAttStages < ntiles) issue(t + kAttStages);
   }
-  // merge the warps -> this chunk's partial (m in log2 units, l, unnormalised acc)
+  // merge the four octets of the warp (lanes o, o + 8, o + 16, o + 24 hold
+  // the same elements), then octet 0 writes the warp's state
 #pragma unroll
-  for (int h = 0; h < REP; ++h) {
-    {
-      float* mg = merge + (static_cast<size_t>(warp) * rep + h) * (D + 2);
+  for (int sh = 8; sh <= 16; sh <<= 1) {
 #pragma unroll
-      for (int k = 0; k < DL; ++k) mg[lane * DL + k] = acc[h][k];
-      if (lane == 0) {
+    for (int h = 0; h < REP; ++h) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m[h], sh);
+      const float lo = __shfl_xor_sync(0xffffffffu, ls[h], sh);
+      const float mn = fmaxf(m[h], mo);
+      const float e1 = (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - mn);
+      const float e2 = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+      ls[h] = ls[h] * e1 + lo * e2;
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int e = 0; e < HALF; ++e) {
+          const float ao = __shfl_xor_sync(0xffffffffu, acc[h][i][e], sh);
+          acc[h][i][e] = acc[h][i][e] * e1 + ao * e2;
+        }
+      m[h] = mn;
+    }
+  }
+  if (oct == 0) {
+#pragma unroll
+    for (int h = 0; h < REP; ++h) {
+      float* mg = merge + (static_cast<size_t>(warp) * REP + h) * (D + 2);
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int e = 0; e < HALF; ++e) mg[i * (D / 2) + o * HALF + e] = acc[h][i][e];
+      if (o == 0) {
         mg[D] = m[h];
         mg[D + 1] = ls[h];
       }
     }
   }
   __syncthreads();
-  for (int t = tid; t < rep * D; t += kAttThreads) {
+  const int HqD = a.Hq * D;
+  // merge the warps: thread t -> (head, element)
+  for (int t = tid; t < REP * D; t += kAttThreads) {
     const int h = t / D, d = t % D;
     float M = -INFINITY;
-    for (int w = 0; w < kAttWarps; ++w) M = fmaxf(M, merge[(w * rep + h) * (D + 2) + D]);
+    for (int w = 0; w < kAttWarps; ++w) M = fmaxf(M, merge[(w * REP + h) * (D + 2) + D]);
     float Ls = 0.f, A = 0.f;
     for (int w = 0; w < kAttWarps; ++w) {
-      const float* mg = merge + (w * rep + h) * (D + 2);
+      const float* mg = merge + (w * REP + h) * (D + 2);
       const float e = (mg[D] == -INFINITY) ? 0.f : exp2f(mg[D] - M);
       Ls += mg[D + 1] * e;
       A += mg[d] * e;
     }
-    float* pp = a.part + ((static_cast<size_t>(b) * a.Hq + g * rep + h) * a.chunks + ci) * (D + 2);
-    pp[d] = A;
-    if (d == 0) {
-      pp[D] = M;
-      pp[D + 1] = Ls;
+    if (nchunk == 1) {  // the whole context: this CTA writes the output
+      put_act(a.out, b, (g * REP + h) * D + d, HqD, A / Ls);
+    } else {
+      float* pp =
+          a.part + ((static_cast<size_t>(b) * a.Hq + g * REP + h) * a.chunks + ci) * (D + 2);
+      pp[d] = A;
+      if (d == 0) {
+        pp[D] = M;
+        pp[D + 1] = Ls;
+      }
     }
   }
+  if (nchunk == 1) return;
   __syncthreads();
   if (tid == 0) {
     __threadfence();
@@ -849,10 +920,9 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const AttnArgs2 a)
   }
   __syncthreads();
   if (!s_last) return;
-  const int HqD = a.Hq * D;
-  for (int t = tid; t < rep * D; t += kAttThreads) {
+  for (int t = tid; t < REP * D; t += kAttThreads) {
     const int h = t / D, d = t % D;
-    const float* pb = a.part + (static_cast<size_t>(b) * a.Hq + g * rep + h) * a.chunks * (D + 2);
+    const float* pb = a.part + (static_cast<size_t>(b) * a.Hq + g * REP + h) * a.chunks * (D + 2);
     float M = -INFINITY;
     for (int c = 0; c < nchunk; ++c) M = fmaxf(M, __ldcg(pb + c * (D + 2) + D));
     float Ls = 0.f, A = 0.f;
@@ -861,12 +931,13 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const AttnArgs2 a)
       Ls += __ldcg(pb + c * (D + 2) + D + 1) * e;
       A += __ldcg(pb + c * (D + 2) + d) * e;
     }
-    put_act(a.out, b, (g * rep + h) * D + d, HqD, A / Ls);
+    put_act(a.out, b, (g * REP + h) * D + d, HqD, A / Ls);
   }
 }
 
 size_t attn_smem(int D, int rep, bool fp8) {
-  return static_cast<size_t>(kAttStages) * kAttTileRows * D * (fp8 ? 1 : 2) * 2 +
+  return static_cast<size_t>(kAttStages) * (kAttTileRows * D * (fp8 ? 1 : 2) * 2 +
+                                            (fp8 ? 2 * kAttTileRows * 4 : 0)) +
          kAttStages * sizeof(uint64_t) + static_cast<size_t>(kAttWarps) * rep * (D + 2) * sizeof(float);
 }
 
@@ -1197,12 +1268,14 @@ cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
     return g;
   };
 
-  // attention chunking: about 4 CTAs per SM over the cache capacity, at most
-  // kMaxAttnChunks chunks per (sequence, KV head)
-  int cr = attention_chunk_rows(io.B, s.Hkv, io.max_ctx, p->sms);
-  const int min_cr = ((io.max_ctx + kMaxAttnChunks - 1) / kMaxAttnChunks + kAttTileRows - 1) /
-                     kAttTileRows * kAttTileRows;
-  if (cr < min_cr) cr = min_cr;
+  // attention chunking: one wave of CTAs (2 resident per SM) over the
+  // (sequence, KV head) pairs, i.e. one chunk per pair once there are enough
+  // pairs; at most kMaxAttnChunks chunks per pair
+  int per_pair = (2 * p->sms) / (io.B * s.Hkv);
+  if (per_pair < 1) per_pair = 1;
+  if (per_pair > kMaxAttnChunks) per_pair = kMaxAttnChunks;
+  int cr = (io.max_ctx + per_pair - 1) / per_pair;
+  cr = (cr + kAttTileRows - 1) / kAttTileRows * kAttTileRows;
   AttnArgs2 at{};
   at.B = io.B;
   at.Hq = s.Hq;

@@ -87,8 +87,12 @@ def test_sequences_are_independent_of_the_batch():
         res.append((ids[:7], logits[:7], hid[:, :7],
                     kv.values[:, :, :7].float().cpu().numpy()))
     assert np.array_equal(res[0][0], res[1][0])
-    for a, b in zip(res[0][1:], res[1][1:]):
+    for a, b in zip(res[0][1:3], res[1][1:3]):        # logits, residual stream
         assert np.max(np.abs(a - b)) <= 1e-4
+    # cache rows of layers >= 1 come from attention outputs that differ by
+    # fp32 rounding: their bf16 storage may differ by one unit in the last place
+    ka, kb = res[0][3], res[1][3]
+    assert np.all(np.abs(ka - kb) <= 2.0 ** -7 * np.maximum(np.abs(ka), np.abs(kb)))
     dec.close()
 
 
