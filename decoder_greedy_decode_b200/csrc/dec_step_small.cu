@@ -708,16 +708,29 @@ struct Cta {
   __device__ void gemv(int K, int nrows, int rpt, bool pair, int sc, int l) {
     const int nv = K >> 3;
     const int per = pair ? R / 2 : R;  // output rows per group
+    // A stage of many tiles (lm_head) gives each tile to one warp: only that
+    // warp waits for it, computes all its groups and releases it for the
+    // whole CTA; the other warps only advance their ring position.  The owner
+    // is the ring slot's warp (slot mod warps), so a warp's consecutive tiles
+    // are never more than one ring lap apart and its parity waits stay
+    // unambiguous.  A stage of a few tiles spreads each tile's groups over
+    // the warps.
+    const bool owned = (nrows + rpt - 1) / rpt > 2 * kCW;
     int gbase = 0;
     for (int r0 = 0; r0 < nrows; r0 += rpt) {
       const int nr = min(rpt, nrows - r0);
       const int ng = (nr + per - 1) / per;
-      wait_tile();
-      if (!ab) {
+      const bool mine = !owned || rs % kCW == warp;
+      if (mine) wait_tile();
+      if (mine && !ab) {
         const uint8_t* tb = ring + static_cast<size_t>(rs) * kSlotBytes;
-        int g0 = (warp - gbase) % kCW;
-        if (g0 < 0) g0 += kCW;
-        for (int gl = g0; gl < ng; gl += kCW) {
+        int g0 = 0, gs = 1;
+        if (!owned) {
+          g0 = (warp - gbase) % kCW;
+          if (g0 < 0) g0 += kCW;
+          gs = kCW;
+        }
+        for (int gl = g0; gl < ng; gl += gs) {
           uint32_t rows[R];
 #pragma unroll
           for (int i = 0; i < R; ++i) {
@@ -725,20 +738,30 @@ struct Cta {
             const int trow = (pair && i >= per) ? nr + j : j;
             rows[i] = smem_u32(tb) + static_cast<uint32_t>(j < nr ? trow : 0) * K * 2;
           }
-          const GroupSums<R, B> gs = group_dot<R, B>(rows, smem_u32(act), kmax, nv, lane);
+          const GroupSums<R, B> gs4 = group_dot<R, B>(rows, smem_u32(act), kmax, nv, lane);
           const int ri = R == 4 ? (lane >> 3) : (R == 2 ? (lane >> 4) : 0);
           const bool leader = R == 4 ? ((lane & 7) == 0) : (R == 2 ? ((lane & 15) == 0) : lane == 0);
           const int j = gl * per + ri;
 #pragma unroll
           for (int b = 0; b < B; ++b) {
-            const float sv = gs.s[b];
+            const float sv = gs4.s[b];
             const float su = __shfl_down_sync(0xffffffffu, sv, 16);
             if (leader && (!pair || ri < per) && j < nr && b < a.B) epilogue(sc, l, r0 + j, b, sv, su);
           }
         }
       }
       gbase += ng;
-      release_tile();
+      if (owned) {
+        __syncwarp();
+        if (mine && lane == 0 && !ring_dead) mbar_arrive_cnt(&empty[rs], kCW);
+        ++rn;
+        if (++rs == a.nslot) {
+          rs = 0;
+          rph ^= 1;
+        }
+      } else {
+        release_tile();
+      }
     }
     // the next stage overwrites act: every warp must be done reading it
     csync();
