@@ -321,6 +321,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       tc_commit(smem_u32(done));
     }
     __syncwarp();
+  } else if (tid >= 64 && tid < 64 + kTileN) {
+    // idle during the main loop: the epilogue's per-sequence inputs
+    pdl_wait();
+    const int b = tid - 64;
+    if constexpr (MODE != kResid) s_inv[b] = b < g.B ? rms_scale(g.ssp_in, g.n_ssp, b, g.H, g.eps) : 0.f;
+    if constexpr (MODE == kQKV) s_pos[b] = b < g.B ? g.pos[b] : 0;
   }
 
   // ---- accumulator: TMEM lane = tile row, column = sequence.  Warp w reads
@@ -342,8 +348,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 
   if constexpr (MODE == kLm) {
     // logits = rsqrt(mean x^2 + eps) * (W (g x)); argmax per sequence
-    if (tid < kTileN) s_inv[tid] = rms_scale(g.ssp_in, g.n_ssp, tid, g.H, g.eps);
-    __syncthreads();
+    __syncthreads();  // s_inv
 #pragma unroll
     for (int c = 0; c < kHalfN; ++c) v[c] *= s_inv[hg * kHalfN + c];
     const int V = g.rows[0];
@@ -405,12 +410,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     // R overlays the operand ring: wait until every CTA of the cluster is
     // past its MMAs before writing into another CTA's ring
     cluster_arrive();
-    if (tid < kTileN) {
-      if constexpr (MODE != kResid) s_inv[tid] = tid < g.B ? rms_scale(g.ssp_in, g.n_ssp, tid, g.H, g.eps) : 0.f;
-      if constexpr (MODE == kQKV) s_pos[tid] = tid < g.B ? g.pos[tid] : 0;
-    }
     const bool bad = MODE == kQKV ? (*g.bad != 0) : false;
-    cluster_wait();
+    cluster_wait();  // also orders s_inv / s_pos (written before the MMAs finished)
     const uint32_t r_addr = smem_u32(R) + 4u * static_cast<uint32_t>(rank * nbmax * kTileM + m);
     {
       int dst = (hg * kHalfN) % S, slot = (hg * kHalfN) / S;  // owner and slot of sequence b

@@ -565,8 +565,7 @@ struct Cta {
         } else if (ld_relaxed_i32(a.abort_flag)) {
           fail = 1;
         }
-        if (fail) pend = 0;
-        else __nanosleep(64);
+        if (fail) pend = 0;  // else re-poll at once: a hop costs one L2 round trip
       }
       more = named_sync_or(1, kCT, pend != 0);
     } while (more);
