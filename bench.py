@@ -215,6 +215,63 @@ def run_bs64(s, wd, dev, ws, seed):
             "gpu_launches_per_step": 1 + 5 * s.n_layers + 2}
 
 
+ATT_LENGTHS = (128, 795, 4096, 16384, 32768)
+ATT_BATCHES = (1, 8, 64)
+
+
+def run_attention_grid(dev, seed):
+    """Isolated GQA decode attention (16 query / 8 KV heads of 128, bf16 K/V
+    ~N(0,1), lengths U[L/2, L]) through dec_attention, per (L, B) cell: device
+    time per call (median of 10 after 3 warm-ups, L2 flushed between calls
+    by the 1 GiB scratch write) and bandwidth over the algorithmic bytes."""
+    import torch
+    from decoder_greedy_decode_b200 import capi, roofline, synth
+    Hq, Hkv, D = 16, 8, 128
+    peak, kind = peaks()
+    flush = torch.empty(1 << 28, dtype=torch.float32, device=dev)  # 1 GiB > L2
+    cells = []
+    g = torch.Generator(device=dev).manual_seed(seed + 20)
+    for L in ATT_LENGTHS:
+        for B in ATT_BATCHES:
+            lengths = synth.ragged_lengths(L // 2, L, B, seed=seed + 21)
+            k = torch.randn((B, Hkv, L, D), generator=g, device=dev).to(torch.bfloat16)
+            v = torch.randn((B, Hkv, L, D), generator=g, device=dev).to(torch.bfloat16)
+            q = torch.randn((B, Hq, D), generator=g, device=dev).to(torch.bfloat16)
+            lens = torch.tensor(lengths, dtype=torch.int32, device=dev)
+            out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+            wsb = capi.dec_attention_workspace_bytes(B, Hq, Hkv, D, L)
+            ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+            stream = torch.cuda.current_stream(dev)
+            call = lambda: capi.dec_attention(B, Hq, Hkv, D, q, k, v, L, lens, out, ws, wsb,
+                                              None, stream)
+            for _ in range(3):
+                call()
+            # queued back to back: the flush kernel in front of every call hides
+            # the host's launch time, so an event pair times the call alone
+            evs = []
+            for _ in range(10):
+                flush.fill_(1.0)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                call()
+                e1.record(stream)
+                evs.append((e0, e1))
+            torch.cuda.synchronize(dev)
+            times = [e0.elapsed_time(e1) for e0, e1 in evs]
+            us = statistics.median(times) * 1e3
+            nbytes = roofline.attention_bytes(lengths, Hkv, D, Hq)
+            gbs = nbytes / (us * 1e-6) / 1e9
+            cells.append({"L": L, "B": B, "us": round(us, 2), "GB/s": round(gbs, 1),
+                          "frac": round(gbs / peak, 4), "bytes": nbytes})
+            del k, v, q, out, ws
+    del flush
+    return {"metric": "isolated GQA decode attention, us/call and GB/s per (L, B) cell",
+            "peak": peak, "peak_source": f"{kind} hbm_gbs", "unit": "GB/s",
+            "config": {"workload": "16 q / 8 kv heads, D 128, bf16 K/V N(0,1), lengths U[L/2, L]",
+                       "l2": "flushed between calls (1 GiB write)"},
+            "cells": cells}
+
+
 def cpu_baseline(s, w, kv_host, tok0, budget_s=20.0):
     """The CPU oracle, as it stands, on a bounded sample of the same workload."""
     import oracle
@@ -359,8 +416,13 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
 
-    # ---- the batched configuration
+    # ---- the batched configuration and the isolated attention grid
     bs64 = run_bs64(s, wd, dev, ws, args.seed)
+    kernel_config = dec.config()
+    dec.close()
+    del kv, wd
+    torch.cuda.empty_cache()
+    attention = run_attention_grid(dev, args.seed) if rank == 0 else None
 
     # ---- max over ranks
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev, ws)
@@ -380,7 +442,7 @@ def run_ours(args):
             "config": {"workload": WORKLOAD, "batch": B, "ctx": N0, "window": WINDOW,
                        "replicas": ws, "parallelism": "replicas" if ws > 1 else "single",
                        "l2": "inputs larger than L2: 1.19 GB of weights streamed per step",
-                       "kernel": dec.config()},
+                       "kernel": kernel_config},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": ncu_traffic(),
                          "peak_source": f"{peak_kind} hbm_gbs",
@@ -394,6 +456,7 @@ def run_ours(args):
             "gpu_launches": K,
             "clocks": clocks,
             "bs64": bs64,
+            "attention": attention,
         }
         if not args.no_cpu_baseline and ws == 1:
             line["cpu_baseline"] = cpu_baseline(s, w, kv_host, tok0)

@@ -7,7 +7,9 @@
 // every CTA takes a chunk of one (sequence, KV head) context, streams its K
 // and V rows through shared memory with 1-D bulk copies, keeps an fp32 online
 // softmax per query head of the group, and the last CTA of the (sequence, KV
-// head) merges the chunks' partial states.  The Baseten Qwen3-ASR article
+// head) merges the chunks' partial states.  Up to 3 (head_dim 128) or 4
+// (head_dim 64) query heads per KV head run the lane-octet kernel (4 rows per
+// warp step); more run the one-row-per-warp kernel.  The Baseten Qwen3-ASR article
 // (KV cache quantization) notes that decode attention is memory-bound: the
 // roofline of this kernel is HBM bandwidth over the K/V bytes.
 #include <cuda_runtime.h>
@@ -194,6 +196,250 @@ __global__ void __launch_bounds__(kAttThreads) attention_kernel(const AttnArgs a
   }
 }
 
+// Lane-octet variant for up to 4 query heads per KV head: 8 warps, each
+// taking 4 rows of a 32-row tile at once with 8 lanes per row (lane o holds
+// elements [o*D/16, (o+1)*D/16) and the same span of the second half of the
+// row: conflict-free 16-byte shared-memory reads; a dot product is 3
+// shuffles), an fp32 online softmax per octet, merged at the end.  A CTA that
+// holds a whole context writes the output directly.
+constexpr int kOctWarps = 8;
+constexpr int kOctThreads = kOctWarps * 32;
+constexpr int kOctRows = kOctWarps * 4;  // rows of a tile
+
+template <int D, int REP>
+__global__ void __launch_bounds__(kOctThreads, 2) attention_octet(const AttnArgs a) {
+  constexpr int HALF = D / 16;
+  constexpr int RB = D * 2;                    // bytes per bf16 row
+  constexpr int kHalfT = kOctRows * RB;        // K (or V) rows of one tile
+  constexpr int kTile = 2 * kHalfT;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* ring = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kAttStages * kTile);
+  float* merge = reinterpret_cast<float*>(full + kAttStages);  // [warps][REP][D + 2]
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int oct = lane >> 3, o = lane & 7;
+  const int ci = blockIdx.x % a.chunks_max;
+  const int bg = blockIdx.x / a.chunks_max;
+  const int b = bg / a.Hkv, g = bg % a.Hkv;
+  const int len = a.lengths[b];
+  if (len < 1 || len > a.max_len) {
+    if (tid == 0 && ci == 0 && g == 0 && a.status) atomicOr(a.status, 1);
+    return;
+  }
+  const int nchunk = (len + a.chunk_rows - 1) / a.chunk_rows;
+  if (ci >= nchunk) return;
+  const int j0 = ci * a.chunk_rows;
+  const int j1 = min(j0 + a.chunk_rows, len);
+  const int ntiles = (j1 - j0 + kOctRows - 1) / kOctRows;
+  const size_t head_row0 = (static_cast<size_t>(b) * a.Hkv + g) * a.max_len;
+  const uint8_t* kbase = reinterpret_cast<const uint8_t*>(a.k + head_row0 * D);
+  const uint8_t* vbase = reinterpret_cast<const uint8_t*>(a.v + head_row0 * D);
+
+  if (tid == 0) {
+    for (int s = 0; s < kAttStages; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const uint64_t pol = policy_evict_first();
+  auto issue = [&](int t) {
+    const int j = j0 + t * kOctRows;
+    const int nr = min(kOctRows, j1 - j);
+    const uint32_t rb = static_cast<uint32_t>(nr) * RB;
+    uint64_t* bar = &full[t % kAttStages];
+    uint8_t* dst = ring + (t % kAttStages) * kTile;
+    mbar_arrive_expect_tx(bar, 2 * rb);
+    bulk_g2s(dst, kbase + static_cast<size_t>(j) * RB, rb, bar, pol);
+    bulk_g2s(dst + kHalfT, vbase + static_cast<size_t>(j) * RB, rb, bar, pol);
+  };
+  if (tid == 0)
+    for (int t = 0; t < ntiles && t < kAttStages; ++t) issue(t);
+
+  const float qscale = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+  float qv[REP][2][HALF], acc[REP][2][HALF], m[REP], ls[REP];
+#pragma unroll
+  for (int h = 0; h < REP; ++h) {
+    m[h] = -INFINITY;
+    ls[h] = 0.f;
+    const uint16_t* qh = a.q + (static_cast<size_t>(b) * a.Hq + g * REP + h) * D;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int e = 0; e < HALF; ++e) {
+        acc[h][i][e] = 0.f;
+        qv[h][i][e] = bf16_to_f(qh[i * (D / 2) + o * HALF + e]) * qscale;
+      }
+  }
+  auto span = [&](const uint8_t* row, int i, float (&x)[HALF]) {
+    const uint8_t* pp = row + 2 * (i * (D / 2) + o * HALF);
+    if constexpr (HALF == 8) {
+      const uint4 w = *reinterpret_cast<const uint4*>(pp);
+      x[0] = bf16lo(w.x); x[1] = bf16hi(w.x); x[2] = bf16lo(w.y); x[3] = bf16hi(w.y);
+      x[4] = bf16lo(w.z); x[5] = bf16hi(w.z); x[6] = bf16lo(w.w); x[7] = bf16hi(w.w);
+    } else {
+      const uint2 w = *reinterpret_cast<const uint2*>(pp);
+      x[0] = bf16lo(w.x); x[1] = bf16hi(w.x); x[2] = bf16lo(w.y); x[3] = bf16hi(w.y);
+    }
+  };
+  for (int t = 0; t < ntiles; ++t) {
+    const int j = j0 + t * kOctRows;
+    const int nr = min(kOctRows, j1 - j);
+    {
+      Spin1 sp;
+      while (!mbar_test(&full[t % kAttStages], (t / kAttStages) & 1))
+        if (sp.expired()) break;
+    }
+    const uint8_t* tb = ring + (t % kAttStages) * kTile;
+    const int r = warp * 4 + oct;
+    const bool valid = r < nr;  // every lane joins the shuffles; short rows are masked
+    const uint8_t* krow = tb + static_cast<size_t>(valid ? r : 0) * RB;
+    float s[REP];
+#pragma unroll
+    for (int h = 0; h < REP; ++h) s[h] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      float kx[HALF];
+      span(krow, i, kx);
+#pragma unroll
+      for (int h = 0; h < REP; ++h)
+#pragma unroll
+        for (int e = 0; e < HALF; ++e) s[h] = fmaf(qv[h][i][e], kx[e], s[h]);
+    }
+#pragma unroll
+    for (int sh = 4; sh > 0; sh >>= 1)
+#pragma unroll
+      for (int h = 0; h < REP; ++h) s[h] += __shfl_xor_sync(0xffffffffu, s[h], sh);
+    if (valid) {
+      float al[REP], p[REP];
+#pragma unroll
+      for (int h = 0; h < REP; ++h) {
+        const float mn = fmaxf(m[h], s[h]);
+        al[h] = exp2f(m[h] - mn);
+        p[h] = exp2f(s[h] - mn);
+        ls[h] = ls[h] * al[h] + p[h];
+        m[h] = mn;
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        float vx[HALF];
+        span(krow + kHalfT, i, vx);
+#pragma unroll
+        for (int h = 0; h < REP; ++h)
+#pragma unroll
+          for (int e = 0; e < HALF; ++e) acc[h][i][e] = fmaf(acc[h][i][e], al[h], p[h] * vx[e]);
+      }
+    }
+    __syncthreads();  // slot t % stages fully read
+    if (tid == 0 && t + kAttStages < ntiles) issue(t + kAttStages);
+  }
+  // merge the four octets of the warp, then octet 0 writes the warp's state
+#pragma unroll
+  for (int sh = 8; sh <= 16; sh <<= 1) {
+#pragma unroll
+    for (int h = 0; h < REP; ++h) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m[h], sh);
+      const float lo = __shfl_xor_sync(0xffffffffu, ls[h], sh);
+      const float mn = fmaxf(m[h], mo);
+      const float e1 = (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - mn);
+      const float e2 = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+      ls[h] = ls[h] * e1 + lo * e2;
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int e = 0; e < HALF; ++e) {
+          const float ao = __shfl_xor_sync(0xffffffffu, acc[h][i][e], sh);
+          acc[h][i][e] = acc[h][i][e] * e1 + ao * e2;
+        }
+      m[h] = mn;
+    }
+  }
+  if (oct == 0) {
+#pragma unroll
+    for (int h = 0; h < REP; ++h) {
+      float* mg = merge + (static_cast<size_t>(warp) * REP + h) * (D + 2);
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int e = 0; e < HALF; ++e) mg[i * (D / 2) + o * HALF + e] = acc[h][i][e];
+      if (o == 0) {
+        mg[D] = m[h];
+        mg[D + 1] = ls[h];
+      }
+    }
+  }
+  __syncthreads();
+  for (int t = tid; t < REP * D; t += kOctThreads) {
+    const int h = t / D, d = t % D;
+    float M = -INFINITY;
+    for (int w = 0; w < kOctWarps; ++w) M = fmaxf(M, merge[(w * REP + h) * (D + 2) + D]);
+    float Ls = 0.f, A = 0.f;
+    for (int w = 0; w < kOctWarps; ++w) {
+      const float* mg = merge + (w * REP + h) * (D + 2);
+      const float e = (mg[D] == -INFINITY) ? 0.f : exp2f(mg[D] - M);
+      Ls += mg[D + 1] * e;
+      A += mg[d] * e;
+    }
+    if (nchunk == 1) {
+      a.out[(static_cast<size_t>(b) * a.Hq + g * REP + h) * D + d] = A / Ls;
+    } else {
+      float* pp = a.part + ((static_cast<size_t>(b) * a.Hq + g * REP + h) * a.chunks_max + ci) * (D + 2);
+      pp[d] = A;
+      if (d == 0) {
+        pp[D] = M;
+        pp[D + 1] = Ls;
+      }
+    }
+  }
+  if (nchunk == 1) return;
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    const unsigned old = atomicAdd(&a.cnt[b * a.Hkv + g], 1u);
+    s_last = (old == static_cast<unsigned>(nchunk - 1));
+    if (s_last) {
+      atomicExch(&a.cnt[b * a.Hkv + g], 0u);
+      __threadfence();
+    }
+  }
+  __syncthreads();
+  if (!s_last) return;
+  for (int t = tid; t < REP * D; t += kOctThreads) {
+    const int h = t / D, d = t % D;
+    const float* pb = a.part + (static_cast<size_t>(b) * a.Hq + g * REP + h) * a.chunks_max * (D + 2);
+    float M = -INFINITY;
+    for (int c = 0; c < nchunk; ++c) M = fmaxf(M, __ldcg(pb + c * (D + 2) + D));
+    float Ls = 0.f, A = 0.f;
+    for (int c = 0; c < nchunk; ++c) {
+      const float e = exp2f(__ldcg(pb + c * (D + 2) + D) - M);
+      Ls += __ldcg(pb + c * (D + 2) + D + 1) * e;
+      A += __ldcg(pb + c * (D + 2) + d) * e;
+    }
+    a.out[(static_cast<size_t>(b) * a.Hq + g * REP + h) * D + d] = A / Ls;
+  }
+}
+
+size_t octet_smem_bytes(int D, int rep) {
+  return static_cast<size_t>(kAttStages) * kOctRows * D * 4 + kAttStages * sizeof(uint64_t) +
+         static_cast<size_t>(kOctWarps) * rep * (D + 2) * sizeof(float);
+}
+
+template <int D, int REP>
+cudaError_t launch_octet(const AttnArgs& a, cudaStream_t s) {
+  static std::once_flag once;
+  static cudaError_t set_err = cudaSuccess;
+  const size_t smem = octet_smem_bytes(D, REP);
+  std::call_once(once, [&] {
+    set_err = cudaFuncSetAttribute(attention_octet<D, REP>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem));
+  });
+  if (set_err != cudaSuccess) return set_err;
+  const dim3 grid(static_cast<unsigned>(a.B) * a.Hkv * a.chunks_max);
+  attention_octet<D, REP><<<grid, kOctThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
 // One warp per row: E4M3 codes and the fp32 row scale (the step kernel's
 // append uses the same routine).
 template <int D>
@@ -244,6 +490,23 @@ int attention_chunk_rows(int B, int Hkv, int max_len, int sms) {
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {
   const int rep = a.Hq / a.Hkv;
+  if (a.D == 128) {
+    switch (rep) {
+      case 1: return launch_octet<128, 1>(a, s);
+      case 2: return launch_octet<128, 2>(a, s);
+      case 3: return launch_octet<128, 3>(a, s);
+      default: break;  // 4 heads of 128 would spill registers
+    }
+  } else if (a.D == 64) {
+    switch (rep) {
+      case 1: return launch_octet<64, 1>(a, s);
+      case 2: return launch_octet<64, 2>(a, s);
+      case 3: return launch_octet<64, 3>(a, s);
+      case 4: return launch_octet<64, 4>(a, s);
+      default: break;
+    }
+  }
+  // 5..8 query heads per KV head: one row per warp step
   const size_t smem = attention_smem_bytes(a.D, rep);
   const dim3 grid(static_cast<unsigned>(a.B) * a.Hkv * a.chunks_max);
   cudaError_t e;

@@ -6,7 +6,8 @@ quick timing.
 
 Weights have the 0.6B (default) or 1.7B widths with --layers layers; every
 sequence's cache holds N(0,1) rows up to a context drawn in [lo, hi]; the
-steps feed their own ids back.  Prints the device time per step."""
+steps feed their own ids back.  Prints the device time per step of the
+--steps steps that follow --warmup untimed ones."""
 from __future__ import annotations
 
 import argparse
@@ -24,6 +25,7 @@ def main() -> None:
     p.add_argument("--batch", type=int, default=64)
     p.add_argument("--ctx", default="200,420")
     p.add_argument("--steps", type=int, default=2)
+    p.add_argument("--warmup", type=int, default=0)
     p.add_argument("--kv", choices=["bf16", "fp8"], default="bf16")
     a = p.parse_args()
     base = synth.QWEN3_0_6B if a.shape == "0.6b" else synth.QWEN3_1_7B
@@ -31,7 +33,7 @@ def main() -> None:
                          base.ffn, base.vocab)
     lo, hi = (int(x) for x in a.ctx.split(","))
     dec = Decoder(s, to_device(synth.model_weights(s, seed=2)), max_batch=a.batch)
-    max_ctx = (hi + a.steps + 15) // 16 * 16
+    max_ctx = (hi + a.warmup + a.steps + 15) // 16 * 16
     kv = dec.kv_cache(a.batch, max_ctx, a.kv)
     g = torch.Generator(device="cuda").manual_seed(1)
     if a.kv == "bf16":
@@ -43,11 +45,13 @@ def main() -> None:
     lengths = synth.ragged_lengths(lo, hi, a.batch, seed=3)
     base_pos = torch.tensor(lengths, dtype=torch.int32, device="cuda")
     tok = torch.randint(0, s.vocab, (a.batch,), generator=g, dtype=torch.int32, device="cuda")
+    for i in range(a.warmup):
+        dec.step(kv, tok, base_pos + i, tok)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     e0.record()
     for i in range(a.steps):
-        dec.step(kv, tok, base_pos + i, tok)
+        dec.step(kv, tok, base_pos + a.warmup + i, tok)
     e1.record()
     torch.cuda.synchronize()
     st = dec.check()
