@@ -77,7 +77,7 @@ constexpr int kAttStages = 4;
 constexpr int kAttTileRows = 32;                // = kAttWarps x 4 rows (lane octets)
 constexpr int kAttMaxRep = 4;  // query heads per KV head (attention template)
 constexpr int kRowThreads = 256;
-constexpr int kProfCtas = 2048;                   // GEMM CTAs with timestamps (profiling builds)
+[[maybe_unused]] constexpr int kProfCtas = 2048;                   // GEMM CTAs with timestamps (profiling builds)
 
 enum GemmMode { kQKV = 0, kResid = 1, kSwiGLU = 2, kLm = 3 };
 

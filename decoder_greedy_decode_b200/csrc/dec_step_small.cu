@@ -54,7 +54,7 @@ enum { SQ = 0, SA, SO, SU, SD, kStages, SLM = kStages };
 // prof[cta][kStampsPerLayer * L + 8] at the points named by the St* indices
 // below (per layer), then lm_head start / gathered / done, consumer end and
 // consumer start.
-constexpr int kStampsPerLayer = 16;
+[[maybe_unused]] constexpr int kStampsPerLayer = 16;
 enum {
   StStart = 0, StQGath, StQNorm, StQkv, StAttIn, StAttRows, StAtt, StOGath, StO, StUGath, StUNorm,
   StU, StDGath, StD
@@ -804,7 +804,7 @@ struct Cta {
   // fourth row and each lane a D/8-wide slice (3-shuffle dot products).  The
   // CTA of chunk 0 combines the chunks' partial softmax states and publishes
   // the head outputs; other chunks publish their partial state and move on.
-  // act holds qs[rep][D], kn[D], vn[D], merge[kCW][D + 2], ownb[rep][D + 2].
+  // act holds qs[rep][D], kn[D], vn[D], merge[kCW][D + 2].
   __device__ void attention(int l) {
     const int rep = a.Hq / a.Hkv;
     const float qscale = 1.4426950408889634f / sqrtf(static_cast<float>(D));  // log2(e)/sqrt(D)
@@ -812,7 +812,6 @@ struct Cta {
     float* kn = act + rep * D;
     float* vn = kn + D;
     float* merge = vn + D;
-    float* ownb = merge + kCW * (D + 2);
     const LayerPtrs& lw = slw[l];
     const uint32_t f = flag(l);
     const int HqD = a.Hq * D;
