@@ -69,7 +69,7 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, kTileN);
 constexpr int kTStride = kTileM + 4;              // accumulator tile in smem: T[b][row]
 constexpr int kWOffset = 40 * 1024;               // reduced rows of this CTA's sequences
 constexpr size_t kGemmSmem = 1024 + kGemmStages * kStageBytes + 256;
-constexpr int kMaxSplits = 8;                     // cluster size (portable)
+constexpr int kMaxSplits = 16;                    // cluster size (16: non-portable, allowed per kernel)
 constexpr int kMaxAttnChunks = 32;
 constexpr int kAttWarps = 8;
 constexpr int kAttThreads = kAttWarps * 32;
@@ -1207,10 +1207,14 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_h
   // kernel attributes, once
   const int smem = static_cast<int>(kGemmSmem);
   const cudaFuncAttribute dyn = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  const cudaFuncAttribute npc = cudaFuncAttributeNonPortableClusterSizeAllowed;
   if (ok) e = cudaFuncSetAttribute(gemm_kernel<kQKV>, dyn, smem);
   if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kResid>, dyn, smem);
   if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kSwiGLU>, dyn, smem);
   if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kLm>, dyn, smem);
+  if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kQKV>, npc, 1);
+  if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kResid>, npc, 1);
+  if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kSwiGLU>, npc, 1);
   const int rep = s.Hq / s.Hkv;
   if (ok && e == cudaSuccess) e = s.D == 128 ? attn_attrs_for<128>(rep) : attn_attrs_for<64>(rep);
   if (!ok || e != cudaSuccess) {
