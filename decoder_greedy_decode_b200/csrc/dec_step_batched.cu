@@ -71,10 +71,10 @@ constexpr int kWOffset = 40 * 1024;               // reduced rows of this CTA's 
 constexpr size_t kGemmSmem = 1024 + kGemmStages * kStageBytes + 256;
 constexpr int kMaxSplits = 16;                    // cluster size (16: non-portable, allowed per kernel)
 constexpr int kMaxAttnChunks = 32;
-constexpr int kAttWarps = 8;
+constexpr int kAttWarps = 4;
 constexpr int kAttThreads = kAttWarps * 32;
-constexpr int kAttStages = 4;
-constexpr int kAttTileRows = 32;                // = kAttWarps x 4 rows (lane octets)
+constexpr int kAttStages = 3;
+constexpr int kAttTileRows = 32;                // passes of kAttWarps x 4 rows (lane octets)
 constexpr int kAttMaxRep = 4;  // query heads per KV head (attention template)
 constexpr int kRowThreads = 256;
 [[maybe_unused]] constexpr int kProfCtas = 2048;                   // GEMM CTAs with timestamps (profiling builds)
@@ -82,7 +82,7 @@ constexpr int kRowThreads = 256;
 enum GemmMode { kQKV = 0, kResid = 1, kSwiGLU = 2, kLm = 3 };
 
 static_assert(kTileN == 64 && kTmemCols == 64, "epilogue reads 4 x 16 accumulator columns");
-static_assert(kAttWarps * 4 == kAttTileRows, "a tile is one row per octet");
+static_assert(kAttTileRows % (kAttWarps * 4) == 0, "a tile is whole passes of one row per octet");
 static_assert(kTileN * kTStride * 4 <= kWOffset, "accumulator tile below the reduced rows");
 static_assert((kTileN + kMaxSplits) * kTileM * 4 <= kWOffset, "split receive rows below them");
 static_assert(kWOffset + kTileN * kTileM * 4 <= kGemmStages * kStageBytes, "both fit the ring");
@@ -646,8 +646,10 @@ __global__ void finish_kernel(const StepArgs2 a) {
 // ================================================================ attention
 // Split-K GQA decode attention over the step's cache: CTA = (sequence b, KV
 // head g, chunk of chunk_rows rows of 0..p_b).  K and V rows of 32-row tiles
-// arrive by 1-D bulk copies into a ring.  Lane octets: each warp takes 4 rows
-// of a tile at once, 8 lanes per row; lane o of an octet holds elements
+// arrive by 1-D bulk copies into a 3-stage ring.  4 warps (4 CTAs fit an SM,
+// so a batch of 64 x 8 (sequence, KV head) pairs is one wave).  Lane octets:
+// each warp takes 4 rows of a tile at once (two passes per 32-row tile), 8
+// lanes per row; lane o of an octet holds elements
 // [o*D/16, (o+1)*D/16) and the same span of the second half of the row (so
 // the 8 lanes of a row read 8 consecutive 16-byte pieces: no bank conflicts),
 // a dot product is 3 shuffles, and every octet keeps its own fp32 online
@@ -704,7 +706,7 @@ __device__ __forceinline__ void load_span(const uint8_t* row, int o, int i, floa
 }
 
 template <int D, bool FP8, int REP>
-__global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const AttnArgs2 a) {
+__global__ void __launch_bounds__(kAttThreads, 4) attn_kernel(const AttnArgs2 a) {
   constexpr int E = FP8 ? 1 : 2;                      // bytes per element
   constexpr int HALF = D / 16;                        // elements per span
   constexpr int RB = D * E;                           // bytes per row
@@ -789,58 +791,61 @@ __global__ void __launch_bounds__(kAttThreads, 2) attn_kernel(const AttnArgs2 a)
         if (sp.expired()) break;
     }
     const uint8_t* tb = ring + (t % kAttStages) * kTile;
-    // 8 warps x 4 rows = the 32 rows of a tile; every lane takes part in the
-    // shuffles, rows past nr are masked out of the softmax
-    const int r = warp * 4 + oct;
-    const bool valid = r < nr;
-    const int rr = valid ? r : 0;
-    const uint8_t* krow = tb + static_cast<size_t>(rr) * RB;
-    const uint8_t* vrow = krow + kHalf;
     const float* tsc = reinterpret_cast<const float*>(tb + 2 * kHalf);
-    const float ks = FP8 ? tsc[rr] : 1.f;
-    float s[REP];
+    // kAttWarps x 4 rows per pass; every lane takes part in the shuffles,
+    // rows past nr are masked out of the softmax
 #pragma unroll
-    for (int h = 0; h < REP; ++h) s[h] = 0.f;
+    for (int pass = 0; pass < kAttTileRows / (kAttWarps * 4); ++pass) {
+      const int r = (pass * kAttWarps + warp) * 4 + oct;
+      const bool valid = r < nr;
+      const int rr = valid ? r : 0;
+      const uint8_t* krow = tb + static_cast<size_t>(rr) * RB;
+      const uint8_t* vrow = krow + kHalf;
+      const float ks = FP8 ? tsc[rr] : 1.f;
+      float s[REP];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      float kx[HALF];
-      load_span<D, FP8>(krow, o, i, kx);
-#pragma unroll
-      for (int h = 0; h < REP; ++h)
-#pragma unroll
-        for (int e = 0; e < HALF; ++e) s[h] = fmaf(qv[h][i][e], kx[e], s[h]);
-    }
-#pragma unroll
-    for (int sh = 4; sh > 0; sh >>= 1)
-#pragma unroll
-      for (int h = 0; h < REP; ++h) s[h] += __shfl_xor_sync(0xffffffffu, s[h], sh);
-    if (FP8) {
-#pragma unroll
-      for (int h = 0; h < REP; ++h) s[h] *= ks;  // q . (code x scale) = scale x (q . code)
-    }
-    if (valid) {
-      float al[REP], p[REP];
-#pragma unroll
-      for (int h = 0; h < REP; ++h) {
-        const float mn = fmaxf(m[h], s[h]);
-        al[h] = exp2f(m[h] - mn);
-        p[h] = exp2f(s[h] - mn);
-        ls[h] = ls[h] * al[h] + p[h];
-        m[h] = mn;
-      }
-      if (FP8) {
-        const float vs = tsc[kAttTileRows + rr];
-#pragma unroll
-        for (int h = 0; h < REP; ++h) p[h] *= vs;  // p (code x scale) = (p scale) code
-      }
+      for (int h = 0; h < REP; ++h) s[h] = 0.f;
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        float vx[HALF];
-        load_span<D, FP8>(vrow, o, i, vx);
+        float kx[HALF];
+        load_span<D, FP8>(krow, o, i, kx);
 #pragma unroll
         for (int h = 0; h < REP; ++h)
 #pragma unroll
-          for (int e = 0; e < HALF; ++e) acc[h][i][e] = fmaf(acc[h][i][e], al[h], p[h] * vx[e]);
+          for (int e = 0; e < HALF; ++e) s[h] = fmaf(qv[h][i][e], kx[e], s[h]);
+      }
+#pragma unroll
+      for (int sh = 4; sh > 0; sh >>= 1)
+#pragma unroll
+        for (int h = 0; h < REP; ++h) s[h] += __shfl_xor_sync(0xffffffffu, s[h], sh);
+      if (FP8) {
+#pragma unroll
+        for (int h = 0; h < REP; ++h) s[h] *= ks;  // q . (code x scale) = scale x (q . code)
+      }
+      if (valid) {
+        float al[REP], p[REP];
+#pragma unroll
+        for (int h = 0; h < REP; ++h) {
+          const float mn = fmaxf(m[h], s[h]);
+          al[h] = exp2f(m[h] - mn);
+          p[h] = exp2f(s[h] - mn);
+          ls[h] = ls[h] * al[h] + p[h];
+          m[h] = mn;
+        }
+        if (FP8) {
+          const float vs = tsc[kAttTileRows + rr];
+#pragma unroll
+          for (int h = 0; h < REP; ++h) p[h] *= vs;  // p (code x scale) = (p scale) code
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          float vx[HALF];
+          load_span<D, FP8>(vrow, o, i, vx);
+#pragma unroll
+          for (int h = 0; h < REP; ++h)
+#pragma unroll
+            for (int e = 0; e < HALF; ++e) acc[h][i][e] = fmaf(acc[h][i][e], al[h], p[h] * vx[e]);
+        }
       }
     }
     __syncthreads();  // slot t % stages fully read
@@ -1273,10 +1278,10 @@ cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
     return g;
   };
 
-  // attention chunking: one wave of CTAs (2 resident per SM) over the
+  // attention chunking: one wave of CTAs (4 resident per SM) over the
   // (sequence, KV head) pairs, i.e. one chunk per pair once there are enough
   // pairs; at most kMaxAttnChunks chunks per pair
-  int per_pair = (2 * p->sms) / (io.B * s.Hkv);
+  int per_pair = (4 * p->sms) / (io.B * s.Hkv);
   if (per_pair < 1) per_pair = 1;
   if (per_pair > kMaxAttnChunks) per_pair = kMaxAttnChunks;
   int cr = (io.max_ctx + per_pair - 1) / per_pair;
