@@ -27,7 +27,7 @@ EXPORTS = (
     "dec_step_debug", "dec_step_host", "dec_check", "dec_set_timeout_ns", "dec_set_debug_stall",
     "dec_error_string", "dec_last_cuda_error", "dec_get_config",
     "dec_attention_workspace_bytes", "dec_attention", "dec_kv_quantize_e4m3",
-    "dec_attention_noalloc",
+    "dec_attention_noalloc", "dec_verify", "dec_accept_greedy",
 )
 
 
@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
             "dec_attention": ([I, I, I, I, P, P, P, I, P, P, P, Z, P, P], I),
             "dec_kv_quantize_e4m3": ([P, I, I, P, P, P], I),
             "dec_attention_noalloc": ([I, I, I, I, P, P, P, I, P, P, P, P], I),
+            "dec_verify": ([P, I, P, P, I, ctypes.POINTER(dec_kv), P, P, P], I),
+            "dec_accept_greedy": ([I, P, P, P, ctypes.POINTER(I)], I),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -150,6 +152,23 @@ def dec_step(h: int, batch: int, token_ids, positions, kv: dec_kv, out_ids, out_
              stream=None) -> None:
     _ok(lib().dec_step(h, batch, _ptr(token_ids), _ptr(positions), ctypes.byref(kv),
                        _ptr(out_ids), _ptr(out_logits), _stream(stream)), "dec_step")
+
+
+def dec_verify(h: int, k: int, token_ids, positions, seq: int, kv: dec_kv, out_ids,
+               out_logits=None, stream=None) -> None:
+    _ok(lib().dec_verify(h, k, _ptr(token_ids), _ptr(positions), seq, ctypes.byref(kv),
+                         _ptr(out_ids), _ptr(out_logits), _stream(stream)), "dec_verify")
+
+
+def dec_accept_greedy(tokens: Sequence[int], out_ids: Sequence[int]) -> list:
+    """Greedy acceptance of a verified block (host lists): the emitted tokens."""
+    k = len(tokens)
+    t = (ctypes.c_int32 * k)(*[int(x) for x in tokens])
+    o = (ctypes.c_int32 * k)(*[int(x) for x in out_ids])
+    e = (ctypes.c_int32 * k)()
+    n = ctypes.c_int()
+    _ok(lib().dec_accept_greedy(k, t, o, e, ctypes.byref(n)), "dec_accept_greedy")
+    return [int(e[i]) for i in range(n.value)]
 
 
 def dec_step_debug(h: int, batch: int, token_ids, positions, kv: dec_kv, out_ids, out_logits,

@@ -257,6 +257,7 @@ static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* 
                              : nullptr;
     io.kv_batch = kv->batch;
     io.max_ctx = kv->max_ctx;
+    io.one_seq = -1;
     io.status = reinterpret_cast<int*>(h->ws + h->wl.status);
     io.timeout_ns = h->timeout_ns;
     cudaError_t e = bt_step(h->bt, io, stream);
@@ -354,6 +355,54 @@ extern "C" int dec_step_host(dec_handle* h, int batch, const int32_t* tok_host,
                         cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e);
+  return DEC_OK;
+}
+
+extern "C" int dec_verify(dec_handle* h, int k, const int32_t* token_ids,
+                          const int32_t* positions, int seq, const dec_kv* kv, int32_t* out_ids,
+                          float* out_logits, void* stream) {
+  if (!h || !kv || !token_ids || !positions || !out_ids || !kv->base) return DEC_ERR_NULL;
+  if (!h->bt) return DEC_ERR_BATCH;  // the handle has no batched step (max_batch <= 4)
+  if (k < 1 || k > h->shape.max_batch) return DEC_ERR_BATCH;
+  if (seq < 0 || seq >= kv->batch) return DEC_ERR_ARG;
+  if (kv->dtype != DEC_KV_BF16 && kv->dtype != DEC_KV_FP8_E4M3) return DEC_ERR_DTYPE;
+  if (kv->bytes < dec_kv_bytes(h, kv->batch, kv->max_ctx, kv->dtype)) return DEC_ERR_KV_SIZE;
+  BtIO io{};
+  io.B = k;
+  io.tok = token_ids;
+  io.pos = positions;
+  io.out = out_ids;
+  io.logits = out_logits;
+  io.hidden = nullptr;
+  io.kv = static_cast<uint8_t*>(kv->base);
+  io.kv_fp8 = kv->dtype == DEC_KV_FP8_E4M3;
+  io.kv_scales = io.kv_fp8 ? reinterpret_cast<float*>(
+                                 static_cast<uint8_t*>(kv->base) +
+                                 dec_kv_scale_offset(h, kv->batch, kv->max_ctx, kv->dtype))
+                           : nullptr;
+  io.kv_batch = kv->batch;
+  io.max_ctx = kv->max_ctx;
+  io.one_seq = seq;
+  io.status = reinterpret_cast<int*>(h->ws + h->wl.status);
+  io.timeout_ns = h->timeout_ns;
+  cudaError_t e = bt_step(h->bt, io, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return DEC_OK;
+}
+
+extern "C" int dec_accept_greedy(int k, const int32_t* tokens, const int32_t* out_ids,
+                                 int32_t* emitted, int* n_emitted) {
+  if (!tokens || !out_ids || !emitted || !n_emitted) return DEC_ERR_NULL;
+  if (k < 1) return DEC_ERR_ARG;
+  for (int i = 0; i < k; ++i)
+    if (out_ids[i] < 0) return DEC_ERR_ARG;  // the verify step was invalid
+  // draft token tokens[i + 1] is checked against the prediction made at the
+  // position before it, out_ids[i]; the first mismatch ends the accepted run
+  int j = 0;
+  while (j < k - 1 && tokens[j + 1] == out_ids[j]) ++j;
+  for (int i = 0; i < j; ++i) emitted[i] = tokens[i + 1];
+  emitted[j] = out_ids[j];  // the correction, or the bonus token after a full match
+  *n_emitted = j + 1;
   return DEC_OK;
 }
 

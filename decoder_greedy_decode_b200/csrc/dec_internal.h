@@ -112,6 +112,7 @@ struct BtIO {
   uint8_t* kv;
   float* kv_scales;
   int kv_batch, max_ctx, kv_fp8;
+  int one_seq;     // -1: row b is cache sequence b; >= 0: every row is that sequence
   int* status;
   unsigned long long timeout_ns;
 };

@@ -159,6 +159,7 @@ struct GemmArgs {
   uint8_t* kv;
   float* kv_scales;
   int kv_batch, max_ctx, layer, kv_fp8;
+  int one_seq;           // -1: row b is cache sequence b; >= 0: every row is that sequence
   const int32_t* pos;
   const int* bad;
   const float* inv_freq;
@@ -481,8 +482,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       } else if (!bad) {  // an invalid step leaves the cache unchanged
         const int kvsel = mat - 1;
         auto crow_of = [&](int b) {
+          const int cs = g.one_seq >= 0 ? g.one_seq : b;  // cache sequence of row b
           const size_t plane =
-              ((static_cast<size_t>(g.layer) * 2 + kvsel) * g.kv_batch + b) * g.Hkv + head;
+              ((static_cast<size_t>(g.layer) * 2 + kvsel) * g.kv_batch + cs) * g.Hkv + head;
           return plane * g.max_ctx + s_pos[b];
         };
         if (!g.kv_fp8) {
@@ -658,6 +660,7 @@ __global__ void finish_kernel(const StepArgs2 a) {
 // planes, otherwise the last chunk CTA of (b, g) merges the chunks.
 struct AttnArgs2 {
   int B, Hq, Hkv, max_ctx, kv_batch, l;
+  int one_seq;     // -1: row b is cache sequence b; >= 0: every row is that sequence
   const uint8_t* kv;
   const float* kv_scales;
   const float* q;
@@ -733,8 +736,9 @@ __global__ void __launch_bounds__(kAttThreads, 4) attn_kernel(const AttnArgs2 a)
   const int j0 = ci * a.chunk_rows;
   const int j1 = min(j0 + a.chunk_rows, len);
   const int ntiles = (j1 - j0 + kAttTileRows - 1) / kAttTileRows;
-  const size_t kplane = ((static_cast<size_t>(a.l) * 2 + 0) * a.kv_batch + b) * a.Hkv + g;
-  const size_t vplane = ((static_cast<size_t>(a.l) * 2 + 1) * a.kv_batch + b) * a.Hkv + g;
+  const int cs = a.one_seq >= 0 ? a.one_seq : b;  // cache sequence of row b
+  const size_t kplane = ((static_cast<size_t>(a.l) * 2 + 0) * a.kv_batch + cs) * a.Hkv + g;
+  const size_t vplane = ((static_cast<size_t>(a.l) * 2 + 1) * a.kv_batch + cs) * a.Hkv + g;
   const uint8_t* kbase = a.kv + kplane * a.max_ctx * RB;
   const uint8_t* vbase = a.kv + vplane * a.max_ctx * RB;
   const float* ksc = FP8 ? a.kv_scales + kplane * a.max_ctx : nullptr;
@@ -1259,6 +1263,7 @@ cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
   base.kv_batch = io.kv_batch;
   base.max_ctx = io.max_ctx;
   base.kv_fp8 = io.kv_fp8;
+  base.one_seq = io.one_seq;
   base.pos = io.pos;
   base.bad = p->bad;
   base.inv_freq = p->inv_freq;
@@ -1292,6 +1297,7 @@ cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
   at.Hkv = s.Hkv;
   at.max_ctx = io.max_ctx;
   at.kv_batch = io.kv_batch;
+  at.one_seq = io.one_seq;
   at.kv = io.kv;
   at.kv_scales = io.kv_scales;
   at.q = p->q;

@@ -88,6 +88,14 @@ class Decoder:
         b = int(token_ids.numel()) if batch is None else batch
         capi.dec_step(self.h, b, token_ids, positions, kv.kv, out_ids, logits, stream)
 
+    def verify(self, kv: KVCache, token_ids, positions, seq: int, out_ids, logits=None,
+               stream=None) -> None:
+        """One step over k consecutive tokens of cache sequence `seq`
+        (positions p0 .. p0+k-1): out_ids[i] is the greedy token after
+        token_ids[i]."""
+        capi.dec_verify(self.h, int(token_ids.numel()), token_ids, positions, seq, kv.kv,
+                        out_ids, logits, stream)
+
     def step_debug(self, kv: KVCache, token_ids, positions, out_ids, logits, hidden,
                    stream=None) -> None:
         capi.dec_step_debug(self.h, int(token_ids.numel()), token_ids, positions, kv.kv,

@@ -195,6 +195,42 @@ int dec_kv_alloc(dec_handle *h, int batch, int max_ctx, int dtype, void *buf,
 int dec_step(dec_handle *h, int batch, const int32_t *token_ids, const int32_t *positions,
              const dec_kv *kv, int32_t *out_ids, float *out_logits, void *stream);
 
+/* ------------------------------------------------------------------ */
+/* Block verification and greedy acceptance (speculative decoding)     */
+/* ------------------------------------------------------------------ */
+
+/* Verify a block of k consecutive tokens of ONE cached sequence in a single
+ * step ("Can CTC make Qwen3-ASR faster?", §11 Phase A steps 2-3: one target
+ * forward over the whole draft block; §03: greedy verification).
+ *   token_ids  int32 [k] (device)  t_0 = the last committed token, then the
+ *                                  draft tokens t_1 .. t_{k-1}
+ *   positions  int32 [k] (device)  p0 + i: row i is written to cache row
+ *                                  p0 + i of sequence `seq` and attends rows
+ *                                  0 .. p0 + i (so the block is causal among
+ *                                  itself)
+ *   out_ids    int32 [k]           out_ids[i] = greedy next token after t_i
+ *                                  (the prediction that checks t_{i+1});
+ *                                  may alias token_ids
+ *   out_logits fp32 [k, vocab] or NULL.
+ * Results equal k single-sequence steps fed t_0 .. t_{k-1} (up to rounding).
+ * Needs a handle created with max_batch > 4 (it runs the batched step) and
+ * 1 <= k <= max_batch.  Asynchronous; invalid positions / tokens behave as in
+ * dec_step.  Cache rows p0 .. p0 + k - 1 of `seq` are overwritten. */
+int dec_verify(dec_handle *h, int k, const int32_t *token_ids, const int32_t *positions,
+               int seq, const dec_kv *kv, int32_t *out_ids, float *out_logits, void *stream);
+
+/* Greedy acceptance of a verified block (HOST arrays, no GPU work): the
+ * pages' contract ("Can CTC make Qwen3-ASR faster?", §03 and §08) — accept
+ * draft token t_{i+1} only while it equals out_ids[i]; at the first mismatch
+ * emit out_ids[i] instead and stop; after a full match emit the bonus token
+ * out_ids[k-1].  Writes the j + 1 emitted tokens (t_1..t_j, then out_ids[j])
+ * to emitted[] (room for k) and j + 1 to *n_emitted.  The cache is valid up
+ * to row p0 + j; the host continues at position p0 + j + 1 with token
+ * emitted[j] (rows beyond are overwritten by later steps: the crop is the
+ * host's position).  DEC_ERR_ARG if out_ids holds -1 (an invalid step). */
+int dec_accept_greedy(int k, const int32_t *tokens, const int32_t *out_ids, int32_t *emitted,
+                      int *n_emitted);
+
 /* dec_step plus the residual stream after the embedding and after every
  * layer: hidden_out fp32 [n_layers + 1][batch][hidden] (device). */
 int dec_step_debug(dec_handle *h, int batch, const int32_t *token_ids,
