@@ -215,6 +215,57 @@ def run_bs64(s, wd, dev, ws, seed):
             "gpu_launches_per_step": 1 + 5 * s.n_layers + 2}
 
 
+VERIFY_BLOCKS = (1, 2, 4, 8, 16, 32)
+
+
+def run_verify(s, wd, dev, seed):
+    """Block verification ("Can CTC make Qwen3-ASR faster?", 11 Phase A:
+    time block sizes 1 .. 32): one sequence of the 0.6B decoder at context
+    795, a block of k tokens per dec_verify call; device time per call (median
+    of 20 after 3 warm-ups) and per committed token if the whole block is
+    accepted.  Bytes: the weights, the sequence's cache rows once, the block's
+    embedding rows."""
+    import torch
+    from decoder_greedy_decode_b200 import roofline
+    from decoder_greedy_decode_b200.decoder import Decoder
+    kmax = max(VERIFY_BLOCKS)
+    dec = Decoder(s, wd, max_batch=kmax)
+    max_ctx = (N0 + kmax + 15) // 16 * 16
+    kv = dec.kv_cache(1, max_ctx)
+    kv.values.normal_(generator=torch.Generator(device=dev).manual_seed(seed + 30))
+    stream = torch.cuda.current_stream(dev)
+    peak, kind = peaks()
+    cells = []
+    for k in VERIFY_BLOCKS:
+        toks = torch.randint(0, s.vocab, (k,), dtype=torch.int32, device=dev)
+        pos = torch.arange(N0, N0 + k, dtype=torch.int32, device=dev)
+        out = torch.empty(k, dtype=torch.int32, device=dev)
+        for _ in range(3):
+            dec.verify(kv, toks, pos, 0, out, None, stream)
+        evs = []
+        for _ in range(20):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dec.verify(kv, toks, pos, 0, out, None, stream)
+            e1.record(stream)
+            evs.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        us = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs) * 1e3
+        nbytes = (roofline.weight_bytes(s) + (N0 + k) * roofline.kv_bytes_per_token(s)
+                  + k * s.hidden * 2)
+        cells.append({"k": k, "us_per_call": round(us, 1), "us_per_token_full_accept": round(us / k, 1),
+                      "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1)})
+    st = dec.check()
+    dec.close()
+    if st != 0:
+        raise RuntimeError(f"verify device status {st}")
+    return {"metric": "block verification: us per dec_verify call and per committed token "
+                      "at full acceptance", "peak": peak, "peak_source": f"{kind} hbm_gbs",
+            "config": {"workload": "qwen3-0.6b-shape decoder, one sequence, context 795, "
+                                   "blocks of k tokens (batched tensor-core step)"},
+            "cells": cells}
+
+
 ATT_LENGTHS = (128, 795, 4096, 16384, 32768)
 ATT_BATCHES = (1, 8, 64)
 
@@ -418,6 +469,7 @@ def run_ours(args):
 
     # ---- the batched configuration and the isolated attention grid
     bs64 = run_bs64(s, wd, dev, ws, args.seed)
+    verify = run_verify(s, wd, dev, args.seed) if rank == 0 else None
     kernel_config = dec.config()
     dec.close()
     del kv, wd
@@ -457,6 +509,7 @@ def run_ours(args):
             "clocks": clocks,
             "bs64": bs64,
             "attention": attention,
+            "verify": verify,
         }
         if not args.no_cpu_baseline and ws == 1:
             line["cpu_baseline"] = cpu_baseline(s, w, kv_host, tok0)
