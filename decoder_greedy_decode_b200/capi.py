@@ -27,7 +27,7 @@ EXPORTS = (
     "dec_step_debug", "dec_step_host", "dec_check", "dec_set_timeout_ns", "dec_set_debug_stall",
     "dec_error_string", "dec_last_cuda_error", "dec_get_config",
     "dec_attention_workspace_bytes", "dec_attention", "dec_kv_quantize_e4m3",
-    "dec_attention_noalloc", "dec_verify", "dec_accept_greedy",
+    "dec_attention_noalloc", "dec_verify", "dec_accept_greedy", "dec_generate",
 )
 
 
@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
             "dec_attention_noalloc": ([I, I, I, I, P, P, P, I, P, P, P, P], I),
             "dec_verify": ([P, I, P, P, I, ctypes.POINTER(dec_kv), P, P, P], I),
             "dec_accept_greedy": ([I, P, P, P, ctypes.POINTER(I)], I),
+            "dec_generate": ([P, I, I, P, P, ctypes.POINTER(dec_kv), P, I, P], I),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -158,6 +159,13 @@ def dec_verify(h: int, k: int, token_ids, positions, seq: int, kv: dec_kv, out_i
                out_logits=None, stream=None) -> None:
     _ok(lib().dec_verify(h, k, _ptr(token_ids), _ptr(positions), seq, ctypes.byref(kv),
                          _ptr(out_ids), _ptr(out_logits), _stream(stream)), "dec_verify")
+
+
+def dec_generate(h: int, batch: int, n_steps: int, token_ids, positions, kv: dec_kv, out_ids,
+                 eos: int = -1, stream=None) -> None:
+    _ok(lib().dec_generate(h, batch, n_steps, _ptr(token_ids), _ptr(positions),
+                           ctypes.byref(kv), _ptr(out_ids), int(eos), _stream(stream)),
+        "dec_generate")
 
 
 def dec_accept_greedy(tokens: Sequence[int], out_ids: Sequence[int]) -> list:

@@ -139,6 +139,7 @@ extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle
   wl.tok_dev = take(sizeof(int32_t) * Bfull);
   wl.pos_dev = take(sizeof(int32_t) * Bfull);
   wl.out_dev = take(sizeof(int32_t) * Bfull);
+  wl.gen_done = take(sizeof(int) * Bfull);
 #ifdef DEC_PROFILE
   wl.prof = take(sizeof(unsigned long long) * h->ctas * (16 * L + 8));
 #endif
@@ -403,6 +404,27 @@ extern "C" int dec_accept_greedy(int k, const int32_t* tokens, const int32_t* ou
   for (int i = 0; i < j; ++i) emitted[i] = tokens[i + 1];
   emitted[j] = out_ids[j];  // the correction, or the bonus token after a full match
   *n_emitted = j + 1;
+  return DEC_OK;
+}
+
+extern "C" int dec_generate(dec_handle* h, int batch, int n_steps, const int32_t* token_ids,
+                            int32_t* positions, const dec_kv* kv, int32_t* out_ids, int eos,
+                            void* stream) {
+  if (!h || !kv || !token_ids || !positions || !out_ids) return DEC_ERR_NULL;
+  if (batch < 1 || batch > h->shape.max_batch || batch > 64) return DEC_ERR_BATCH;
+  if (n_steps < 1) return DEC_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* done = reinterpret_cast<int*>(h->ws + h->wl.gen_done);
+  cudaError_t e = launch_gen_reset(done, batch, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  for (int i = 0; i < n_steps; ++i) {
+    const int32_t* tok = i == 0 ? token_ids : out_ids + static_cast<size_t>(i - 1) * batch;
+    int32_t* out = out_ids + static_cast<size_t>(i) * batch;
+    const int rc = do_step(h, batch, tok, positions, kv, out, nullptr, nullptr, st);
+    if (rc) return rc;
+    e = launch_gen_advance(out, positions, done, batch, eos, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   return DEC_OK;
 }
 

@@ -63,7 +63,7 @@ struct StepArgs {
 // Scratch layout inside the library workspace (byte offsets).
 struct WorkspaceLayout {
   size_t x_qkv, x_o, x_mid, x_u, x_out, part, amax_key, exit_cnt, seq, status, abort_flag,
-      inv_freq, tok_dev, pos_dev, out_dev, prof, total;
+      inv_freq, tok_dev, pos_dev, out_dev, gen_done, prof, total;
   int part_chunks;
 };
 
@@ -90,6 +90,10 @@ size_t attention_smem_bytes(int D, int rep);
 int attention_chunk_rows(int B, int Hkv, int max_len, int sms);
 cudaError_t launch_quantize(const float* x, int rows, int dim, uint8_t* codes, float* scales,
                             cudaStream_t s);
+// dec_generate's between-step bookkeeping (dec_generate.cu)
+cudaError_t launch_gen_reset(int* done, int batch, cudaStream_t s);
+cudaError_t launch_gen_advance(int32_t* out, int32_t* pos, int* done, int batch, int eos,
+                               cudaStream_t s);
 
 // ---- batched step (batch > kMaxBatchSmall): tensor-core projections
 struct BtShape {

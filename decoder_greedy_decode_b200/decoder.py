@@ -88,6 +88,12 @@ class Decoder:
         b = int(token_ids.numel()) if batch is None else batch
         capi.dec_step(self.h, b, token_ids, positions, kv.kv, out_ids, logits, stream)
 
+    def generate(self, kv: KVCache, token_ids, positions, out_ids, eos: int = -1,
+                 stream=None) -> None:
+        """out_ids.shape[0] greedy steps on the device; positions advance in place."""
+        capi.dec_generate(self.h, int(token_ids.numel()), int(out_ids.shape[0]), token_ids,
+                          positions, kv.kv, out_ids, eos, stream)
+
     def verify(self, kv: KVCache, token_ids, positions, seq: int, out_ids, logits=None,
                stream=None) -> None:
         """One step over k consecutive tokens of cache sequence `seq`

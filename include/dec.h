@@ -195,6 +195,22 @@ int dec_kv_alloc(dec_handle *h, int batch, int max_ctx, int dtype, void *buf,
 int dec_step(dec_handle *h, int batch, const int32_t *token_ids, const int32_t *positions,
              const dec_kv *kv, int32_t *out_ids, float *out_logits, void *stream);
 
+/* n greedy steps on the device, the host out of the loop (faster-qwen-asr
+ * GB10 record, notes.configuration: token fed back on the device; Baseten
+ * article, "Minimizing host-to-device syncs").
+ *   token_ids  int32 [batch] (device)   the current tokens
+ *   positions  int32 [batch] (device)   the rows the first step writes;
+ *                                       advanced IN PLACE after every step
+ *   out_ids    int32 [n_steps][batch]   step i's ids (the input of step i+1)
+ *   eos        end-of-sequence id, or -1 for none.  A sequence that emits
+ *              it is retired: its position stays at that step's row and its
+ *              later outputs are eos.
+ * Equivalent to n_steps dec_step calls that feed out_ids back and advance
+ * the positions by one; asynchronous (no host read-back inside); device
+ * errors as in dec_step (dec_check). */
+int dec_generate(dec_handle *h, int batch, int n_steps, const int32_t *token_ids,
+                 int32_t *positions, const dec_kv *kv, int32_t *out_ids, int eos, void *stream);
+
 /* ------------------------------------------------------------------ */
 /* Block verification and greedy acceptance (speculative decoding)     */
 /* ------------------------------------------------------------------ */

@@ -1,0 +1,132 @@
+"""The on-device decode loop (dec_generate) against step-by-step decoding and
+the CPU oracle.
+
+faster-qwen-asr GB10 record (notes.configuration): the emitted token is fed
+back on the device; Baseten article ("Minimizing host-to-device syncs"): no
+host read-back inside the loop.  dec_generate must equal n dec_step calls
+that feed their ids back and advance the positions, and retire a sequence at
+its end-of-sequence token."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import oracle_cache, oracle_shape, oracle_weights
+from decoder_greedy_decode_b200 import capi, synth
+from decoder_greedy_decode_b200.decoder import Decoder, to_device
+from gpu_util import NEAR_TIE, i32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    capi.lib()
+
+
+def _fixture(batch, seed, n0s, max_ctx=96, max_batch=None):
+    s = synth.TINY
+    w = synth.model_weights(s, seed=seed)
+    kv_host, _ = synth.kv_prefill(s, batch, max_ctx, n0s, seed=seed + 1)
+    dec = Decoder(s, to_device(w), max_batch=max_batch or batch)
+    toks = [int(t) for t in synth.tokens(s.vocab, batch, seed=seed + 2)]
+    return s, w, kv_host, dec, toks
+
+
+def _cache(dec, batch, max_ctx, kv_host):
+    kv = dec.kv_cache(batch, max_ctx)
+    kv.values.copy_(kv_host.cuda())
+    return kv
+
+
+def _step_loop(dec, kv, toks, n0s, n, eos=-1):
+    """dec_step n times, feeding the ids back; positions advance by one, and
+    stop for a sequence after it emits eos (whose later outputs are eos)."""
+    B = len(toks)
+    tok, pos, done = i32(toks), i32(n0s), [False] * B
+    out_all = []
+    for _ in range(n):
+        out = torch.empty(B, dtype=torch.int32, device="cuda")
+        dec.step(kv, tok, pos, out)
+        ids = out.cpu().tolist()
+        p = pos.cpu().tolist()
+        for b in range(B):
+            if done[b]:
+                ids[b] = eos
+            elif eos >= 0 and ids[b] == eos:
+                done[b] = True
+            else:
+                p[b] += 1
+        out_all.append(ids)
+        tok, pos = i32(ids), i32(p)
+    return out_all, pos.cpu().tolist()
+
+
+@pytest.mark.parametrize("batch,max_batch", [(2, 2), (6, 8)])
+def test_generate_equals_step_loop(batch, max_batch):
+    n0s = [20 + 7 * b for b in range(batch)]
+    s, w, kv_host, dec, toks = _fixture(batch, 100 + batch, n0s, max_batch=max_batch)
+    n = 12
+    kv_a = _cache(dec, batch, 96, kv_host)
+    out = torch.empty((n, batch), dtype=torch.int32, device="cuda")
+    pos = i32(n0s)
+    dec.generate(kv_a, i32(toks), pos, out)
+    assert dec.check() == 0
+    kv_b = _cache(dec, batch, 96, kv_host)
+    ref, ref_pos = _step_loop(dec, kv_b, toks, n0s, n)
+    assert out.cpu().tolist() == ref          # the same kernels: identical ids
+    assert pos.cpu().tolist() == ref_pos == [p + n for p in n0s]
+    assert torch.equal(kv_a.buf, kv_b.buf)
+    # and the oracle's greedy sequence, up to a permitted near-tie
+    m = oracle.Model(oracle_shape(s), oracle_weights(w))
+    got = np.array(ref)
+    for b in range(batch):
+        cache = oracle_cache(kv_host, None, b)
+        tok = toks[b]
+        for i in range(n):
+            r = m.step(cache, tok, n0s[b] + i)
+            if got[i, b] != r.token:
+                assert r.margin < NEAR_TIE, f"seq {b} step {i}"
+                break
+            tok = r.token
+    dec.close()
+
+
+def test_generate_retires_a_sequence_at_eos():
+    batch, n = 2, 10
+    n0s = [30, 40]
+    s, w, kv_host, dec, toks = _fixture(batch, 120, n0s)
+    # the token sequence 0 emits at step 4 becomes the end token
+    kv_r = _cache(dec, batch, 96, kv_host)
+    free, _ = _step_loop(dec, kv_r, toks, n0s, n)
+    eos = free[4][0]
+    first = {b: next((i for i in range(n) if free[i][b] == eos), None) for b in range(batch)}
+    kv_a = _cache(dec, batch, 96, kv_host)
+    out = torch.empty((n, batch), dtype=torch.int32, device="cuda")
+    pos = i32(n0s)
+    dec.generate(kv_a, i32(toks), pos, out, eos=eos)
+    assert dec.check() == 0
+    got = out.cpu().tolist()
+    kv_b = _cache(dec, batch, 96, kv_host)
+    ref, ref_pos = _step_loop(dec, kv_b, toks, n0s, n, eos=eos)
+    assert got == ref and pos.cpu().tolist() == ref_pos
+    f0 = first[0]
+    assert f0 is not None and f0 <= 4
+    assert all(got[i][0] == eos for i in range(f0, n))
+    assert ref_pos[0] == n0s[0] + f0          # the position stopped at the eos step
+    if first[1] is None:
+        assert ref_pos[1] == n0s[1] + n
+    dec.close()
+
+
+def test_generate_rejects_bad_arguments():
+    s, w, kv_host, dec, toks = _fixture(1, 130, [10])
+    kv = _cache(dec, 1, 96, kv_host)
+    out = torch.empty((2, 1), dtype=torch.int32, device="cuda")
+    with pytest.raises(RuntimeError):
+        capi.dec_generate(dec.h, 1, 0, i32(toks), i32([10]), kv.kv, out)
+    with pytest.raises(RuntimeError):
+        capi.dec_generate(dec.h, 2, 2, i32(toks), i32([10]), kv.kv, out)
+    dec.close()
