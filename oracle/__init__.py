@@ -70,7 +70,12 @@ def lib() -> ctypes.CDLL:
         L.or_attend.argtypes = [P, I, I, I, P, P, P, P, P, P, ctypes.c_size_t, P, P]
         L.or_attend.restype = None
         L.or_argmax.argtypes, L.or_argmax.restype = [P, I, P], I
-        L.or_step.argtypes = [P, P, P, P, P, P, I, P, P, P, I, I, I, P, P, P, P, P]
+        L.or_int8_quantize_row.argtypes = [P, I, P]
+        L.or_int8_quantize_row.restype = F
+        L.or_int8_quantize_rows.argtypes = [P, I, I, P, P]
+        L.or_int8_quantize_rows.restype = None
+        L.or_gemv_i8.argtypes, L.or_gemv_i8.restype = [P, P, P, I, I, P], None
+        L.or_step.argtypes = [P, P, P, P, P, P, I, P, P, I, P, P, P, I, I, I, P, P, P, P, P]
         L.or_step.restype = I
         L.or_set_threads.argtypes, L.or_set_threads.restype = [I], None
         L.or_get_threads.argtypes, L.or_get_threads.restype = [], I
@@ -122,6 +127,17 @@ def e4m3_quantize_row(x) -> tuple:
     return codes, float(s)
 
 
+def int8_quantize_rows(W_bits) -> tuple:
+    """Per-row symmetric int8 codes and fp32 scales of a bf16 matrix [rows, cols]
+    (reading in dec_oracle.c, or_int8_quantize_row)."""
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    W2 = W.reshape(-1, W.shape[-1])
+    codes = np.zeros(W2.shape, dtype=np.int8)
+    scales = np.zeros(W2.shape[0], dtype=np.float32)
+    lib().or_int8_quantize_rows(_p(W2), W2.shape[0], W2.shape[1], _p(codes), _p(scales))
+    return codes.reshape(W.shape), scales.reshape(W.shape[:-1])
+
+
 # ---------------------------------------------------------- building blocks
 def rmsnorm(x, g_bits, eps: float) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float64)
@@ -136,6 +152,15 @@ def gemv(W_bits, x) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float64)
     y = np.zeros(W.shape[0], dtype=np.float64)
     lib().or_gemv(_p(W), _p(x), W.shape[0], W.shape[1], _p(y))
+    return y
+
+
+def gemv_i8(codes, scales, x) -> np.ndarray:
+    C = np.ascontiguousarray(codes, dtype=np.int8)
+    sc = np.ascontiguousarray(scales, dtype=np.float32)
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.zeros(C.shape[0], dtype=np.float64)
+    lib().or_gemv_i8(_p(C), _p(sc), _p(x), C.shape[0], C.shape[1], _p(y))
     return y
 
 
@@ -194,13 +219,39 @@ class Shape:
     rope_theta: float = 1e6
 
 
+PROJ_KEYS = ("q", "k", "v", "o", "gate", "up", "down")
+
+
 @dataclass
 class Weights:
-    """bf16 bits (np.uint16) of every tensor; layer tensors keyed by LAYER_KEYS."""
+    """bf16 bits (np.uint16) of every tensor; layer tensors keyed by LAYER_KEYS.
+
+    kind "int8": the PROJ_KEYS tensors of every layer and lm_head are int8
+    codes, with fp32 row scales in `scales` (per layer, keyed by PROJ_KEYS)
+    and `lm_scale`; the embedding and the norm gains stay bf16."""
     embed: np.ndarray
     lm_head: np.ndarray
     final_norm: np.ndarray
     layers: List[Dict[str, np.ndarray]]
+    kind: str = "bf16"
+    lm_scale: Optional[np.ndarray] = None
+    scales: Optional[List[Dict[str, np.ndarray]]] = None
+
+
+def quantize_weights_int8(w: Weights) -> Weights:
+    """The int8 weight-only model of a bf16 one: every projection and lm_head
+    quantised per row (int8_quantize_rows)."""
+    assert w.kind == "bf16"
+    layers, scales = [], []
+    for lw in w.layers:
+        nl, ns = dict(lw), {}
+        for key in PROJ_KEYS:
+            nl[key], ns[key] = int8_quantize_rows(lw[key])
+        layers.append(nl)
+        scales.append(ns)
+    lm, lms = int8_quantize_rows(w.lm_head)
+    return Weights(embed=w.embed, lm_head=lm, final_norm=w.final_norm, layers=layers,
+                   kind="int8", lm_scale=lms, scales=scales)
 
 
 @dataclass
@@ -234,15 +285,28 @@ class Model:
         self.w = w
         self._keep = []
         L = shape.n_layers
+        i8 = w.kind == "int8"
+        if w.kind not in ("bf16", "int8"):
+            raise ValueError(w.kind)
         ptrs = (ctypes.c_void_p * (L * len(LAYER_KEYS)))()
+        sptrs = (ctypes.c_void_p * (L * len(LAYER_KEYS)))()
         for l, lw in enumerate(w.layers):
             for j, key in enumerate(LAYER_KEYS):
-                a = np.ascontiguousarray(lw[key], dtype=np.uint16)
+                proj = i8 and key in PROJ_KEYS
+                a = np.ascontiguousarray(lw[key], dtype=np.int8 if proj else np.uint16)
                 self._keep.append(a)
                 ptrs[l * len(LAYER_KEYS) + j] = a.ctypes.data
+                if proj:
+                    sc = np.ascontiguousarray(w.scales[l][key], dtype=np.float32)
+                    assert sc.shape == (a.shape[0],)
+                    self._keep.append(sc)
+                    sptrs[l * len(LAYER_KEYS) + j] = sc.ctypes.data
         self._ptrs = ptrs
+        self._sptrs = sptrs
+        self._wkind = 1 if i8 else 0
         self._emb = np.ascontiguousarray(w.embed, dtype=np.uint16)
-        self._lm = np.ascontiguousarray(w.lm_head, dtype=np.uint16)
+        self._lm = np.ascontiguousarray(w.lm_head, dtype=np.int8 if i8 else np.uint16)
+        self._lms = np.ascontiguousarray(w.lm_scale, dtype=np.float32) if i8 else None
         self._fn = np.ascontiguousarray(w.final_norm, dtype=np.uint16)
         s = shape
         self._sh = np.array([s.n_layers, s.hidden, s.n_q_heads, s.n_kv_heads, s.head_dim,
@@ -272,7 +336,9 @@ class Model:
         else:
             raise ValueError(cache.kind)
         tok = lib().or_step(_p(self._sh), _p(self._shd), _p(self._emb), _p(self._lm),
-                            _p(self._fn), ctypes.cast(self._ptrs, ctypes.c_void_p), kind,
+                            _p(self._fn), ctypes.cast(self._ptrs, ctypes.c_void_p),
+                            self._wkind, _p(self._lms),
+                            ctypes.cast(self._sptrs, ctypes.c_void_p), kind,
                             _p(k16), _p(k8), _p(ks), cache.max_ctx, int(token), int(pos),
                             _p(logits), _p(hidden), _p(nk), _p(nv), ctypes.byref(margin))
         return StepResult(int(tok), float(margin.value), logits, hidden, nk, nv)

@@ -7,8 +7,9 @@
  * code, header, table or constant with the CUDA library.
  *
  * Arithmetic: every activation is a double; weights and the KV cache are held
- * as the bytes the pages' system stores (bf16, or OCP FP8 E4M3 + fp32 scale)
- * and widened to double on use.  Sums run in the order the definition writes
+ * as the bytes the pages' system stores (bf16, or OCP FP8 E4M3 + fp32 scale
+ * for the cache, or int8 + fp32 row scale for the projection weights) and
+ * widened to double on use.  Sums run in the order the definition writes
  * them (ascending index), no blocking, no reordering.
  *
  * Sources (page title, section):
@@ -21,6 +22,8 @@
  *    is the argmax of the target logits).
  *  - Baseten Qwen3-ASR batch-transcription article, KV cache quantization
  *    (the cache is stored in FP8; attention math stays in full precision).
+ *  - faster-qwen-asr GB10 benchmark record, "cuda_graph_int8" entries
+ *    (int8 weight-only quantisation of the text decoder and lm_head).
  * Readings where the pages are silent (per-head q/k RMSNorm placement,
  * rotate-half RoPE pairing, consecutive GQA grouping, eps 1e-6, theta 1e6,
  * E4M3 encoding with one fp32 scale per (layer, K/V, head, token)) are listed
@@ -131,6 +134,43 @@ float or_e4m3_quantize_row(const float *x, int n, uint8_t *codes) {
   return scale;
 }
 
+/* Per-row symmetric int8 quantisation of one bf16 weight row (faster-qwen-asr
+ * GB10 benchmark record, "cuda_graph_int8" entries of the 0.6B and 1.7B
+ * models: int8 weight-only quantisation of the text decoder and lm_head).
+ * Reading (the record names the format only): one fp32 scale per output row,
+ * scale = amax / 127 in fp32, code_i = round_half_even(fp32(w_i) / scale)
+ * with the division in fp32, clamped to [-127, 127]; a row of zeros has
+ * scale 0 and codes 0.  The decision that yields each integer code is taken
+ * in fp32, as the kernel takes it.  Returns the scale. */
+float or_int8_quantize_row(const uint16_t *w, int n, int8_t *codes) {
+  float amax = 0.0f;
+  for (int i = 0; i < n; ++i) {
+    float a = fabsf((float)or_bf16_to_double(w[i]));
+    if (a > amax) amax = a;
+  }
+  if (amax == 0.0f) {
+    for (int i = 0; i < n; ++i) codes[i] = 0;
+    return 0.0f;
+  }
+  float scale = amax / 127.0f;
+  for (int i = 0; i < n; ++i) {
+    float q = (float)or_bf16_to_double(w[i]) / scale;  /* IEEE fp32 division */
+    float r = rintf(q);  /* default rounding mode: to nearest, ties to even */
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    codes[i] = (int8_t)r;
+  }
+  return scale;
+}
+
+/* Every row of a row-major bf16 W[rows, cols]; rows are independent. */
+void or_int8_quantize_rows(const uint16_t *W, int rows, int cols, int8_t *codes,
+                           float *scales) {
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < rows; ++r)
+    scales[r] = or_int8_quantize_row(W + (size_t)r * cols, cols, codes + (size_t)r * cols);
+}
+
 /* ------------------------------------------------------------------ */
 /* Building blocks                                                     */
 /* ------------------------------------------------------------------ */
@@ -156,6 +196,29 @@ void or_gemv(const uint16_t *W, const double *x, int rows, int cols, double *y) 
     for (int c = 0; c < cols; ++c) acc += or_bf16_to_double(w[c]) * x[c];
     y[r] = acc;
   }
+}
+
+/* y = W x for int8 codes C[rows, cols] with one fp32 scale per row: the
+ * weight is the dequantised value code * scale, widened to double; double
+ * dot products in ascending column order, as or_gemv. */
+void or_gemv_i8(const int8_t *C, const float *s, const double *x, int rows, int cols,
+                double *y) {
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < rows; ++r) {
+    const int8_t *c = C + (size_t)r * cols;
+    const double sr = (double)s[r];
+    double acc = 0.0;
+    for (int j = 0; j < cols; ++j) acc += ((double)c[j] * sr) * x[j];
+    y[r] = acc;
+  }
+}
+
+/* A projection in either weight format: wkind 0 -> bf16 W, 1 -> int8 codes
+ * with row scales s. */
+static void project(int wkind, const void *W, const float *s, const double *x, int rows,
+                    int cols, double *y) {
+  if (wkind == 0) or_gemv((const uint16_t *)W, x, rows, cols, y);
+  else or_gemv_i8((const int8_t *)W, s, x, rows, cols, y);
 }
 
 /* Rotary embedding of one head vector at position p ("MRoPE, fp32" in
@@ -269,6 +332,10 @@ enum { W_IN_NORM, W_Q, W_K, W_V, W_Q_NORM, W_K_NORM, W_O, W_POST_NORM,
  *    h = rmsnorm(x, g_post);  x += Wd (silu(Wg h) * (Wu h))
  *  logits = W_lm rmsnorm(x, g_final);  token' = argmax(logits)
  *
+ * Weights: wkind 0 -> every tensor bf16 bits; wkind 1 -> the seven
+ * projections of every layer (q, k, v, o, gate, up, down) and lm_head are
+ * int8 codes with fp32 row scales (lsc[l * W_N + idx], lm_scale), the
+ * embedding and the norm gains stay bf16.
  * KV cache of this sequence: kind 0 -> bf16 bits kv16[L][2][Hkv][max_ctx][D];
  * kind 1 -> codes kv8[L][2][Hkv][max_ctx][D] and scales kvs[L][2][Hkv][max_ctx].
  * hidden_out (optional): x after the embedding and after every layer,
@@ -276,8 +343,9 @@ enum { W_IN_NORM, W_Q, W_K, W_V, W_Q_NORM, W_K_NORM, W_O, W_POST_NORM,
  * they are stored, [L][Hkv][D].  Returns the argmax.
  */
 int or_step(const int *sh, const double *shd,
-            const uint16_t *embed, const uint16_t *lm_head, const uint16_t *final_norm,
-            const uint16_t *const *lw,
+            const uint16_t *embed, const void *lm_head, const uint16_t *final_norm,
+            const void *const *lw, int wkind, const float *lm_scale,
+            const float *const *lsc,
             int kind, uint16_t *kv16, uint8_t *kv8, float *kvs, int max_ctx,
             int token, int p,
             double *logits, double *hidden_out, double *new_k, double *new_v,
@@ -299,11 +367,13 @@ int or_step(const int *sh, const double *shd,
   if (hidden_out) memcpy(hidden_out, x, sizeof(double) * H);
 
   for (int l = 0; l < L; ++l) {
-    const uint16_t *const *w = lw + (size_t)l * W_N;
+    const void *const *w = lw + (size_t)l * W_N;
+    const float *const *sc = wkind ? lsc + (size_t)l * W_N : NULL;
+#define OR_SC(i) (sc ? sc[i] : NULL)
     or_rmsnorm(x, w[W_IN_NORM], H, eps, h);
-    or_gemv(w[W_Q], h, nq, H, q);
-    or_gemv(w[W_K], h, nkv, H, k);
-    or_gemv(w[W_V], h, nkv, H, v);
+    project(wkind, w[W_Q], OR_SC(W_Q), h, nq, H, q);
+    project(wkind, w[W_K], OR_SC(W_K), h, nkv, H, k);
+    project(wkind, w[W_V], OR_SC(W_V), h, nkv, H, v);
     for (int hh = 0; hh < Hq; ++hh) {
       or_rmsnorm(q + hh * D, w[W_Q_NORM], D, eps, tmp);
       memcpy(q + hh * D, tmp, sizeof(double) * D);
@@ -345,20 +415,21 @@ int or_step(const int *sh, const double *shd,
                   kvs + kbase, kvs + vbase, D, o + hh * D, NULL);
     }
 
-    or_gemv(w[W_O], o, H, nq, t);
+    project(wkind, w[W_O], OR_SC(W_O), o, H, nq, t);
     for (int i = 0; i < H; ++i) x[i] += t[i];
 
     or_rmsnorm(x, w[W_POST_NORM], H, eps, h);
-    or_gemv(w[W_GATE], h, F, H, g);
-    or_gemv(w[W_UP], h, F, H, u);
+    project(wkind, w[W_GATE], OR_SC(W_GATE), h, F, H, g);
+    project(wkind, w[W_UP], OR_SC(W_UP), h, F, H, u);
     for (int i = 0; i < F; ++i) u[i] = or_silu(g[i]) * u[i];
-    or_gemv(w[W_DOWN], u, H, F, t);
+    project(wkind, w[W_DOWN], OR_SC(W_DOWN), u, H, F, t);
+#undef OR_SC
     for (int i = 0; i < H; ++i) x[i] += t[i];
     if (hidden_out) memcpy(hidden_out + (size_t)(l + 1) * H, x, sizeof(double) * H);
   }
 
   or_rmsnorm(x, final_norm, H, eps, h);
-  or_gemv(lm_head, h, V, H, logits);
+  project(wkind, lm_head, lm_scale, h, V, H, logits);
   int id = or_argmax(logits, V, margin);
 
   free(x); free(h); free(q); free(k); free(v); free(o); free(t);
