@@ -266,6 +266,66 @@ def run_verify(s, wd, dev, seed):
             "cells": cells}
 
 
+INT8_STEPS = 260
+INT8_HANDLES = 3
+
+
+def run_int8(s, wd, kv_host, tok0, dev, seed):
+    """Weight-only int8 (faster-qwen-asr GB10 record, "cuda_graph_int8": int8
+    text decoder + lm_head): the same batch-1 workload (context 795, the
+    130-step window, self-feeding) with every projection and lm_head
+    quantised per row by dec_quantize_int8.  Device time per step over
+    INT8_STEPS steps after 5 warm-ups, on INT8_HANDLES live handles (the
+    step time depends by a few per cent on where a handle's workspace lands
+    in memory): the median handle is the value, all are listed.  Bytes: int8
+    weights + row scales, the KV rows and the embedding row."""
+    import torch
+    from decoder_greedy_decode_b200 import capi, roofline
+    from decoder_greedy_decode_b200.decoder import Decoder, quantize_int8
+    w8 = quantize_int8(wd)
+    decs = [Decoder(s, w8, max_batch=1) for _ in range(INT8_HANDLES)]
+    kv = decs[0].kv_cache(1, 928)
+    stream = torch.cuda.current_stream(dev)
+    pos = torch.tensor([N0 + (i % WINDOW) for i in range(INT8_STEPS)], dtype=torch.int32,
+                       device=dev)
+    per_handle = []
+    for dec in decs:
+        kv.values.copy_(kv_host.to(dev))
+        tok = torch.tensor([tok0], dtype=torch.int32, device=dev)
+        for i in range(5):
+            capi.dec_step(dec.h, 1, tok, pos.data_ptr() + 4 * i, kv.kv, tok, None, stream)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(INT8_STEPS + 1)]
+        torch.cuda.synchronize(dev)
+        evs[0].record(stream)
+        for i in range(INT8_STEPS):
+            capi.dec_step(dec.h, 1, tok, pos.data_ptr() + 4 * i, kv.kv, tok, None, stream)
+            evs[i + 1].record(stream)
+        torch.cuda.synchronize(dev)
+        st = dec.check()
+        if st != 0:
+            raise RuntimeError(f"int8 device status {st}")
+        per_handle.append(statistics.fmean(evs[i].elapsed_time(evs[i + 1])
+                                           for i in range(INT8_STEPS)) * 1e3)
+    for dec in decs:
+        dec.close()
+    del w8
+    us = statistics.median(per_handle)
+    nbytes = statistics.fmean(roofline.step_bytes(s, [N0 + (i % WINDOW)], weights="int8")
+                              for i in range(WINDOW))
+    peak, kind = peaks()
+    achieved = nbytes / (us * 1e-6) / 1e9
+    return {"metric": "us/token, weight-only int8", "value": us, "unit": "us/token",
+            "steps": INT8_STEPS, "dtype": "int8 weights x fp32 activations",
+            "us_per_token_per_handle": [round(v, 1) for v in per_handle],
+            "config": {"workload": "qwen3-0.6b-shape decoder, batch 1, context 795, 130-step "
+                                   "window, int8 projections + lm_head (per-row fp32 scales), "
+                                   "bf16 KV"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": f"{kind} hbm_gbs",
+                         "algorithmic_bytes_per_launch": nbytes},
+            "gpu_launches": INT8_STEPS}
+
+
 ATT_LENGTHS = (128, 795, 4096, 16384, 32768)
 ATT_BATCHES = (1, 8, 64)
 
@@ -470,6 +530,7 @@ def run_ours(args):
     # ---- the batched configuration and the isolated attention grid
     bs64 = run_bs64(s, wd, dev, ws, args.seed)
     verify = run_verify(s, wd, dev, args.seed) if rank == 0 else None
+    int8 = run_int8(s, wd, kv_host, tok0, dev, args.seed) if rank == 0 else None
     kernel_config = dec.config()
     dec.close()
     del kv, wd
@@ -510,6 +571,7 @@ def run_ours(args):
             "bs64": bs64,
             "attention": attention,
             "verify": verify,
+            "int8": int8,
         }
         if not args.no_cpu_baseline and ws == 1:
             line["cpu_baseline"] = cpu_baseline(s, w, kv_host, tok0)

@@ -28,7 +28,10 @@ EXPORTS = (
     "dec_error_string", "dec_last_cuda_error", "dec_get_config",
     "dec_attention_workspace_bytes", "dec_attention", "dec_kv_quantize_e4m3",
     "dec_attention_noalloc", "dec_verify", "dec_accept_greedy", "dec_generate",
+    "dec_init_int8", "dec_quantize_int8",
 )
+#: the projections an int8 handle holds as int8 codes + row scales
+PROJ_KEYS = ("q", "k", "v", "o", "gate", "up", "down")
 
 
 class dec_shape(ctypes.Structure):
@@ -41,6 +44,13 @@ class dec_shape(ctypes.Structure):
 class dec_weights(ctypes.Structure):
     _fields_ = [("embed", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
                 ("final_norm", ctypes.c_void_p), ("layers", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class dec_weights_int8(ctypes.Structure):
+    _fields_ = [("embed", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
+                ("lm_head_scale", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
+                ("layers", ctypes.POINTER(ctypes.c_void_p)),
+                ("scales", ctypes.POINTER(ctypes.c_void_p))]
 
 
 class dec_kv(ctypes.Structure):
@@ -89,6 +99,9 @@ def lib() -> ctypes.CDLL:
             "dec_verify": ([P, I, P, P, I, ctypes.POINTER(dec_kv), P, P, P], I),
             "dec_accept_greedy": ([I, P, P, P, ctypes.POINTER(I)], I),
             "dec_generate": ([P, I, I, P, P, ctypes.POINTER(dec_kv), P, I, P], I),
+            "dec_init_int8": ([ctypes.POINTER(dec_shape), ctypes.POINTER(dec_weights_int8),
+                               ctypes.POINTER(P)], I),
+            "dec_quantize_int8": ([P, I, I, P, P, P], I),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -128,6 +141,25 @@ def dec_init(shape: dec_shape, embed, lm_head, final_norm, layer_ptrs: Sequence[
     h = ctypes.c_void_p()
     _ok(lib().dec_init(ctypes.byref(shape), ctypes.byref(w), ctypes.byref(h)), "dec_init")
     return h.value
+
+
+def dec_init_int8(shape: dec_shape, embed, lm_head, lm_head_scale, final_norm,
+                  layer_ptrs: Sequence[int], scale_ptrs: Sequence[Optional[int]]) -> int:
+    arr = (ctypes.c_void_p * len(layer_ptrs))(*[int(p) for p in layer_ptrs])
+    sarr = (ctypes.c_void_p * len(scale_ptrs))(*[None if p is None else int(p)
+                                                 for p in scale_ptrs])
+    w = dec_weights_int8(_ptr(embed), _ptr(lm_head), _ptr(lm_head_scale), _ptr(final_norm),
+                         ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)),
+                         ctypes.cast(sarr, ctypes.POINTER(ctypes.c_void_p)))
+    h = ctypes.c_void_p()
+    _ok(lib().dec_init_int8(ctypes.byref(shape), ctypes.byref(w), ctypes.byref(h)),
+        "dec_init_int8")
+    return h.value
+
+
+def dec_quantize_int8(w, rows: int, cols: int, codes, scales, stream=None) -> None:
+    _ok(lib().dec_quantize_int8(_ptr(w), rows, cols, _ptr(codes), _ptr(scales),
+                                _stream(stream)), "dec_quantize_int8")
 
 
 def dec_free(h: int) -> None:

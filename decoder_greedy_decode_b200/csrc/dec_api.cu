@@ -36,6 +36,10 @@ struct dec_handle {
   const uint16_t* lm_head = nullptr;
   const uint16_t* final_norm = nullptr;
   LayerPtrs* layers_dev = nullptr;
+  int w8 = 0;                         // weight-only int8 handle
+  const float* lm_scale = nullptr;    // int8: lm_head row scales
+  LayerScales* scales_dev = nullptr;  // int8: projection row scales
+  int wsc_n = 0;
   uint8_t* ws = nullptr;
   WorkspaceLayout wl{};
   float* logits_dev = nullptr;
@@ -61,6 +65,25 @@ static int check_shape(const dec_shape* s) {
   return DEC_OK;
 }
 
+namespace {
+// The weights either entry point passes on (checked by the caller).
+struct InitWeights {
+  const void* embed;
+  const void* lm_head;
+  const void* final_norm;
+  const void* const* layers;
+  int w8;
+  const float* lm_scale;
+  const float* const* scales;
+};
+bool is_projection(int j) {
+  return j == DEC_LW_Q || j == DEC_LW_K || j == DEC_LW_V || j == DEC_LW_O || j == DEC_LW_GATE ||
+         j == DEC_LW_UP || j == DEC_LW_DOWN;
+}
+}  // namespace
+
+static int init_handle(const dec_shape* shape, const InitWeights& w, dec_handle** out);
+
 extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle** out) {
   if (!shape || !w || !out) return DEC_ERR_NULL;
   *out = nullptr;
@@ -74,6 +97,40 @@ extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle
     if (!w->layers[i]) return DEC_ERR_NULL;
     if (!aligned(w->layers[i], 16)) return DEC_ERR_ALIGN;
   }
+  const InitWeights iw{w->embed, w->lm_head, w->final_norm, w->layers, 0, nullptr, nullptr};
+  return init_handle(shape, iw, out);
+}
+
+extern "C" int dec_init_int8(const dec_shape* shape, const dec_weights_int8* w,
+                             dec_handle** out) {
+  if (!shape || !w || !out) return DEC_ERR_NULL;
+  *out = nullptr;
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (shape->max_batch > kMaxBatchSmall) return DEC_ERR_BATCH;
+  if (!w->embed || !w->lm_head || !w->lm_head_scale || !w->final_norm || !w->layers ||
+      !w->scales)
+    return DEC_ERR_NULL;
+  if (!aligned(w->embed, 16) || !aligned(w->lm_head, 16) || !aligned(w->final_norm, 16) ||
+      !aligned(w->lm_head_scale, 4))
+    return DEC_ERR_ALIGN;
+  const int L = shape->n_layers;
+  for (int i = 0; i < L * DEC_LW_COUNT; ++i) {
+    if (!w->layers[i]) return DEC_ERR_NULL;
+    if (!aligned(w->layers[i], 16)) return DEC_ERR_ALIGN;
+    if (is_projection(i % DEC_LW_COUNT)) {
+      if (!w->scales[i]) return DEC_ERR_NULL;
+      if (!aligned(w->scales[i], 4)) return DEC_ERR_ALIGN;
+    }
+  }
+  const InitWeights iw{w->embed, w->lm_head, w->final_norm, w->layers,
+                       1, w->lm_head_scale, w->scales};
+  return init_handle(shape, iw, out);
+}
+
+static int init_handle(const dec_shape* shape, const InitWeights& w, dec_handle** out) {
+  int rc = DEC_OK;
+  const int L = shape->n_layers;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -102,20 +159,23 @@ extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle
     return DEC_ERR_SHAPE;
   }
   const int nchunks = h->ctas + 1;
+  const int nqkv = (Hq + 2 * Hkv) * D;
+  h->w8 = w.w8;
+  h->lm_scale = w.lm_scale;
+  h->wsc_n = w.w8 ? step_wsc_slots(H, F, nqkv, shape->vocab, h->ctas) : 0;
   for (int b = 1; b <= B; ++b) {
-    h->nslot[b] = step_max_slots(b, H, F, HqD, D, rep, h->smem_optin);
+    h->nslot[b] = step_max_slots(b, H, F, HqD, D, rep, h->wsc_n, h->smem_optin);
     if (h->nslot[b] < 2) {
       delete h;
       return DEC_ERR_DEVICE;
     }
-    h->smem[b] = step_smem_bytes(h->nslot[b], b, H, F, HqD, D, rep);
+    h->smem[b] = step_smem_bytes(h->nslot[b], b, H, F, HqD, D, rep, h->wsc_n);
   }
-  h->embed = static_cast<const uint16_t*>(w->embed);
-  h->lm_head = static_cast<const uint16_t*>(w->lm_head);
-  h->final_norm = static_cast<const uint16_t*>(w->final_norm);
+  h->embed = static_cast<const uint16_t*>(w.embed);
+  h->lm_head = static_cast<const uint16_t*>(w.lm_head);
+  h->final_norm = static_cast<const uint16_t*>(w.final_norm);
 
   // ---- workspace
-  const int nqkv = (Hq + 2 * Hkv) * D;
   WorkspaceLayout& wl = h->wl;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -144,6 +204,7 @@ extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle
   wl.prof = take(sizeof(unsigned long long) * h->ctas * (16 * L + 8));
 #endif
   size_t layers_off = take(sizeof(LayerPtrs) * L);
+  size_t scales_off = w.w8 ? take(sizeof(LayerScales) * L) : 0;
   size_t logits_off = take(sizeof(float) * static_cast<size_t>(Bfull) * shape->vocab);
   wl.total = o;
   e = cudaMalloc(&h->ws, wl.total);
@@ -163,10 +224,19 @@ extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle
   std::vector<LayerPtrs> lp(L);
   for (int l = 0; l < L; ++l)
     for (int j = 0; j < DEC_LW_COUNT; ++j)
-      lp[l].w[j] = static_cast<const uint16_t*>(w->layers[l * DEC_LW_COUNT + j]);
+      lp[l].w[j] = static_cast<const uint16_t*>(w.layers[l * DEC_LW_COUNT + j]);
   h->layers_dev = reinterpret_cast<LayerPtrs*>(h->ws + layers_off);
   if (e == cudaSuccess)
     e = cudaMemcpy(h->layers_dev, lp.data(), sizeof(LayerPtrs) * L, cudaMemcpyHostToDevice);
+  if (w.w8) {
+    std::vector<LayerScales> ls(L);
+    for (int l = 0; l < L; ++l)
+      for (int j = 0; j < DEC_LW_COUNT; ++j)
+        ls[l].s[j] = is_projection(j) ? w.scales[l * DEC_LW_COUNT + j] : nullptr;
+    h->scales_dev = reinterpret_cast<LayerScales*>(h->ws + scales_off);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(h->scales_dev, ls.data(), sizeof(LayerScales) * L, cudaMemcpyHostToDevice);
+  }
   h->logits_dev = reinterpret_cast<float*>(h->ws + logits_off);
   if (e != cudaSuccess) {
     cudaFree(h->ws);
@@ -279,6 +349,10 @@ static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* 
   a.lm_head = h->lm_head;
   a.final_norm = h->final_norm;
   a.layers = h->layers_dev;
+  a.w8 = h->w8;
+  a.lm_scale = h->lm_scale;
+  a.wscale = h->scales_dev;
+  a.wsc_n = h->wsc_n;
   a.kv = static_cast<uint8_t*>(kv->base);
   a.kv_fp8 = kv->dtype == DEC_KV_FP8_E4M3;
   a.kv_scales = a.kv_fp8 ? reinterpret_cast<float*>(static_cast<uint8_t*>(kv->base) +
@@ -550,6 +624,18 @@ extern "C" int dec_kv_quantize_e4m3(const float* x, int rows, int dim, uint8_t* 
   if (dim != 64 && dim != 128) return DEC_ERR_SHAPE;
   if (rows == 0) return DEC_OK;
   cudaError_t e = launch_quantize(x, rows, dim, codes, scales, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return DEC_OK;
+}
+
+extern "C" int dec_quantize_int8(const void* w, int rows, int cols, int8_t* codes,
+                                 float* scales, void* stream) {
+  if (!w || !codes || !scales) return DEC_ERR_NULL;
+  if (rows < 0 || cols < 8 || cols % 8) return DEC_ERR_ARG;
+  if (!aligned(w, 16) || !aligned(codes, 8) || !aligned(scales, 4)) return DEC_ERR_ALIGN;
+  if (rows == 0) return DEC_OK;
+  cudaError_t e = launch_quantize_int8(static_cast<const uint16_t*>(w), rows, cols, codes, scales,
+                                       static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return DEC_OK;
 }

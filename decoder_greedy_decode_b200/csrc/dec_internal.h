@@ -15,7 +15,12 @@ constexpr int kLayerPtrs = 11;
 constexpr int kMaxBatch = 64;                       // batched step: the N of the tensor-core tiles
 
 struct LayerPtrs {
-  const uint16_t* w[kLayerPtrs];  // dec_layer_weight order
+  const uint16_t* w[kLayerPtrs];  // dec_layer_weight order (int8 codes for the
+                                  // projections of an int8 handle)
+};
+// fp32 row scales of an int8 handle's projections (norm slots unused).
+struct LayerScales {
+  const float* s[kLayerPtrs];
 };
 
 // Everything one launch of the persistent step kernel reads.
@@ -28,6 +33,12 @@ struct StepArgs {
   const uint16_t* lm_head;
   const uint16_t* final_norm;
   const LayerPtrs* layers;  // device array [L]
+  // weight-only int8: projections and lm_head are int8 codes with one fp32
+  // scale per output row (the embedding and the norm gains stay bf16)
+  int w8;
+  const float* lm_scale;        // [V]
+  const LayerScales* wscale;    // device array [L]
+  int wsc_n;                    // shared-memory scale slots (0 unless w8)
   // KV cache
   uint8_t* kv;          // values (bf16) or codes (fp8)
   float* kv_scales;     // fp8 only
@@ -67,8 +78,13 @@ struct WorkspaceLayout {
   int part_chunks;
 };
 
-size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep);
-int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int smem_optin);
+size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep, int wsc_n);
+int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int wsc_n, int smem_optin);
+// Shared-memory row-scale slots an int8 step needs: the most rows one CTA
+// computes in any stage (gate and up rows counted twice).
+int step_wsc_slots(int H, int F, int nqkv, int V, int ctas);
+cudaError_t launch_quantize_int8(const uint16_t* w, int rows, int cols, int8_t* codes,
+                                 float* scales, cudaStream_t s);
 cudaError_t launch_step_small(const StepArgs& a, int ctas, size_t smem, cudaStream_t s);
 
 // Isolated split-K decode attention.

@@ -81,12 +81,12 @@ constexpr int kMaxLayers = 64;  // layer pointer table kept in shared memory
 constexpr int kMinChunkRows = 96;
 
 struct Carve {
-  size_t ring, bars, act, stg, xown, bred, ints, lw, total;
+  size_t ring, bars, act, stg, xown, bred, ints, lw, wsc, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline Carve carve(int nslot, int B, int kmax, int D, int rep) {
+__host__ __device__ inline Carve carve(int nslot, int B, int kmax, int D, int rep, int wsc_n) {
   Carve c;
   size_t o = 0;
   c.ring = o;
@@ -107,6 +107,8 @@ __host__ __device__ inline Carve carve(int nslot, int B, int kmax, int D, int re
   o += 64 * sizeof(int);
   c.lw = o;
   o += align_up(sizeof(LayerPtrs) * kMaxLayers, 16);
+  c.wsc = o;
+  o += align_up(static_cast<size_t>(wsc_n) * sizeof(float), 16);
   c.total = o;
   return c;
 }
@@ -230,8 +232,82 @@ __device__ __noinline__ GroupSums<R, B> group_dot(const uint32_t* rows, uint32_t
   return out;
 }
 
+// Signed int8 byte j of w (given as w ^ 0x80808080, i.e. biased to code + 128)
+// as a float, exactly: the byte becomes the low mantissa bits of 2^23, so the
+// float is 2^23 + code + 128, and subtracting 2^23 + 128 leaves the code.
+__device__ __forceinline__ float i8_at(uint32_t biased, uint32_t j) {
+  return __uint_as_float(__byte_perm(biased, 0x4B000000u, 0x7540u + j)) - 8388736.0f;
+}
+__device__ __forceinline__ float dot8_i8(uint32_t w0, uint32_t w1, const float* x) {
+  const uint32_t u0 = w0 ^ 0x80808080u, u1 = w1 ^ 0x80808080u;
+  float s = i8_at(u0, 0) * x[0];
+  s = fmaf(i8_at(u0, 1), x[1], s);
+  s = fmaf(i8_at(u0, 2), x[2], s);
+  s = fmaf(i8_at(u0, 3), x[3], s);
+  s = fmaf(i8_at(u1, 0), x[4], s);
+  s = fmaf(i8_at(u1, 1), x[5], s);
+  s = fmaf(i8_at(u1, 2), x[6], s);
+  s = fmaf(i8_at(u1, 3), x[7], s);
+  return s;
+}
+
+// group_dot for int8 weight rows (row i at rows[i], K bytes): the sums of
+// code * x (the row scale is applied by the caller).  The columns go in
+// blocks of 256; lane l takes columns 4l..4l+3 and 128+4l..128+4l+3 of each
+// block, so that a warp's weight reads (4 bytes a lane) and activation reads
+// (16 bytes a lane) are contiguous and free of bank conflicts.
+template <int R, int B>
+__device__ __noinline__ GroupSums<R, B> group_dot_i8(const uint32_t* rows, uint32_t act,
+                                                     int act_stride, int nblk, int lane) {
+  float acc[R][B], acc2[R][B];
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int b = 0; b < B; ++b) acc[i][b] = acc2[i][b] = 0.f;
+#pragma unroll 2
+  for (int c = 0; c < nblk; ++c) {
+    const bool odd = c & 1;
+    const uint32_t col = static_cast<uint32_t>(c * 256 + lane * 4);
+    uint32_t w[R][2];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[i][0]) : "r"(rows[i] + col));
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[i][1]) : "r"(rows[i] + col + 128));
+    }
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      float x[8];
+      const uint32_t xa = act + static_cast<uint32_t>(b * act_stride) * 4u + col * 4u;
+      asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                   : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3]) : "r"(xa));
+      asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                   : "=f"(x[4]), "=f"(x[5]), "=f"(x[6]), "=f"(x[7]) : "r"(xa + 512));
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const float d = dot8_i8(w[i][0], w[i][1], x);
+        if (odd) acc2[i][b] += d;
+        else acc[i][b] += d;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int b = 0; b < B; ++b) acc[i][b] += acc2[i][b];
+  GroupSums<R, B> out;
+#pragma unroll
+  for (int b = 0; b < B; ++b) {
+    float col[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) col[i] = acc[i][b];
+    out.s[b] = tbfly_lane<R>(col, lane);
+  }
+  return out;
+}
+
 // The per-launch state of one CTA.  FP8: the cache holds E4M3 codes + scales.
-template <int B, int D, bool FP8>
+// W8: the projections and lm_head are int8 codes with fp32 row scales.
+template <int B, int D, bool FP8, bool W8>
 struct Cta {
   static constexpr int DL = D / 32;  // attention dims per lane
   const StepArgs& a;
@@ -245,6 +321,8 @@ struct Cta {
   int* bredi;
   int* sints;
   const LayerPtrs* slw;  // layer pointer table copied to shared memory
+  float* wsc;                               // int8: row scales of the current stage
+  static constexpr int eb = W8 ? 1 : 2;     // bytes per weight element
   int tid, warp, lane, cta, nc;
   int kmax, nqkv;
   uint32_t seq;
@@ -259,7 +337,7 @@ struct Cta {
 
   __device__ Cta(const StepArgs& args, uint8_t* smem, int kmax_) : a(args), kmax(kmax_) {
     const int rep = a.Hq / a.Hkv;
-    Carve c = carve(a.nslot, B, kmax, D, rep);
+    Carve c = carve(a.nslot, B, kmax, D, rep, a.wsc_n);
     ring = smem + c.ring;
     full = reinterpret_cast<uint64_t*>(smem + c.bars);
     empty = full + a.nslot;
@@ -270,6 +348,7 @@ struct Cta {
     bredi = reinterpret_cast<int*>(bredf + 2 * kCW * B);
     sints = reinterpret_cast<int*>(smem + c.ints);
     slw = reinterpret_cast<const LayerPtrs*>(smem + c.lw);
+    wsc = reinterpret_cast<float*>(smem + c.wsc);
     pos = sints + 8;
     tok = sints + 16;
     nchunk = sints + 24;
@@ -287,10 +366,10 @@ struct Cta {
     f1 = split_at(a.F, nc, cta + 1);
     v0 = split_at(a.V, nc, cta);
     v1 = split_at(a.V, nc, cta + 1);
-    rpt_h = kSlotBytes / (2 * a.H);
-    rpt_o = kSlotBytes / (2 * a.Hq * D);
-    rpt_u = kSlotBytes / (4 * a.H);
-    rpt_d = kSlotBytes / (2 * a.F);
+    rpt_h = kSlotBytes / (eb * a.H);
+    rpt_o = kSlotBytes / (eb * a.Hq * D);
+    rpt_u = kSlotBytes / (2 * eb * a.H);
+    rpt_d = kSlotBytes / (eb * a.F);
     if constexpr (FP8) {
       art = (kSlotBytes / (2 * D + 8)) & ~15;
     } else {
@@ -373,12 +452,17 @@ struct Cta {
       }
     };
     const int H = a.H, HqD = a.Hq * D, HkvD = a.Hkv * D;
+    const uint32_t e = static_cast<uint32_t>(eb);
+    // byte address of row r of a [rows, K] weight matrix
+    auto wrow = [&](const void* base, int r, int K) {
+      return static_cast<const uint8_t*>(base) + static_cast<size_t>(r) * K * e;
+    };
     for (int l = 0; l < a.L && !dead; ++l) {
       const LayerPtrs& lw = slw[l];
       // ---- QKV rows [q0, q1) of [Wq; Wk; Wv]
       for (int r = q0; r < q1 && !dead; r += rpt_h) {
         const int nr = min(rpt_h, q1 - r);
-        uint8_t* dst = acquire(static_cast<uint32_t>(nr) * H * 2);
+        uint8_t* dst = acquire(static_cast<uint32_t>(nr) * H * e);
         if (!dst) break;
         int rr = r, left = nr;
         while (left > 0) {
@@ -391,9 +475,8 @@ struct Cta {
           } else {
             base = lw.w[3]; lo = rr - HqD - HkvD; cnt = left;
           }
-          bulk_g2s(dst, base + static_cast<size_t>(lo) * H, static_cast<uint32_t>(cnt) * H * 2,
-                   fb, pol);
-          dst += static_cast<size_t>(cnt) * H * 2;
+          bulk_g2s(dst, wrow(base, lo, H), static_cast<uint32_t>(cnt) * H * e, fb, pol);
+          dst += static_cast<size_t>(cnt) * H * e;
           rr += cnt;
           left -= cnt;
         }
@@ -431,39 +514,36 @@ struct Cta {
       // ---- o_proj rows [h0, h1), K = Hq*D
       for (int r = h0; r < h1 && !dead; r += rpt_o) {
         const int nr = min(rpt_o, h1 - r);
-        uint8_t* dst = acquire(static_cast<uint32_t>(nr) * HqD * 2);
+        uint8_t* dst = acquire(static_cast<uint32_t>(nr) * HqD * e);
         if (!dst) break;
-        bulk_g2s(dst, lw.w[6] + static_cast<size_t>(r) * HqD, static_cast<uint32_t>(nr) * HqD * 2,
-                 fb, pol);
+        bulk_g2s(dst, wrow(lw.w[6], r, HqD), static_cast<uint32_t>(nr) * HqD * e, fb, pol);
         advance();
       }
       // ---- gate / up rows [f0, f1): a tile is nr gate rows then nr up rows
       for (int r = f0; r < f1 && !dead; r += rpt_u) {
         const int nr = min(rpt_u, f1 - r);
-        const uint32_t rb = static_cast<uint32_t>(nr) * H * 2;
+        const uint32_t rb = static_cast<uint32_t>(nr) * H * e;
         uint8_t* dst = acquire(2 * rb);
         if (!dst) break;
-        bulk_g2s(dst, lw.w[8] + static_cast<size_t>(r) * H, rb, fb, pol);
-        bulk_g2s(dst + rb, lw.w[9] + static_cast<size_t>(r) * H, rb, fb, pol);
+        bulk_g2s(dst, wrow(lw.w[8], r, H), rb, fb, pol);
+        bulk_g2s(dst + rb, wrow(lw.w[9], r, H), rb, fb, pol);
         advance();
       }
       // ---- down rows [h0, h1), K = F
       for (int r = h0; r < h1 && !dead; r += rpt_d) {
         const int nr = min(rpt_d, h1 - r);
-        uint8_t* dst = acquire(static_cast<uint32_t>(nr) * a.F * 2);
+        uint8_t* dst = acquire(static_cast<uint32_t>(nr) * a.F * e);
         if (!dst) break;
-        bulk_g2s(dst, lw.w[10] + static_cast<size_t>(r) * a.F,
-                 static_cast<uint32_t>(nr) * a.F * 2, fb, pol);
+        bulk_g2s(dst, wrow(lw.w[10], r, a.F), static_cast<uint32_t>(nr) * a.F * e, fb, pol);
         advance();
       }
     }
     // ---- lm_head rows [v0, v1)
     for (int r = v0; r < v1 && !dead; r += rpt_h) {
       const int nr = min(rpt_h, v1 - r);
-      uint8_t* dst = acquire(static_cast<uint32_t>(nr) * H * 2);
+      uint8_t* dst = acquire(static_cast<uint32_t>(nr) * H * e);
       if (!dst) break;
-      bulk_g2s(dst, a.lm_head + static_cast<size_t>(r) * H, static_cast<uint32_t>(nr) * H * 2,
-               fb, pol);
+      bulk_g2s(dst, wrow(a.lm_head, r, H), static_cast<uint32_t>(nr) * H * e, fb, pol);
       advance();
     }
     // Every copy issued must land before the CTA exits: wait for the last
@@ -658,6 +738,41 @@ struct Cta {
     csync();
   }
 
+  // int8 weights: the row scales of this CTA's rows of stage sc of layer l
+  // into wsc (cp.async, 4 bytes each), issued before the stage's input
+  // gather so that their latency overlaps it; the gather's wait and barrier
+  // complete them.  QKV: rows [q0, q1) of [Wq; Wk; Wv]; gate/up: the gate
+  // rows, then the up rows; lm_head: rows [v0, v1).
+  __device__ void load_scales(int sc, int l) {
+    const float* src0 = nullptr;
+    const float* src1 = nullptr;
+    int lo = 0, n = 0;
+    if (sc == SLM) {
+      src0 = a.lm_scale; lo = v0; n = v1 - v0;
+    } else if (sc == SQ) {
+      const LayerScales& ls = a.wscale[l];
+      const int HqD = a.Hq * D, HkvD = a.Hkv * D;
+      for (int i = tid; i < q1 - q0; i += kCT) {
+        const int r = q0 + i;
+        const float* p = r < HqD ? ls.s[1] + r
+                       : r < HqD + HkvD ? ls.s[2] + (r - HqD)
+                                        : ls.s[3] + (r - HqD - HkvD);
+        cp_async4(wsc + i, p);
+      }
+      return;
+    } else if (sc == SO) {
+      src0 = a.wscale[l].s[6]; lo = h0; n = h1 - h0;
+    } else if (sc == SU) {
+      src0 = a.wscale[l].s[8]; src1 = a.wscale[l].s[9]; lo = f0; n = f1 - f0;
+    } else {
+      src0 = a.wscale[l].s[10]; lo = h0; n = h1 - h0;
+    }
+    for (int i = tid; i < n; i += kCT) {
+      cp_async4(wsc + i, src0 + lo + i);
+      if (src1) cp_async4(wsc + n + i, src1 + lo + i);
+    }
+  }
+
   // What each projection does with its output row r of sequence b.
   __device__ __forceinline__ void epilogue(int sc, int l, int r, int b, float s0, float s1) {
     switch (sc) {
@@ -706,6 +821,7 @@ struct Cta {
   template <int R>
   __device__ void gemv(int K, int nrows, int rpt, bool pair, int sc, int l) {
     const int nv = K >> 3;
+    const uint32_t row_bytes = static_cast<uint32_t>(K * eb);
     const int per = pair ? R / 2 : R;  // output rows per group
     // A stage of many tiles (lm_head) gives each tile to one warp: only that
     // warp waits for it, computes all its groups and releases it for the
@@ -735,17 +851,29 @@ struct Cta {
           for (int i = 0; i < R; ++i) {
             const int j = gl * per + (i % per);
             const int trow = (pair && i >= per) ? nr + j : j;
-            rows[i] = smem_u32(tb) + static_cast<uint32_t>(j < nr ? trow : 0) * K * 2;
+            rows[i] = smem_u32(tb) + static_cast<uint32_t>(j < nr ? trow : 0) * row_bytes;
           }
-          const GroupSums<R, B> gs4 = group_dot<R, B>(rows, smem_u32(act), kmax, nv, lane);
+          const GroupSums<R, B> gs4 =
+              W8 ? group_dot_i8<R, B>(rows, smem_u32(act), kmax, K >> 8, lane)
+                 : group_dot<R, B>(rows, smem_u32(act), kmax, nv, lane);
           const int ri = R == 4 ? (lane >> 3) : (R == 2 ? (lane >> 4) : 0);
           const bool leader = R == 4 ? ((lane & 7) == 0) : (R == 2 ? ((lane & 15) == 0) : lane == 0);
           const int j = gl * per + ri;
+          // int8 rows: the sums are of codes; scale them by their rows' scales
+          // (gate row r0 + j, and its up row nrows + r0 + j for a pair)
+          float s0 = 1.f, s1 = 1.f;
+          if constexpr (W8) {
+            if (j < nr) {
+              s0 = wsc[r0 + j];
+              if (pair) s1 = wsc[nrows + r0 + j];
+            }
+          }
 #pragma unroll
           for (int b = 0; b < B; ++b) {
             const float sv = gs4.s[b];
             const float su = __shfl_down_sync(0xffffffffu, sv, 16);
-            if (leader && (!pair || ri < per) && j < nr && b < a.B) epilogue(sc, l, r0 + j, b, sv, su);
+            if (leader && (!pair || ri < per) && j < nr && b < a.B)
+              epilogue(sc, l, r0 + j, b, sv * s0, su * s1);
           }
         }
       }
@@ -1106,11 +1234,20 @@ struct Cta {
           src = a.x_u; K = F; fin = flag(l); nrows = h1 - h0; rpt = rpt_d; sc = SD;
         }
         if (gain) load_gains(K, gain, gr);
-        if (st == SQ && l == 0) embed_rows();
-        else gather_x(src, K, fin);
+        if constexpr (W8) load_scales(sc, l);
+        if (st == SQ && l == 0) {
+          if constexpr (W8) cp_async_wait_all();  // made visible by embed_rows' barrier
+          embed_rows();
+        } else {
+          gather_x(src, K, fin);
+        }
         if (st == SQ) DEC_STAMP(kStampsPerLayer * l + StQGath);
+        if (st == SO) DEC_STAMP(kStampsPerLayer * l + StOGath);
+        if (st == SU) DEC_STAMP(kStampsPerLayer * l + StUGath);
+        if (st == SD) DEC_STAMP(kStampsPerLayer * l + StDGath);
         if (gain) rmsnorm_act(K, gain, gr);
         if (st == SQ) DEC_STAMP(kStampsPerLayer * l + StQNorm);
+        if (st == SU) DEC_STAMP(kStampsPerLayer * l + StUNorm);
         if (pair || nrows > 2 * kCW) gemv<4>(K, nrows, rpt, pair, sc, l);
         else gemv<1>(K, nrows, rpt, pair, sc, l);
         if (st == SO) DEC_STAMP(kStampsPerLayer * l + StO);
@@ -1161,10 +1298,10 @@ struct Cta {
   }
 };
 
-template <int B, int D, bool FP8>
+template <int B, int D, bool FP8, bool W8>
 __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a, int kmax) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  Cta<B, D, FP8> c(a, smem, kmax);
+  Cta<B, D, FP8, W8> c(a, smem, kmax);
   // ---- set-up: layer pointer table, barriers, step inputs, validation
   {
     const uint64_t* src = reinterpret_cast<const uint64_t*>(a.layers);
@@ -1220,10 +1357,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
   }
 }
 
-template <int B, int D, bool FP8>
+template <int B, int D, bool FP8, bool W8>
 cudaError_t launch_bd(const StepArgs& a, int ctas, size_t smem, int kmax,
                       cudaStream_t s) {
-  auto k = step_kernel<B, D, FP8>;
+  auto k = step_kernel<B, D, FP8, W8>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -1239,16 +1376,32 @@ static int kmax_of(int H, int F, int HqD) {
   int k = H > F ? H : F;
   return k > HqD ? k : HqD;
 }
-size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep) {
-  return carve(nslot, B, kmax_of(H, F, HqD), D, rep).total;
+size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep, int wsc_n) {
+  return carve(nslot, B, kmax_of(H, F, HqD), D, rep, wsc_n).total;
 }
 
-int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int smem_optin) {
+int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int wsc_n, int smem_optin) {
   int best = 0;
   for (int n = 1; n <= 16; ++n)
-    if (step_smem_bytes(n, B, H, F, HqD, D, rep) <= static_cast<size_t>(smem_optin))
+    if (step_smem_bytes(n, B, H, F, HqD, D, rep, wsc_n) <= static_cast<size_t>(smem_optin))
       best = n;
   return best;
+}
+
+int step_wsc_slots(int H, int F, int nqkv, int V, int ctas) {
+  auto most = [&](int n) {  // the largest split_at range over the CTAs
+    int m = 0;
+    for (int i = 0; i < ctas; ++i) {
+      const int c = split_at(n, ctas, i + 1) - split_at(n, ctas, i);
+      m = c > m ? c : m;
+    }
+    return m;
+  };
+  int m = most(nqkv);
+  m = most(H) > m ? most(H) : m;
+  m = 2 * most(F) > m ? 2 * most(F) : m;
+  m = most(V) > m ? most(V) : m;
+  return m;
 }
 
 cudaError_t launch_step_small(const StepArgs& a, int ctas, size_t smem, cudaStream_t s) {
@@ -1257,8 +1410,10 @@ cudaError_t launch_step_small(const StepArgs& a, int ctas, size_t smem, cudaStre
   const bool f8 = a.kv_fp8 != 0;
 #define DEC_CASE(BB, DD)                                                            \
   if (a.B == BB && a.D == DD)                                                       \
-    return f8 ? launch_bd<BB, DD, true>(a, ctas, smem, kmax, s)                     \
-              : launch_bd<BB, DD, false>(a, ctas, smem, kmax, s);
+    return f8 ? (a.w8 ? launch_bd<BB, DD, true, true>(a, ctas, smem, kmax, s)        \
+                      : launch_bd<BB, DD, true, false>(a, ctas, smem, kmax, s))      \
+              : (a.w8 ? launch_bd<BB, DD, false, true>(a, ctas, smem, kmax, s)       \
+                      : launch_bd<BB, DD, false, false>(a, ctas, smem, kmax, s));
   DEC_CASE(1, 128) DEC_CASE(2, 128) DEC_CASE(3, 128) DEC_CASE(4, 128)
   DEC_CASE(1, 64) DEC_CASE(2, 64) DEC_CASE(3, 64) DEC_CASE(4, 64)
 #undef DEC_CASE

@@ -23,6 +23,29 @@ def to_device(w: Dict[str, object], device: str = "cuda") -> Dict[str, object]:
             "layers": [{k: t.to(device) for k, t in lw.items()} for lw in w["layers"]]}
 
 
+def quantize_int8(w: Dict[str, object]) -> Dict[str, object]:
+    """Weight-only int8 copy of device weights (to_device(...) layout): every
+    projection and lm_head quantised per output row by dec_quantize_int8
+    (codes int8 + fp32 row scales); embedding and norm gains shared."""
+    def q(t):
+        rows, cols = t.shape
+        codes = torch.empty((rows, cols), dtype=torch.int8, device=t.device)
+        scales = torch.empty(rows, dtype=torch.float32, device=t.device)
+        capi.dec_quantize_int8(t, rows, cols, codes, scales)
+        return codes, scales
+
+    layers, scales = [], []
+    for lw in w["layers"]:
+        nl, ns = dict(lw), {}
+        for key in capi.PROJ_KEYS:
+            nl[key], ns[key] = q(lw[key])
+        layers.append(nl)
+        scales.append(ns)
+    lm, lms = q(w["lm_head"])
+    return {"kind": "int8", "embed": w["embed"], "lm_head": lm, "lm_head_scale": lms,
+            "final_norm": w["final_norm"], "layers": layers, "scales": scales}
+
+
 class KVCache:
     """A caller-owned cache buffer (torch) bound through dec_kv_alloc."""
 
@@ -62,8 +85,15 @@ class Decoder:
                             shape.rope_theta, max_batch)
         ptrs = [weights["layers"][l][k].data_ptr() for l in range(shape.n_layers)
                 for k in capi.LW_ORDER]
-        self.h = capi.dec_init(cs, weights["embed"], weights["lm_head"], weights["final_norm"],
-                               ptrs)
+        if weights.get("kind") == "int8":
+            sptrs = [weights["scales"][l][k].data_ptr() if k in capi.PROJ_KEYS else None
+                     for l in range(shape.n_layers) for k in capi.LW_ORDER]
+            self.h = capi.dec_init_int8(cs, weights["embed"], weights["lm_head"],
+                                        weights["lm_head_scale"], weights["final_norm"], ptrs,
+                                        sptrs)
+        else:
+            self.h = capi.dec_init(cs, weights["embed"], weights["lm_head"],
+                                   weights["final_norm"], ptrs)
         self.max_batch = max_batch
 
     def close(self) -> None:

@@ -6,8 +6,10 @@ quick timing.
 
 Weights have the 0.6B (default) or 1.7B widths with --layers layers; every
 sequence's cache holds N(0,1) rows up to a context drawn in [lo, hi]; the
-steps feed their own ids back.  Prints the device time per step of the
---steps steps that follow --warmup untimed ones."""
+steps feed their own ids back.  --weights int8 quantises every projection and
+lm_head per row (dec_quantize_int8) and runs the weight-only int8 step
+(batch 1..4).  Prints the device time per step of the --steps steps that
+follow --warmup untimed ones."""
 from __future__ import annotations
 
 import argparse
@@ -15,7 +17,7 @@ import argparse
 import torch
 
 from . import synth
-from .decoder import Decoder, to_device
+from .decoder import Decoder, quantize_int8, to_device
 
 
 def main() -> None:
@@ -27,12 +29,16 @@ def main() -> None:
     p.add_argument("--steps", type=int, default=2)
     p.add_argument("--warmup", type=int, default=0)
     p.add_argument("--kv", choices=["bf16", "fp8"], default="bf16")
+    p.add_argument("--weights", choices=["bf16", "int8"], default="bf16")
     a = p.parse_args()
     base = synth.QWEN3_0_6B if a.shape == "0.6b" else synth.QWEN3_1_7B
     s = synth.ModelShape(a.layers, base.hidden, base.n_q_heads, base.n_kv_heads, base.head_dim,
                          base.ffn, base.vocab)
     lo, hi = (int(x) for x in a.ctx.split(","))
-    dec = Decoder(s, to_device(synth.model_weights(s, seed=2)), max_batch=a.batch)
+    w = to_device(synth.model_weights(s, seed=2))
+    if a.weights == "int8":
+        w = quantize_int8(w)
+    dec = Decoder(s, w, max_batch=a.batch)
     max_ctx = (hi + a.warmup + a.steps + 15) // 16 * 16
     kv = dec.kv_cache(a.batch, max_ctx, a.kv)
     g = torch.Generator(device="cuda").manual_seed(1)
@@ -57,7 +63,7 @@ def main() -> None:
     st = dec.check()
     if st != 0:
         raise SystemExit(f"device status {st}")
-    print(f"{a.steps} steps, batch {a.batch}, {a.layers} layers: "
+    print(f"{a.steps} steps, batch {a.batch}, {a.layers} layers, {a.weights} weights: "
           f"{e0.elapsed_time(e1) / a.steps * 1e3:.1f} us/step")
     dec.close()
 

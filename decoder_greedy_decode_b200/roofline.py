@@ -32,9 +32,24 @@ def lm_head_bytes(s) -> int:
     return s.vocab * s.hidden * BF16
 
 
-def weight_bytes(s) -> int:
-    """Every weight the step reads once: layers + lm_head + final norm."""
-    return (s.n_layers * layer_weight_params(s) + s.vocab * s.hidden + s.hidden) * BF16
+def projection_rows(s) -> int:
+    """Output rows of one layer's seven projections (q, k, v, o, gate, up, down)."""
+    nq, nkv = s.n_q_heads * s.head_dim, s.n_kv_heads * s.head_dim
+    return nq + 2 * nkv + s.hidden + 2 * s.ffn + s.hidden
+
+
+def weight_bytes(s, weights: str = "bf16") -> int:
+    """Every weight the step reads once: layers + lm_head + final norm.
+
+    weights "int8": the projections and lm_head as int8 codes (1 byte each)
+    plus one fp32 scale per output row; norm gains stay bf16."""
+    if weights == "bf16":
+        return (s.n_layers * layer_weight_params(s) + s.vocab * s.hidden + s.hidden) * BF16
+    assert weights == "int8"
+    norms = 2 * s.hidden + 2 * s.head_dim
+    proj = layer_weight_params(s) - norms
+    per_layer = proj + 4 * projection_rows(s) + norms * BF16
+    return s.n_layers * per_layer + s.vocab * s.hidden + 4 * s.vocab + s.hidden * BF16
 
 
 def kv_bytes_per_token(s, kind: str = "bf16") -> int:
@@ -43,12 +58,12 @@ def kv_bytes_per_token(s, kind: str = "bf16") -> int:
     return s.n_layers * 2 * s.n_kv_heads * per_head
 
 
-def step_bytes(s, positions: Iterable[int], kind: str = "bf16") -> int:
+def step_bytes(s, positions: Iterable[int], kind: str = "bf16", weights: str = "bf16") -> int:
     """Algorithmic bytes of one step: weights + for every sequence b the KV
     rows 0..p_b-1 read, row p_b written, and its embedding row."""
+    positions = list(positions)
     kv = sum((int(p) + 1) * kv_bytes_per_token(s, kind) for p in positions)
-    n = len(list(positions)) if not isinstance(positions, Sequence) else len(positions)
-    return weight_bytes(s) + kv + n * s.hidden * BF16
+    return weight_bytes(s, weights) + kv + len(positions) * s.hidden * BF16
 
 
 def attention_bytes(lengths: Sequence[int], n_kv_heads: int, head_dim: int,

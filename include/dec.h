@@ -137,6 +137,35 @@ typedef struct dec_handle dec_handle;
  * and DEC_ERR_DEVICE if the device is not compute capability 10.0. */
 int dec_init(const dec_shape *shape, const dec_weights *weights, dec_handle **out);
 
+/* Weight-only int8 model (faster-qwen-asr GB10 benchmark record,
+ * "cuda_graph_int8" entries of the 0.6B and 1.7B models: int8 weight-only
+ * quantisation of the text decoder and lm_head).  The seven projections of
+ * every layer (DEC_LW_Q, _K, _V, _O, _GATE, _UP, _DOWN) and lm_head are int8
+ * codes [out, in] (row-major, like the bf16 tensors they replace) with one
+ * fp32 scale per output row; the weight the step multiplies is code * scale
+ * (dec_quantize_int8 makes both from bf16).  The embedding and the norm
+ * gains stay bf16. */
+typedef struct dec_weights_int8 {
+  const void *embed;           /* bf16 [vocab, hidden] */
+  const void *lm_head;         /* int8 [vocab, hidden] codes, 16-byte aligned */
+  const float *lm_head_scale;  /* fp32 [vocab] */
+  const void *final_norm;      /* bf16 [hidden] */
+  /* HOST array of n_layers * DEC_LW_COUNT device pointers in dec_layer_weight
+   * order: bf16 norm gains, int8 codes for the projections; every pointer
+   * 16-byte aligned.  Copied by dec_init_int8. */
+  const void *const *layers;
+  /* HOST array of n_layers * DEC_LW_COUNT device pointers: the fp32 row
+   * scales [out] of each projection (4-byte aligned); the norm slots are
+   * ignored (may be NULL).  Copied by dec_init_int8. */
+  const float *const *scales;
+} dec_weights_int8;
+
+/* dec_init for a weight-only int8 model.  Same ownership and errors as
+ * dec_init; max_batch must be 1..4 (DEC_ERR_BATCH otherwise): int8 weights
+ * run on the single persistent kernel (dec_step, dec_step_host,
+ * dec_generate); dec_verify needs a bf16 handle. */
+int dec_init_int8(const dec_shape *shape, const dec_weights_int8 *weights, dec_handle **out);
+
 /* Release the handle and its workspace (synchronises the device first). */
 void dec_free(dec_handle *h);
 
@@ -338,6 +367,21 @@ int dec_attention(int batch, int n_q_heads, int n_kv_heads, int head_dim, const 
 int dec_attention_noalloc(int batch, int n_q_heads, int n_kv_heads, int head_dim, const void *q,
                           const void *k_cache, const void *v_cache, int max_len,
                           const int32_t *lengths, float *out, int *status, void *stream);
+
+/* ------------------------------------------------------------------ */
+/* int8 weights                                                        */
+/* ------------------------------------------------------------------ */
+
+/* Quantise a bf16 weight matrix w [rows, cols] (row-major, device) to int8
+ * codes [rows, cols] and one fp32 scale per row (device), the format
+ * dec_init_int8 reads: scale = amax/127 (IEEE fp32 division; 0 for a row of
+ * zeros), code = round-half-even(w/scale) (IEEE fp32 division), clamped to
+ * [-127, 127] (faster-qwen-asr GB10 record, "cuda_graph_int8": int8
+ * weight-only, per output row).  cols must be a multiple of 8 (DEC_ERR_ARG);
+ * w 16-byte, codes 8-byte and scales 4-byte aligned (DEC_ERR_ALIGN).
+ * Asynchronous on `stream`. */
+int dec_quantize_int8(const void *w, int rows, int cols, int8_t *codes, float *scales,
+                      void *stream);
 
 /* ------------------------------------------------------------------ */
 /* FP8 cache rows                                                      */

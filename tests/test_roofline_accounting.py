@@ -32,3 +32,14 @@ def test_step_bytes_0_6b_ctx_795():
 
 def test_step_bytes_1_7b():
     assert roofline.weight_bytes(synth.QWEN3_1_7B) == 3_441_149_952
+
+
+def test_int8_weight_bytes_0_6b():
+    """Weight-only int8: 28 x (15,728,640 projection codes + 12,288 row scales
+    x 4 + 2,304 bf16 gains x 2) + lm_head (151,936 x 1,024 codes + 151,936 x 4)
+    + the final norm (1,024 x 2)."""
+    s = synth.QWEN3_0_6B
+    assert roofline.projection_rows(s) == 12_288
+    assert roofline.weight_bytes(s, "int8") == 28 * 15_782_400 + 156_190_208 + 2_048
+    assert roofline.step_bytes(s, [795], weights="int8") == (
+        598_099_456 + 796 * 114_688 + 2048)
