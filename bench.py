@@ -80,9 +80,10 @@ def peaks():
     return 6650.0, "fallback"
 
 
-def ncu_traffic():
-    """Per-launch DRAM bytes of the step kernel from the committed ncu summary."""
-    path = os.path.join(ROOT, "profiles", "step_kernel_0p6b_bs1_ctx795.json")
+def ncu_traffic(summary="step_kernel_0p6b_bs1_ctx795"):
+    """Per-launch DRAM bytes of the step kernel from the committed ncu summary
+    (null once the kernel's sources have changed since the capture)."""
+    path = os.path.join(ROOT, "profiles", summary + ".json")
     if os.path.exists(path):
         d = json.load(open(path))
         if d.get("kernel_source_hash") == source_hash():
@@ -322,8 +323,9 @@ def run_int8(s, wd, kv_host, tok0, dev, seed):
                                    "bf16 KV"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_source": f"{kind} hbm_gbs",
+                         "traffic": ncu_traffic("step_kernel_int8_0p6b_bs1_ctx795"),
                          "algorithmic_bytes_per_launch": nbytes},
-            "gpu_launches": INT8_STEPS}
+            "gpu_launches": INT8_STEPS * INT8_HANDLES}
 
 
 ATT_LENGTHS = (128, 795, 4096, 16384, 32768)
