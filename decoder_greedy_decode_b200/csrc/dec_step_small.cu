@@ -7,7 +7,7 @@
 // step launch-bound (~300 attention kernels per token, 07 Root causes); here
 // there is one launch per step and no host involvement inside it.
 //
-// Structure (one CTA per SM, 8 consumer warps + 1 producer warp):
+// Structure (one CTA per SM, 7 consumer warps + 1 producer warp):
 //  * Every weight and KV byte the CTA will need is known before the step
 //    starts, independent of activations.  The producer warp streams them with
 //    1-D bulk copies (TMA engine) into a ring of 24 KB shared-memory slots,
@@ -21,8 +21,9 @@
 //  * Rows of every projection are split evenly over CTAs.  Each CTA owns the
 //    same hidden rows in o_proj and down, so it keeps those residual entries
 //    in shared memory.  Attention is split-K over (sequence, KV head, chunk)
-//    items; the last CTA to finish a (sequence, KV head) merges the partials
-//    (flash-decoding combine) and publishes the head outputs.
+//    items; the CTA of chunk 0 of a (sequence, KV head) gathers the other
+//    chunks' partials as they are published, merges them (flash-decoding
+//    combine) and publishes the head outputs.
 //  * Every wait is bounded (globaltimer).  A wait that runs out raises a
 //    status bit and a global abort flag; all CTAs then drain their in-flight
 //    copies without computing and leave; out_ids becomes -1.
@@ -145,13 +146,17 @@ __device__ __forceinline__ float dot8(const uint4 w, const float* x) {
   return s;
 }
 
-// Dot products of R weight rows (shared memory, rows row_bytes apart, row i
-// at rows[i]) with the activation rows of B sequences (shared memory, act_stride
-// floats apart), K = 8 * nv columns; lane l takes 16-byte column vectors l,
-// l + 32, ...  Returns the transposed-butterfly reduction: every lane gets the
-// full sum of row (R == 4: lane >> 3; R == 2: lane >> 4; R == 1: 0) for each b.
-// Compiled on its own (not inlined) so that its register allocation and
-// scheduling do not depend on the rest of the persistent kernel.
+// Dot products of R weight rows (shared memory, row i at rows[i]) with the
+// activation rows of B sequences (shared memory, act_stride floats apart),
+// K = 256 * nblk columns (group_dot: bf16 rows, group_dot_i8: int8 codes).
+// The columns go in blocks of 256; lane l takes columns 4l..4l+3 and
+// 128+4l..128+4l+3 of each block, so that a warp's weight reads (8 or 4
+// bytes a lane) and activation reads (16 bytes a lane) are contiguous and
+// free of bank conflicts.  Returns the transposed-butterfly reduction: every
+// lane gets the full sum of row (R == 4: lane >> 3; R == 2: lane >> 4;
+// R == 1: 0) for each b.  Compiled on their own (not inlined) so that their
+// register allocation and scheduling do not depend on the rest of the
+// persistent kernel.
 template <int R, int B>
 struct GroupSums {
   float s[B];
@@ -182,56 +187,6 @@ __device__ __forceinline__ float tbfly_lane(float (&p)[R], int lane) {
   }
 }
 
-template <int R, int B>
-__device__ __noinline__ GroupSums<R, B> group_dot(const uint32_t* rows, uint32_t act, int act_stride,
-                                                  int nv, int lane) {
-  // two accumulator banks (even / odd column vectors): twice the independent
-  // FMA chains
-  float acc[R][B], acc2[R][B];
-#pragma unroll
-  for (int i = 0; i < R; ++i)
-#pragma unroll
-    for (int b = 0; b < B; ++b) acc[i][b] = acc2[i][b] = 0.f;
-#pragma unroll 2
-  for (int v = lane; v < nv; v += 32) {
-    const bool odd = (v >> 5) & 1;
-    float x[B][8];
-#pragma unroll
-    for (int b = 0; b < B; ++b) {
-      const uint32_t xa = act + static_cast<uint32_t>(b * act_stride + v * 8) * 4u;
-      asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
-                   : "=f"(x[b][0]), "=f"(x[b][1]), "=f"(x[b][2]), "=f"(x[b][3]) : "r"(xa));
-      asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
-                   : "=f"(x[b][4]), "=f"(x[b][5]), "=f"(x[b][6]), "=f"(x[b][7]) : "r"(xa + 16));
-    }
-#pragma unroll
-    for (int i = 0; i < R; ++i) {
-      uint4 w;
-      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                   : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w) : "r"(rows[i] + v * 16));
-#pragma unroll
-      for (int b = 0; b < B; ++b) {
-        const float d = dot8(w, x[b]);
-        if (odd) acc2[i][b] += d;
-        else acc[i][b] += d;
-      }
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < R; ++i)
-#pragma unroll
-    for (int b = 0; b < B; ++b) acc[i][b] += acc2[i][b];
-  GroupSums<R, B> out;
-#pragma unroll
-  for (int b = 0; b < B; ++b) {
-    float col[R];
-#pragma unroll
-    for (int i = 0; i < R; ++i) col[i] = acc[i][b];
-    out.s[b] = tbfly_lane<R>(col, lane);
-  }
-  return out;
-}
-
 // Signed int8 byte j of w (given as w ^ 0x80808080, i.e. biased to code + 128)
 // as a float, exactly: the byte becomes the low mantissa bits of 2^23, so the
 // float is 2^23 + code + 128, and subtracting 2^23 + 128 leaves the code.
@@ -251,11 +206,7 @@ __device__ __forceinline__ float dot8_i8(uint32_t w0, uint32_t w1, const float* 
   return s;
 }
 
-// group_dot for int8 weight rows (row i at rows[i], K bytes): the sums of
-// code * x (the row scale is applied by the caller).  The columns go in
-// blocks of 256; lane l takes columns 4l..4l+3 and 128+4l..128+4l+3 of each
-// block, so that a warp's weight reads (4 bytes a lane) and activation reads
-// (16 bytes a lane) are contiguous and free of bank conflicts.
+// int8 rows (K bytes): the sums of code * x; the caller applies the row scale.
 template <int R, int B>
 __device__ __noinline__ GroupSums<R, B> group_dot_i8(const uint32_t* rows, uint32_t act,
                                                      int act_stride, int nblk, int lane) {
@@ -285,6 +236,59 @@ __device__ __noinline__ GroupSums<R, B> group_dot_i8(const uint32_t* rows, uint3
 #pragma unroll
       for (int i = 0; i < R; ++i) {
         const float d = dot8_i8(w[i][0], w[i][1], x);
+        if (odd) acc2[i][b] += d;
+        else acc[i][b] += d;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int b = 0; b < B; ++b) acc[i][b] += acc2[i][b];
+  GroupSums<R, B> out;
+#pragma unroll
+  for (int b = 0; b < B; ++b) {
+    float col[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) col[i] = acc[i][b];
+    out.s[b] = tbfly_lane<R>(col, lane);
+  }
+  return out;
+}
+
+// bf16 rows (2K bytes).
+template <int R, int B>
+__device__ __noinline__ GroupSums<R, B> group_dot(const uint32_t* rows, uint32_t act,
+                                                    int act_stride, int nblk, int lane) {
+  float acc[R][B], acc2[R][B];
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int b = 0; b < B; ++b) acc[i][b] = acc2[i][b] = 0.f;
+#pragma unroll 2
+  for (int c = 0; c < nblk; ++c) {
+    const bool odd = c & 1;
+    const uint32_t col = static_cast<uint32_t>(c * 256 + lane * 4);
+    uint2 w[R][2];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
+                   : "=r"(w[i][0].x), "=r"(w[i][0].y) : "r"(rows[i] + col * 2));
+      asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
+                   : "=r"(w[i][1].x), "=r"(w[i][1].y) : "r"(rows[i] + col * 2 + 256));
+    }
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      float x[8];
+      const uint32_t xa = act + static_cast<uint32_t>(b * act_stride) * 4u + col * 4u;
+      asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                   : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3]) : "r"(xa));
+      asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                   : "=f"(x[4]), "=f"(x[5]), "=f"(x[6]), "=f"(x[7]) : "r"(xa + 512));
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const uint4 wv = make_uint4(w[i][0].x, w[i][0].y, w[i][1].x, w[i][1].y);
+        const float d = dot8(wv, x);
         if (odd) acc2[i][b] += d;
         else acc[i][b] += d;
       }
@@ -820,7 +824,6 @@ struct Cta {
   // ring ahead of the others) and releases it.
   template <int R>
   __device__ void gemv(int K, int nrows, int rpt, bool pair, int sc, int l) {
-    const int nv = K >> 3;
     const uint32_t row_bytes = static_cast<uint32_t>(K * eb);
     const int per = pair ? R / 2 : R;  // output rows per group
     // A stage of many tiles (lm_head) gives each tile to one warp: only that
@@ -855,7 +858,7 @@ struct Cta {
           }
           const GroupSums<R, B> gs4 =
               W8 ? group_dot_i8<R, B>(rows, smem_u32(act), kmax, K >> 8, lane)
-                 : group_dot<R, B>(rows, smem_u32(act), kmax, nv, lane);
+                 : group_dot<R, B>(rows, smem_u32(act), kmax, K >> 8, lane);
           const int ri = R == 4 ? (lane >> 3) : (R == 2 ? (lane >> 4) : 0);
           const bool leader = R == 4 ? ((lane & 7) == 0) : (R == 2 ? ((lane & 15) == 0) : lane == 0);
           const int j = gl * per + ri;
