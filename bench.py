@@ -13,8 +13,12 @@ One step = one dec_step launch (the whole hot path).  Prints one JSON line.
 The line also carries a "bs64" object: the same decoder serving 64
 sequences at once (contexts drawn in [200, 420], a 128-step window; the
 Baseten Qwen3-ASR article, "KV cache quantization": many concurrent
-30-second windows), in tokens/s, through the batched tensor-core step.
-`--impl reference` times the CPU oracle on a bounded sample instead.
+30-second windows), in tokens/s, through the batched tensor-core step; a
+"verify" object (block verification, "Can CTC make Qwen3-ASR faster?", 11
+Phase A); an "int8" object (the batch-1 workload with weight-only int8
+projections and lm_head, faster-qwen-asr GB10 record, "cuda_graph_int8");
+and an "attention" object (isolated decode attention over a length x batch
+grid).  `--impl reference` times the CPU oracle on a bounded sample instead.
 """
 from __future__ import annotations
 

@@ -19,6 +19,8 @@
  *     lengths are owned by the host; no step reads device data back) and
  *     "KV cache quantization" (an FP8 cache, attention math in full
  *     precision).
+ *   - faster-qwen-asr GB10 benchmark record, "cuda_graph_int8" entries
+ *     (int8 weight-only text decoder and lm_head: dec_init_int8).
  *
  * Conventions.  Every pointer is a DEVICE pointer unless its comment says
  * "host".  `stream` is a cudaStream_t (NULL = the legacy default stream).
@@ -45,7 +47,9 @@
  *   - argmax ties go to the lowest token id;
  *   - FP8 cache: OCP E4M3 codes with one fp32 scale per (layer, K/V, sequence,
  *     KV head, token): scale = max(amax, 2^-126)/448, code = RNE-satfinite of
- *     x/scale, both in fp32.
+ *     x/scale, both in fp32;
+ *   - int8 weights: one fp32 scale per output row, scale = amax/127,
+ *     code = round-half-even(w/scale), both in fp32, clamped to [-127, 127].
  */
 #ifndef DEC_H
 #define DEC_H
