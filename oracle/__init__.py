@@ -342,3 +342,37 @@ class Model:
                             _p(k16), _p(k8), _p(ks), cache.max_ctx, int(token), int(pos),
                             _p(logits), _p(hidden), _p(nk), _p(nv), ctypes.byref(margin))
         return StepResult(int(tok), float(margin.value), logits, hidden, nk, nv)
+
+
+# ------------------------------------------------- input marshalling helpers
+# Views of the seeded synthetic inputs (torch tensors from the input
+# generators) in the oracle's numpy form: raw bytes only, no arithmetic.
+
+def _bits16(t) -> np.ndarray:
+    """The raw 16-bit patterns of a bf16 torch tensor as numpy uint16."""
+    import torch
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def shape_from(s) -> Shape:
+    """A model shape (any object with the Shape field names) as a Shape."""
+    return Shape(s.n_layers, s.hidden, s.n_q_heads, s.n_kv_heads, s.head_dim, s.ffn, s.vocab,
+                 s.rms_eps, s.rope_theta)
+
+
+def weights_from(w) -> Weights:
+    """{"embed", "lm_head", "final_norm", "layers": [dict per layer]} of bf16
+    torch tensors as Weights of uint16 bit patterns."""
+    layers = [{k: _bits16(t) for k, t in lw.items()} for lw in w["layers"]]
+    return Weights(embed=_bits16(w["embed"]), lm_head=_bits16(w["lm_head"]),
+                   final_norm=_bits16(w["final_norm"]), layers=layers)
+
+
+def cache_from(kv, scales, b: int) -> Cache:
+    """Sequence b of a [L, 2, B, Hkv, max_ctx, D] cache (bf16 values, or E4M3
+    codes with fp32 scales [L, 2, B, Hkv, max_ctx]) as a Cache (a copy)."""
+    if scales is None:
+        return Cache("bf16", np.ascontiguousarray(_bits16(kv[:, :, b])))
+    codes = np.ascontiguousarray(kv[:, :, b].cpu().numpy())
+    sc = np.ascontiguousarray(scales[:, :, b].cpu().numpy())
+    return Cache("fp8", codes, sc)

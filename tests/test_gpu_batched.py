@@ -247,6 +247,14 @@ def test_0p6b_bs64_ragged(big06):
     _full_size(s, w, wd, 64, lengths, 432, "bf16", sampled, steps=2, seed=71)
 
 
+def test_0p6b_bs64_every_sequence_one_step(big06):
+    """0.6B shape, 64 sequences, contexts U[200, 420]: every sequence of the
+    batch against the oracle for one step."""
+    s, w, wd = big06
+    lengths = synth.ragged_lengths(200, 420, 64, seed=74)
+    _full_size(s, w, wd, 64, lengths, 432, "bf16", list(range(64)), steps=1, seed=75)
+
+
 @pytest.fixture(scope="module")
 def big17():
     s = synth.QWEN3_1_7B

@@ -185,8 +185,8 @@ def big06_int8():
 
 def test_0p6b_int8_bs1_ctx795(big06_int8):
     """The 0.6B shape with int8 weights, batch 1, 795 prefilled rows: the
-    codes of every projection equal the oracle's, and three teacher-forced
-    steps match the oracle's int8 model."""
+    codes of every projection equal the oracle's, and the 130 teacher-forced
+    steps of the window match the oracle's int8 model."""
     s, w, m = big06_int8
     wd = to_device(w)
     w8 = quantize_int8(wd)
@@ -200,18 +200,19 @@ def test_0p6b_int8_bs1_ctx795(big06_int8):
     del wd
     dec = Decoder(s, w8, 1)
     n0 = 795
-    kv_host, _ = synth.kv_prefill(s, 1, 800, [n0], seed=3)
+    kv_host, _ = synth.kv_prefill(s, 1, 928, [n0], seed=3)
     cache = oracle_cache(kv_host, None, 0)
-    kv = dec.kv_cache(1, 800)
+    kv = dec.kv_cache(1, 928)
     kv.values.copy_(kv_host.cuda())
     tok = int(synth.tokens(s.vocab, 1, seed=4)[0])
-    for t in range(3):
+    # the whole 130-token window (positions 795 .. 924), teacher-forced
+    for t in range(130):
         p = n0 + t
         r = m.step(cache, tok, p, want_hidden=True)
         ids, logits, hid = _step(dec, kv, [tok], [p])
         tag = f"0.6B int8 p={p}"
         assert_close(logits[0], r.logits, tag + " logits")
-        for l in (0, 1, 14, 27, 28):
+        for l in range(s.n_layers + 1):
             assert_close(hid[l, 0], r.hidden[l], tag + f" hidden {l}")
         assert_id(int(ids[0]), r, tag)
         _check_kv_row(kv, cache, 0, p, tag)

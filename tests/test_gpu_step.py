@@ -266,6 +266,67 @@ def test_0p6b_bs1_ctx795_teacher_forced(big06):
     dec.close()
 
 
+def test_0p6b_bs1_window_130_teacher_forced(big06):
+    """The whole 130-token window of the 0.6B workload ("Qwen3-ASR -- Latency &
+    Bottleneck Analysis", 01 Method & setup: 795 prompt tokens, then 130
+    generated), positions 795 .. 924, teacher-forced: every step's logits,
+    every layer's residual stream, the emitted id and the appended cache row
+    against the oracle."""
+    s, w, m, wd = big06
+    dec = Decoder(s, wd, 1)
+    kv_host, _ = synth.kv_prefill(s, 1, 928, [795], seed=3)
+    cache = oracle_cache(kv_host, None, 0)
+    kv = dec.kv_cache(1, 928)
+    kv.values.copy_(kv_host.cuda())
+    tok = int(synth.tokens(s.vocab, 1, seed=4)[0])
+    worst = (0.0, 0.0)
+    for t in range(130):
+        p = 795 + t
+        r = m.step(cache, tok, p, want_hidden=True)
+        ids, logits, hid = _gpu_step(dec, kv, [tok], [p])
+        tag = f"0.6B window p={p}"
+        ma, rl = assert_close(logits[0], r.logits, tag + " logits")
+        worst = (max(worst[0], ma), max(worst[1], rl))
+        for l in range(s.n_layers + 1):
+            assert_close(hid[l, 0], r.hidden[l], tag + f" hidden {l}")
+        assert_id(int(ids[0]), r, tag)
+        _check_kv_row(kv, cache, 0, p, tag)
+        tok = r.token
+    print(f"130-step window: worst logits max-abs {worst[0]:.3g}, rel-L2 {worst[1]:.3g}")
+    del kv
+    dec.close()
+
+
+def test_0p6b_bs1_free_running_follows_oracle_greedy(big06):
+    """The device feeds its own ids back (out_ids aliases token_ids) from
+    position 795; the ids equal the oracle's own greedy sequence up to the
+    oracle's first near-tie (top-2 margin below 1e-2), after which the two
+    may legitimately part."""
+    s, w, m, wd = big06
+    dec = Decoder(s, wd, 1)
+    kv_host, _ = synth.kv_prefill(s, 1, 928, [795], seed=3)
+    cache = oracle_cache(kv_host, None, 0)
+    kv = dec.kv_cache(1, 928)
+    kv.values.copy_(kv_host.cuda())
+    tok = int(synth.tokens(s.vocab, 1, seed=4)[0])
+    buf = i32([tok])
+    n = 0
+    for t in range(130):
+        p = 795 + t
+        r = m.step(cache, tok, p)
+        dec.step(kv, buf, i32([p]), buf)
+        assert dec.check() == 0
+        if r.margin < 1e-2:
+            break
+        assert int(buf[0]) == r.token, f"free-running step {t} (p={p})"
+        tok = r.token
+        n += 1
+    assert n >= 1
+    print(f"free-running: {n} steps equal to the oracle's greedy ids before its first near-tie")
+    del kv
+    dec.close()
+
+
 def test_0p6b_batch4_ragged(big06):
     s, w, m, wd = big06
     dec = Decoder(s, wd, 4)
