@@ -209,15 +209,12 @@ def run_bs64(s, wd, dev, ws, seed):
                               for i in range(BS64_STEPS))
     peak, kind = peaks()
     achieved = nbytes / (step_ms * 1e-3) / 1e9
-    return {"metric": "tokens/s at bs64", "value": replica_throughput(BS64, step_ms, ws),
-            "unit": "tokens/s", "ms_per_step": step_ms, "steps": BS64_STEPS,
-            "config": {"workload": "qwen3-0.6b-shape decoder, batch 64, contexts U[200,420], "
-                                   "128-step window, bf16 KV", "batch": BS64,
-                       "max_ctx": max_ctx},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_source": f"{kind} hbm_gbs",
-                         "algorithmic_bytes_per_step": nbytes},
-            "gpu_launches_per_step": 1 + 5 * s.n_layers + 2}
+    return {"value": round(replica_throughput(BS64, step_ms, ws), 1), "unit": "tokens/s",
+            "ms_per_step": round(step_ms, 4), "steps": BS64_STEPS,
+            "workload": "0.6b, batch 64, contexts U[200,420], bf16 KV",
+            "roofline": {"achieved": round(achieved, 1), "peak": peak,
+                         "frac": round(achieved / peak, 4)},
+            "launches_per_step": 1 + 5 * s.n_layers + 2}
 
 
 VERIFY_BLOCKS = (1, 2, 4, 8, 16, 32)
@@ -258,17 +255,14 @@ def run_verify(s, wd, dev, seed):
         us = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs) * 1e3
         nbytes = (roofline.weight_bytes(s) + (N0 + k) * roofline.kv_bytes_per_token(s)
                   + k * s.hidden * 2)
-        cells.append({"k": k, "us_per_call": round(us, 1), "us_per_token_full_accept": round(us / k, 1),
-                      "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1)})
+        cells.append((k, round(us, 1), round(us / k, 1), round(nbytes / (us * 1e-6) / 1e9, 1)))
     st = dec.check()
     dec.close()
     if st != 0:
         raise RuntimeError(f"verify device status {st}")
-    return {"metric": "block verification: us per dec_verify call and per committed token "
-                      "at full acceptance", "peak": peak, "peak_source": f"{kind} hbm_gbs",
-            "config": {"workload": "qwen3-0.6b-shape decoder, one sequence, context 795, "
-                                   "blocks of k tokens (batched tensor-core step)"},
-            "cells": cells}
+    return {"workload": "0.6b, one sequence, context 795, blocks of k tokens",
+            "k": [c[0] for c in cells], "us_per_call": [c[1] for c in cells],
+            "us_per_token_full_accept": [c[2] for c in cells], "GB/s": [c[3] for c in cells]}
 
 
 INT8_STEPS = 260
@@ -319,17 +313,12 @@ def run_int8(s, wd, kv_host, tok0, dev, seed):
                               for i in range(WINDOW))
     peak, kind = peaks()
     achieved = nbytes / (us * 1e-6) / 1e9
-    return {"metric": "us/token, weight-only int8", "value": us, "unit": "us/token",
-            "steps": INT8_STEPS, "dtype": "int8 weights x fp32 activations",
-            "us_per_token_per_handle": [round(v, 1) for v in per_handle],
-            "config": {"workload": "qwen3-0.6b-shape decoder, batch 1, context 795, 130-step "
-                                   "window, int8 projections + lm_head (per-row fp32 scales), "
-                                   "bf16 KV"},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_source": f"{kind} hbm_gbs",
-                         "traffic": ncu_traffic("step_kernel_int8_0p6b_bs1_ctx795"),
-                         "algorithmic_bytes_per_launch": nbytes},
-            "gpu_launches": INT8_STEPS * INT8_HANDLES}
+    return {"value": round(us, 1), "unit": "us/token",
+            "workload": "0.6b, batch 1, ctx 795 window, int8 projections + lm_head",
+            "us_per_handle": [round(v, 1) for v in per_handle],
+            "roofline": {"achieved": round(achieved, 1), "peak": peak,
+                         "frac": round(achieved / peak, 4),
+                         "traffic": ncu_traffic("step_kernel_int8_0p6b_bs1_ctx795")}}
 
 
 ATT_LENGTHS = (128, 795, 4096, 16384, 32768)
@@ -378,24 +367,149 @@ def run_attention_grid(dev, seed):
             us = statistics.median(times) * 1e3
             nbytes = roofline.attention_bytes(lengths, Hkv, D, Hq)
             gbs = nbytes / (us * 1e-6) / 1e9
-            cells.append({"L": L, "B": B, "us": round(us, 2), "GB/s": round(gbs, 1),
-                          "frac": round(gbs / peak, 4), "bytes": nbytes})
+            cells.append([L, B, round(us, 2), round(gbs / peak, 4)])
             del k, v, q, out, ws
     del flush
-    return {"metric": "isolated GQA decode attention, us/call and GB/s per (L, B) cell",
-            "peak": peak, "peak_source": f"{kind} hbm_gbs", "unit": "GB/s",
-            "config": {"workload": "16 q / 8 kv heads, D 128, bf16 K/V N(0,1), lengths U[L/2, L]",
-                       "l2": "flushed between calls (1 GiB write)"},
-            "cells": cells}
+    return {"workload": "16 q / 8 kv heads, D 128, bf16 K/V, lengths U[L/2, L], L2 flushed",
+            "peak": peak, "cells [L, B, us, frac]": cells}
+
+
+def device_weights(s, dev, seed):
+    """Random-init bf16 weights of shape s drawn on the device (N(0, 0.02),
+    gains 1): the timing-only configurations have no oracle leg."""
+    import torch
+    from decoder_greedy_decode_b200 import synth
+    g = torch.Generator(device=dev).manual_seed(seed)
+
+    def n(*shape):
+        return (torch.randn(shape, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+
+    shp = synth.layer_shapes(s)
+    layers = [{k: (torch.ones(v, dtype=torch.bfloat16, device=dev) if len(v) == 1 else n(*v))
+               for k, v in shp.items()} for _ in range(s.n_layers)]
+    return {"embed": n(s.vocab, s.hidden), "lm_head": n(s.vocab, s.hidden),
+            "final_norm": torch.ones(s.hidden, dtype=torch.bfloat16, device=dev),
+            "layers": layers}
+
+
+def fill_cache(kv, kind, dev, seed):
+    import torch
+    g = torch.Generator(device=dev).manual_seed(seed)
+    if kind == "bf16":
+        kv.values.normal_(generator=g)
+    else:
+        z = torch.randn(kv.codes.shape, generator=g, device=dev) * 32.0
+        kv.codes.copy_(z.to(torch.float8_e4m3fn).view(torch.uint8))
+        kv.scales.uniform_(0.02, 0.04, generator=g)
+
+
+CFG5_BS1_CTX, CFG5_BS1_STEPS = 3968, 20
+CFG5_BS64_LO, CFG5_BS64_HI, CFG5_BS64_STEPS = 2048, 4064, 10
+
+
+def run_cfg5(dev, ws, seed):
+    """The 1.7B-shaped decoder (28 layers, hidden 2048, 16/8 heads of 128,
+    FFN 6144): batch 1 at context ~4000 and batch 64 with contexts U[2048,
+    4064], each with a bf16 and an E4M3 cache (Baseten Qwen3-ASR article,
+    "KV cache quantization": 64 concurrent 1.7B requests, FP8 KV).  Device
+    time per step (CUDA events over the steps after 3 warm-ups), tokens/s
+    and the fraction of the HBM roofline over the algorithmic bytes."""
+    import torch
+    from decoder_greedy_decode_b200 import roofline, synth
+    from decoder_greedy_decode_b200.decoder import Decoder
+    s = synth.QWEN3_1_7B
+    wd = device_weights(s, dev, seed + 40)
+    peak, kind_src = peaks()
+    stream = torch.cuda.current_stream(dev)
+    out = {"workload": "qwen3-1.7b-shape decoder (random-init bf16 weights)",
+           "peak_source": f"{kind_src} hbm_gbs"}
+    for batch in (1, 64):
+        dec = Decoder(s, wd, max_batch=batch)
+        if batch == 1:
+            lengths, steps = [CFG5_BS1_CTX], CFG5_BS1_STEPS
+        else:
+            lengths = synth.ragged_lengths(CFG5_BS64_LO, CFG5_BS64_HI, 64, seed=seed + 41)
+            steps = CFG5_BS64_STEPS
+        max_ctx = (max(lengths) + steps + 3 + 15) // 16 * 16
+        for kind in ("bf16", "fp8"):
+            kv = dec.kv_cache(batch, max_ctx, kind)
+            fill_cache(kv, kind, dev, seed + 42)
+            base = torch.tensor(lengths, dtype=torch.int32, device=dev)
+            pos = [base + i for i in range(steps + 3)]
+            tok = torch.randint(0, s.vocab, (batch,), dtype=torch.int32, device=dev)
+            for i in range(3):
+                dec.step(kv, tok, pos[i], tok, None, stream)
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(steps):
+                dec.step(kv, tok, pos[3 + i], tok, None, stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            st = dec.check()
+            if st != 0:
+                raise RuntimeError(f"cfg5 device status {st}")
+            ms = max_over_ranks([e0.elapsed_time(e1)], dev, ws)[0] / steps
+            nbytes = statistics.fmean(
+                roofline.step_bytes(s, [n + 3 + i for n in lengths], kind=kind)
+                for i in range(steps))
+            frac = nbytes / (ms * 1e-3) / 1e9 / peak
+            key = f"bs{batch}_{kind}"
+            if batch == 1:
+                out[key] = {"us_per_token": round(ms * 1e3, 1), "frac": round(frac, 4),
+                            "ctx": lengths[0]}
+            else:
+                out[key] = {"tokens_per_s": round(replica_throughput(batch, ms, ws), 1),
+                            "ms_per_step": round(ms, 3), "frac": round(frac, 4),
+                            "ctx": [CFG5_BS64_LO, CFG5_BS64_HI]}
+            del kv
+        dec.close()
+    del wd
+    torch.cuda.empty_cache()
+    return out
+
+
+GEN_STEPS = 130
+
+
+def run_generate(s, wd, kv_host, tok0, dev):
+    """dec_generate on the batch-1 workload: the 130-token window from
+    position 795 in one call (ids fed back and positions advanced on the
+    device); device time per generated token over 3 calls after one warm-up
+    call."""
+    import torch
+    from decoder_greedy_decode_b200.decoder import Decoder
+    dec = Decoder(s, wd, max_batch=1)
+    kv = dec.kv_cache(1, 928)
+    stream = torch.cuda.current_stream(dev)
+    out = torch.empty((GEN_STEPS, 1), dtype=torch.int32, device=dev)
+    times = []
+    for rep in range(4):
+        kv.values.copy_(kv_host.to(dev))
+        tok = torch.tensor([tok0], dtype=torch.int32, device=dev)
+        pos = torch.tensor([N0], dtype=torch.int32, device=dev)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        dec.generate(kv, tok, pos, out, -1, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if rep > 0:
+            times.append(e0.elapsed_time(e1))
+    st = dec.check()
+    dec.close()
+    if st != 0:
+        raise RuntimeError(f"generate device status {st}")
+    ms = statistics.median(times)
+    return {"us_per_token": round(ms * 1e3 / GEN_STEPS, 1), "steps_per_call": GEN_STEPS,
+            "ms_per_call": round(ms, 3)}
 
 
 def cpu_baseline(s, w, kv_host, tok0, budget_s=20.0):
     """The CPU oracle, as it stands, on a bounded sample of the same workload."""
     import oracle
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from conftest import oracle_cache, oracle_shape, oracle_weights
-    m = oracle.Model(oracle_shape(s), oracle_weights(w))
-    cache = oracle_cache(kv_host, None, 0)
+    m = oracle.Model(oracle.shape_from(s), oracle.weights_from(w))
+    cache = oracle.cache_from(kv_host, None, 0)
     tok, n, t0 = tok0, 0, time.perf_counter()
     while n < WINDOW:
         r = m.step(cache, tok, N0 + n)
@@ -422,12 +536,10 @@ def run_reference(args):
     # warm-up and timed steps, bounded so that the run ends within minutes
     budget = 90.0
     import oracle
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from conftest import oracle_cache, oracle_shape, oracle_weights
-    m = oracle.Model(oracle_shape(s), oracle_weights(w))
-    cache = oracle_cache(kv_host, None, 0)
+    m = oracle.Model(oracle.shape_from(s), oracle.weights_from(w))
+    cache = oracle.cache_from(kv_host, None, 0)
     tok = tok0
-    for i in range(min(args.warmup, 2)):
+    for i in range(args.warmup):
         tok = m.step(cache, tok, N0 + i).token
     t0 = time.perf_counter()
     n = 0
@@ -440,7 +552,7 @@ def run_reference(args):
     v = dt / n * 1e6
     cores = oracle.get_threads()
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": n, "warmup": min(args.warmup, 2), "ms_per_step": dt / n * 1e3,
+            "steps": n, "warmup": args.warmup, "ms_per_step": dt / n * 1e3,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": WORKLOAD, "batch": 1, "ctx": N0},
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -533,14 +645,16 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
 
-    # ---- the batched configuration and the isolated attention grid
+    # ---- the other configurations (rank 0 prints their summaries)
     bs64 = run_bs64(s, wd, dev, ws, args.seed)
     verify = run_verify(s, wd, dev, args.seed) if rank == 0 else None
     int8 = run_int8(s, wd, kv_host, tok0, dev, args.seed) if rank == 0 else None
+    generate = run_generate(s, wd, kv_host, tok0, dev) if rank == 0 else None
     kernel_config = dec.config()
     dec.close()
     del kv, wd
     torch.cuda.empty_cache()
+    cfg5 = run_cfg5(dev, ws, args.seed)
     attention = run_attention_grid(dev, args.seed) if rank == 0 else None
 
     # ---- max over ranks
@@ -553,6 +667,9 @@ def run_ours(args):
         bytes_mean = statistics.fmean(roofline.step_bytes(s, [p]) for p in positions[:WINDOW])
         peak, peak_kind = peaks()
         achieved = bytes_mean / (mean_launch_ms * 1e-3) / 1e9
+        # Key order: the driver keeps the END of the line, so the long
+        # attention grid comes first and the compact summaries of the other
+        # configurations last.
         line = {
             "metric": METRIC, "value": us_per_tok, "unit": UNIT, "n_gpus": ws, "steps": K,
             "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": False,
@@ -574,15 +691,16 @@ def run_ours(args):
                     "steps": KE, "api": "dec_step_host"},
             "gpu_launches": K,
             "clocks": clocks,
-            "bs64": bs64,
             "attention": attention,
             "verify": verify,
             "int8": int8,
+            "bs64": bs64,
+            "cfg5": cfg5,
+            "generate": generate,
         }
         if not args.no_cpu_baseline and ws == 1:
             line["cpu_baseline"] = cpu_baseline(s, w, kv_host, tok0)
         print(json.dumps(line), flush=True)
-    dec.close()
     if ws > 1:
         dist.destroy_process_group()
 

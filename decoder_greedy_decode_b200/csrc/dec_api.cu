@@ -40,6 +40,7 @@ struct dec_handle {
   const float* lm_scale = nullptr;    // int8: lm_head row scales
   LayerScales* scales_dev = nullptr;  // int8: projection row scales
   int wsc_n = 0;
+  int prow = 0;
   uint8_t* ws = nullptr;
   WorkspaceLayout wl{};
   float* logits_dev = nullptr;
@@ -163,13 +164,19 @@ static int init_handle(const dec_shape* shape, const InitWeights& w, dec_handle*
   h->w8 = w.w8;
   h->lm_scale = w.lm_scale;
   h->wsc_n = w.w8 ? step_wsc_slots(H, F, nqkv, shape->vocab, h->ctas) : 0;
+  h->prow = step_part_rows(H, F, nqkv, h->ctas);
   for (int b = 1; b <= B; ++b) {
-    h->nslot[b] = step_max_slots(b, H, F, HqD, D, rep, h->wsc_n, h->smem_optin);
+    h->nslot[b] = step_max_slots(b, H, F, HqD, D, rep, h->wsc_n, h->prow, h->smem_optin);
     if (h->nslot[b] < 2) {
       delete h;
       return DEC_ERR_DEVICE;
     }
-    h->smem[b] = step_smem_bytes(h->nslot[b], b, H, F, HqD, D, rep, h->wsc_n);
+    h->smem[b] = step_smem_bytes(h->nslot[b], b, H, F, HqD, D, rep, h->wsc_n, h->prow);
+    e = step_set_smem(b, D, w.w8 != 0, h->smem[b]);
+    if (e != cudaSuccess) {
+      delete h;
+      return cuda_fail(e);
+    }
   }
   h->embed = static_cast<const uint16_t*>(w.embed);
   h->lm_head = static_cast<const uint16_t*>(w.lm_head);
@@ -191,6 +198,8 @@ static int init_handle(const dec_shape* shape, const InitWeights& w, dec_handle*
   wl.x_out = take(sizeof(uint64_t) * B * H);
   wl.part = take(sizeof(uint64_t) * B * Hq * wl.part_chunks * (D + 2));
   wl.amax_key = take(sizeof(unsigned long long) * B);
+  wl.tokw = take(sizeof(uint64_t) * B);
+  wl.step_cnt = take(sizeof(unsigned));
   wl.exit_cnt = take(sizeof(unsigned));
   wl.seq = take(sizeof(unsigned));
   wl.status = take(sizeof(int));
@@ -201,7 +210,7 @@ static int init_handle(const dec_shape* shape, const InitWeights& w, dec_handle*
   wl.out_dev = take(sizeof(int32_t) * Bfull);
   wl.gen_done = take(sizeof(int) * Bfull);
 #ifdef DEC_PROFILE
-  wl.prof = take(sizeof(unsigned long long) * h->ctas * (16 * L + 8));
+  wl.prof = take(sizeof(unsigned long long) * h->ctas * (kProfStampsPerLayer * L + 8));
 #endif
   size_t layers_off = take(sizeof(LayerPtrs) * L);
   size_t scales_off = w.w8 ? take(sizeof(LayerScales) * L) : 0;
@@ -304,9 +313,12 @@ extern "C" int dec_kv_alloc(dec_handle* h, int batch, int max_ctx, int dtype, vo
   return DEC_OK;
 }
 
+// n_steps > 1 (batch <= kMaxBatchSmall only): the persistent kernel runs the
+// steps itself, feeding the ids back and advancing gen_pos (== pos) in place.
 static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* pos,
                    const dec_kv* kv, int32_t* out_ids, float* logits, float* hidden,
-                   cudaStream_t stream) {
+                   cudaStream_t stream, int n_steps = 1, int eos = -1,
+                   int32_t* gen_pos = nullptr, const int* retired = nullptr) {
   if (!h || !kv || !tok || !pos || !out_ids || !kv->base) return DEC_ERR_NULL;
   if (batch < 1 || batch > h->shape.max_batch || batch > kv->batch) return DEC_ERR_BATCH;
   if (kv->dtype != DEC_KV_BF16 && kv->dtype != DEC_KV_FP8_E4M3) return DEC_ERR_DTYPE;
@@ -329,6 +341,7 @@ static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* 
     io.kv_batch = kv->batch;
     io.max_ctx = kv->max_ctx;
     io.one_seq = -1;
+    io.retired = retired;
     io.status = reinterpret_cast<int*>(h->ws + h->wl.status);
     io.timeout_ns = h->timeout_ns;
     cudaError_t e = bt_step(h->bt, io, stream);
@@ -364,6 +377,9 @@ static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* 
   a.token_ids = tok;
   a.positions = pos;
   a.out_ids = out_ids;
+  a.n_steps = n_steps;
+  a.eos = eos;
+  a.gen_pos = gen_pos;
   a.out_logits = logits;
   a.hidden_out = hidden;
   const WorkspaceLayout& wl = h->wl;
@@ -375,6 +391,8 @@ static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* 
   a.part = reinterpret_cast<uint64_t*>(h->ws + wl.part);
   a.part_chunks = wl.part_chunks;
   a.amax_key = reinterpret_cast<unsigned long long*>(h->ws + wl.amax_key);
+  a.tokw = reinterpret_cast<uint64_t*>(h->ws + wl.tokw);
+  a.step_cnt = reinterpret_cast<unsigned*>(h->ws + wl.step_cnt);
   a.exit_cnt = reinterpret_cast<unsigned*>(h->ws + wl.exit_cnt);
   a.seq = reinterpret_cast<unsigned*>(h->ws + wl.seq);
   a.status = reinterpret_cast<int*>(h->ws + wl.status);
@@ -383,6 +401,7 @@ static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* 
   a.timeout_ns = h->timeout_ns;
   a.stall_cta = h->stall_cta;
   a.nslot = h->nslot[batch];
+  a.prow = h->prow;
 #ifdef DEC_PROFILE
   a.prof = reinterpret_cast<unsigned long long*>(h->ws + wl.prof);
 #else
@@ -486,15 +505,21 @@ extern "C" int dec_generate(dec_handle* h, int batch, int n_steps, const int32_t
                             void* stream) {
   if (!h || !kv || !token_ids || !positions || !out_ids) return DEC_ERR_NULL;
   if (batch < 1 || batch > h->shape.max_batch || batch > 64) return DEC_ERR_BATCH;
-  if (n_steps < 1) return DEC_ERR_ARG;
+  if (n_steps < 1 || eos < -1 || eos >= h->shape.vocab) return DEC_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (batch <= kMaxBatchSmall)  // one launch: the persistent kernel loops over the steps
+    return do_step(h, batch, token_ids, positions, kv, out_ids, nullptr, nullptr, st, n_steps,
+                   eos, positions);
+  // the batched step: one step per launch, a small kernel in between feeds
+  // the ids back, advances the positions and retires sequences at eos
   int* done = reinterpret_cast<int*>(h->ws + h->wl.gen_done);
   cudaError_t e = launch_gen_reset(done, batch, st);
   if (e != cudaSuccess) return cuda_fail(e);
   for (int i = 0; i < n_steps; ++i) {
     const int32_t* tok = i == 0 ? token_ids : out_ids + static_cast<size_t>(i - 1) * batch;
     int32_t* out = out_ids + static_cast<size_t>(i) * batch;
-    const int rc = do_step(h, batch, tok, positions, kv, out, nullptr, nullptr, st);
+    const int rc = do_step(h, batch, tok, positions, kv, out, nullptr, nullptr, st, 1, -1,
+                           nullptr, done);
     if (rc) return rc;
     e = launch_gen_advance(out, positions, done, batch, eos, st);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -567,7 +592,8 @@ extern "C" int dec_last_cuda_error(void) { return g_last_cuda; }
 // ------------------------------------------------------------ attention
 extern "C" size_t dec_attention_workspace_bytes(int batch, int n_q_heads, int n_kv_heads,
                                                 int head_dim, int max_len) {
-  if (batch < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads || max_len < 1) return 0;
+  if (batch < 1 || n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % n_kv_heads || max_len < 1)
+    return 0;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -584,7 +610,8 @@ extern "C" int dec_attention(int batch, int n_q_heads, int n_kv_heads, int head_
   if (!q || !k_cache || !v_cache || !lengths || !out || !workspace) return DEC_ERR_NULL;
   if (batch < 1) return DEC_ERR_BATCH;
   if (head_dim != 64 && head_dim != 128) return DEC_ERR_SHAPE;
-  if (n_kv_heads < 1 || n_q_heads % n_kv_heads || n_q_heads / n_kv_heads > 8) return DEC_ERR_SHAPE;
+  if (n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % n_kv_heads || n_q_heads / n_kv_heads > 8)
+    return DEC_ERR_SHAPE;
   if (max_len < 1) return DEC_ERR_ARG;
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(workspace, 256))
     return DEC_ERR_ALIGN;
@@ -652,10 +679,10 @@ extern "C" int dec_bt_prof_read(dec_handle* h, unsigned long long* host, size_t 
 }
 
 // Profiling builds only (not part of dec.h): copy the per-phase timestamps of
-// the last step, [ctas][16 * n_layers + 8] globaltimer values, to `host`.
+// the last step, [ctas][32 * n_layers + 8] globaltimer values, to `host`.
 extern "C" int dec_prof_read(dec_handle* h, unsigned long long* host, size_t n) {
   if (!h || !host) return DEC_ERR_NULL;
-  const size_t need = static_cast<size_t>(h->ctas) * (16 * h->shape.n_layers + 8);
+  const size_t need = static_cast<size_t>(h->ctas) * (kProfStampsPerLayer * h->shape.n_layers + 8);
   if (n < need) return DEC_ERR_ARG;
   cudaError_t e = cudaMemcpy(host, h->ws + h->wl.prof, need * sizeof(unsigned long long),
                              cudaMemcpyDeviceToHost);

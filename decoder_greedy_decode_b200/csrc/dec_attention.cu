@@ -560,7 +560,8 @@ extern "C" int dec_attention_noalloc(int batch, int n_q_heads, int n_kv_heads, i
   if (!q || !k_cache || !v_cache || !lengths || !out) return DEC_ERR_NULL;
   if (batch < 1) return DEC_ERR_BATCH;
   if (head_dim != 64 && head_dim != 128) return DEC_ERR_SHAPE;
-  if (n_kv_heads < 1 || n_q_heads % n_kv_heads || n_q_heads / n_kv_heads > 8) return DEC_ERR_SHAPE;
+  if (n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % n_kv_heads || n_q_heads / n_kv_heads > 8)
+    return DEC_ERR_SHAPE;
   if (max_len < 1) return DEC_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15)
     return DEC_ERR_ALIGN;

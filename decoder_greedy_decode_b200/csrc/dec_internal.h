@@ -5,7 +5,7 @@
 
 namespace dec {
 
-constexpr int kConsumerWarps = 7;
+constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kStepThreads = kConsumerThreads + 32;  // + one producer warp
 constexpr int kSlotBytes = 24576;                   // ring slot: 12 rows of 1024 bf16
@@ -13,6 +13,7 @@ constexpr int kMaxBatchSmall = 4;                   // batch handled by the GEMV
 constexpr int kMaxRep = 4;                          // query heads per KV head (step kernel)
 constexpr int kLayerPtrs = 11;
 constexpr int kMaxBatch = 64;                       // batched step: the N of the tensor-core tiles
+constexpr int kProfStampsPerLayer = 32;             // profiling builds: timestamps per layer and CTA
 
 struct LayerPtrs {
   const uint16_t* w[kLayerPtrs];  // dec_layer_weight order (int8 codes for the
@@ -48,7 +49,10 @@ struct StepArgs {
   // step inputs / outputs
   const int32_t* token_ids;
   const int32_t* positions;
-  int32_t* out_ids;
+  int32_t* out_ids;     // [n_steps][B]
+  int n_steps;          // greedy steps this launch runs (ids fed back on the device)
+  int eos;              // end-of-sequence id, or -1
+  int32_t* gen_pos;     // n_steps > 1: the caller's positions, advanced in place; else null
   float* out_logits;    // [B, V] or null
   float* hidden_out;    // [L+1, B, H] or null
   // workspace
@@ -60,6 +64,8 @@ struct StepArgs {
   uint64_t* part;       // tagged attention partials [B, Hq, part_chunks, D + 2]
   int part_chunks;
   unsigned long long* amax_key;  // [B]
+  uint64_t* tokw;       // tagged ids of the last finished step [B]
+  unsigned* step_cnt;   // CTAs past their argmax, over the launch's steps
   unsigned* exit_cnt;
   unsigned* seq;
   int* status;
@@ -68,18 +74,26 @@ struct StepArgs {
   unsigned long long timeout_ns;
   int stall_cta;        // -1: off
   int nslot;            // ring slots per CTA
+  int prow;             // most output rows of one CTA in a K-split stage
   unsigned long long* prof;  // per-phase timestamps (profiling builds) or null
 };
 
 // Scratch layout inside the library workspace (byte offsets).
 struct WorkspaceLayout {
-  size_t x_qkv, x_o, x_mid, x_u, x_out, part, amax_key, exit_cnt, seq, status, abort_flag,
-      inv_freq, tok_dev, pos_dev, out_dev, gen_done, prof, total;
+  size_t x_qkv, x_o, x_mid, x_u, x_out, part, amax_key, tokw, step_cnt, exit_cnt, seq, status,
+      abort_flag, inv_freq, tok_dev, pos_dev, out_dev, gen_done, prof, total;
   int part_chunks;
 };
 
-size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep, int wsc_n);
-int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int wsc_n, int smem_optin);
+size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep, int wsc_n,
+                       int prow);
+int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int wsc_n, int prow,
+                   int smem_optin);
+// The most output rows one CTA computes in a K-split stage (gate and up rows
+// counted separately).
+int step_part_rows(int H, int F, int nqkv, int ctas);
+// Dynamic shared-memory limit of the step kernels a handle launches.
+cudaError_t step_set_smem(int B, int D, bool w8, size_t smem);
 // Shared-memory row-scale slots an int8 step needs: the most rows one CTA
 // computes in any stage (gate and up rows counted twice).
 int step_wsc_slots(int H, int F, int nqkv, int V, int ctas);
@@ -133,6 +147,7 @@ struct BtIO {
   float* kv_scales;
   int kv_batch, max_ctx, kv_fp8;
   int one_seq;     // -1: row b is cache sequence b; >= 0: every row is that sequence
+  const int* retired;  // [B] or null: rows whose new cache row is not written
   int* status;
   unsigned long long timeout_ns;
 };

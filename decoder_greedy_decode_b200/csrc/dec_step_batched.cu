@@ -161,6 +161,7 @@ struct GemmArgs {
   int kv_batch, max_ctx, layer, kv_fp8;
   int one_seq;           // -1: row b is cache sequence b; >= 0: every row is that sequence
   const int32_t* pos;
+  const int* retired;    // [B] or null: rows whose cache row is not written
   const int* bad;
   const float* inv_freq;
   unsigned long long* keys;  // kLm: [64]
@@ -487,11 +488,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
               ((static_cast<size_t>(g.layer) * 2 + kvsel) * g.kv_batch + cs) * g.Hkv + head;
           return plane * g.max_ctx + s_pos[b];
         };
+        auto live = [&](int b) { return g.retired == nullptr || g.retired[b] == 0; };
         if (!g.kv_fp8) {
 #pragma unroll 4
           for (int bi = hg; bi < nb; bi += 2) {
             const int b = rank + S * bi;
-            reinterpret_cast<uint16_t*>(g.kv)[crow_of(b) * D + d] = f_to_bf16(value(bi));
+            if (live(b))
+              reinterpret_cast<uint16_t*>(g.kv)[crow_of(b) * D + d] = f_to_bf16(value(bi));
           }
         } else {
           // E4M3 with one fp32 scale per row: scale = max(amax, 2^-126) / 448
@@ -509,9 +512,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             hm = fmaxf(hm, 1.17549435e-38f);
             const float sc = __fdiv_rn(hm, 448.0f);
             const size_t cr = crow_of(b);
-            g.kv[cr * D + d] =
-                static_cast<uint8_t>(f2_to_e4m3x2(__fdiv_rn(value(bi), sc), 0.f) & 0xFF);
-            if (d == 0) g.kv_scales[cr] = sc;
+            if (live(b)) {
+              g.kv[cr * D + d] =
+                  static_cast<uint8_t>(f2_to_e4m3x2(__fdiv_rn(value(bi), sc), 0.f) & 0xFF);
+              if (d == 0) g.kv_scales[cr] = sc;
+            }
           }
         }
       }
@@ -1265,6 +1270,7 @@ cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
   base.kv_fp8 = io.kv_fp8;
   base.one_seq = io.one_seq;
   base.pos = io.pos;
+  base.retired = io.retired;
   base.bad = p->bad;
   base.inv_freq = p->inv_freq;
   base.keys = p->keys;

@@ -7,23 +7,33 @@
 // step launch-bound (~300 attention kernels per token, 07 Root causes); here
 // there is one launch per step and no host involvement inside it.
 //
-// Structure (one CTA per SM, 7 consumer warps + 1 producer warp):
+// Structure (one CTA per SM, 8 consumer warps + 1 producer warp):
 //  * Every weight and KV byte the CTA will need is known before the step
 //    starts, independent of activations.  The producer warp streams them with
 //    1-D bulk copies (TMA engine) into a ring of 24 KB shared-memory slots,
-//    running up to a whole ring (~190 KB, about one layer's share) ahead of
+//    running up to a whole ring (~170 KB, most of one layer's share) ahead of
 //    the consumers.  HBM therefore keeps streaming while consumers wait for
 //    activations.
 //  * Activations move between CTAs as 8-byte words {fp32 value, 32-bit flag}
 //    in global memory (L2).  A consumer polls the words it needs until their
 //    flags equal the expected (step, layer) tag: data and readiness arrive
 //    in one load, with no separate barrier round trip.
-//  * Rows of every projection are split evenly over CTAs.  Each CTA owns the
+//  * Rows of every projection are split evenly over CTAs; each CTA owns the
 //    same hidden rows in o_proj and down, so it keeps those residual entries
-//    in shared memory.  Attention is split-K over (sequence, KV head, chunk)
-//    items; the CTA of chunk 0 of a (sequence, KV head) gathers the other
-//    chunks' partials as they are published, merges them (flash-decoding
-//    combine) and publishes the head outputs.
+//    in shared memory.  Inside a CTA the K dimension of a projection is split
+//    over the consumer warps in blocks of 128 columns: each warp polls only
+//    the input words of its own blocks and computes its partial dot products
+//    as soon as they are there, so the arrival skew of the producing CTAs
+//    overlaps the arithmetic.  One CTA barrier per projection then sums the
+//    warps' partials in a fixed order (deterministic) and applies the RMSNorm
+//    factor of the input, computed from the warps' partial sums of squares:
+//    W (g * x * s) = s * W (g * x).
+//  * Attention is split-K over (sequence, KV head, chunk) items; every lane
+//    octet scores a cached row against all query heads of its head group
+//    (each K/V row is read once per group); the CTA of chunk 0 of a
+//    (sequence, KV head) gathers the other chunks' partials as they are
+//    published, merges them (flash-decoding combine) and publishes the head
+//    outputs.
 //  * Every wait is bounded (globaltimer).  A wait that runs out raises a
 //    status bit and a global abort flag; all CTAs then drain their in-flight
 //    copies without computing and leave; out_ids becomes -1.
@@ -44,8 +54,10 @@ constexpr int kMaxHRows = 64;  // hidden rows a CTA may own
 constexpr int kDevTimeout = 4;
 constexpr int kDevBadPos = 1;
 constexpr int kDevBadTok = 2;
-// Tagged words one gather pass stages in shared memory (24 KB).
-constexpr int kStageWords = 3072;
+constexpr int kBlk = 128;                      // columns of one K block
+constexpr int kWarpStage = 384;                // tagged words a warp stages per poll round
+constexpr int kStageWords = kCW * kWarpStage;  // whole staging buffer (CTA-wide gathers)
+constexpr int kMaxGainBlk = 6;                 // K blocks per warp of a normalised input (H <= 6144)
 
 // Stages of one layer; the lm_head runs as stage SQ of layer L (code SLM).
 enum { SQ = 0, SA, SO, SU, SD, kStages, SLM = kStages };
@@ -55,10 +67,14 @@ enum { SQ = 0, SA, SO, SU, SD, kStages, SLM = kStages };
 // prof[cta][kStampsPerLayer * L + 8] at the points named by the St* indices
 // below (per layer), then lm_head start / gathered / done, consumer end and
 // consumer start.
-[[maybe_unused]] constexpr int kStampsPerLayer = 16;
+[[maybe_unused]] constexpr int kStampsPerLayer = kProfStampsPerLayer;
 enum {
-  StStart = 0, StQGath, StQNorm, StQkv, StAttIn, StAttRows, StAtt, StOGath, StO, StUGath, StUNorm,
-  StU, StDGath, StD
+  StAttTile = 0, StQIn, StQDot, StQkv, StAttIn, StAttRows, StAtt, StOIn, StO, StUIn, StUDot,
+  StU, StDIn, StD, StODot, StDDot,
+  // the producer's issue time of the first tile of each stage
+  StPQ, StPA, StPO, StPU, StPD,
+  // ns warp 0 spent waiting for ring tiles in each stage
+  StWQ, StWA, StWO, StWU, StWD
 };
 enum { StLmStart = 0, StLmGath, StLmDone, StEnd, StBegin };
 #ifdef DEC_PROFILE
@@ -67,9 +83,25 @@ enum { StLmStart = 0, StLmGath, StLmDone, StEnd, StBegin };
     if (a.prof && tid == 0)                                                            \
       a.prof[static_cast<size_t>(cta) * (kStampsPerLayer * a.L + 8) + (i)] = globaltimer(); \
   } while (0)
+// the producer lane's stamps, and a stored value instead of a time
+#define DEC_PSTAMP(i)                                                                  \
+  do {                                                                                 \
+    if (a.prof)                                                                        \
+      a.prof[static_cast<size_t>(cta) * (kStampsPerLayer * a.L + 8) + (i)] = globaltimer(); \
+  } while (0)
+#define DEC_SVAL(i, v)                                                                 \
+  do {                                                                                 \
+    if (a.prof && tid == 0) a.prof[static_cast<size_t>(cta) * (kStampsPerLayer * a.L + 8) + (i)] = (v); \
+  } while (0)
 #else
 #define DEC_STAMP(i) \
   do {               \
+  } while (0)
+#define DEC_PSTAMP(i) \
+  do {                \
+  } while (0)
+#define DEC_SVAL(i, v) \
+  do {                 \
   } while (0)
 #endif
 
@@ -81,13 +113,25 @@ constexpr int kMaxLayers = 64;  // layer pointer table kept in shared memory
 // Fewer, longer attention chunks keep the combine to one round of loads.
 constexpr int kMinChunkRows = 96;
 
+// The sequences of the current step and its attention work split: items
+// (b, g, chunk) over contexts 0..p_b, chunk rows `crow`.  The consumers and
+// the producer each keep their own copy (they reach a step at different
+// times) and compute it identically.
+struct Plan {
+  int crow, n_items, all_done, bad;
+  int nchunk[kMaxBatchSmall], pos[kMaxBatchSmall], tok[kMaxBatchSmall], done[kMaxBatchSmall];
+};
+
 struct Carve {
-  size_t ring, bars, act, stg, xown, bred, ints, lw, wsc, total;
+  size_t ring, bars, act, stg, xown, part, bred, ints, lw, wsc, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline Carve carve(int nslot, int B, int kmax, int D, int rep, int wsc_n) {
+// prow: the most output rows one CTA computes in a K-split stage (gate and up
+// rows counted separately).
+__host__ __device__ inline Carve carve(int nslot, int B, int kmax, int D, int rep, int wsc_n,
+                                       int prow) {
   Carve c;
   size_t o = 0;
   c.ring = o;
@@ -95,17 +139,19 @@ __host__ __device__ inline Carve carve(int nslot, int B, int kmax, int D, int re
   c.bars = o;
   o += align_up(2 * nslot * sizeof(uint64_t), 16);
   size_t act_f = static_cast<size_t>(B) * kmax;
-  size_t att_f = static_cast<size_t>(rep + 2) * D + static_cast<size_t>(kCW + rep) * (D + 2);
+  size_t att_f = static_cast<size_t>(rep + 2) * D + static_cast<size_t>(kCW) * rep * (D + 2);
   c.act = o;
   o += align_up((act_f > att_f ? act_f : att_f) * sizeof(float), 16);
   c.stg = o;
   o += static_cast<size_t>(kStageWords) * sizeof(uint64_t);
   c.xown = o;
   o += align_up(static_cast<size_t>(kMaxHRows) * B * sizeof(float), 16);
+  c.part = o;  // two buffers of [kCW][prow][B] partial sums + [kCW][B] sums of squares
+  o += align_up(2ull * kCW * (prow + 1) * B * sizeof(float), 16);
   c.bred = o;
   o += align_up(2ull * kCW * B * sizeof(float) + 2ull * kCW * B * sizeof(int), 16);
-  c.ints = o;
-  o += 64 * sizeof(int);
+  c.ints = o;  // two Plans (consumers, producer) + a few ints
+  o += align_up(2 * sizeof(Plan) + 16 * sizeof(int), 16);
   c.lw = o;
   o += align_up(sizeof(LayerPtrs) * kMaxLayers, 16);
   c.wsc = o;
@@ -156,7 +202,7 @@ __device__ __forceinline__ float dot8(const uint4 w, const float* x) {
 // lane gets the full sum of row (R == 4: lane >> 3; R == 2: lane >> 4;
 // R == 1: 0) for each b.  Compiled on their own (not inlined) so that their
 // register allocation and scheduling do not depend on the rest of the
-// persistent kernel.
+// persistent kernel.  (The lm_head: whole rows per warp.)
 template <int R, int B>
 struct GroupSums {
   float s[B];
@@ -309,11 +355,74 @@ __device__ __noinline__ GroupSums<R, B> group_dot(const uint32_t* rows, uint32_t
   return out;
 }
 
+// Partial dot products of 4 tile rows (shared memory, row i at rows[i]) with
+// the activations of B sequences over the K blocks blk0, blk0 + kCW, ...
+// (nb of them): lane l takes columns 4l..4l+3 of each 128-column block, so
+// that the warp reads 256 contiguous bytes of a bf16 row (128 of an int8 row)
+// and 512 contiguous bytes of activations: no bank conflicts.  Returns the
+// transposed-butterfly reduction (lane gets row lane >> 3's sum for each b).
+template <int B, bool W8>
+__device__ __noinline__ GroupSums<4, B> kdot4(const uint32_t* rows, uint32_t act, int act_stride,
+                                              int blk0, int nb, int lane) {
+  float acc[4][B];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int b = 0; b < B; ++b) acc[i][b] = 0.f;
+  for (int j = 0; j < nb; ++j) {
+    const uint32_t col = static_cast<uint32_t>((blk0 + j * kCW) * kBlk + lane * 4);
+    float wf[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if constexpr (W8) {
+        uint32_t w;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(rows[i] + col));
+        const uint32_t u = w ^ 0x80808080u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) wf[i][e] = i8_at(u, e);
+      } else {
+        uint32_t w0, w1;
+        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(rows[i] + col * 2));
+        wf[i][0] = bf16lo(w0);
+        wf[i][1] = bf16hi(w0);
+        wf[i][2] = bf16lo(w1);
+        wf[i][3] = bf16hi(w1);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      float x0, x1, x2, x3;
+      const uint32_t xa = act + static_cast<uint32_t>(b * act_stride + col) * 4u;
+      asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                   : "=f"(x0), "=f"(x1), "=f"(x2), "=f"(x3) : "r"(xa));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float s = acc[i][b];
+        s = fmaf(wf[i][0], x0, s);
+        s = fmaf(wf[i][1], x1, s);
+        s = fmaf(wf[i][2], x2, s);
+        s = fmaf(wf[i][3], x3, s);
+        acc[i][b] = s;
+      }
+    }
+  }
+  GroupSums<4, B> out;
+#pragma unroll
+  for (int b = 0; b < B; ++b) {
+    float col[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) col[i] = acc[i][b];
+    out.s[b] = tbfly_lane<4>(col, lane);
+  }
+  return out;
+}
+
 // The per-launch state of one CTA.  FP8: the cache holds E4M3 codes + scales.
 // W8: the projections and lm_head are int8 codes with fp32 row scales.
 template <int B, int D, bool FP8, bool W8>
 struct Cta {
-  static constexpr int DL = D / 32;  // attention dims per lane
+  static constexpr int DL = D / 32;  // attention dims per lane (warp-wide vectors)
+  static constexpr int DQ = D / 8;   // attention dims per lane (lane octets)
   const StepArgs& a;
   uint8_t* ring;
   uint64_t* full;
@@ -321,41 +430,43 @@ struct Cta {
   float* act;
   float* xown;
   uint64_t* stg;  // gather staging: tagged words
+  float* part;    // K-split partial sums, two buffers
   float* bredf;
   int* bredi;
-  int* sints;
   const LayerPtrs* slw;  // layer pointer table copied to shared memory
   float* wsc;                               // int8: row scales of the current stage
   static constexpr int eb = W8 ? 1 : 2;     // bytes per weight element
   int tid, warp, lane, cta, nc;
-  int kmax, nqkv;
-  uint32_t seq;
+  int kmax, nqkv, prow;
+  uint32_t seq0;  // step counter of the launch's first step
+  uint32_t seq;   // step counter of the consumers' current step
   // per-CTA row ranges
   int q0, q1, h0, h1, f0, f1, v0, v1;
   int rpt_h, rpt_o, rpt_u, rpt_d, art;
-  // attention work split
-  int crow, n_items;
-  int* pos;     // [B] positions (shared memory)
-  int* tok;     // [B] tokens (shared memory)
-  int* nchunk;  // [B] attention chunks per KV head (shared memory)
+  // this side's plan of the current step (shared memory)
+  Plan* pl;
+  Plan* cplan;  // the consumers' copy
+  Plan* pplan;  // the producer's copy
+  int* sints;   // a few shared ints after the plans
 
   __device__ Cta(const StepArgs& args, uint8_t* smem, int kmax_) : a(args), kmax(kmax_) {
     const int rep = a.Hq / a.Hkv;
-    Carve c = carve(a.nslot, B, kmax, D, rep, a.wsc_n);
+    prow = a.prow;
+    Carve c = carve(a.nslot, B, kmax, D, rep, a.wsc_n, prow);
     ring = smem + c.ring;
     full = reinterpret_cast<uint64_t*>(smem + c.bars);
     empty = full + a.nslot;
     act = reinterpret_cast<float*>(smem + c.act);
     xown = reinterpret_cast<float*>(smem + c.xown);
     stg = reinterpret_cast<uint64_t*>(smem + c.stg);
+    part = reinterpret_cast<float*>(smem + c.part);
     bredf = reinterpret_cast<float*>(smem + c.bred);
     bredi = reinterpret_cast<int*>(bredf + 2 * kCW * B);
-    sints = reinterpret_cast<int*>(smem + c.ints);
+    cplan = reinterpret_cast<Plan*>(smem + c.ints);
+    pplan = cplan + 1;
+    sints = reinterpret_cast<int*>(pplan + 1);
     slw = reinterpret_cast<const LayerPtrs*>(smem + c.lw);
     wsc = reinterpret_cast<float*>(smem + c.wsc);
-    pos = sints + 8;
-    tok = sints + 16;
-    nchunk = sints + 24;
     tid = threadIdx.x;
     warp = tid >> 5;
     lane = tid & 31;
@@ -379,39 +490,75 @@ struct Cta {
     } else {
       art = kSlotBytes / (4 * D);
     }
+    pl = warp == kCW ? pplan : cplan;
   }
 
+  // Tag of the words a layer publishes in the current step (seq counts the
+  // steps of all launches on the handle), and of the ids of step st of this
+  // launch.
   __device__ __forceinline__ uint32_t flag(int layer) const {
     return seq * 256u + static_cast<uint32_t>(layer) + 1u;
   }
+  __device__ __forceinline__ uint32_t tok_flag(int st) const {
+    return (seq0 + static_cast<uint32_t>(st)) * 256u + 255u;
+  }
 
-  // Attention items: (b, g, chunk) over contexts 0..p_b, chunk rows `crow`,
-  // so that the items fit the grid when possible.  Same on every CTA.
-  __device__ void plan_attention() {
+  // The attention items of plan P's positions: chunk rows sized so that the
+  // items fit the grid when possible.  Same on every CTA and both sides.
+  __device__ void make_plan(Plan& P) const {
     long long T = 0;
-    for (int b = 0; b < a.B; ++b) T += static_cast<long long>(pos[b] + 1) * a.Hkv;
+    for (int b = 0; b < a.B; ++b) T += static_cast<long long>(P.pos[b] + 1) * a.Hkv;
     int slots = nc - a.B * a.Hkv;
     if (slots < 1) slots = 1;
     long long cr = (T + slots - 1) / slots;
     cr = (cr + 15) / 16 * 16;
     if (cr < kMinChunkRows) cr = kMinChunkRows;
-    crow = static_cast<int>(cr);
-    n_items = 0;
+    P.crow = static_cast<int>(cr);
+    P.n_items = 0;
+    int all = 1;
     for (int b = 0; b < a.B; ++b) {
-      const int nb = (pos[b] + 1 + crow - 1) / crow;
-      if (tid == 0) nchunk[b] = nb;
-      n_items += nb * a.Hkv;
+      const int nb = (P.pos[b] + 1 + P.crow - 1) / P.crow;
+      P.nchunk[b] = nb;
+      P.n_items += nb * a.Hkv;
+      all &= P.done[b];
     }
+    P.all_done = all;
   }
   __device__ void item(int it, int& b, int& g, int& ci) const {
     int bb = 0;
-    while (bb < a.B - 1 && it >= nchunk[bb] * a.Hkv) {
-      it -= nchunk[bb] * a.Hkv;
+    while (bb < a.B - 1 && it >= pl->nchunk[bb] * a.Hkv) {
+      it -= pl->nchunk[bb] * a.Hkv;
       ++bb;
     }
     b = bb;
-    g = it / nchunk[bb];
-    ci = it % nchunk[bb];
+    g = it / pl->nchunk[bb];
+    ci = it % pl->nchunk[bb];
+  }
+
+  // The ids of step s (tagged words published by the CTA that finished the
+  // step last), then plan P of step s + 1: a sequence that has emitted the
+  // end token is retired (its position stays, its input is the end token,
+  // the cache is not written); the others advance by one row.  Polled by one
+  // thread; false when the wait gave up.
+  __device__ bool next_step(Plan& P, uint32_t f) const {
+    Spin sp;
+    for (int b = 0; b < a.B; ++b) {
+      uint64_t w;
+      for (;;) {
+        w = ld_tagged(a.tokw + b);
+        if (static_cast<uint32_t>(w >> 32) == f) break;
+        if (sp.tick(a, true)) return false;
+      }
+      const int id = static_cast<int>(static_cast<uint32_t>(w));
+      if (!P.done[b]) {
+        if (a.eos >= 0 && id == a.eos) P.done[b] = 1;
+        else P.pos[b] += 1;
+      }
+      P.tok[b] = P.done[b] ? a.eos : id;
+      if (!P.done[b] && P.pos[b] >= a.max_ctx) P.bad = 1;
+    }
+    make_plan(P);
+    return true;
   }
 
   __device__ __forceinline__ size_t kv_row(int l, int kvsel, int b, int g, int j) const {
@@ -461,6 +608,8 @@ struct Cta {
     auto wrow = [&](const void* base, int r, int K) {
       return static_cast<const uint8_t*>(base) + static_cast<size_t>(r) * K * e;
     };
+    bool stop = false;
+    for (int st = 0; !dead && !stop; ++st) {
     for (int l = 0; l < a.L && !dead; ++l) {
       const LayerPtrs& lw = slw[l];
       // ---- QKV rows [q0, q1) of [Wq; Wk; Wv]
@@ -468,6 +617,7 @@ struct Cta {
         const int nr = min(rpt_h, q1 - r);
         uint8_t* dst = acquire(static_cast<uint32_t>(nr) * H * e);
         if (!dst) break;
+        if (r == q0) DEC_PSTAMP(kStampsPerLayer * l + StPQ);
         int rr = r, left = nr;
         while (left > 0) {
           const uint16_t* base;
@@ -486,18 +636,29 @@ struct Cta {
         }
         advance();
       }
+      // A later step's attention rows depend on the ids of the step before
+      // (a sequence that emitted the end token keeps its position): wait for
+      // them once the first layer's QKV rows are on their way.
+      if (l == 0 && st > 0) {
+        if (!next_step(*pplan, tok_flag(st - 1))) dead = true;
+        if (dead || pplan->bad || pplan->all_done) {
+          stop = true;
+          break;
+        }
+      }
       // ---- attention: cached rows [j0, min(j1, p_b)) of every item of this CTA
-      for (int it = cta; it < n_items && !dead; it += nc) {
+      for (int it = cta; it < pl->n_items && !dead; it += nc) {
         int b, g, ci;
         item(it, b, g, ci);
-        const int j0 = ci * crow;
-        const int jc = min(j0 + crow, pos[b]);
+        const int j0 = ci * pl->crow;
+        const int jc = min(j0 + pl->crow, pl->pos[b]);
         for (int j = j0; j < jc && !dead; j += art) {
           const int nr = min(art, jc - j);
           if constexpr (!FP8) {
             const uint32_t rb = static_cast<uint32_t>(nr) * D * 2;
             uint8_t* dst = acquire(2 * rb);
             if (!dst) break;
+            if (j == j0) DEC_PSTAMP(kStampsPerLayer * l + StPA);
             const uint16_t* kvb = reinterpret_cast<const uint16_t*>(a.kv);
             bulk_g2s(dst, kvb + kv_row(l, 0, b, g, j) * D, rb, fb, pol);
             bulk_g2s(dst + rb, kvb + kv_row(l, 1, b, g, j) * D, rb, fb, pol);
@@ -520,6 +681,7 @@ struct Cta {
         const int nr = min(rpt_o, h1 - r);
         uint8_t* dst = acquire(static_cast<uint32_t>(nr) * HqD * e);
         if (!dst) break;
+        if (r == h0) DEC_PSTAMP(kStampsPerLayer * l + StPO);
         bulk_g2s(dst, wrow(lw.w[6], r, HqD), static_cast<uint32_t>(nr) * HqD * e, fb, pol);
         advance();
       }
@@ -529,6 +691,7 @@ struct Cta {
         const uint32_t rb = static_cast<uint32_t>(nr) * H * e;
         uint8_t* dst = acquire(2 * rb);
         if (!dst) break;
+        if (r == f0) DEC_PSTAMP(kStampsPerLayer * l + StPU);
         bulk_g2s(dst, wrow(lw.w[8], r, H), rb, fb, pol);
         bulk_g2s(dst + rb, wrow(lw.w[9], r, H), rb, fb, pol);
         advance();
@@ -538,10 +701,12 @@ struct Cta {
         const int nr = min(rpt_d, h1 - r);
         uint8_t* dst = acquire(static_cast<uint32_t>(nr) * a.F * e);
         if (!dst) break;
+        if (r == h0) DEC_PSTAMP(kStampsPerLayer * l + StPD);
         bulk_g2s(dst, wrow(lw.w[10], r, a.F), static_cast<uint32_t>(nr) * a.F * e, fb, pol);
         advance();
       }
     }
+    if (stop) break;
     // ---- lm_head rows [v0, v1)
     for (int r = v0; r < v1 && !dead; r += rpt_h) {
       const int nr = min(rpt_h, v1 - r);
@@ -549,6 +714,8 @@ struct Cta {
       if (!dst) break;
       bulk_g2s(dst, wrow(a.lm_head, r, H), static_cast<uint32_t>(nr) * H * e, fb, pol);
       advance();
+    }
+    if (st + 1 >= a.n_steps) break;
     }
     // Every copy issued must land before the CTA exits: wait for the last
     // phase armed on each slot (returns at once when consumers already did).
@@ -568,6 +735,8 @@ struct Cta {
   uint32_t rph = 0;        // full-barrier phase parity of tile rn
   int ab = 0;              // aborted: keep the barrier sequence, compute nothing
   bool ring_dead = false;  // a ring wait ran out: stop waiting on the ring
+  int pb = 0;              // partial-sum buffer of the current K-split stage
+  uint64_t wacc = 0;       // profiling builds: ns spent in ring waits
   float best_v[B];         // lm_head argmax of this thread, per sequence
   int best_i[B];
 
@@ -583,6 +752,9 @@ struct Cta {
     const uint32_t par = rph;
     int st = 1;
     if (lane == 0) {
+#ifdef DEC_PROFILE
+      const uint64_t tw = globaltimer();
+#endif
       Spin sp;
       while (!mbar_wait(&full[slot], par, kWaitHintNs)) {
         if (sp.tick(a, false)) {
@@ -590,6 +762,9 @@ struct Cta {
           break;
         }
       }
+#ifdef DEC_PROFILE
+      wacc += globaltimer() - tw;
+#endif
     }
     st = __shfl_sync(0xffffffffu, st, 0);
     if (!st) {
@@ -625,11 +800,12 @@ struct Cta {
     }
     int fail = 0;
     uint64_t t0 = 0;
-    int more;
+    int more, round = 0;
     do {
       int k = 0;
       for (int c = tid; c < nch; c += kCT, ++k)
         if (pend & (1u << k)) cp_async16_cg(stg + 2 * c, src_of(2 * c));
+      const int abf = (pend && round++ > 0) ? ld_relaxed_i32(a.abort_flag) : 0;
       cp_async_wait_all();
       k = 0;
       for (int c = tid; c < nch; c += kCT, ++k) {
@@ -646,7 +822,7 @@ struct Cta {
           atomicOr(a.status, kDevTimeout);
           atomicExch(a.abort_flag, 1);
           fail = 1;
-        } else if (ld_relaxed_i32(a.abort_flag)) {
+        } else if (abf) {
           fail = 1;
         }
         if (fail) pend = 0;  // else re-poll at once: a hop costs one L2 round trip
@@ -656,95 +832,213 @@ struct Cta {
     ab = named_sync_or(1, kCT, fail | ab);
   }
 
-  // B rows of K tagged words (row stride K) -> act rows (row stride kmax).
-  __device__ void gather_x(const uint64_t* src, int K, uint32_t f) {
-    const int n = a.B * K;
-    for (int w0 = 0; w0 < n; w0 += kStageWords) {
-      const int nw = min(kStageWords, n - w0);
-      gather(nw, f, [=](int w) { return src + w0 + w; });
-      if (!ab)
-        for (int i = tid; i < nw; i += kCT) {
-          const int idx = w0 + i;
-          act[(idx / K) * kmax + idx % K] = __uint_as_float(static_cast<uint32_t>(stg[i]));
+  // Warp-collective version for one warp's own words: n (even, <=
+  // kWarpStage) tagged words into ws (this warp's part of stg).  Sets ab
+  // (warp-uniform) when the wait gave up; ends with every word visible to
+  // every lane of the warp.
+  template <class Src>
+  __device__ void warp_gather(uint64_t* ws, int n, uint32_t f, Src src_of) {
+    __syncwarp();  // the previous round's words are consumed
+    const int np = n >> 1;
+    uint32_t pend = 0;
+    if (!ab)
+      for (int k = 0, c = lane; c < np; c += 32, ++k) pend |= 1u << k;
+    uint64_t t0 = 0;
+    for (int round = 0;; ++round) {
+      for (int k = 0, c = lane; c < np; c += 32, ++k)
+        if (pend & (1u << k)) cp_async16_cg(ws + 2 * c, src_of(2 * c));
+      // the abort flag travels with every later round (its load overlaps the
+      // copies' round trip instead of following it)
+      const int abf = (lane == 0 && round > 0) ? ld_relaxed_i32(a.abort_flag) : 0;
+      cp_async_wait_all();
+      for (int k = 0, c = lane; c < np; c += 32, ++k)
+        if ((pend & (1u << k)) && static_cast<uint32_t>(ws[2 * c] >> 32) == f &&
+            static_cast<uint32_t>(ws[2 * c + 1] >> 32) == f)
+          pend &= ~(1u << k);
+      if (!__any_sync(0xffffffffu, pend != 0)) break;
+      int fail = 0;
+      if (lane == 0) {
+        const uint64_t now = globaltimer();
+        if (t0 == 0) t0 = now;
+        if (now - t0 > a.timeout_ns) {
+          atomicOr(a.status, kDevTimeout);
+          atomicExch(a.abort_flag, 1);
+          fail = 1;
+        } else if (abf) {
+          fail = 1;
         }
-      csync();
+      }
+      if (__shfl_sync(0xffffffffu, fail, 0)) {
+        ab = 1;
+        break;
+      }
+    }
+    __syncwarp();
+  }
+
+  // K blocks of 128 columns are dealt to the consumer warps round-robin:
+  // warp w owns blocks w, w + kCW, ...
+  __device__ __forceinline__ int my_blocks(int nblk) const {
+    return nblk > warp ? (nblk - 1 - warp) / kCW + 1 : 0;
+  }
+
+  // This warp's share of a stage input: for every sequence b and every K
+  // block the warp owns, the 128 values src[b][k] (tagged words, flag f; or,
+  // with src == nullptr, the embedding row of the step's token) times the
+  // gain g[k] (g == nullptr: 1) into act[b][k]; ss[b] gets the warp's share
+  // of sum_k x[b][k]^2 (before the gain), reduced over the warp.
+  __device__ void warp_input(const uint64_t* src, int K, uint32_t f, const uint16_t* g,
+                             float (&ss)[B]) {
+#pragma unroll
+    for (int b = 0; b < B; ++b) ss[b] = 0.f;
+    const int nbw = my_blocks(K / kBlk);
+    const int units = a.B * nbw;  // 128-word units: (b, block)
+    constexpr int per = kWarpStage / kBlk;
+    uint64_t* ws = stg + warp * kWarpStage;
+    // the gains of the warp's blocks, loaded before the polls so that their
+    // latency overlaps them (K <= kMaxGainBlk * kCW * kBlk for a gained input)
+    uint2 gv[kMaxGainBlk];
+#pragma unroll
+    for (int j = 0; j < kMaxGainBlk; ++j)
+      gv[j] = (g && j < nbw) ? __ldg(reinterpret_cast<const uint2*>(
+                                   g + (warp + j * kCW) * kBlk + lane * 4))
+                             : make_uint2(0u, 0u);
+    for (int u0 = 0; u0 < units; u0 += per) {
+      const int nu = min(per, units - u0);
+      if (src)
+        warp_gather(ws, nu * kBlk, f, [=](int i) {
+          const int u = u0 + i / kBlk, b = u / nbw, blk = warp + (u % nbw) * kCW;
+          return src + static_cast<size_t>(b) * K + blk * kBlk + (i % kBlk);
+        });
+      if (ab) continue;
+      for (int uu = 0; uu < nu; ++uu) {
+        const int u = u0 + uu, b = u / nbw, blk = warp + (u % nbw) * kCW;
+        const int k = blk * kBlk + lane * 4;
+        float v[4];
+        if (src) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            v[j] = __uint_as_float(static_cast<uint32_t>(ws[uu * kBlk + lane * 4 + j]));
+        } else {
+          const uint2 e = *reinterpret_cast<const uint2*>(
+              a.embed + static_cast<size_t>(pl->tok[b]) * a.H + k);
+          v[0] = bf16lo(e.x);
+          v[1] = bf16hi(e.x);
+          v[2] = bf16lo(e.y);
+          v[3] = bf16hi(e.y);
+        }
+        const float q = v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
+#pragma unroll
+        for (int bb = 0; bb < B; ++bb)
+          if (bb == b) ss[bb] += q;
+        if (g) {
+          const int j = u % nbw;
+          uint2 gs = gv[0];
+#pragma unroll
+          for (int jj = 1; jj < kMaxGainBlk; ++jj)
+            if (jj == j) gs = gv[jj];
+          v[0] *= bf16lo(gs.x);
+          v[1] *= bf16hi(gs.x);
+          v[2] *= bf16lo(gs.y);
+          v[3] *= bf16hi(gs.y);
+        }
+        *reinterpret_cast<float4*>(act + b * kmax + k) = make_float4(v[0], v[1], v[2], v[3]);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < B; ++b) ss[b] = warp_sum(ss[b]);
+  }
+
+  // The K-split GEMV of a stage over ring tiles: rows [0, nrows) of the
+  // stage arrive rpt per tile (pair: rpt rows of the first matrix, then the
+  // same rows of the second).  Every warp reads every tile and computes the
+  // partial dot products of all its rows over the warp's own K blocks, 4 rows
+  // at a time; the partials of row r (pair: the second matrix's row r at
+  // nrows + r) go to pbuf[warp][r][b].
+  __device__ void kgemv(int K, int nrows, int rpt, bool pair, float* pbuf) {
+    const int nbw = my_blocks(K / kBlk);
+    const uint32_t row_bytes = static_cast<uint32_t>(K * eb);
+    for (int r0 = 0; r0 < nrows; r0 += rpt) {
+      const int nr = min(rpt, nrows - r0);
+      const int ntr = pair ? 2 * nr : nr;
+      wait_tile();
+      if (!ab && nbw > 0) {
+        const uint32_t tb = smem_u32(ring + static_cast<size_t>(rs) * kSlotBytes);
+        for (int g0 = 0; g0 < ntr; g0 += 4) {
+          uint32_t rows[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            rows[i] = tb + static_cast<uint32_t>(min(g0 + i, ntr - 1)) * row_bytes;
+          const GroupSums<4, B> s = kdot4<B, W8>(rows, smem_u32(act), kmax, warp, nbw, lane);
+          const int tr = g0 + (lane >> 3);
+          if ((lane & 7) == 0 && tr < ntr) {
+            const int r = pair ? (tr < nr ? r0 + tr : nrows + r0 + tr - nr) : r0 + tr;
+#pragma unroll
+            for (int b = 0; b < B; ++b) pbuf[(warp * prow + r) * B + b] = s.s[b];
+          }
+        }
+      }
+      release_tile();
     }
   }
 
-  // Layer 0 input: the embedding rows of the step's tokens.
-  __device__ void embed_rows() {
-    const int H = a.H;
-    for (int i = tid; i < a.B * H; i += kCT) {
-      const int b = i / H, k = i % H;
-      act[b * kmax + k] = bf16_to_f(a.embed[static_cast<size_t>(tok[b]) * H + k]);
+  // End of a K-split stage: publish the warp's sums of squares, one CTA
+  // barrier, then the sums of the warps' partials (fixed order) times the
+  // RMSNorm factor of the input (norm) and the int8 row scales, through the
+  // stage's epilogue.
+  __device__ void kstage_end(int sc, int l, int K, int nrows, bool pair, bool norm,
+                             const float (&ss)[B]) {
+    float* pbuf = part + pb * (kCW * (prow + 1) * B);
+    float* sbuf = pbuf + kCW * prow * B;
+    if (lane == 0) {
+#pragma unroll
+      for (int b = 0; b < B; ++b) sbuf[warp * B + b] = ss[b];
     }
-    csync();
-    for (int i = tid; i < (h1 - h0) * a.B; i += kCT) {
-      const int r = i / a.B, b = i % a.B;
-      xown[r * B + b] = act[b * kmax + h0 + r];
-      if (a.hidden_out) a.hidden_out[static_cast<size_t>(b) * H + h0 + r] = xown[r * B + b];
+    cp_async_wait_all();  // int8 row scales of the stage
+    ab = named_sync_or(1, kCT, ab);
+    pb ^= 1;
+    if (ab) return;
+    const int nw = min(kCW, K / kBlk);
+    for (int t = tid; t < nrows * a.B; t += kCT) {
+      const int r = t / a.B, b = t % a.B;
+      float s0 = 0.f, s1 = 0.f;
+      for (int w = 0; w < nw; ++w) {
+        s0 += pbuf[(w * prow + r) * B + b];
+        if (pair) s1 += pbuf[(w * prow + nrows + r) * B + b];
+      }
+      float f = 1.f;
+      if (norm) {
+        float t2 = 0.f;
+        for (int w = 0; w < nw; ++w) t2 += sbuf[w * B + b];
+        f = rsqrtf(t2 / static_cast<float>(K) + a.eps);
+      }
+      float c0 = f, c1 = f;
+      if constexpr (W8) {
+        c0 *= wsc[r];
+        if (pair) c1 *= wsc[nrows + r];
+      }
+      epilogue(sc, l, r, b, s0 * c0, s1 * c1);
     }
   }
 
-  // Gains of an RMSNorm over K (thread tid handles k = tid + kCT * j), loaded
-  // before the gather that precedes the norm so that their latency overlaps it.
-  static constexpr int kGainRegs = 8;
-  __device__ __forceinline__ void load_gains(int K, const uint16_t* g, float (&gr)[kGainRegs]) const {
-#pragma unroll
-    for (int j = 0; j < kGainRegs; ++j) {
-      const int k = tid + kCT * j;
-      gr[j] = k < K ? bf16_to_f(__ldg(g + k)) : 0.f;
-    }
-  }
-  // In-place RMSNorm of rows act[b][0..K) with bf16 gains g (the first
-  // kGainRegs * kCT of them already in gr).
-  __device__ void rmsnorm_act(int K, const uint16_t* g, const float (&gr)[kGainRegs]) {
-    if (!ab) {
-      float ss[B];
-#pragma unroll
-      for (int b = 0; b < B; ++b) ss[b] = 0.f;
-      for (int k = tid; k < K; k += kCT) {
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-          const float x = act[b * kmax + k];
-          ss[b] = fmaf(x, x, ss[b]);
-        }
-      }
-#pragma unroll
-      for (int b = 0; b < B; ++b) {
-        ss[b] = warp_sum(ss[b]);
-        if (lane == 0) bredf[warp * B + b] = ss[b];
-      }
-    }
-    csync();
-    if (!ab) {
-      float inv[B];
-#pragma unroll
-      for (int b = 0; b < B; ++b) {
-        float t = 0.f;
-        for (int w = 0; w < kCW; ++w) t += bredf[w * B + b];
-        inv[b] = rsqrtf(t / static_cast<float>(K) + a.eps);
-      }
-#pragma unroll
-      for (int j = 0; j < kGainRegs; ++j) {
-        const int k = tid + kCT * j;
-        if (k < K) {
-#pragma unroll
-          for (int b = 0; b < B; ++b) act[b * kmax + k] = act[b * kmax + k] * inv[b] * gr[j];
-        }
-      }
-      for (int k = tid + kCT * kGainRegs; k < K; k += kCT) {
-        const float gk = bf16_to_f(g[k]);
-#pragma unroll
-        for (int b = 0; b < B; ++b) act[b * kmax + k] = act[b * kmax + k] * inv[b] * gk;
-      }
-    }
-    csync();
+  // One K-split projection stage: this warp's input, the GEMV over the
+  // stage's tiles, the CTA sum and the epilogue.
+  __device__ void kstage(int sc, int l, const uint64_t* src, uint32_t f, const uint16_t* g,
+                         int K, int nrows, int rpt, bool pair, bool norm) {
+    float ss[B];
+    if constexpr (W8) load_scales(sc, l);
+    warp_input(src, K, f, g, ss);
+    DEC_STAMP(kStampsPerLayer * l + (sc == SQ ? StQIn : sc == SO ? StOIn : sc == SU ? StUIn : StDIn));
+    wacc = 0;
+    kgemv(K, nrows, rpt, pair, part + pb * (kCW * (prow + 1) * B));
+    DEC_STAMP(kStampsPerLayer * l + (sc == SQ ? StQDot : sc == SO ? StODot : sc == SU ? StUDot : StDDot));
+    DEC_SVAL(kStampsPerLayer * l + (sc == SQ ? StWQ : sc == SO ? StWO : sc == SU ? StWU : StWD), wacc);
+    kstage_end(sc, l, K, nrows, pair, norm, ss);
   }
 
   // int8 weights: the row scales of this CTA's rows of stage sc of layer l
-  // into wsc (cp.async, 4 bytes each), issued before the stage's input
-  // gather so that their latency overlaps it; the gather's wait and barrier
+  // into wsc (cp.async, 4 bytes each), issued before the stage's input polls
+  // so that their latency overlaps them; the stage end's wait and barrier
   // complete them.  QKV: rows [q0, q1) of [Wq; Wk; Wv]; gate/up: the gate
   // rows, then the up rows; lm_head: rows [v0, v1).
   __device__ void load_scales(int sc, int l) {
@@ -813,31 +1107,26 @@ struct Cta {
     }
   }
 
-  // Row-group GEMV over ring tiles.  Rows [0, nrows) of the stage arrive
-  // `rpt` per tile, K columns (K % 256 == 0).  One warp computes whole dot
-  // products for a group of R rows (pair: R/2 rows of the first matrix and the
-  // same R/2 rows of the second, which follow them in the tile), reading the
-  // activations act[b][k] from shared memory, and reduces its lanes' R partial
-  // sums with one transposed butterfly (R = 4: 6 shuffles instead of 20).
-  // Groups are dealt to warps round-robin over the whole stage, so there is no
-  // CTA barrier per tile.  Every warp waits for every tile (no warp can run a
-  // ring ahead of the others) and releases it.
+  // Row-group GEMV over ring tiles (the lm_head): rows [0, nrows) arrive
+  // `rpt` per tile, K columns (K % 256 == 0); act holds the whole input.
+  // One warp computes whole dot products for a group of R rows and reduces
+  // its lanes' R partial sums with one transposed butterfly (R = 4: 6
+  // shuffles instead of 20); every output is multiplied by rsc[b] (the final
+  // RMSNorm factor) and, for int8 rows, the row scale.
   template <int R>
-  __device__ void gemv(int K, int nrows, int rpt, bool pair, int sc, int l) {
+  __device__ void gemv(int K, int nrows, int rpt, int sc, int l, const float (&rsc)[B]) {
     const uint32_t row_bytes = static_cast<uint32_t>(K * eb);
-    const int per = pair ? R / 2 : R;  // output rows per group
-    // A stage of many tiles (lm_head) gives each tile to one warp: only that
-    // warp waits for it, computes all its groups and releases it for the
-    // whole CTA; the other warps only advance their ring position.  The owner
-    // is the ring slot's warp (slot mod warps), so a warp's consecutive tiles
-    // are never more than one ring lap apart and its parity waits stay
-    // unambiguous.  A stage of a few tiles spreads each tile's groups over
-    // the warps.
+    // A stage of many tiles gives each tile to one warp: only that warp waits
+    // for it, computes all its groups and releases it for the whole CTA; the
+    // other warps only advance their ring position.  The owner is the ring
+    // slot's warp (slot mod warps), so a warp's consecutive tiles are never
+    // more than one ring lap apart and its parity waits stay unambiguous.  A
+    // stage of a few tiles spreads each tile's groups over the warps.
     const bool owned = (nrows + rpt - 1) / rpt > 2 * kCW;
     int gbase = 0;
     for (int r0 = 0; r0 < nrows; r0 += rpt) {
       const int nr = min(rpt, nrows - r0);
-      const int ng = (nr + per - 1) / per;
+      const int ng = (nr + R - 1) / R;
       const bool mine = !owned || rs % kCW == warp;
       if (mine) wait_tile();
       if (mine && !ab) {
@@ -852,32 +1141,22 @@ struct Cta {
           uint32_t rows[R];
 #pragma unroll
           for (int i = 0; i < R; ++i) {
-            const int j = gl * per + (i % per);
-            const int trow = (pair && i >= per) ? nr + j : j;
-            rows[i] = smem_u32(tb) + static_cast<uint32_t>(j < nr ? trow : 0) * row_bytes;
+            const int j = gl * R + i;
+            rows[i] = smem_u32(tb) + static_cast<uint32_t>(j < nr ? j : 0) * row_bytes;
           }
           const GroupSums<R, B> gs4 =
               W8 ? group_dot_i8<R, B>(rows, smem_u32(act), kmax, K >> 8, lane)
                  : group_dot<R, B>(rows, smem_u32(act), kmax, K >> 8, lane);
           const int ri = R == 4 ? (lane >> 3) : (R == 2 ? (lane >> 4) : 0);
           const bool leader = R == 4 ? ((lane & 7) == 0) : (R == 2 ? ((lane & 15) == 0) : lane == 0);
-          const int j = gl * per + ri;
-          // int8 rows: the sums are of codes; scale them by their rows' scales
-          // (gate row r0 + j, and its up row nrows + r0 + j for a pair)
-          float s0 = 1.f, s1 = 1.f;
+          const int j = gl * R + ri;
+          float s0 = 1.f;
           if constexpr (W8) {
-            if (j < nr) {
-              s0 = wsc[r0 + j];
-              if (pair) s1 = wsc[nrows + r0 + j];
-            }
+            if (j < nr) s0 = wsc[r0 + j];
           }
 #pragma unroll
-          for (int b = 0; b < B; ++b) {
-            const float sv = gs4.s[b];
-            const float su = __shfl_down_sync(0xffffffffu, sv, 16);
-            if (leader && (!pair || ri < per) && j < nr && b < a.B)
-              epilogue(sc, l, r0 + j, b, sv * s0, su * s1);
-          }
+          for (int b = 0; b < B; ++b)
+            if (leader && j < nr && b < a.B) epilogue(sc, l, r0 + j, b, gs4.s[b] * s0 * rsc[b], 0.f);
         }
       }
       gbase += ng;
@@ -893,15 +1172,12 @@ struct Cta {
         release_tile();
       }
     }
-    // the next stage overwrites act: every warp must be done reading it
-    csync();
   }
 
   // ------------------------------------------------------------- attention
   // One K (or V) row slice of the lane from a ring tile: the lane holds dims
   // [e8 * DQ, e8 * DQ + DQ) of tile row r (bf16 rows, or E4M3 codes with the
   // row scales stored after the codes).
-  static constexpr int DQ = D / 8;
   __device__ __forceinline__ void tile_row(const uint8_t* tb, int nr, int r, int e8, int kvsel,
                                            float (&o)[DQ]) const {
     if constexpr (!FP8) {
@@ -931,13 +1207,20 @@ struct Cta {
   // head g of sequence b over cached rows [j0, jc) streamed through the ring,
   // plus the new row p_b (from the gathered q/k/v, rotated and rounded as the
   // cache stores it; the CTA whose chunk holds p_b writes it to the cache).
-  // Warp w serves query head w % rep; within a warp, lane octet q8 takes every
-  // fourth row and each lane a D/8-wide slice (3-shuffle dot products).  The
-  // CTA of chunk 0 combines the chunks' partial softmax states and publishes
-  // the head outputs; other chunks publish their partial state and move on.
-  // act holds qs[rep][D], kn[D], vn[D], merge[kCW][D + 2].
+  // The query heads of a KV head form groups of at most two; every lane octet
+  // serves one group and scores each of its rows against both heads, so a
+  // K/V row is read once per group.  Octet i of a group takes rows i, i +
+  // octets per group, ...; each lane holds a D/8-wide slice (3-shuffle dot
+  // products).  The CTA of chunk 0 combines the chunks' partial softmax
+  // states and publishes the head outputs; other chunks publish their partial
+  // state and move on.  act holds qs[rep][D], kn[D], vn[D], merge[kCW][rep][D + 2].
   __device__ void attention(int l) {
     const int rep = a.Hq / a.Hkv;
+    const int ngrp = (rep + 1) >> 1;               // head groups of <= 2 heads
+    const int q8 = lane >> 3, e8 = lane & 7;
+    const int octet = warp * 4 + q8;
+    const int hg = octet % ngrp, oi = octet / ngrp, ostep = 32 / ngrp;
+    const int hb = 2 * hg, nh = min(2, rep - hb);  // this octet's heads hb, hb + 1
     const float qscale = 1.4426950408889634f / sqrtf(static_cast<float>(D));  // log2(e)/sqrt(D)
     float* qs = act;
     float* kn = act + rep * D;
@@ -946,192 +1229,217 @@ struct Cta {
     const LayerPtrs& lw = slw[l];
     const uint32_t f = flag(l);
     const int HqD = a.Hq * D;
-    const int rstep = kCW / rep;
-    const int hw = warp % rep, rw = warp / rep;
-    const bool attw = warp < rstep * rep;
-    const int q8 = lane >> 3, e8 = lane & 7;
-    for (int it = cta; it < n_items; it += nc) {
+    for (int it = cta; it < pl->n_items; it += nc) {
       int b, g, ci;
       item(it, b, g, ci);
-      const int p = pos[b];
-      const int j0 = ci * crow;
-      const int j1 = min(j0 + crow, p + 1);
+      const int p = pl->pos[b];
+      const bool live = !pl->done[b];  // a retired sequence writes no cache row
+      const int j0 = ci * pl->crow;
+      const int j1 = min(j0 + pl->crow, p + 1);
       const int jc = min(j1, p);  // cached rows [j0, jc)
       const bool has_new = (p >= j0 && p < j1);
-      // norm gains and rotation frequencies, fetched before the gather
-      float gq[DL], invf[DL / 2];
-      {
+      // -- inputs: warp w < rep takes query head g*rep + w, warp rep the key
+      //    and warp rep + 1 the value (both only for the chunk holding p_b)
+      if (warp < rep || (has_new && warp < rep + 2)) {
         const uint16_t* gn = warp < rep ? lw.w[4] : lw.w[5];
+        float gq[DL], invf[DL / 2];
 #pragma unroll
         for (int k = 0; k < DL; ++k) gq[k] = warp <= rep ? bf16_to_f(__ldg(gn + lane + 32 * k)) : 0.f;
 #pragma unroll
         for (int k = 0; k < DL / 2; ++k) invf[k] = __ldg(a.inv_freq + lane + 32 * k);
-      }
-      // -- q heads of the group, k_g and v_g of sequence b -> qs, kn, vn
-      {
-        const uint64_t* src = a.x_qkv + static_cast<size_t>(b) * nqkv;
-        const int qn = rep * D;
-        const int qoff = g * rep * D, koff = HqD + g * D, voff = HqD + a.Hkv * D + g * D;
-        gather(qn + 2 * D, f, [=](int w) {
-          return src + (w < qn ? qoff + w : (w < qn + D ? koff + (w - qn) : voff + (w - qn - D)));
-        });
-        if (!ab)
-          for (int i = tid; i < qn + 2 * D; i += kCT)
-            act[i] = __uint_as_float(static_cast<uint32_t>(stg[i]));
-        csync();
-      }
-      // -- q/k RMSNorm + RoPE (warp w < rep: q head; rep: k; rep+1: v)
-      if (!ab && warp < rep + 2) {
-        float* x = warp < rep ? qs + warp * D : (warp == rep ? kn : vn);
-        float v[DL];
+        const uint64_t* src = a.x_qkv + static_cast<size_t>(b) * nqkv +
+                              (warp < rep ? (g * rep + warp) * D
+                                          : HqD + (warp - rep) * a.Hkv * D + g * D);
+        uint64_t* ws = stg + warp * kWarpStage;
+        warp_gather(ws, D, f, [=](int i) { return src + i; });
+        if (!ab) {
+          float v[DL];
 #pragma unroll
-        for (int k = 0; k < DL; ++k) v[k] = x[lane + 32 * k];
-        if (warp <= rep) {
-          float ss = 0.f;
+          for (int k = 0; k < DL; ++k) v[k] = __uint_as_float(static_cast<uint32_t>(ws[lane + 32 * k]));
+          if (warp <= rep) {  // q/k RMSNorm + RoPE
+            float ss = 0.f;
 #pragma unroll
-          for (int k = 0; k < DL; ++k) ss = fmaf(v[k], v[k], ss);
-          ss = warp_sum(ss);
-          const float inv = rsqrtf(ss / static_cast<float>(D) + a.eps);
+            for (int k = 0; k < DL; ++k) ss = fmaf(v[k], v[k], ss);
+            ss = warp_sum(ss);
+            const float inv = rsqrtf(ss / static_cast<float>(D) + a.eps);
 #pragma unroll
-          for (int k = 0; k < DL; ++k) v[k] = v[k] * inv * gq[k];
+            for (int k = 0; k < DL; ++k) v[k] = v[k] * inv * gq[k];
 #pragma unroll
-          for (int k = 0; k < DL / 2; ++k) {
-            const float ang = __fmul_rn(static_cast<float>(p), invf[k]);
-            float sn, cs;
-            rope_sincos(ang, &sn, &cs);
-            const float x1 = v[k], x2 = v[k + DL / 2];
-            v[k] = x1 * cs - x2 * sn;
-            v[k + DL / 2] = x2 * cs + x1 * sn;
-          }
-        }
-        if (warp >= rep) {
-          // the new K / V row as the cache stores it
-          const size_t row = kv_row(l, warp - rep, b, g, p);
-          if constexpr (!FP8) {
-            uint16_t* dstp = reinterpret_cast<uint16_t*>(a.kv) + row * D;
-#pragma unroll
-            for (int k = 0; k < DL; ++k) {
-              const uint16_t h = f_to_bf16(v[k]);
-              v[k] = bf16_to_f(h);
-              if (has_new) dstp[lane + 32 * k] = h;
-            }
-          } else {
-            uint8_t code[DL];
-            const float sc = quantize_row_e4m3<DL>(v, code);
-            if (has_new) {
-              uint8_t* dstp = a.kv + row * D;
-#pragma unroll
-              for (int k = 0; k < DL; ++k) dstp[lane + 32 * k] = code[k];
-              if (lane == 0) a.kv_scales[row] = sc;
+            for (int k = 0; k < DL / 2; ++k) {
+              const float ang = __fmul_rn(static_cast<float>(p), invf[k]);
+              float sn, cs;
+              rope_sincos(ang, &sn, &cs);
+              const float x1 = v[k], x2 = v[k + DL / 2];
+              v[k] = x1 * cs - x2 * sn;
+              v[k + DL / 2] = x2 * cs + x1 * sn;
             }
           }
-        }
+          if (warp >= rep) {
+            // the new K / V row as the cache stores it, written by this chunk
+            const size_t row = kv_row(l, warp - rep, b, g, p);
+            if constexpr (!FP8) {
+              uint16_t* dstp = reinterpret_cast<uint16_t*>(a.kv) + row * D;
 #pragma unroll
-        for (int k = 0; k < DL; ++k) x[lane + 32 * k] = v[k];
+              for (int k = 0; k < DL; ++k) {
+                const uint16_t h = f_to_bf16(v[k]);
+                v[k] = bf16_to_f(h);
+                if (live) dstp[lane + 32 * k] = h;
+              }
+            } else {
+              uint8_t code[DL];
+              const float sc = quantize_row_e4m3<DL>(v, code);
+              if (live) {
+                uint8_t* dstp = a.kv + row * D;
+#pragma unroll
+                for (int k = 0; k < DL; ++k) dstp[lane + 32 * k] = code[k];
+                if (lane == 0) a.kv_scales[row] = sc;
+              }
+            }
+          }
+          float* x = warp < rep ? qs + warp * D : (warp == rep ? kn : vn);
+#pragma unroll
+          for (int k = 0; k < DL; ++k) x[lane + 32 * k] = v[k];
+        }
       }
-      csync();
+      ab = named_sync_or(1, kCT, ab);
       DEC_STAMP(kStampsPerLayer * l + StAttIn);
-      // -- this chunk's rows: online softmax per lane octet
-      float qv[DQ], acc[DQ];
-      float m = -INFINITY, ls = 0.f;
+      wacc = 0;
+      // -- this chunk's rows: online softmax per (lane octet, head)
+      float qv[2][DQ], acc[2][DQ], m[2], ls[2];
 #pragma unroll
-      for (int k = 0; k < DQ; ++k) {
-        acc[k] = 0.f;
-        qv[k] = (attw && !ab) ? qs[hw * D + e8 * DQ + k] * qscale : 0.f;
+      for (int hh = 0; hh < 2; ++hh) {
+        m[hh] = -INFINITY;
+        ls[hh] = 0.f;
+#pragma unroll
+        for (int k = 0; k < DQ; ++k) {
+          acc[hh][k] = 0.f;
+          qv[hh][k] = (!ab && hh < nh) ? qs[(hb + hh) * D + e8 * DQ + k] * qscale : 0.f;
+        }
       }
       for (int j = j0; j < jc; j += art) {
         const int nr = min(art, jc - j);
         wait_tile();
-        if (!ab && attw) {
+        if (j == j0) DEC_STAMP(kStampsPerLayer * l + StAttTile);
+        if (!ab) {
           const uint8_t* tb = ring + static_cast<size_t>(rs) * kSlotBytes;
-          for (int r4 = rw * 4; r4 < nr; r4 += rstep * 4) {
-            const int r = r4 + q8;
+          for (int r0 = 0; r0 < nr; r0 += ostep) {  // warp-uniform trip count
+            const int r = r0 + oi;
             const bool ok = r < nr;
             float kr[DQ];
             tile_row(tb, nr, ok ? r : 0, e8, 0, kr);
-            float s = 0.f;
+            float s[2];
 #pragma unroll
-            for (int k = 0; k < DQ; ++k) s = fmaf(qv[k], kr[k], s);
-            s += __shfl_xor_sync(0xffffffffu, s, 4);
-            s += __shfl_xor_sync(0xffffffffu, s, 2);
-            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            for (int hh = 0; hh < 2; ++hh) {
+              float t = 0.f;
+#pragma unroll
+              for (int k = 0; k < DQ; ++k) t = fmaf(qv[hh][k], kr[k], t);
+              t += __shfl_xor_sync(0xffffffffu, t, 4);
+              t += __shfl_xor_sync(0xffffffffu, t, 2);
+              t += __shfl_xor_sync(0xffffffffu, t, 1);
+              s[hh] = t;
+            }
             if (ok) {
               float vr[DQ];
               tile_row(tb, nr, r, e8, 1, vr);
-              const float mn = fmaxf(m, s);
-              const float al = exp2f(m - mn), pe = exp2f(s - mn);
-              ls = ls * al + pe;
 #pragma unroll
-              for (int k = 0; k < DQ; ++k) acc[k] = fmaf(acc[k], al, pe * vr[k]);
-              m = mn;
+              for (int hh = 0; hh < 2; ++hh) {
+                if (hh < nh) {
+                  const float mn = fmaxf(m[hh], s[hh]);
+                  const float al = exp2f(m[hh] - mn), pe = exp2f(s[hh] - mn);
+                  ls[hh] = ls[hh] * al + pe;
+#pragma unroll
+                  for (int k = 0; k < DQ; ++k) acc[hh][k] = fmaf(acc[hh][k], al, pe * vr[k]);
+                  m[hh] = mn;
+                }
+              }
             }
           }
         }
         release_tile();
       }
-      if (!ab && attw && rw == 0 && has_new) {  // the new row, by octet 0
-        float s = 0.f;
+      if (!ab && has_new && warp == 0) {  // the new row, kept by the first octet of each group
+        float s[2];
 #pragma unroll
-        for (int k = 0; k < DQ; ++k) s = fmaf(qv[k], kn[e8 * DQ + k], s);
-        s += __shfl_xor_sync(0xffffffffu, s, 4);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        if (q8 == 0) {
-          const float mn = fmaxf(m, s);
-          const float al = exp2f(m - mn), pe = exp2f(s - mn);
-          ls = ls * al + pe;
+        for (int hh = 0; hh < 2; ++hh) {
+          float t = 0.f;
 #pragma unroll
-          for (int k = 0; k < DQ; ++k) acc[k] = fmaf(acc[k], al, pe * vn[e8 * DQ + k]);
-          m = mn;
+          for (int k = 0; k < DQ; ++k) t = fmaf(qv[hh][k], kn[e8 * DQ + k], t);
+          t += __shfl_xor_sync(0xffffffffu, t, 4);
+          t += __shfl_xor_sync(0xffffffffu, t, 2);
+          t += __shfl_xor_sync(0xffffffffu, t, 1);
+          s[hh] = t;
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          if (hh < nh && oi == 0) {
+            const float mn = fmaxf(m[hh], s[hh]);
+            const float al = exp2f(m[hh] - mn), pe = exp2f(s[hh] - mn);
+            ls[hh] = ls[hh] * al + pe;
+#pragma unroll
+            for (int k = 0; k < DQ; ++k) acc[hh][k] = fmaf(acc[hh][k], al, pe * vn[e8 * DQ + k]);
+            m[hh] = mn;
+          }
         }
       }
-      // merge the four octets of the warp, octet 0 writes the warp's state
-      if (!ab && attw) {
+      // merge the octets of the warp that serve the same head group (xor 16,
+      // and xor 8 when there is one group); the first octet of each group
+      // writes the warp's state
+      if (!ab) {
 #pragma unroll
         for (int o = 8; o <= 16; o <<= 1) {
-          const float mo = __shfl_xor_sync(0xffffffffu, m, o);
-          const float lo = __shfl_xor_sync(0xffffffffu, ls, o);
-          const float mn = fmaxf(m, mo);
-          const float e1 = (m == -INFINITY) ? 0.f : exp2f(m - mn);
-          const float e2 = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
-          ls = ls * e1 + lo * e2;
+          if (o == 8 && ngrp != 1) continue;
 #pragma unroll
-          for (int k = 0; k < DQ; ++k) {
-            const float ao = __shfl_xor_sync(0xffffffffu, acc[k], o);
-            acc[k] = acc[k] * e1 + ao * e2;
+          for (int hh = 0; hh < 2; ++hh) {
+            const float mo = __shfl_xor_sync(0xffffffffu, m[hh], o);
+            const float lo = __shfl_xor_sync(0xffffffffu, ls[hh], o);
+            const float mn = fmaxf(m[hh], mo);
+            const float e1 = (m[hh] == -INFINITY) ? 0.f : exp2f(m[hh] - mn);
+            const float e2 = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+            ls[hh] = ls[hh] * e1 + lo * e2;
+#pragma unroll
+            for (int k = 0; k < DQ; ++k) {
+              const float ao = __shfl_xor_sync(0xffffffffu, acc[hh][k], o);
+              acc[hh][k] = acc[hh][k] * e1 + ao * e2;
+            }
+            m[hh] = mn;
           }
-          m = mn;
         }
-        if (q8 == 0) {
-          float* mg = merge + static_cast<size_t>(warp) * (D + 2);
+        if (q8 < ngrp) {
 #pragma unroll
-          for (int k = 0; k < DQ; ++k) mg[e8 * DQ + k] = acc[k];
-          if (e8 == 0) {
-            mg[D] = m;
-            mg[D + 1] = ls;
+          for (int hh = 0; hh < 2; ++hh) {
+            if (hh < nh) {
+              float* mg = merge + (static_cast<size_t>(warp) * rep + hb + hh) * (D + 2);
+#pragma unroll
+              for (int k = 0; k < DQ; ++k) mg[e8 * DQ + k] = acc[hh][k];
+              if (e8 == 0) {
+                mg[D] = m[hh];
+                mg[D + 1] = ls[hh];
+              }
+            }
           }
         }
       }
       csync();
       DEC_STAMP(kStampsPerLayer * l + StAttRows);
+      DEC_SVAL(kStampsPerLayer * l + StWA, wacc);
       // -- this chunk's partial state (m in log2 units, l, unnormalised acc)
       const bool combiner = (ci == 0);
       const int pc = a.part_chunks;
       const uint64_t* pbase =
           a.part + (static_cast<size_t>(b) * a.Hq + g * rep) * pc * (D + 2);
-      float RM[3], RL[3], RA[3];  // (h, d) = t / D, t % D for t = tid + kCT * i
+      float RM[2], RL[2], RA[2];  // (h, d) = t / D, t % D for t = tid + kCT * i
 #pragma unroll
-      for (int i = 0; i < 3; ++i) {
+      for (int i = 0; i < 2; ++i) {
         const int t = tid + kCT * i;
         RM[i] = -INFINITY;
         RL[i] = RA[i] = 0.f;
         if (!ab && t < rep * D) {
           const int h = t / D, d = t % D;
           float M = -INFINITY;
-          for (int w = h; w < rstep * rep; w += rep) M = fmaxf(M, merge[w * (D + 2) + D]);
+          for (int w = 0; w < kCW; ++w) M = fmaxf(M, merge[(w * rep + h) * (D + 2) + D]);
           float Ls = 0.f, A = 0.f;
-          for (int w = h; w < rstep * rep; w += rep) {
-            const float* mg = merge + w * (D + 2);
+          for (int w = 0; w < kCW; ++w) {
+            const float* mg = merge + (w * rep + h) * (D + 2);
             const float e = (mg[D] == -INFINITY) ? 0.f : exp2f(mg[D] - M);
             Ls += mg[D + 1] * e;
             A += mg[d] * e;
@@ -1151,7 +1459,7 @@ struct Cta {
         }
       }
       if (combiner) {  // uniform over the CTA: ci is the item's
-        const int nc1 = nchunk[b] - 1;
+        const int nc1 = pl->nchunk[b] - 1;
         const int win = kStageWords / (rep * (D + 2));
         for (int c0 = 1; c0 <= nc1; c0 += win) {
           const int nw = min(win, nc1 - c0 + 1);
@@ -1162,7 +1470,7 @@ struct Cta {
           });
           if (!ab) {
 #pragma unroll
-            for (int i = 0; i < 3; ++i) {
+            for (int i = 0; i < 2; ++i) {
               const int t = tid + kCT * i;
               if (t < rep * D) {
                 const int h = t / D, d = t % D;
@@ -1184,7 +1492,7 @@ struct Cta {
         }
         if (!ab) {
 #pragma unroll
-          for (int i = 0; i < 3; ++i) {
+          for (int i = 0; i < 2; ++i) {
             const int t = tid + kCT * i;
             if (t < rep * D) {
               const int h = t / D, d = t % D;
@@ -1198,65 +1506,61 @@ struct Cta {
   }
 
   // ------------------------------------------------------------- one step
-  __device__ void consumer() {
+  __device__ void one_step() {
     const int H = a.H, F = a.F, HqD = a.Hq * D;
 #pragma unroll
     for (int b = 0; b < B; ++b) {
       best_v[b] = -INFINITY;
       best_i[b] = 0x7fffffff;
     }
-    float gr[kGainRegs];
     DEC_STAMP(kStampsPerLayer * a.L + StBegin);
-    // Stages of a layer: QKV, attention, o_proj, gate/up, down; the lm_head
-    // runs as stage QKV of layer L.  One copy of each piece of code.
-    for (int l = 0; l <= a.L; ++l) {
-      const bool lm = (l == a.L);
-      for (int st = 0; st < kStages; ++st) {
-        if (lm && st != SQ) break;
-        if (st == SA) {
-          DEC_STAMP(kStampsPerLayer * l + StQkv);
-          attention(l);
-          DEC_STAMP(kStampsPerLayer * l + StAtt);
-          continue;
-        }
-        const uint64_t* src;
-        const uint16_t* gain = nullptr;
-        int K, nrows, rpt, sc;
-        uint32_t fin;
-        bool pair = false;
-        if (st == SQ) {
-          src = a.x_out; K = H; fin = flag(l - 1);
-          gain = lm ? a.final_norm : slw[l].w[0];
-          nrows = lm ? v1 - v0 : q1 - q0; rpt = rpt_h; sc = lm ? SLM : SQ;
-        } else if (st == SO) {
-          src = a.x_o; K = HqD; fin = flag(l); nrows = h1 - h0; rpt = rpt_o; sc = SO;
-        } else if (st == SU) {
-          src = a.x_mid; K = H; fin = flag(l); gain = slw[l].w[7];
-          nrows = f1 - f0; rpt = rpt_u; pair = true; sc = SU;
-        } else {
-          src = a.x_u; K = F; fin = flag(l); nrows = h1 - h0; rpt = rpt_d; sc = SD;
-        }
-        if (gain) load_gains(K, gain, gr);
-        if constexpr (W8) load_scales(sc, l);
-        if (st == SQ && l == 0) {
-          if constexpr (W8) cp_async_wait_all();  // made visible by embed_rows' barrier
-          embed_rows();
-        } else {
-          gather_x(src, K, fin);
-        }
-        if (st == SQ) DEC_STAMP(kStampsPerLayer * l + StQGath);
-        if (st == SO) DEC_STAMP(kStampsPerLayer * l + StOGath);
-        if (st == SU) DEC_STAMP(kStampsPerLayer * l + StUGath);
-        if (st == SD) DEC_STAMP(kStampsPerLayer * l + StDGath);
-        if (gain) rmsnorm_act(K, gain, gr);
-        if (st == SQ) DEC_STAMP(kStampsPerLayer * l + StQNorm);
-        if (st == SU) DEC_STAMP(kStampsPerLayer * l + StUNorm);
-        if (pair || nrows > 2 * kCW) gemv<4>(K, nrows, rpt, pair, sc, l);
-        else gemv<1>(K, nrows, rpt, pair, sc, l);
-        if (st == SO) DEC_STAMP(kStampsPerLayer * l + StO);
-        if (st == SU) DEC_STAMP(kStampsPerLayer * l + StU);
-        if (st == SD) DEC_STAMP(kStampsPerLayer * l + StD);
+    // the CTA's residual rows start as the embedding rows
+    for (int i = tid; i < (h1 - h0) * a.B; i += kCT) {
+      const int r = i / a.B, b = i % a.B;
+      const float x = bf16_to_f(a.embed[static_cast<size_t>(pl->tok[b]) * H + h0 + r]);
+      xown[r * B + b] = x;
+      if (a.hidden_out) a.hidden_out[static_cast<size_t>(b) * H + h0 + r] = x;
+    }
+    for (int l = 0; l < a.L; ++l) {
+      const LayerPtrs& lw = slw[l];
+      const uint32_t f = flag(l);
+      // QKV (the layer-0 input is the embedding row)
+      kstage(SQ, l, l == 0 ? nullptr : a.x_out, flag(l - 1), lw.w[0], H, q1 - q0, rpt_h, false,
+             true);
+      DEC_STAMP(kStampsPerLayer * l + StQkv);
+      attention(l);
+      DEC_STAMP(kStampsPerLayer * l + StAtt);
+      kstage(SO, l, a.x_o, f, nullptr, HqD, h1 - h0, rpt_o, false, false);
+      DEC_STAMP(kStampsPerLayer * l + StO);
+      kstage(SU, l, a.x_mid, f, lw.w[7], H, f1 - f0, rpt_u, true, true);
+      DEC_STAMP(kStampsPerLayer * l + StU);
+      kstage(SD, l, a.x_u, f, nullptr, F, h1 - h0, rpt_d, false, false);
+      DEC_STAMP(kStampsPerLayer * l + StD);
+    }
+    // final norm + lm_head: the whole input in act, the norm factor applied
+    // to every logit
+    DEC_STAMP(kStampsPerLayer * a.L + StLmStart);
+    {
+      float ss[B], rsc[B];
+      if constexpr (W8) load_scales(SLM, a.L);
+      warp_input(a.x_out, H, flag(a.L - 1), a.final_norm, ss);
+      float* sbuf = part + pb * (kCW * (prow + 1) * B) + kCW * prow * B;
+      if (lane == 0) {
+#pragma unroll
+        for (int b = 0; b < B; ++b) sbuf[warp * B + b] = ss[b];
       }
+      cp_async_wait_all();
+      ab = named_sync_or(1, kCT, ab);
+      pb ^= 1;
+      const int nw = min(kCW, H / kBlk);
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        float t2 = 0.f;
+        for (int w = 0; w < nw; ++w) t2 += sbuf[w * B + b];
+        rsc[b] = rsqrtf(t2 / static_cast<float>(H) + a.eps);
+      }
+      DEC_STAMP(kStampsPerLayer * a.L + StLmGath);
+      gemv<4>(H, v1 - v0, rpt_h, SLM, a.L, rsc);
     }
     DEC_STAMP(kStampsPerLayer * a.L + StLmDone);
     // CTA argmax -> one 64-bit atomicMax per sequence (ties: lowest id)
@@ -1299,13 +1603,66 @@ struct Cta {
     }
     DEC_STAMP(kStampsPerLayer * a.L + StEnd);
   }
+
+  // After this CTA's argmax of step st is in: the CTA that arrives last takes
+  // the step's ids from the argmax keys (clearing them for the next step),
+  // writes out_ids[st] and publishes the ids as tagged words for the next
+  // step.  A retired sequence keeps emitting the end token.  For a multi-step
+  // launch it also advances the caller's positions (a sequence stays at the
+  // row of the step that emitted the end token) and, when every sequence has
+  // retired or the next step would be invalid, fills the remaining steps'
+  // ids.  One thread.
+  __device__ void step_end(int st) {
+    __threadfence();
+    const unsigned old = atomicAdd(a.step_cnt, 1u);
+    if (old != static_cast<unsigned>(st + 1) * static_cast<unsigned>(nc) - 1u) return;
+    __threadfence();
+    int32_t* out = a.out_ids + static_cast<size_t>(st) * a.B;
+    int all = 1, bad = 0;
+    for (int b = 0; b < a.B; ++b) {
+      const unsigned long long key = atomicExch(&a.amax_key[b], 0ull);
+      int id = key == 0ull ? -1 : static_cast<int>(~static_cast<uint32_t>(key & 0xffffffffull));
+      const bool was_done = cplan->done[b] != 0;
+      if (was_done) id = a.eos;
+      out[b] = id;
+      const bool done = was_done || (a.eos >= 0 && id == a.eos);
+      const int np = done ? cplan->pos[b] : cplan->pos[b] + 1;
+      if (a.gen_pos) a.gen_pos[b] = np;
+      all &= done;
+      if (!done && (id < 0 || id >= a.V)) bad |= kDevBadTok;
+      if (!done && np >= a.max_ctx) bad |= kDevBadPos;
+      st_tagged(a.tokw + b, __int_as_float(id), tok_flag(st));
+    }
+    if (st + 1 < a.n_steps && (all || bad)) {
+      if (bad) atomicOr(a.status, bad);
+      for (int s2 = st + 1; s2 < a.n_steps; ++s2)
+        for (int b = 0; b < a.B; ++b)
+          a.out_ids[static_cast<size_t>(s2) * a.B + b] = bad ? -1 : a.eos;
+    }
+  }
+
+  // The consumers' step loop: one step per iteration, then the next step's
+  // ids and plan (thread 0 polls, the others wait at the barrier).
+  __device__ void consumer() {
+    for (int st = 0;; ++st) {
+      seq = seq0 + static_cast<uint32_t>(st);
+      one_step();
+      csync();  // this CTA's argmax keys are in
+      if (tid == 0 && !ab) step_end(st);
+      if (st + 1 >= a.n_steps || ab) break;
+      if (tid == 0) sints[0] = next_step(*cplan, tok_flag(st)) ? 0 : 1;
+      ab = named_sync_or(1, kCT, tid == 0 ? sints[0] : 0);
+      if (ab || cplan->bad || cplan->all_done) break;
+    }
+  }
 };
 
 template <int B, int D, bool FP8, bool W8>
 __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a, int kmax) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Cta<B, D, FP8, W8> c(a, smem, kmax);
-  // ---- set-up: layer pointer table, barriers, step inputs, validation
+  // ---- set-up: layer pointer table, barriers, the first step's inputs and
+  // plan (both sides' copies), validation
   {
     const uint64_t* src = reinterpret_cast<const uint64_t*>(a.layers);
     uint64_t* dst = reinterpret_cast<uint64_t*>(const_cast<LayerPtrs*>(c.slw));
@@ -1318,43 +1675,46 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     }
     fence_mbar_init();
     int bad = 0;
+    Plan& P = *c.cplan;
     for (int b = 0; b < a.B; ++b) {
       const int p = a.positions[b], t = a.token_ids[b];
-      c.sints[8 + b] = p;
-      c.sints[16 + b] = t;
+      P.pos[b] = p;
+      P.tok[b] = t;
+      P.done[b] = 0;
       if (p < 0 || p >= a.max_ctx) bad |= kDevBadPos;
       if (t < 0 || t >= a.V) bad |= kDevBadTok;
     }
+    P.bad = bad;
+    if (!bad) c.make_plan(P);
+    *c.pplan = P;
     c.sints[1] = bad;
     c.sints[2] = static_cast<int>(ld_relaxed_u32(a.seq));
     if (bad && blockIdx.x == 0) atomicOr(a.status, bad);
   }
   __syncthreads();
   const int bad = c.sints[1];
-  c.seq = static_cast<uint32_t>(c.sints[2]);
-  if (!bad) c.plan_attention();
-  __syncthreads();
+  c.seq0 = c.seq = static_cast<uint32_t>(c.sints[2]);
   if (!bad) {
     if (c.warp == kCW) c.producer();
     else c.consumer();
   }
   __syncthreads();
-  // ---- exit: the last CTA publishes the ids and resets the step state
+  // ---- exit: the last CTA resets the launch state; a launch that saw an
+  // invalid input or ran out of a wait reports -1 for every id
   if (threadIdx.x == 0) {
     __threadfence();
     const unsigned old = atomicAdd(a.exit_cnt, 1u);
     if (old == gridDim.x - 1) {
       __threadfence();
       const int aborted = ld_relaxed_i32(a.abort_flag);
-      for (int b = 0; b < a.B; ++b) {
-        const unsigned long long key = atomicExch(&a.amax_key[b], 0ull);
-        a.out_ids[b] = (bad || aborted || key == 0ull)
-                           ? -1
-                           : static_cast<int32_t>(~static_cast<uint32_t>(key & 0xffffffffull));
+      if (bad || aborted) {
+        for (int i = 0; i < a.n_steps * a.B; ++i) a.out_ids[i] = -1;
+        for (int b = 0; b < a.B; ++b) atomicExch(&a.amax_key[b], 0ull);
       }
       atomicExch(a.abort_flag, 0);
+      atomicExch(a.step_cnt, 0u);
       atomicExch(a.exit_cnt, 0u);
-      atomicAdd(a.seq, 1u);
+      atomicAdd(a.seq, static_cast<unsigned>(a.n_steps));
       __threadfence();
     }
   }
@@ -1364,13 +1724,16 @@ template <int B, int D, bool FP8, bool W8>
 cudaError_t launch_bd(const StepArgs& a, int ctas, size_t smem, int kmax,
                       cudaStream_t s) {
   auto k = step_kernel<B, D, FP8, W8>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
   StepArgs args = a;
   void* params[] = {&args, &kmax};
   return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k), dim3(ctas),
                                      dim3(kStepThreads), params, smem, s);
+}
+
+template <int B, int D, bool FP8, bool W8>
+cudaError_t attr_bd(size_t smem) {
+  return cudaFuncSetAttribute(step_kernel<B, D, FP8, W8>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
 }
 
 }  // namespace
@@ -1379,32 +1742,59 @@ static int kmax_of(int H, int F, int HqD) {
   int k = H > F ? H : F;
   return k > HqD ? k : HqD;
 }
-size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep, int wsc_n) {
-  return carve(nslot, B, kmax_of(H, F, HqD), D, rep, wsc_n).total;
+size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep, int wsc_n,
+                       int prow) {
+  return carve(nslot, B, kmax_of(H, F, HqD), D, rep, wsc_n, prow).total;
 }
 
-int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int wsc_n, int smem_optin) {
+int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int wsc_n, int prow,
+                   int smem_optin) {
   int best = 0;
   for (int n = 1; n <= 16; ++n)
-    if (step_smem_bytes(n, B, H, F, HqD, D, rep, wsc_n) <= static_cast<size_t>(smem_optin))
+    if (step_smem_bytes(n, B, H, F, HqD, D, rep, wsc_n, prow) <= static_cast<size_t>(smem_optin))
       best = n;
   return best;
 }
 
-int step_wsc_slots(int H, int F, int nqkv, int V, int ctas) {
-  auto most = [&](int n) {  // the largest split_at range over the CTAs
-    int m = 0;
-    for (int i = 0; i < ctas; ++i) {
-      const int c = split_at(n, ctas, i + 1) - split_at(n, ctas, i);
-      m = c > m ? c : m;
-    }
-    return m;
-  };
-  int m = most(nqkv);
-  m = most(H) > m ? most(H) : m;
-  m = 2 * most(F) > m ? 2 * most(F) : m;
-  m = most(V) > m ? most(V) : m;
+// The largest split_at range of n over `ctas` parts.
+static int most_rows(int n, int ctas) {
+  int m = 0;
+  for (int i = 0; i < ctas; ++i) {
+    const int c = split_at(n, ctas, i + 1) - split_at(n, ctas, i);
+    m = c > m ? c : m;
+  }
   return m;
+}
+
+int step_wsc_slots(int H, int F, int nqkv, int V, int ctas) {
+  int m = most_rows(nqkv, ctas);
+  m = most_rows(H, ctas) > m ? most_rows(H, ctas) : m;
+  m = 2 * most_rows(F, ctas) > m ? 2 * most_rows(F, ctas) : m;
+  m = most_rows(V, ctas) > m ? most_rows(V, ctas) : m;
+  return m;
+}
+
+int step_part_rows(int H, int F, int nqkv, int ctas) {
+  int m = most_rows(nqkv, ctas);
+  m = most_rows(H, ctas) > m ? most_rows(H, ctas) : m;
+  m = 2 * most_rows(F, ctas) > m ? 2 * most_rows(F, ctas) : m;
+  return m;
+}
+
+// Sets the dynamic shared-memory limit of the kernel instantiations a
+// handle launches (once, when the handle is created).
+cudaError_t step_set_smem(int B, int D, bool w8, size_t smem) {
+  cudaError_t e = cudaErrorInvalidValue;
+#define DEC_ATTR(BB, DD)                                                        \
+  if (B == BB && D == DD) {                                                     \
+    e = w8 ? attr_bd<BB, DD, false, true>(smem) : attr_bd<BB, DD, false, false>(smem); \
+    if (e == cudaSuccess)                                                       \
+      e = w8 ? attr_bd<BB, DD, true, true>(smem) : attr_bd<BB, DD, true, false>(smem); \
+  }
+  DEC_ATTR(1, 128) DEC_ATTR(2, 128) DEC_ATTR(3, 128) DEC_ATTR(4, 128)
+  DEC_ATTR(1, 64) DEC_ATTR(2, 64) DEC_ATTR(3, 64) DEC_ATTR(4, 64)
+#undef DEC_ATTR
+  return e;
 }
 
 cudaError_t launch_step_small(const StepArgs& a, int ctas, size_t smem, cudaStream_t s) {

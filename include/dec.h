@@ -133,7 +133,9 @@ typedef struct dec_weights {
 
 typedef struct dec_handle dec_handle;
 
-/* Create a handle for the current CUDA device.  Validates the shape, copies
+/* Create a handle for the current CUDA device (the pages define no API: this
+ * call, like dec_kv_bytes, dec_kv_alloc and dec_check, is the library's own
+ * boundary around the step they describe).  Validates the shape, copies
  * the weight pointer table (not the weights: they stay caller-owned and must
  * stay alive and unchanged), allocates the workspace (activation exchange
  * buffers, attention partials, counters; a few MB) and picks the kernel
@@ -194,13 +196,16 @@ typedef struct dec_kv {
   int dtype;          /* dec_kv_dtype */
 } dec_kv;
 
-/* Bytes a cache of this size needs (0 for an invalid request). */
+/* Bytes a cache of this size needs (0 for an invalid request).  No page
+ * defines this call; the layout above is the library's own. */
 size_t dec_kv_bytes(const dec_handle *h, int batch, int max_ctx, int dtype);
 
 /* Byte offset of the fp32 scale array inside an fp8 cache (0 for bf16). */
 size_t dec_kv_scale_offset(const dec_handle *h, int batch, int max_ctx, int dtype);
 
-/* Bind a caller-owned device buffer as a KV cache.  Allocates nothing and
+/* Bind a caller-owned device buffer as a KV cache (no page defines this call;
+ * the caller owning the cache follows the Baseten article's host-owned
+ * sequence state, "Minimizing host-to-device syncs").  Allocates nothing and
  * does not touch the buffer's contents.  DEC_ERR_KV_SIZE if buf_bytes <
  * dec_kv_bytes(), DEC_ERR_ALIGN unless buf is 256-byte aligned. */
 int dec_kv_alloc(dec_handle *h, int batch, int max_ctx, int dtype, void *buf,
@@ -235,12 +240,19 @@ int dec_step(dec_handle *h, int batch, const int32_t *token_ids, const int32_t *
  *   positions  int32 [batch] (device)   the rows the first step writes;
  *                                       advanced IN PLACE after every step
  *   out_ids    int32 [n_steps][batch]   step i's ids (the input of step i+1)
- *   eos        end-of-sequence id, or -1 for none.  A sequence that emits
- *              it is retired: its position stays at that step's row and its
- *              later outputs are eos.
- * Equivalent to n_steps dec_step calls that feed out_ids back and advance
- * the positions by one; asynchronous (no host read-back inside); device
- * errors as in dec_step (dec_check). */
+ *   eos        end-of-sequence id in [0, vocab), or -1 for none.  A sequence
+ *              that emits it is retired: its position stays at the row of
+ *              that step, its later outputs are eos and no later step writes
+ *              its cache.
+ * Equivalent to n_steps dec_step calls that feed out_ids back and advance the
+ * positions by one.  Batches of 1..4 run as ONE launch of the persistent
+ * kernel, which loops over the steps itself; once every sequence has retired
+ * it stops early (the remaining out_ids rows are eos).  A sequence whose next
+ * position would reach max_ctx stops the loop: DEC_DEV_BAD_POSITION, and the
+ * steps that could not run report -1.  Batches of 5..64 launch the batched
+ * step once per step with a small bookkeeping kernel in between.
+ * Asynchronous (no host read-back inside); other device errors as in dec_step
+ * (dec_check). */
 int dec_generate(dec_handle *h, int batch, int n_steps, const int32_t *token_ids,
                  int32_t *positions, const dec_kv *kv, int32_t *out_ids, int eos, void *stream);
 
@@ -294,7 +306,9 @@ int dec_step_host(dec_handle *h, int batch, const int32_t *token_ids_host,
                   const int32_t *positions_host, const dec_kv *kv, int32_t *out_ids_host,
                   float *out_logits_host, void *stream);
 
-/* Synchronise `stream`, then return and clear the device status bits
+/* (No page defines this call: it reports the conditions the device detected
+ * without any read-back inside a step.)
+ * Synchronise `stream`, then return and clear the device status bits
  * (DEC_DEV_*; 0 when every step since the last check was clean), or a
  * negative dec_status if the synchronisation itself failed. */
 int dec_check(dec_handle *h, void *stream);

@@ -94,10 +94,20 @@ def test_generate_equals_step_loop(batch, max_batch):
     dec.close()
 
 
-def test_generate_retires_a_sequence_at_eos():
-    batch, n = 2, 10
-    n0s = [30, 40]
-    s, w, kv_host, dec, toks = _fixture(batch, 120, n0s)
+def _seq_rows(kv, b, lo, hi):
+    """Cache rows [lo, hi) of sequence b (all layers, K and V) as raw bits."""
+    return kv.values[:, :, b, :, lo:hi].contiguous().view(torch.int16)
+
+
+@pytest.mark.parametrize("batch,max_batch", [(2, 2), (6, 8)])
+def test_generate_retires_a_sequence_at_eos(batch, max_batch):
+    """A sequence that emits the end token stops: its later ids are the end
+    token, its position stays at the row of that step, and its cache holds
+    exactly what a loop that stops stepping it there leaves (no later write
+    into its rows)."""
+    n = 10
+    n0s = [30 + 10 * b for b in range(batch)]
+    s, w, kv_host, dec, toks = _fixture(batch, 120, n0s, max_batch=max_batch)
     # the token sequence 0 emits at step 4 becomes the end token
     kv_r = _cache(dec, batch, 96, kv_host)
     free, _ = _step_loop(dec, kv_r, toks, n0s, n)
@@ -118,6 +128,51 @@ def test_generate_retires_a_sequence_at_eos():
     assert ref_pos[0] == n0s[0] + f0          # the position stopped at the eos step
     if first[1] is None:
         assert ref_pos[1] == n0s[1] + n
+    # sequence 0's cache: rows 0 .. n0 + f0 equal those of a loop that ran
+    # only the steps up to and including the eos step; every later row still
+    # holds the prefill
+    kv_c = _cache(dec, batch, 96, kv_host)
+    _step_loop(dec, kv_c, toks, n0s, f0 + 1)
+    last = n0s[0] + f0 + 1
+    assert torch.equal(_seq_rows(kv_a, 0, 0, last), _seq_rows(kv_c, 0, 0, last))
+    init = _cache(dec, batch, 96, kv_host)
+    assert torch.equal(_seq_rows(kv_a, 0, last, 96), _seq_rows(init, 0, last, 96))
+    dec.close()
+
+
+def test_generate_stops_when_every_sequence_retired():
+    """When every sequence has emitted the end token the remaining steps are
+    not run: their ids are the end token and the positions stay."""
+    n = 12
+    n0s = [25]
+    s, w, kv_host, dec, toks = _fixture(1, 140, n0s)
+    kv_r = _cache(dec, 1, 96, kv_host)
+    free, _ = _step_loop(dec, kv_r, toks, n0s, n)
+    eos = free[2][0]
+    f0 = next(i for i in range(n) if free[i][0] == eos)
+    kv_a = _cache(dec, 1, 96, kv_host)
+    out = torch.full((n, 1), -7, dtype=torch.int32, device="cuda")
+    pos = i32(n0s)
+    dec.generate(kv_a, i32(toks), pos, out, eos=eos)
+    assert dec.check() == 0
+    got = [r[0] for r in out.cpu().tolist()]
+    assert got[:f0 + 1] == [free[i][0] for i in range(f0 + 1)]
+    assert all(g == eos for g in got[f0:])
+    assert pos.cpu().tolist() == [n0s[0] + f0]
+    dec.close()
+
+
+def test_generate_position_past_the_cache_is_reported():
+    """A sequence that would step past max_ctx stops the loop: DEC_DEV_BAD_POSITION,
+    and the steps that could not run report -1."""
+    s, w, kv_host, dec, toks = _fixture(1, 150, [90])
+    kv = _cache(dec, 1, 96, kv_host)
+    out = torch.full((8, 1), -7, dtype=torch.int32, device="cuda")
+    pos = i32([90])
+    dec.generate(kv, i32(toks), pos, out)
+    assert dec.check() == capi.DEC_DEV_BAD_POSITION
+    got = [r[0] for r in out.cpu().tolist()]
+    assert all(0 <= g < s.vocab for g in got[:6]) and got[6:] == [-1, -1]
     dec.close()
 
 
