@@ -31,6 +31,7 @@ struct dec_handle {
   int ctas = 0;
   int smem_optin = 0;
   int nslot[kMaxBatchSmall + 1] = {0};
+  int slot_bytes[kMaxBatchSmall + 1] = {0};
   size_t smem[kMaxBatchSmall + 1] = {0};
   const uint16_t* embed = nullptr;
   const uint16_t* lm_head = nullptr;
@@ -166,12 +167,14 @@ static int init_handle(const dec_shape* shape, const InitWeights& w, dec_handle*
   h->wsc_n = w.w8 ? step_wsc_slots(H, F, nqkv, shape->vocab, h->ctas) : 0;
   h->prow = step_part_rows(H, F, nqkv, h->ctas);
   for (int b = 1; b <= B; ++b) {
-    h->nslot[b] = step_max_slots(b, H, F, HqD, D, rep, h->wsc_n, h->prow, h->smem_optin);
+    step_ring(b, H, F, HqD, D, rep, h->wsc_n, h->prow, h->smem_optin, &h->nslot[b],
+              &h->slot_bytes[b]);
     if (h->nslot[b] < 2) {
       delete h;
       return DEC_ERR_DEVICE;
     }
-    h->smem[b] = step_smem_bytes(h->nslot[b], b, H, F, HqD, D, rep, h->wsc_n, h->prow);
+    h->smem[b] = step_smem_bytes(h->nslot[b], h->slot_bytes[b], b, H, F, HqD, D, rep, h->wsc_n,
+                                 h->prow);
     e = step_set_smem(b, D, w.w8 != 0, h->smem[b]);
     if (e != cudaSuccess) {
       delete h;
@@ -401,6 +404,7 @@ static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* 
   a.timeout_ns = h->timeout_ns;
   a.stall_cta = h->stall_cta;
   a.nslot = h->nslot[batch];
+  a.slot_bytes = h->slot_bytes[batch];
   a.prow = h->prow;
 #ifdef DEC_PROFILE
   a.prof = reinterpret_cast<unsigned long long*>(h->ws + wl.prof);
@@ -557,7 +561,7 @@ extern "C" int dec_get_config(const dec_handle* h, int* ctas, int* ring_slots, i
   if (!h) return DEC_ERR_NULL;
   if (ctas) *ctas = h->ctas;
   if (ring_slots) *ring_slots = h->nslot[1];
-  if (slot_bytes) *slot_bytes = kSlotBytes;
+  if (slot_bytes) *slot_bytes = h->slot_bytes[1];
   return DEC_OK;
 }
 

@@ -8,7 +8,12 @@ namespace dec {
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kStepThreads = kConsumerThreads + 32;  // + one producer warp
-constexpr int kSlotBytes = 24576;                   // ring slot: 12 rows of 1024 bf16
+// Ring slot sizes of the persistent step: the large one when at least
+// kMinLargeSlots of them fit shared memory (fewer, larger tiles mean fewer
+// waits per stage), else the small one.
+constexpr int kSlotBytesLarge = 49152;
+constexpr int kSlotBytesSmall = 24576;
+constexpr int kMinLargeSlots = 3;
 constexpr int kMaxBatchSmall = 4;                   // batch handled by the GEMV step kernel
 constexpr int kMaxRep = 4;                          // query heads per KV head (step kernel)
 constexpr int kLayerPtrs = 11;
@@ -74,6 +79,7 @@ struct StepArgs {
   unsigned long long timeout_ns;
   int stall_cta;        // -1: off
   int nslot;            // ring slots per CTA
+  int slot_bytes;       // bytes per ring slot
   int prow;             // most output rows of one CTA in a K-split stage
   unsigned long long* prof;  // per-phase timestamps (profiling builds) or null
 };
@@ -85,10 +91,12 @@ struct WorkspaceLayout {
   int part_chunks;
 };
 
-size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep, int wsc_n,
-                       int prow);
-int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int wsc_n, int prow,
-                   int smem_optin);
+size_t step_smem_bytes(int nslot, int slot_bytes, int B, int H, int F, int HqD, int D, int rep,
+                       int wsc_n, int prow);
+// The ring of the persistent step for batch B: slot size and count (0 slots:
+// the shape does not fit).
+void step_ring(int B, int H, int F, int HqD, int D, int rep, int wsc_n, int prow, int smem_optin,
+               int* nslot, int* slot_bytes);
 // The most output rows one CTA computes in a K-split stage (gate and up rows
 // counted separately).
 int step_part_rows(int H, int F, int nqkv, int ctas);

@@ -58,6 +58,10 @@ constexpr int kBlk = 128;                      // columns of one K block
 constexpr int kWarpStage = 384;                // tagged words a warp stages per poll round
 constexpr int kStageWords = kCW * kWarpStage;  // whole staging buffer (CTA-wide gathers)
 constexpr int kMaxGainBlk = 6;                 // K blocks per warp of a normalised input (H <= 6144)
+// bf16 projection rows sit in the ring kRowPad bytes apart beyond their
+// length, so that the 8 rows an 8x8 matrix load touches fall in different
+// banks (row stride = 16 mod 128 bytes); the activation planes likewise.
+constexpr int kRowPad = 16;
 
 // Stages of one layer; the lm_head runs as stage SQ of layer L (code SLM).
 enum { SQ = 0, SA, SO, SU, SD, kStages, SLM = kStages };
@@ -73,8 +77,10 @@ enum {
   StU, StDIn, StD, StODot, StDDot,
   // the producer's issue time of the first tile of each stage
   StPQ, StPA, StPO, StPU, StPD,
-  // ns warp 0 spent waiting for ring tiles in each stage
-  StWQ, StWA, StWO, StWU, StWD
+  // SM cycles warp 0 spent waiting for ring tiles in each stage
+  StWQ, StWA, StWO, StWU, StWD,
+  // SM cycles of warp 0's GEMV of each stage (waits included)
+  StCQ, StCO, StCU, StCD
 };
 enum { StLmStart = 0, StLmGath, StLmDone, StEnd, StBegin };
 #ifdef DEC_PROFILE
@@ -130,18 +136,20 @@ __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a -
 
 // prow: the most output rows one CTA computes in a K-split stage (gate and up
 // rows counted separately).
-__host__ __device__ inline Carve carve(int nslot, int B, int kmax, int D, int rep, int wsc_n,
-                                       int prow) {
+__host__ __device__ inline Carve carve(int nslot, int slot_bytes, int B, int kmax, int D, int rep,
+                                       int wsc_n, int prow) {
   Carve c;
   size_t o = 0;
   c.ring = o;
-  o += static_cast<size_t>(nslot) * kSlotBytes;
+  o += static_cast<size_t>(nslot) * slot_bytes;
   c.bars = o;
   o += align_up(2 * nslot * sizeof(uint64_t), 16);
-  size_t act_f = static_cast<size_t>(B) * kmax;
-  size_t att_f = static_cast<size_t>(rep + 2) * D + static_cast<size_t>(kCW) * rep * (D + 2);
+  // fp32 activations [B][kmax], or their bf16 hi/lo planes [B][2][kmax + pad]
+  size_t act_b = static_cast<size_t>(B) * kmax * sizeof(float) + 2ull * B * kRowPad;
+  size_t att_b = (static_cast<size_t>(rep + 2) * D + static_cast<size_t>(kCW) * rep * (D + 2)) *
+                 sizeof(float);
   c.act = o;
-  o += align_up((act_f > att_f ? act_f : att_f) * sizeof(float), 16);
+  o += align_up(act_b > att_b ? act_b : att_b, 16);
   c.stg = o;
   o += static_cast<size_t>(kStageWords) * sizeof(uint64_t);
   c.xown = o;
@@ -150,8 +158,8 @@ __host__ __device__ inline Carve carve(int nslot, int B, int kmax, int D, int re
   o += align_up(2ull * kCW * (prow + 1) * B * sizeof(float), 16);
   c.bred = o;
   o += align_up(2ull * kCW * B * sizeof(float) + 2ull * kCW * B * sizeof(int), 16);
-  c.ints = o;  // two Plans (consumers, producer) + a few ints
-  o += align_up(2 * sizeof(Plan) + 16 * sizeof(int), 16);
+  c.ints = o;  // two Plans (consumers, producer), a few ints, a 16-byte zero row
+  o += align_up(2 * sizeof(Plan) + 16 * sizeof(int), 16) + 16;
   c.lw = o;
   o += align_up(sizeof(LayerPtrs) * kMaxLayers, 16);
   c.wsc = o;
@@ -355,66 +363,107 @@ __device__ __noinline__ GroupSums<R, B> group_dot(const uint32_t* rows, uint32_t
   return out;
 }
 
-// Partial dot products of 4 tile rows (shared memory, row i at rows[i]) with
-// the activations of B sequences over the K blocks blk0, blk0 + kCW, ...
-// (nb of them): lane l takes columns 4l..4l+3 of each 128-column block, so
-// that the warp reads 256 contiguous bytes of a bf16 row (128 of an int8 row)
-// and 512 contiguous bytes of activations: no bank conflicts.  Returns the
-// transposed-butterfly reduction (lane gets row lane >> 3's sum for each b).
-template <int B, bool W8>
-__device__ __noinline__ GroupSums<4, B> kdot4(const uint32_t* rows, uint32_t act, int act_stride,
-                                              int blk0, int nb, int lane) {
-  float acc[4][B];
+// Partial dot products of R (4 or 8) tile rows (shared memory, row i at
+// rows[i]) with the activations of B sequences over the K blocks blk0,
+// blk0 + kCW, ... (nb of them): lane l takes columns 4l..4l+3 of each
+// 128-column block, so that the warp reads 256 contiguous bytes of a bf16 row
+// (128 of an int8 row) and 512 contiguous bytes of activations: no bank
+// conflicts.  All R rows' loads of a block are issued before their
+// multiply-adds, so R independent chains hide the shared-memory latency.
+// Returns the transposed-butterfly reductions: lane gets the sums of rows
+// (lane >> 3) and, for R == 8, 4 + (lane >> 3), for each b.
+template <int R, int B>
+struct KSums {
+  float s[R / 4][B];
+};
+
+template <int R, int B, bool W8>
+__device__ __forceinline__ KSums<R, B> kdot(const uint32_t (&rows)[R], uint32_t act,
+                                            int act_stride, int blk0, int nb, int lane) {
+  float acc[R][B];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < R; ++i)
 #pragma unroll
     for (int b = 0; b < B; ++b) acc[i][b] = 0.f;
   for (int j = 0; j < nb; ++j) {
     const uint32_t col = static_cast<uint32_t>((blk0 + j * kCW) * kBlk + lane * 4);
-    float wf[4][4];
+    uint32_t w[R][2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < R; ++i) {
       if constexpr (W8) {
-        uint32_t w;
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(rows[i] + col));
-        const uint32_t u = w ^ 0x80808080u;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) wf[i][e] = i8_at(u, e);
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[i][0]) : "r"(rows[i] + col));
+        w[i][1] = 0u;
       } else {
-        uint32_t w0, w1;
-        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(rows[i] + col * 2));
-        wf[i][0] = bf16lo(w0);
-        wf[i][1] = bf16hi(w0);
-        wf[i][2] = bf16lo(w1);
-        wf[i][3] = bf16hi(w1);
+        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
+                     : "=r"(w[i][0]), "=r"(w[i][1]) : "r"(rows[i] + col * 2));
       }
     }
+    float x[B][4];
 #pragma unroll
     for (int b = 0; b < B; ++b) {
-      float x0, x1, x2, x3;
       const uint32_t xa = act + static_cast<uint32_t>(b * act_stride + col) * 4u;
       asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
-                   : "=f"(x0), "=f"(x1), "=f"(x2), "=f"(x3) : "r"(xa));
+                   : "=f"(x[b][0]), "=f"(x[b][1]), "=f"(x[b][2]), "=f"(x[b][3]) : "r"(xa));
+    }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float s = acc[i][b];
-        s = fmaf(wf[i][0], x0, s);
-        s = fmaf(wf[i][1], x1, s);
-        s = fmaf(wf[i][2], x2, s);
-        s = fmaf(wf[i][3], x3, s);
-        acc[i][b] = s;
+    for (int i = 0; i < R; ++i) {
+      float wf[4];
+      if constexpr (W8) {
+        const uint32_t u = w[i][0] ^ 0x80808080u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) wf[e] = i8_at(u, e);
+      } else {
+        wf[0] = bf16lo(w[i][0]);
+        wf[1] = bf16hi(w[i][0]);
+        wf[2] = bf16lo(w[i][1]);
+        wf[3] = bf16hi(w[i][1]);
+      }
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        float t = fmaf(wf[0], x[b][0], acc[i][b]);
+        t = fmaf(wf[1], x[b][1], t);
+        t = fmaf(wf[2], x[b][2], t);
+        acc[i][b] = fmaf(wf[3], x[b][3], t);
       }
     }
   }
-  GroupSums<4, B> out;
+  KSums<R, B> out;
 #pragma unroll
-  for (int b = 0; b < B; ++b) {
-    float col[4];
+  for (int q = 0; q < R / 4; ++q)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) col[i] = acc[i][b];
-    out.s[b] = tbfly_lane<4>(col, lane);
-  }
+    for (int b = 0; b < B; ++b) {
+      float c4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) c4[i] = acc[4 * q + i][b];
+      out.s[q][b] = tbfly_lane<4>(c4, lane);
+    }
   return out;
+}
+
+// Warp-level tensor-core pieces of the batch-1..4 projections: an 8x8
+// matrix load per lane group and the m16n8k16 bf16 MMA with fp32
+// accumulation.  With a handful of sequences the projections are matrix x
+// vector products; one MMA multiplies 16 weight rows x 16 columns by the 8
+// activation columns (hi and lo bf16 planes of up to 4 sequences), which
+// replaces ~40 unpack/FMA/shuffle instructions per lane.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t (&r)[2]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
+                                          const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(uint16_t lo, uint16_t hi) {
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
 // The per-launch state of one CTA.  FP8: the cache holds E4M3 codes + scales.
@@ -442,7 +491,12 @@ struct Cta {
   uint32_t seq;   // step counter of the consumers' current step
   // per-CTA row ranges
   int q0, q1, h0, h1, f0, f1, v0, v1;
-  int rpt_h, rpt_o, rpt_u, rpt_d, art;
+  int slot;  // bytes per ring slot
+  int rpt_lm, rpt_h, rpt_o, rpt_u, rpt_d, art;
+  uint32_t zrow;  // 16 zero bytes (shared memory)
+  static constexpr int pad = W8 ? 0 : kRowPad;  // ring row padding of the projections
+  // ring bytes between two rows of a projection with K columns
+  __device__ __forceinline__ int rstride(int K) const { return K * eb + pad; }
   // this side's plan of the current step (shared memory)
   Plan* pl;
   Plan* cplan;  // the consumers' copy
@@ -452,7 +506,8 @@ struct Cta {
   __device__ Cta(const StepArgs& args, uint8_t* smem, int kmax_) : a(args), kmax(kmax_) {
     const int rep = a.Hq / a.Hkv;
     prow = a.prow;
-    Carve c = carve(a.nslot, B, kmax, D, rep, a.wsc_n, prow);
+    slot = a.slot_bytes;
+    Carve c = carve(a.nslot, slot, B, kmax, D, rep, a.wsc_n, prow);
     ring = smem + c.ring;
     full = reinterpret_cast<uint64_t*>(smem + c.bars);
     empty = full + a.nslot;
@@ -465,6 +520,7 @@ struct Cta {
     cplan = reinterpret_cast<Plan*>(smem + c.ints);
     pplan = cplan + 1;
     sints = reinterpret_cast<int*>(pplan + 1);
+    zrow = smem_u32(smem + c.ints + align_up(2 * sizeof(Plan) + 16 * sizeof(int), 16));
     slw = reinterpret_cast<const LayerPtrs*>(smem + c.lw);
     wsc = reinterpret_cast<float*>(smem + c.wsc);
     tid = threadIdx.x;
@@ -481,14 +537,15 @@ struct Cta {
     f1 = split_at(a.F, nc, cta + 1);
     v0 = split_at(a.V, nc, cta);
     v1 = split_at(a.V, nc, cta + 1);
-    rpt_h = kSlotBytes / (eb * a.H);
-    rpt_o = kSlotBytes / (eb * a.Hq * D);
-    rpt_u = kSlotBytes / (2 * eb * a.H);
-    rpt_d = kSlotBytes / (eb * a.F);
+    rpt_lm = slot / (eb * a.H);
+    rpt_h = slot / rstride(a.H);
+    rpt_o = slot / rstride(a.Hq * D);
+    rpt_u = slot / (2 * rstride(a.H));
+    rpt_d = slot / rstride(a.F);
     if constexpr (FP8) {
-      art = (kSlotBytes / (2 * D + 8)) & ~15;
+      art = (slot / (2 * D + 8)) & ~15;
     } else {
-      art = kSlotBytes / (4 * D);
+      art = slot / (4 * D);
     }
     pl = warp == kCW ? pplan : cplan;
   }
@@ -589,11 +646,14 @@ struct Cta {
             dead = true;
             return nullptr;
           }
+#ifdef DEC_PRODUCER_NAP
+          __nanosleep(DEC_PRODUCER_NAP);  // the ring runs far ahead: issue slots go to the consumers
+#endif
         }
       }
       fb = &full[ps];
       mbar_arrive_expect_tx(fb, bytes);
-      return ring + static_cast<size_t>(ps) * kSlotBytes;
+      return ring + static_cast<size_t>(ps) * slot;
     };
     auto advance = [&]() {
       ++n;
@@ -607,6 +667,16 @@ struct Cta {
     // byte address of row r of a [rows, K] weight matrix
     auto wrow = [&](const void* base, int r, int K) {
       return static_cast<const uint8_t*>(base) + static_cast<size_t>(r) * K * e;
+    };
+    // cnt rows lo.. of a [rows, K] projection to dst, rstride(K) bytes apart
+    auto rows_to = [&](uint8_t* dst, const void* base, int lo, int cnt, int K) {
+      if (pad == 0) {
+        bulk_g2s(dst, wrow(base, lo, K), static_cast<uint32_t>(cnt) * K * e, fb, pol);
+      } else {
+        for (int i = 0; i < cnt; ++i)
+          bulk_g2s(dst + static_cast<size_t>(i) * rstride(K), wrow(base, lo + i, K),
+                   static_cast<uint32_t>(K) * e, fb, pol);
+      }
     };
     bool stop = false;
     for (int st = 0; !dead && !stop; ++st) {
@@ -629,8 +699,8 @@ struct Cta {
           } else {
             base = lw.w[3]; lo = rr - HqD - HkvD; cnt = left;
           }
-          bulk_g2s(dst, wrow(base, lo, H), static_cast<uint32_t>(cnt) * H * e, fb, pol);
-          dst += static_cast<size_t>(cnt) * H * e;
+          rows_to(dst, base, lo, cnt, H);
+          dst += static_cast<size_t>(cnt) * rstride(H);
           rr += cnt;
           left -= cnt;
         }
@@ -682,7 +752,7 @@ struct Cta {
         uint8_t* dst = acquire(static_cast<uint32_t>(nr) * HqD * e);
         if (!dst) break;
         if (r == h0) DEC_PSTAMP(kStampsPerLayer * l + StPO);
-        bulk_g2s(dst, wrow(lw.w[6], r, HqD), static_cast<uint32_t>(nr) * HqD * e, fb, pol);
+        rows_to(dst, lw.w[6], r, nr, HqD);
         advance();
       }
       // ---- gate / up rows [f0, f1): a tile is nr gate rows then nr up rows
@@ -692,8 +762,8 @@ struct Cta {
         uint8_t* dst = acquire(2 * rb);
         if (!dst) break;
         if (r == f0) DEC_PSTAMP(kStampsPerLayer * l + StPU);
-        bulk_g2s(dst, wrow(lw.w[8], r, H), rb, fb, pol);
-        bulk_g2s(dst + rb, wrow(lw.w[9], r, H), rb, fb, pol);
+        rows_to(dst, lw.w[8], r, nr, H);
+        rows_to(dst + static_cast<size_t>(nr) * rstride(H), lw.w[9], r, nr, H);
         advance();
       }
       // ---- down rows [h0, h1), K = F
@@ -702,14 +772,14 @@ struct Cta {
         uint8_t* dst = acquire(static_cast<uint32_t>(nr) * a.F * e);
         if (!dst) break;
         if (r == h0) DEC_PSTAMP(kStampsPerLayer * l + StPD);
-        bulk_g2s(dst, wrow(lw.w[10], r, a.F), static_cast<uint32_t>(nr) * a.F * e, fb, pol);
+        rows_to(dst, lw.w[10], r, nr, a.F);
         advance();
       }
     }
     if (stop) break;
     // ---- lm_head rows [v0, v1)
-    for (int r = v0; r < v1 && !dead; r += rpt_h) {
-      const int nr = min(rpt_h, v1 - r);
+    for (int r = v0; r < v1 && !dead; r += rpt_lm) {
+      const int nr = min(rpt_lm, v1 - r);
       uint8_t* dst = acquire(static_cast<uint32_t>(nr) * H * e);
       if (!dst) break;
       bulk_g2s(dst, wrow(a.lm_head, r, H), static_cast<uint32_t>(nr) * H * e, fb, pol);
@@ -753,7 +823,7 @@ struct Cta {
     int st = 1;
     if (lane == 0) {
 #ifdef DEC_PROFILE
-      const uint64_t tw = globaltimer();
+      const long long tw = clock64();
 #endif
       Spin sp;
       while (!mbar_wait(&full[slot], par, kWaitHintNs)) {
@@ -763,7 +833,7 @@ struct Cta {
         }
       }
 #ifdef DEC_PROFILE
-      wacc += globaltimer() - tw;
+      wacc += static_cast<uint64_t>(clock64() - tw);
 #endif
     }
     st = __shfl_sync(0xffffffffu, st, 0);
@@ -772,7 +842,11 @@ struct Cta {
       ab = 1;
       return;
     }
+#ifdef DEC_LEAN_WAIT
+    __syncwarp();  // lane 0 observed the completed phase; the warp is ordered after it
+#else
     (void)mbar_test(&full[slot], par);  // every lane observes the completed phase
+#endif
   }
   __device__ __forceinline__ void release_tile() {
     __syncwarp();
@@ -840,22 +914,34 @@ struct Cta {
   __device__ void warp_gather(uint64_t* ws, int n, uint32_t f, Src src_of) {
     __syncwarp();  // the previous round's words are consumed
     const int np = n >> 1;
+    constexpr int kPer = kWarpStage / 64;  // pairs per lane at most
     uint32_t pend = 0;
-    if (!ab)
-      for (int k = 0, c = lane; c < np; c += 32, ++k) pend |= 1u << k;
+    const uint64_t* sp[kPer];  // this lane's source pairs, computed once
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int c = lane + 32 * k;
+      sp[k] = c < np ? src_of(2 * c) : nullptr;
+      if (!ab && c < np) pend |= 1u << k;
+    }
     uint64_t t0 = 0;
     for (int round = 0;; ++round) {
-      for (int k = 0, c = lane; c < np; c += 32, ++k)
-        if (pend & (1u << k)) cp_async16_cg(ws + 2 * c, src_of(2 * c));
-      // the abort flag travels with every later round (its load overlaps the
-      // copies' round trip instead of following it)
-      const int abf = (lane == 0 && round > 0) ? ld_relaxed_i32(a.abort_flag) : 0;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k)
+        if (pend & (1u << k)) cp_async16_cg(ws + 2 * (lane + 32 * k), sp[k]);
+      // every 8th round also reads the abort flag (its load overlaps the
+      // copies' round trip) and checks the time limit
+      const bool slow = (round & 7) == 7;
+      const int abf = (lane == 0 && slow) ? ld_relaxed_i32(a.abort_flag) : 0;
       cp_async_wait_all();
-      for (int k = 0, c = lane; c < np; c += 32, ++k)
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int c = lane + 32 * k;
         if ((pend & (1u << k)) && static_cast<uint32_t>(ws[2 * c] >> 32) == f &&
             static_cast<uint32_t>(ws[2 * c + 1] >> 32) == f)
           pend &= ~(1u << k);
+      }
       if (!__any_sync(0xffffffffu, pend != 0)) break;
+      if (!slow) continue;
       int fail = 0;
       if (lane == 0) {
         const uint64_t now = globaltimer();
@@ -887,12 +973,15 @@ struct Cta {
   // with src == nullptr, the embedding row of the step's token) times the
   // gain g[k] (g == nullptr: 1) into act[b][k]; ss[b] gets the warp's share
   // of sum_k x[b][k]^2 (before the gain), reduced over the warp.
+  // With `planes` (bf16 weights) the values go to act as two bf16 planes per
+  // sequence instead, hi = bf16(x) and lo = bf16(x - hi) (row 2b + plane,
+  // rstride(K) bytes apart): the operands of the tensor-core projections.
   __device__ void warp_input(const uint64_t* src, int K, uint32_t f, const uint16_t* g,
-                             float (&ss)[B]) {
+                             float (&ss)[B], bool planes) {
 #pragma unroll
     for (int b = 0; b < B; ++b) ss[b] = 0.f;
     const int nbw = my_blocks(K / kBlk);
-    const int units = a.B * nbw;  // 128-word units: (b, block)
+    const int units = B * nbw;  // 128-word units: (b, block)
     constexpr int per = kWarpStage / kBlk;
     uint64_t* ws = stg + warp * kWarpStage;
     // the gains of the warp's blocks, loaded before the polls so that their
@@ -942,11 +1031,93 @@ struct Cta {
           v[2] *= bf16lo(gs.y);
           v[3] *= bf16hi(gs.y);
         }
-        *reinterpret_cast<float4*>(act + b * kmax + k) = make_float4(v[0], v[1], v[2], v[3]);
+        if (planes) {
+          uint16_t hi[4], lo[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            hi[q] = f_to_bf16(v[q]);
+            lo[q] = f_to_bf16(v[q] - bf16_to_f(hi[q]));
+          }
+          uint8_t* pl0 = reinterpret_cast<uint8_t*>(act) +
+                         static_cast<size_t>(2 * b) * (K * 2 + kRowPad) + k * 2;
+          *reinterpret_cast<uint2*>(pl0) =
+              make_uint2(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]));
+          *reinterpret_cast<uint2*>(pl0 + K * 2 + kRowPad) =
+              make_uint2(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]));
+        } else {
+          *reinterpret_cast<float4*>(act + b * kmax + k) = make_float4(v[0], v[1], v[2], v[3]);
+        }
       }
     }
 #pragma unroll
     for (int b = 0; b < B; ++b) ss[b] = warp_sum(ss[b]);
+  }
+
+  // The bf16 K-split GEMV on the tensor cores: for every ring tile, 16-row
+  // MMA tiles (rows past the tile repeat its last row; their sums are
+  // dropped) over the warp's K blocks, 8 MMAs of k16 per block.  Matrix loads
+  // of the A (weight rows, rstride(K) apart) and B (activation planes) tiles
+  // are conflict-free thanks to the 16-byte row padding.  Output column n of
+  // an MMA is plane n & 1 of sequence n >> 1 (zero for sequences past a.B), so
+  // lane (g, t) holds rows g and g + 8 of sequence t as hi + lo.
+  __device__ void kgemv_mma(int K, int nrows, int rpt, bool pair, float* pbuf) {
+    const int nbw = my_blocks(K / kBlk);
+    const uint32_t rsb = static_cast<uint32_t>(rstride(K));
+    const uint32_t psb = static_cast<uint32_t>(K * 2 + kRowPad);
+    // this lane's row address of the B matrix loads (lanes 0..15: rows n of
+    // the k8 halves 0 / 1), or the zero row
+    const int bn = lane & 7, bh = (lane >> 3) & 1;
+    const bool bval = bn < 2 * B;
+    const uint32_t bbase = bval ? smem_u32(act) + bn * psb + bh * 16 : zrow;
+    const uint32_t bstep = bval ? 2u : 0u;  // bytes per column
+    const int am = lane >> 3, ar = lane & 7;
+    const int g = lane >> 2, t = lane & 3;
+    for (int r0 = 0; r0 < nrows; r0 += rpt) {
+      const int nr = min(rpt, nrows - r0);
+      const int ntr = pair ? 2 * nr : nr;
+      wait_tile();
+      if (!ab && nbw > 0) {
+        const uint32_t tb = smem_u32(ring + static_cast<size_t>(rs) * slot);
+        for (int mt = 0; mt < ntr; mt += 16) {
+          const int arow = min(mt + ar + 8 * (am & 1), ntr - 1);
+          const uint32_t abase = tb + static_cast<uint32_t>(arow) * rsb + (am >> 1) * 16;
+          // one accumulator per k16 step of a block: the MMAs of a block are
+          // independent (a dependent chain would cost the MMA latency per step)
+          float cs[kBlk / 16][4];
+#pragma unroll
+          for (int st = 0; st < kBlk / 16; ++st) cs[st][0] = cs[st][1] = cs[st][2] = cs[st][3] = 0.f;
+          for (int j = 0; j < nbw; ++j) {
+            const uint32_t k0 = static_cast<uint32_t>((warp + j * kCW) * kBlk);
+            uint32_t af[kBlk / 16][4], bf[kBlk / 16][2];
+#pragma unroll
+            for (int st = 0; st < kBlk / 16; ++st) {
+              const uint32_t k = k0 + st * 16;
+              ldsm_x4(abase + k * 2, af[st]);
+              ldsm_x2(bbase + k * bstep, bf[st]);
+            }
+#pragma unroll
+            for (int st = 0; st < kBlk / 16; ++st) mma_16816(cs[st], af[st], bf[st]);
+          }
+          float c[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            c[q] = ((cs[0][q] + cs[1][q]) + (cs[2][q] + cs[3][q])) +
+                   ((cs[4][q] + cs[5][q]) + (cs[6][q] + cs[7][q]));
+          }
+          if (t < B) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int tr = mt + g + 8 * h;
+              if (tr < ntr) {
+                const int r = pair ? (tr < nr ? r0 + tr : nrows + r0 + tr - nr) : r0 + tr;
+                pbuf[(warp * prow + r) * B + t] = c[2 * h] + c[2 * h + 1];
+              }
+            }
+          }
+        }
+      }
+      release_tile();
+    }
   }
 
   // The K-split GEMV of a stage over ring tiles: rows [0, nrows) of the
@@ -956,26 +1127,43 @@ struct Cta {
   // at a time; the partials of row r (pair: the second matrix's row r at
   // nrows + r) go to pbuf[warp][r][b].
   __device__ void kgemv(int K, int nrows, int rpt, bool pair, float* pbuf) {
+    if constexpr (!W8) {
+      kgemv_mma(K, nrows, rpt, pair, pbuf);
+      return;
+    }
     const int nbw = my_blocks(K / kBlk);
-    const uint32_t row_bytes = static_cast<uint32_t>(K * eb);
+    const uint32_t row_bytes = static_cast<uint32_t>(rstride(K));
     for (int r0 = 0; r0 < nrows; r0 += rpt) {
       const int nr = min(rpt, nrows - r0);
       const int ntr = pair ? 2 * nr : nr;
       wait_tile();
       if (!ab && nbw > 0) {
-        const uint32_t tb = smem_u32(ring + static_cast<size_t>(rs) * kSlotBytes);
-        for (int g0 = 0; g0 < ntr; g0 += 4) {
+        const uint32_t tb = smem_u32(ring + static_cast<size_t>(rs) * slot);
+        // the partials of tile row tr go to stage row r
+        auto put = [&](int tr, const float (&v)[B]) {
+          if ((lane & 7) == 0 && tr < ntr) {
+            const int r = pair ? (tr < nr ? r0 + tr : nrows + r0 + tr - nr) : r0 + tr;
+#pragma unroll
+            for (int b = 0; b < B; ++b) pbuf[(warp * prow + r) * B + b] = v[b];
+          }
+        };
+        int g0 = 0;
+        for (; g0 + 4 < ntr; g0 += 8) {  // 8 rows at a time while more than 4 remain
+          uint32_t rows[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            rows[i] = tb + static_cast<uint32_t>(min(g0 + i, ntr - 1)) * row_bytes;
+          const KSums<8, B> s = kdot<8, B, W8>(rows, smem_u32(act), kmax, warp, nbw, lane);
+          put(g0 + (lane >> 3), s.s[0]);
+          put(g0 + 4 + (lane >> 3), s.s[1]);
+        }
+        if (g0 < ntr) {
           uint32_t rows[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             rows[i] = tb + static_cast<uint32_t>(min(g0 + i, ntr - 1)) * row_bytes;
-          const GroupSums<4, B> s = kdot4<B, W8>(rows, smem_u32(act), kmax, warp, nbw, lane);
-          const int tr = g0 + (lane >> 3);
-          if ((lane & 7) == 0 && tr < ntr) {
-            const int r = pair ? (tr < nr ? r0 + tr : nrows + r0 + tr - nr) : r0 + tr;
-#pragma unroll
-            for (int b = 0; b < B; ++b) pbuf[(warp * prow + r) * B + b] = s.s[b];
-          }
+          const KSums<4, B> s = kdot<4, B, W8>(rows, smem_u32(act), kmax, warp, nbw, lane);
+          put(g0 + (lane >> 3), s.s[0]);
         }
       }
       release_tile();
@@ -999,19 +1187,24 @@ struct Cta {
     pb ^= 1;
     if (ab) return;
     const int nw = min(kCW, K / kBlk);
-    for (int t = tid; t < nrows * a.B; t += kCT) {
-      const int r = t / a.B, b = t % a.B;
-      float s0 = 0.f, s1 = 0.f;
-      for (int w = 0; w < nw; ++w) {
-        s0 += pbuf[(w * prow + r) * B + b];
-        if (pair) s1 += pbuf[(w * prow + nrows + r) * B + b];
-      }
+    // a fixed pairwise tree over the warps (deterministic; warps without K
+    // blocks count as zero), all loads issued before the adds
+    auto tree = [&](const float* p, int stride) {
+      float v[kCW];
+#pragma unroll
+      for (int w = 0; w < kCW; ++w) v[w] = w < nw ? p[w * stride] : 0.f;
+#pragma unroll
+      for (int h = kCW / 2; h > 0; h >>= 1)
+#pragma unroll
+        for (int w = 0; w < h; ++w) v[w] += v[w + h];
+      return v[0];
+    };
+    for (int t = tid; t < nrows * B; t += kCT) {
+      const int r = t / B, b = t % B;
+      const float s0 = tree(pbuf + r * B + b, prow * B);
+      const float s1 = pair ? tree(pbuf + (nrows + r) * B + b, prow * B) : 0.f;
       float f = 1.f;
-      if (norm) {
-        float t2 = 0.f;
-        for (int w = 0; w < nw; ++w) t2 += sbuf[w * B + b];
-        f = rsqrtf(t2 / static_cast<float>(K) + a.eps);
-      }
+      if (norm) f = rsqrtf(tree(sbuf + b, B) / static_cast<float>(K) + a.eps);
       float c0 = f, c1 = f;
       if constexpr (W8) {
         c0 *= wsc[r];
@@ -1027,12 +1220,19 @@ struct Cta {
                          int K, int nrows, int rpt, bool pair, bool norm) {
     float ss[B];
     if constexpr (W8) load_scales(sc, l);
-    warp_input(src, K, f, g, ss);
+    warp_input(src, K, f, g, ss, !W8);
     DEC_STAMP(kStampsPerLayer * l + (sc == SQ ? StQIn : sc == SO ? StOIn : sc == SU ? StUIn : StDIn));
     wacc = 0;
+#ifdef DEC_PROFILE
+    const long long tg = clock64();
+#endif
     kgemv(K, nrows, rpt, pair, part + pb * (kCW * (prow + 1) * B));
     DEC_STAMP(kStampsPerLayer * l + (sc == SQ ? StQDot : sc == SO ? StODot : sc == SU ? StUDot : StDDot));
     DEC_SVAL(kStampsPerLayer * l + (sc == SQ ? StWQ : sc == SO ? StWO : sc == SU ? StWU : StWD), wacc);
+#ifdef DEC_PROFILE
+    DEC_SVAL(kStampsPerLayer * l + (sc == SQ ? StCQ : sc == SO ? StCO : sc == SU ? StCU : StCD),
+             static_cast<uint64_t>(clock64() - tg));
+#endif
     kstage_end(sc, l, K, nrows, pair, norm, ss);
   }
 
@@ -1122,7 +1322,7 @@ struct Cta {
     // slot's warp (slot mod warps), so a warp's consecutive tiles are never
     // more than one ring lap apart and its parity waits stay unambiguous.  A
     // stage of a few tiles spreads each tile's groups over the warps.
-    const bool owned = (nrows + rpt - 1) / rpt > 2 * kCW;
+    const bool owned = (nrows + rpt - 1) / rpt > 2 * kCW && a.nslot >= kCW - 1;
     int gbase = 0;
     for (int r0 = 0; r0 < nrows; r0 += rpt) {
       const int nr = min(rpt, nrows - r0);
@@ -1130,7 +1330,7 @@ struct Cta {
       const bool mine = !owned || rs % kCW == warp;
       if (mine) wait_tile();
       if (mine && !ab) {
-        const uint8_t* tb = ring + static_cast<size_t>(rs) * kSlotBytes;
+        const uint8_t* tb = ring + static_cast<size_t>(rs) * slot;
         int g0 = 0, gs = 1;
         if (!owned) {
           g0 = (warp - gbase) % kCW;
@@ -1321,34 +1521,50 @@ struct Cta {
         wait_tile();
         if (j == j0) DEC_STAMP(kStampsPerLayer * l + StAttTile);
         if (!ab) {
-          const uint8_t* tb = ring + static_cast<size_t>(rs) * kSlotBytes;
-          for (int r0 = 0; r0 < nr; r0 += ostep) {  // warp-uniform trip count
-            const int r = r0 + oi;
-            const bool ok = r < nr;
-            float kr[DQ];
-            tile_row(tb, nr, ok ? r : 0, e8, 0, kr);
-            float s[2];
+          const uint8_t* tb = ring + static_cast<size_t>(rs) * slot;
+          // two rows per octet per pass (independent chains; one rescale for both)
+          for (int r0 = 0; r0 < nr; r0 += 2 * ostep) {  // warp-uniform trip count
+            const int ra = r0 + oi, rb = r0 + ostep + oi;
+            const bool oka = ra < nr, okb = rb < nr;
+            float sa[2], sb[2];
+            {
+              float ka[DQ], kb[DQ];
+              tile_row(tb, nr, oka ? ra : 0, e8, 0, ka);
+              tile_row(tb, nr, okb ? rb : 0, e8, 0, kb);
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              float t = 0.f;
+              for (int hh = 0; hh < 2; ++hh) {
+                float ta[4] = {0.f, 0.f, 0.f, 0.f}, tb4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-              for (int k = 0; k < DQ; ++k) t = fmaf(qv[hh][k], kr[k], t);
-              t += __shfl_xor_sync(0xffffffffu, t, 4);
-              t += __shfl_xor_sync(0xffffffffu, t, 2);
-              t += __shfl_xor_sync(0xffffffffu, t, 1);
-              s[hh] = t;
+                for (int k = 0; k < DQ; ++k) {
+                  ta[k & 3] = fmaf(qv[hh][k], ka[k], ta[k & 3]);
+                  tb4[k & 3] = fmaf(qv[hh][k], kb[k], tb4[k & 3]);
+                }
+                sa[hh] = (ta[0] + ta[1]) + (ta[2] + ta[3]);
+                sb[hh] = (tb4[0] + tb4[1]) + (tb4[2] + tb4[3]);
+              }
             }
-            if (ok) {
-              float vr[DQ];
-              tile_row(tb, nr, r, e8, 1, vr);
+#pragma unroll
+            for (int o = 4; o > 0; o >>= 1)
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                sa[hh] += __shfl_xor_sync(0xffffffffu, sa[hh], o);
+                sb[hh] += __shfl_xor_sync(0xffffffffu, sb[hh], o);
+              }
+            if (oka) {
+              float va[DQ], vb[DQ];
+              tile_row(tb, nr, ra, e8, 1, va);
+              tile_row(tb, nr, okb ? rb : ra, e8, 1, vb);
 #pragma unroll
               for (int hh = 0; hh < 2; ++hh) {
                 if (hh < nh) {
-                  const float mn = fmaxf(m[hh], s[hh]);
-                  const float al = exp2f(m[hh] - mn), pe = exp2f(s[hh] - mn);
-                  ls[hh] = ls[hh] * al + pe;
+                  const float xb = okb ? sb[hh] : -INFINITY;
+                  const float mn = fmaxf(m[hh], fmaxf(sa[hh], xb));
+                  const float al = exp2f(m[hh] - mn), pa = exp2f(sa[hh] - mn);
+                  const float pbv = exp2f(xb - mn);
+                  ls[hh] = ls[hh] * al + (pa + pbv);
 #pragma unroll
-                  for (int k = 0; k < DQ; ++k) acc[hh][k] = fmaf(acc[hh][k], al, pe * vr[k]);
+                  for (int k = 0; k < DQ; ++k)
+                    acc[hh][k] = fmaf(acc[hh][k], al, fmaf(pa, va[k], pbv * vb[k]));
                   m[hh] = mn;
                 }
               }
@@ -1515,8 +1731,8 @@ struct Cta {
     }
     DEC_STAMP(kStampsPerLayer * a.L + StBegin);
     // the CTA's residual rows start as the embedding rows
-    for (int i = tid; i < (h1 - h0) * a.B; i += kCT) {
-      const int r = i / a.B, b = i % a.B;
+    for (int i = tid; i < (h1 - h0) * B; i += kCT) {
+      const int r = i / B, b = i % B;
       const float x = bf16_to_f(a.embed[static_cast<size_t>(pl->tok[b]) * H + h0 + r]);
       xown[r * B + b] = x;
       if (a.hidden_out) a.hidden_out[static_cast<size_t>(b) * H + h0 + r] = x;
@@ -1543,7 +1759,7 @@ struct Cta {
     {
       float ss[B], rsc[B];
       if constexpr (W8) load_scales(SLM, a.L);
-      warp_input(a.x_out, H, flag(a.L - 1), a.final_norm, ss);
+      warp_input(a.x_out, H, flag(a.L - 1), a.final_norm, ss, false);
       float* sbuf = part + pb * (kCW * (prow + 1) * B) + kCW * prow * B;
       if (lane == 0) {
 #pragma unroll
@@ -1560,7 +1776,7 @@ struct Cta {
         rsc[b] = rsqrtf(t2 / static_cast<float>(H) + a.eps);
       }
       DEC_STAMP(kStampsPerLayer * a.L + StLmGath);
-      gemv<4>(H, v1 - v0, rpt_h, SLM, a.L, rsc);
+      gemv<4>(H, v1 - v0, rpt_lm, SLM, a.L, rsc);
     }
     DEC_STAMP(kStampsPerLayer * a.L + StLmDone);
     // CTA argmax -> one 64-bit atomicMax per sequence (ties: lowest id)
@@ -1668,6 +1884,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
     uint64_t* dst = reinterpret_cast<uint64_t*>(const_cast<LayerPtrs*>(c.slw));
     for (int i = threadIdx.x; i < a.L * kLayerPtrs; i += blockDim.x) dst[i] = src[i];
   }
+  if (threadIdx.x < 4) asm volatile("st.shared.u32 [%0], %1;" ::"r"(c.zrow + 4 * threadIdx.x), "r"(0u));
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.nslot; ++s) {
       mbar_init(&c.full[s], 1);
@@ -1742,18 +1959,29 @@ static int kmax_of(int H, int F, int HqD) {
   int k = H > F ? H : F;
   return k > HqD ? k : HqD;
 }
-size_t step_smem_bytes(int nslot, int B, int H, int F, int HqD, int D, int rep, int wsc_n,
-                       int prow) {
-  return carve(nslot, B, kmax_of(H, F, HqD), D, rep, wsc_n, prow).total;
+size_t step_smem_bytes(int nslot, int slot_bytes, int B, int H, int F, int HqD, int D, int rep,
+                       int wsc_n, int prow) {
+  return carve(nslot, slot_bytes, B, kmax_of(H, F, HqD), D, rep, wsc_n, prow).total;
 }
 
-int step_max_slots(int B, int H, int F, int HqD, int D, int rep, int wsc_n, int prow,
-                   int smem_optin) {
-  int best = 0;
-  for (int n = 1; n <= 16; ++n)
-    if (step_smem_bytes(n, B, H, F, HqD, D, rep, wsc_n, prow) <= static_cast<size_t>(smem_optin))
-      best = n;
-  return best;
+void step_ring(int B, int H, int F, int HqD, int D, int rep, int wsc_n, int prow, int smem_optin,
+               int* nslot, int* slot_bytes) {
+  auto most = [&](int sb) {
+    int best = 0;
+    for (int n = 1; n <= 16; ++n)
+      if (step_smem_bytes(n, sb, B, H, F, HqD, D, rep, wsc_n, prow) <=
+          static_cast<size_t>(smem_optin))
+        best = n;
+    return best;
+  };
+  const int nl = most(kSlotBytesLarge);
+  if (nl >= kMinLargeSlots) {
+    *nslot = nl;
+    *slot_bytes = kSlotBytesLarge;
+  } else {
+    *nslot = most(kSlotBytesSmall);
+    *slot_bytes = kSlotBytesSmall;
+  }
 }
 
 // The largest split_at range of n over `ctas` parts.
