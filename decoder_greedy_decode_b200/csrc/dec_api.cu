@@ -321,9 +321,10 @@ extern "C" int dec_kv_alloc(dec_handle* h, int batch, int max_ctx, int dtype, vo
 static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* pos,
                    const dec_kv* kv, int32_t* out_ids, float* logits, float* hidden,
                    cudaStream_t stream, int n_steps = 1, int eos = -1,
-                   int32_t* gen_pos = nullptr, const int* retired = nullptr) {
+                   int32_t* gen_pos = nullptr, const int* retired = nullptr, int vseq = -1) {
   if (!h || !kv || !tok || !pos || !out_ids || !kv->base) return DEC_ERR_NULL;
-  if (batch < 1 || batch > h->shape.max_batch || batch > kv->batch) return DEC_ERR_BATCH;
+  if (batch < 1 || batch > h->shape.max_batch || (vseq < 0 && batch > kv->batch))
+    return DEC_ERR_BATCH;
   if (kv->dtype != DEC_KV_BF16 && kv->dtype != DEC_KV_FP8_E4M3) return DEC_ERR_DTYPE;
   if (kv->bytes < dec_kv_bytes(h, kv->batch, kv->max_ctx, kv->dtype)) return DEC_ERR_KV_SIZE;
   const dec_shape& s = h->shape;
@@ -383,6 +384,7 @@ static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* 
   a.n_steps = n_steps;
   a.eos = eos;
   a.gen_pos = gen_pos;
+  a.vseq = vseq;
   a.out_logits = logits;
   a.hidden_out = hidden;
   const WorkspaceLayout& wl = h->wl;
@@ -460,11 +462,15 @@ extern "C" int dec_verify(dec_handle* h, int k, const int32_t* token_ids,
                           const int32_t* positions, int seq, const dec_kv* kv, int32_t* out_ids,
                           float* out_logits, void* stream) {
   if (!h || !kv || !token_ids || !positions || !out_ids || !kv->base) return DEC_ERR_NULL;
-  if (!h->bt) return DEC_ERR_BATCH;  // the handle has no batched step (max_batch <= 4)
   if (k < 1 || k > h->shape.max_batch) return DEC_ERR_BATCH;
   if (seq < 0 || seq >= kv->batch) return DEC_ERR_ARG;
   if (kv->dtype != DEC_KV_BF16 && kv->dtype != DEC_KV_FP8_E4M3) return DEC_ERR_DTYPE;
   if (kv->bytes < dec_kv_bytes(h, kv->batch, kv->max_ctx, kv->dtype)) return DEC_ERR_KV_SIZE;
+  const int rep = h->shape.n_q_heads / h->shape.n_kv_heads;
+  if (k <= kMaxBatchSmall && k * rep <= kMaxVerifyHeads)  // the persistent kernel: one launch
+    return do_step(h, k, token_ids, positions, kv, out_ids, out_logits, nullptr,
+                   static_cast<cudaStream_t>(stream), 1, -1, nullptr, nullptr, seq);
+  if (!h->bt) return DEC_ERR_BATCH;  // larger blocks need the batched step (max_batch > 4)
   BtIO io{};
   io.B = k;
   io.tok = token_ids;

@@ -16,6 +16,7 @@ constexpr int kSlotBytesSmall = 24576;
 constexpr int kMinLargeSlots = 3;
 constexpr int kMaxBatchSmall = 4;                   // batch handled by the GEMV step kernel
 constexpr int kMaxRep = 4;                          // query heads per KV head (step kernel)
+constexpr int kMaxVerifyHeads = 8;                  // query heads per KV head of a block the step kernel verifies
 constexpr int kLayerPtrs = 11;
 constexpr int kMaxBatch = 64;                       // batched step: the N of the tensor-core tiles
 constexpr int kProfStampsPerLayer = 32;             // profiling builds: timestamps per layer and CTA
@@ -58,6 +59,7 @@ struct StepArgs {
   int n_steps;          // greedy steps this launch runs (ids fed back on the device)
   int eos;              // end-of-sequence id, or -1
   int32_t* gen_pos;     // n_steps > 1: the caller's positions, advanced in place; else null
+  int vseq;             // >= 0: block verification, every row is a token of cache sequence vseq
   float* out_logits;    // [B, V] or null
   float* hidden_out;    // [L+1, B, H] or null
   // workspace

@@ -146,8 +146,10 @@ __host__ __device__ inline Carve carve(int nslot, int slot_bytes, int B, int kma
   o += align_up(2 * nslot * sizeof(uint64_t), 16);
   // fp32 activations [B][kmax], or their bf16 hi/lo planes [B][2][kmax + pad]
   size_t act_b = static_cast<size_t>(B) * kmax * sizeof(float) + 2ull * B * kRowPad;
-  size_t att_b = (static_cast<size_t>(rep + 2) * D + static_cast<size_t>(kCW) * rep * (D + 2)) *
-                 sizeof(float);
+  // attention: qs[hm][D], kn/vn[B][D], merge[kCW][hm][D + 2] for hm query
+  // heads per item (a verification block: B * rep of them, at most 8)
+  const size_t hm = static_cast<size_t>(B * rep <= 8 && B * rep > rep ? B * rep : rep);
+  size_t att_b = ((hm + 2ull * B) * D + static_cast<size_t>(kCW) * hm * (D + 2)) * sizeof(float);
   c.act = o;
   o += align_up(act_b > att_b ? act_b : att_b, 16);
   c.stg = o;
@@ -562,10 +564,16 @@ struct Cta {
 
   // The attention items of plan P's positions: chunk rows sized so that the
   // items fit the grid when possible.  Same on every CTA and both sides.
+  // Block verification (a.vseq >= 0): the rows are consecutive tokens of one
+  // cached sequence; its committed prefix [0, pos[0]) is split into chunks
+  // shared by all rows, and chunk 0 also holds the block's own new rows.
   __device__ void make_plan(Plan& P) const {
+    const bool ver = a.vseq >= 0;
     long long T = 0;
-    for (int b = 0; b < a.B; ++b) T += static_cast<long long>(P.pos[b] + 1) * a.Hkv;
-    int slots = nc - a.B * a.Hkv;
+    if (ver) T = static_cast<long long>(P.pos[0] + a.B) * a.Hkv;
+    else
+      for (int b = 0; b < a.B; ++b) T += static_cast<long long>(P.pos[b] + 1) * a.Hkv;
+    int slots = nc - (ver ? 1 : a.B) * a.Hkv;
     if (slots < 1) slots = 1;
     long long cr = (T + slots - 1) / slots;
     cr = (cr + 15) / 16 * 16;
@@ -573,15 +581,27 @@ struct Cta {
     P.crow = static_cast<int>(cr);
     P.n_items = 0;
     int all = 1;
-    for (int b = 0; b < a.B; ++b) {
-      const int nb = (P.pos[b] + 1 + P.crow - 1) / P.crow;
-      P.nchunk[b] = nb;
-      P.n_items += nb * a.Hkv;
-      all &= P.done[b];
+    if (ver) {
+      const int nb = max(1, (P.pos[0] + P.crow - 1) / P.crow);
+      P.nchunk[0] = nb;
+      P.n_items = nb * a.Hkv;
+    } else {
+      for (int b = 0; b < a.B; ++b) {
+        const int nb = (P.pos[b] + 1 + P.crow - 1) / P.crow;
+        P.nchunk[b] = nb;
+        P.n_items += nb * a.Hkv;
+      }
     }
+    for (int b = 0; b < a.B; ++b) all &= P.done[b];
     P.all_done = all;
   }
   __device__ void item(int it, int& b, int& g, int& ci) const {
+    if (a.vseq >= 0) {
+      b = 0;
+      g = it / pl->nchunk[0];
+      ci = it % pl->nchunk[0];
+      return;
+    }
     int bb = 0;
     while (bb < a.B - 1 && it >= pl->nchunk[bb] * a.Hkv) {
       it -= pl->nchunk[bb] * a.Hkv;
@@ -721,7 +741,8 @@ struct Cta {
         int b, g, ci;
         item(it, b, g, ci);
         const int j0 = ci * pl->crow;
-        const int jc = min(j0 + pl->crow, pl->pos[b]);
+        const int jc = min(j0 + pl->crow, pl->pos[b]);  // (verify: b = 0, the prefix end)
+        if (a.vseq >= 0) b = a.vseq;                     // the cache sequence
         for (int j = j0; j < jc && !dead; j += art) {
           const int nr = min(art, jc - j);
           if constexpr (!FP8) {
@@ -1407,56 +1428,73 @@ struct Cta {
   // head g of sequence b over cached rows [j0, jc) streamed through the ring,
   // plus the new row p_b (from the gathered q/k/v, rotated and rounded as the
   // cache stores it; the CTA whose chunk holds p_b writes it to the cache).
-  // The query heads of a KV head form groups of at most two; every lane octet
-  // serves one group and scores each of its rows against both heads, so a
-  // K/V row is read once per group.  Octet i of a group takes rows i, i +
-  // octets per group, ...; each lane holds a D/8-wide slice (3-shuffle dot
-  // products).  The CTA of chunk 0 combines the chunks' partial softmax
-  // states and publishes the head outputs; other chunks publish their partial
-  // state and move on.  act holds qs[rep][D], kn[D], vn[D], merge[kCW][rep][D + 2].
+  // In block verification (a.vseq >= 0) an item (g, chunk) serves the query
+  // heads of every row of the block at once over the shared prefix, and
+  // chunk 0 adds the block's new rows, causally: row i sees new rows 0..i.
+  // The item's query heads form groups of two; every lane octet serves one
+  // group and scores each of its rows against both heads, so a K/V row is
+  // read once per group.  Octet i of a group takes rows i, i + octets per
+  // group, ...; each lane holds a D/8-wide slice (3-shuffle dot products).
+  // The CTA of chunk 0 combines the chunks' partial softmax states and
+  // publishes the head outputs; other chunks publish their partial state and
+  // move on.  act holds qs[hi][D], kn[nn][D], vn[nn][D], merge[kCW][hi][D + 2]
+  // (hi heads and nn new rows of the item).
   __device__ void attention(int l) {
+    const bool ver = a.vseq >= 0;
     const int rep = a.Hq / a.Hkv;
-    const int ngrp = (rep + 1) >> 1;               // head groups of <= 2 heads
+    const int hi = ver ? B * rep : rep;        // query heads of an item (<= 8 when verifying)
+    const int nn = ver ? B : 1;                // new rows of an item
+    const int ng0 = (hi + 1) >> 1;
+    const int ngrp = ng0 <= 1 ? 1 : (ng0 <= 2 ? 2 : 4);  // head groups (of <= 2 heads)
     const int q8 = lane >> 3, e8 = lane & 7;
     const int octet = warp * 4 + q8;
     const int hg = octet % ngrp, oi = octet / ngrp, ostep = 32 / ngrp;
-    const int hb = 2 * hg, nh = min(2, rep - hb);  // this octet's heads hb, hb + 1
+    const int hb = 2 * hg, nh = max(0, min(2, hi - hb));  // this octet's heads hb, hb + 1
     const float qscale = 1.4426950408889634f / sqrtf(static_cast<float>(D));  // log2(e)/sqrt(D)
     float* qs = act;
-    float* kn = act + rep * D;
-    float* vn = kn + D;
-    float* merge = vn + D;
+    float* kn = act + hi * D;
+    float* vn = kn + nn * D;
+    float* merge = vn + nn * D;
     const LayerPtrs& lw = slw[l];
     const uint32_t f = flag(l);
-    const int HqD = a.Hq * D;
+    const int HqD = a.Hq * D, HkvD = a.Hkv * D;
+    // sequence (row) and query head of item head h
+    auto hrow = [&](int h, int b) { return ver ? h / rep : b; };
+    auto hq = [&](int h, int g) { return g * rep + (ver ? h % rep : h); };
     for (int it = cta; it < pl->n_items; it += nc) {
       int b, g, ci;
       item(it, b, g, ci);
-      const int p = pl->pos[b];
-      const bool live = !pl->done[b];  // a retired sequence writes no cache row
+      const int p = ver ? pl->pos[0] : pl->pos[b];  // verify: the prefix length
+      const bool live = ver || !pl->done[b];        // a retired sequence writes no cache row
+      const int cs = ver ? a.vseq : b;              // cache sequence
       const int j0 = ci * pl->crow;
-      const int j1 = min(j0 + pl->crow, p + 1);
+      const int j1 = ver ? min(j0 + pl->crow, p) : min(j0 + pl->crow, p + 1);
       const int jc = min(j1, p);  // cached rows [j0, jc)
-      const bool has_new = (p >= j0 && p < j1);
-      // -- inputs: warp w < rep takes query head g*rep + w, warp rep the key
-      //    and warp rep + 1 the value (both only for the chunk holding p_b)
-      if (warp < rep || (has_new && warp < rep + 2)) {
-        const uint16_t* gn = warp < rep ? lw.w[4] : lw.w[5];
+      const bool has_new = ver ? ci == 0 : (p >= j0 && p < j1);
+      // -- inputs: vector v < hi is the query head v, then (only for the chunk
+      //    holding the new rows) the keys and the values of the nn new rows;
+      //    warp w takes vectors w, w + kCW, ...
+      const int nvec = hi + (has_new ? 2 * nn : 0);
+      for (int v0 = warp; v0 < nvec; v0 += kCW) {
+        const int kind = v0 < hi ? 0 : (v0 < hi + nn ? 1 : 2);  // q, k, v
+        const int j = kind == 0 ? 0 : (v0 - hi - (kind == 2 ? nn : 0));  // new row
+        const int row = kind == 0 ? hrow(v0, b) : (ver ? j : b);
+        const int prow = pl->pos[row];
+        const uint16_t* gn = kind == 0 ? lw.w[4] : lw.w[5];
         float gq[DL], invf[DL / 2];
 #pragma unroll
-        for (int k = 0; k < DL; ++k) gq[k] = warp <= rep ? bf16_to_f(__ldg(gn + lane + 32 * k)) : 0.f;
+        for (int k = 0; k < DL; ++k) gq[k] = kind < 2 ? bf16_to_f(__ldg(gn + lane + 32 * k)) : 0.f;
 #pragma unroll
         for (int k = 0; k < DL / 2; ++k) invf[k] = __ldg(a.inv_freq + lane + 32 * k);
-        const uint64_t* src = a.x_qkv + static_cast<size_t>(b) * nqkv +
-                              (warp < rep ? (g * rep + warp) * D
-                                          : HqD + (warp - rep) * a.Hkv * D + g * D);
+        const uint64_t* src = a.x_qkv + static_cast<size_t>(row) * nqkv +
+                              (kind == 0 ? hq(v0, g) * D : HqD + (kind - 1) * HkvD + g * D);
         uint64_t* ws = stg + warp * kWarpStage;
         warp_gather(ws, D, f, [=](int i) { return src + i; });
         if (!ab) {
           float v[DL];
 #pragma unroll
           for (int k = 0; k < DL; ++k) v[k] = __uint_as_float(static_cast<uint32_t>(ws[lane + 32 * k]));
-          if (warp <= rep) {  // q/k RMSNorm + RoPE
+          if (kind < 2) {  // q/k RMSNorm + RoPE
             float ss = 0.f;
 #pragma unroll
             for (int k = 0; k < DL; ++k) ss = fmaf(v[k], v[k], ss);
@@ -1466,19 +1504,19 @@ struct Cta {
             for (int k = 0; k < DL; ++k) v[k] = v[k] * inv * gq[k];
 #pragma unroll
             for (int k = 0; k < DL / 2; ++k) {
-              const float ang = __fmul_rn(static_cast<float>(p), invf[k]);
-              float sn, cs;
-              rope_sincos(ang, &sn, &cs);
+              const float ang = __fmul_rn(static_cast<float>(prow), invf[k]);
+              float sn, c;
+              rope_sincos(ang, &sn, &c);
               const float x1 = v[k], x2 = v[k + DL / 2];
-              v[k] = x1 * cs - x2 * sn;
-              v[k + DL / 2] = x2 * cs + x1 * sn;
+              v[k] = x1 * c - x2 * sn;
+              v[k + DL / 2] = x2 * c + x1 * sn;
             }
           }
-          if (warp >= rep) {
+          if (kind > 0) {
             // the new K / V row as the cache stores it, written by this chunk
-            const size_t row = kv_row(l, warp - rep, b, g, p);
+            const size_t crow = kv_row(l, kind - 1, cs, g, prow);
             if constexpr (!FP8) {
-              uint16_t* dstp = reinterpret_cast<uint16_t*>(a.kv) + row * D;
+              uint16_t* dstp = reinterpret_cast<uint16_t*>(a.kv) + crow * D;
 #pragma unroll
               for (int k = 0; k < DL; ++k) {
                 const uint16_t h = f_to_bf16(v[k]);
@@ -1489,14 +1527,14 @@ struct Cta {
               uint8_t code[DL];
               const float sc = quantize_row_e4m3<DL>(v, code);
               if (live) {
-                uint8_t* dstp = a.kv + row * D;
+                uint8_t* dstp = a.kv + crow * D;
 #pragma unroll
                 for (int k = 0; k < DL; ++k) dstp[lane + 32 * k] = code[k];
-                if (lane == 0) a.kv_scales[row] = sc;
+                if (lane == 0) a.kv_scales[crow] = sc;
               }
             }
           }
-          float* x = warp < rep ? qs + warp * D : (warp == rep ? kn : vn);
+          float* x = kind == 0 ? qs + v0 * D : (kind == 1 ? kn : vn) + j * D;
 #pragma unroll
           for (int k = 0; k < DL; ++k) x[lane + 32 * k] = v[k];
         }
@@ -1573,58 +1611,66 @@ struct Cta {
         }
         release_tile();
       }
-      if (!ab && has_new && warp == 0) {  // the new row, kept by the first octet of each group
-        float s[2];
+      // the new rows, kept by the first octet of each group (a warp-uniform
+      // loop: the warps holding those octets shuffle as a whole); head h sees
+      // new row j when j <= its own row
+      if (!ab && has_new && 4 * warp < ngrp) {
+        for (int j = 0; j < nn; ++j) {
+          float sv[2];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float t = 0.f;
+          for (int hh = 0; hh < 2; ++hh) {
+            float t = 0.f;
 #pragma unroll
-          for (int k = 0; k < DQ; ++k) t = fmaf(qv[hh][k], kn[e8 * DQ + k], t);
-          t += __shfl_xor_sync(0xffffffffu, t, 4);
-          t += __shfl_xor_sync(0xffffffffu, t, 2);
-          t += __shfl_xor_sync(0xffffffffu, t, 1);
-          s[hh] = t;
-        }
+            for (int k = 0; k < DQ; ++k) t = fmaf(qv[hh][k], kn[j * D + e8 * DQ + k], t);
+            t += __shfl_xor_sync(0xffffffffu, t, 4);
+            t += __shfl_xor_sync(0xffffffffu, t, 2);
+            t += __shfl_xor_sync(0xffffffffu, t, 1);
+            sv[hh] = t;
+          }
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          if (hh < nh && oi == 0) {
-            const float mn = fmaxf(m[hh], s[hh]);
-            const float al = exp2f(m[hh] - mn), pe = exp2f(s[hh] - mn);
-            ls[hh] = ls[hh] * al + pe;
+          for (int hh = 0; hh < 2; ++hh) {
+            if (hh < nh && oi == 0 && (!ver || j <= (hb + hh) / rep)) {
+              const float mn = fmaxf(m[hh], sv[hh]);
+              const float al = exp2f(m[hh] - mn), pe = exp2f(sv[hh] - mn);
+              ls[hh] = ls[hh] * al + pe;
 #pragma unroll
-            for (int k = 0; k < DQ; ++k) acc[hh][k] = fmaf(acc[hh][k], al, pe * vn[e8 * DQ + k]);
-            m[hh] = mn;
+              for (int k = 0; k < DQ; ++k) acc[hh][k] = fmaf(acc[hh][k], al, pe * vn[j * D + e8 * DQ + k]);
+              m[hh] = mn;
+            }
           }
         }
       }
       // merge the octets of the warp that serve the same head group (xor 16,
-      // and xor 8 when there is one group); the first octet of each group
-      // writes the warp's state
+      // and xor 8 when there is one group; with four groups every octet of a
+      // warp serves its own); the first octet of each group writes the warp's
+      // state
       if (!ab) {
+        if (ngrp < 4) {
 #pragma unroll
-        for (int o = 8; o <= 16; o <<= 1) {
-          if (o == 8 && ngrp != 1) continue;
+          for (int o = 8; o <= 16; o <<= 1) {
+            if (o == 8 && ngrp != 1) continue;
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const float mo = __shfl_xor_sync(0xffffffffu, m[hh], o);
-            const float lo = __shfl_xor_sync(0xffffffffu, ls[hh], o);
-            const float mn = fmaxf(m[hh], mo);
-            const float e1 = (m[hh] == -INFINITY) ? 0.f : exp2f(m[hh] - mn);
-            const float e2 = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
-            ls[hh] = ls[hh] * e1 + lo * e2;
+            for (int hh = 0; hh < 2; ++hh) {
+              const float mo = __shfl_xor_sync(0xffffffffu, m[hh], o);
+              const float lo = __shfl_xor_sync(0xffffffffu, ls[hh], o);
+              const float mn = fmaxf(m[hh], mo);
+              const float e1 = (m[hh] == -INFINITY) ? 0.f : exp2f(m[hh] - mn);
+              const float e2 = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+              ls[hh] = ls[hh] * e1 + lo * e2;
 #pragma unroll
-            for (int k = 0; k < DQ; ++k) {
-              const float ao = __shfl_xor_sync(0xffffffffu, acc[hh][k], o);
-              acc[hh][k] = acc[hh][k] * e1 + ao * e2;
+              for (int k = 0; k < DQ; ++k) {
+                const float ao = __shfl_xor_sync(0xffffffffu, acc[hh][k], o);
+                acc[hh][k] = acc[hh][k] * e1 + ao * e2;
+              }
+              m[hh] = mn;
             }
-            m[hh] = mn;
           }
         }
         if (q8 < ngrp) {
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             if (hh < nh) {
-              float* mg = merge + (static_cast<size_t>(warp) * rep + hb + hh) * (D + 2);
+              float* mg = merge + (static_cast<size_t>(warp) * hi + hb + hh) * (D + 2);
 #pragma unroll
               for (int k = 0; k < DQ; ++k) mg[e8 * DQ + k] = acc[hh][k];
               if (e8 == 0) {
@@ -1639,23 +1685,27 @@ struct Cta {
       DEC_STAMP(kStampsPerLayer * l + StAttRows);
       DEC_SVAL(kStampsPerLayer * l + StWA, wacc);
       // -- this chunk's partial state (m in log2 units, l, unnormalised acc)
+      // for thread slots t = tid + kCT * i: (head, element) = t / D, t % D
+      constexpr int kSlots = (8 * D + kCT - 1) / kCT;
       const bool combiner = (ci == 0);
       const int pc = a.part_chunks;
-      const uint64_t* pbase =
-          a.part + (static_cast<size_t>(b) * a.Hq + g * rep) * pc * (D + 2);
-      float RM[2], RL[2], RA[2];  // (h, d) = t / D, t % D for t = tid + kCT * i
+      // partial state of chunk c for item head h
+      auto pstate = [&](int h, int c) {
+        return a.part + ((static_cast<size_t>(hrow(h, b)) * a.Hq + hq(h, g)) * pc + c) * (D + 2);
+      };
+      float RM[kSlots], RL[kSlots], RA[kSlots];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < kSlots; ++i) {
         const int t = tid + kCT * i;
         RM[i] = -INFINITY;
         RL[i] = RA[i] = 0.f;
-        if (!ab && t < rep * D) {
+        if (!ab && t < hi * D) {
           const int h = t / D, d = t % D;
           float M = -INFINITY;
-          for (int w = 0; w < kCW; ++w) M = fmaxf(M, merge[(w * rep + h) * (D + 2) + D]);
+          for (int w = 0; w < kCW; ++w) M = fmaxf(M, merge[(w * hi + h) * (D + 2) + D]);
           float Ls = 0.f, A = 0.f;
           for (int w = 0; w < kCW; ++w) {
-            const float* mg = merge + (w * rep + h) * (D + 2);
+            const float* mg = merge + (w * hi + h) * (D + 2);
             const float e = (mg[D] == -INFINITY) ? 0.f : exp2f(mg[D] - M);
             Ls += mg[D + 1] * e;
             A += mg[d] * e;
@@ -1665,7 +1715,7 @@ struct Cta {
             RL[i] = Ls;
             RA[i] = A;
           } else {
-            uint64_t* pp = a.part + ((static_cast<size_t>(b) * a.Hq + g * rep + h) * pc + ci) * (D + 2);
+            uint64_t* pp = pstate(h, ci);
             st_tagged(pp + d, A, f);
             if (d == 0) {
               st_tagged(pp + D, M, f);
@@ -1675,23 +1725,22 @@ struct Cta {
         }
       }
       if (combiner) {  // uniform over the CTA: ci is the item's
-        const int nc1 = pl->nchunk[b] - 1;
-        const int win = kStageWords / (rep * (D + 2));
+        const int nc1 = pl->nchunk[ver ? 0 : b] - 1;
+        const int win = kStageWords / (hi * (D + 2));
         for (int c0 = 1; c0 <= nc1; c0 += win) {
           const int nw = min(win, nc1 - c0 + 1);
-          gather(nw * rep * (D + 2), f, [=](int w) {
+          gather(nw * hi * (D + 2), f, [=](int w) {
             const int sg = w / (D + 2), off = w % (D + 2);
-            const int c = c0 + sg / rep, h = sg % rep;
-            return pbase + (static_cast<size_t>(h) * pc + c) * (D + 2) + off;
+            return pstate(sg % hi, c0 + sg / hi) + off;
           });
           if (!ab) {
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
+            for (int i = 0; i < kSlots; ++i) {
               const int t = tid + kCT * i;
-              if (t < rep * D) {
+              if (t < hi * D) {
                 const int h = t / D, d = t % D;
                 for (int cc = 0; cc < nw; ++cc) {
-                  const uint64_t* pw = stg + (cc * rep + h) * (D + 2);
+                  const uint64_t* pw = stg + (cc * hi + h) * (D + 2);
                   const float Mc = __uint_as_float(static_cast<uint32_t>(pw[D]));
                   const float Lc = __uint_as_float(static_cast<uint32_t>(pw[D + 1]));
                   const float Ac = __uint_as_float(static_cast<uint32_t>(pw[d]));
@@ -1708,11 +1757,12 @@ struct Cta {
         }
         if (!ab) {
 #pragma unroll
-          for (int i = 0; i < 2; ++i) {
+          for (int i = 0; i < kSlots; ++i) {
             const int t = tid + kCT * i;
-            if (t < rep * D) {
+            if (t < hi * D) {
               const int h = t / D, d = t % D;
-              st_tagged(a.x_o + static_cast<size_t>(b) * HqD + (g * rep + h) * D + d, RA[i] / RL[i], f);
+              st_tagged(a.x_o + static_cast<size_t>(hrow(h, b)) * HqD + hq(h, g) * D + d,
+                        RA[i] / RL[i], f);
             }
           }
         }
@@ -1899,6 +1949,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
       P.tok[b] = t;
       P.done[b] = 0;
       if (p < 0 || p >= a.max_ctx) bad |= kDevBadPos;
+      if (a.vseq >= 0 && p != a.positions[0] + b) bad |= kDevBadPos;  // a block is consecutive
       if (t < 0 || t >= a.V) bad |= kDevBadTok;
     }
     P.bad = bad;

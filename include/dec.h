@@ -169,7 +169,7 @@ typedef struct dec_weights_int8 {
 /* dec_init for a weight-only int8 model.  Same ownership and errors as
  * dec_init; max_batch must be 1..4 (DEC_ERR_BATCH otherwise): int8 weights
  * run on the single persistent kernel (dec_step, dec_step_host,
- * dec_generate); dec_verify needs a bf16 handle. */
+ * dec_generate, and dec_verify for blocks of up to 4). */
 int dec_init_int8(const dec_shape *shape, const dec_weights_int8 *weights, dec_handle **out);
 
 /* Release the handle and its workspace (synchronises the device first). */
@@ -262,7 +262,10 @@ int dec_generate(dec_handle *h, int batch, int n_steps, const int32_t *token_ids
 
 /* Verify a block of k consecutive tokens of ONE cached sequence in a single
  * step ("Can CTC make Qwen3-ASR faster?", §11 Phase A steps 2-3: one target
- * forward over the whole draft block; §03: greedy verification).
+ * forward over the whole draft block; §03: greedy verification).  Blocks of
+ * k <= 4 (with k * n_q_heads / n_kv_heads <= 8) run as one launch of the
+ * persistent kernel, which reads the committed prefix of the sequence once
+ * for the whole block; larger blocks run the batched step.
  *   token_ids  int32 [k] (device)  t_0 = the last committed token, then the
  *                                  draft tokens t_1 .. t_{k-1}
  *   positions  int32 [k] (device)  p0 + i: row i is written to cache row
@@ -274,9 +277,12 @@ int dec_generate(dec_handle *h, int batch, int n_steps, const int32_t *token_ids
  *                                  may alias token_ids
  *   out_logits fp32 [k, vocab] or NULL.
  * Results equal k single-sequence steps fed t_0 .. t_{k-1} (up to rounding).
- * Needs a handle created with max_batch > 4 (it runs the batched step) and
- * 1 <= k <= max_batch.  Asynchronous; invalid positions / tokens behave as in
- * dec_step.  Cache rows p0 .. p0 + k - 1 of `seq` are overwritten. */
+ * Needs 1 <= k <= max_batch; blocks the persistent kernel does not take need
+ * a handle created with max_batch > 4 (DEC_ERR_BATCH otherwise).  int8
+ * handles verify blocks of up to 4.  Asynchronous; invalid positions /
+ * tokens, and positions that are not p0, p0 + 1, ..., behave as in dec_step
+ * (DEC_DEV_BAD_POSITION).  Cache rows p0 .. p0 + k - 1 of `seq` are
+ * overwritten. */
 int dec_verify(dec_handle *h, int k, const int32_t *token_ids, const int32_t *positions,
                int seq, const dec_kv *kv, int32_t *out_ids, float *out_logits, void *stream);
 

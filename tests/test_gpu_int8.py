@@ -88,12 +88,12 @@ def test_quantizer_rejects_bad_arguments():
         capi.dec_quantize_int8(w2.data_ptr() + 2, 4, 16, codes, scales)  # misaligned
 
 
-def _setup_int8(s, seed, batch, max_ctx, lengths, kind="bf16", gain_std=0.0):
+def _setup_int8(s, seed, batch, max_ctx, lengths, kind="bf16", gain_std=0.0, max_batch=None):
     w = synth.model_weights(s, seed=seed, gain_std=gain_std)
     kv_host, sc_host = synth.kv_prefill(s, batch, max_ctx, lengths, seed=seed + 100, kind=kind)
     m = oracle.Model(oracle_shape(s), oracle.quantize_weights_int8(oracle_weights(w)))
     caches = [oracle_cache(kv_host, sc_host, b) for b in range(batch)]
-    dec = Decoder(s, quantize_int8(to_device(w)), max_batch=batch)
+    dec = Decoder(s, quantize_int8(to_device(w)), max_batch=max_batch or batch)
     kv = dec.kv_cache(batch, max_ctx, kind)
     if kind == "bf16":
         kv.values.copy_(kv_host.cuda())
@@ -146,9 +146,29 @@ def test_int8_handle_limits():
         Decoder(s, w8, max_batch=5)          # int8 runs on the persistent kernel only
     dec = Decoder(s, w8, max_batch=4)
     kv = dec.kv_cache(1, 32)
-    out = torch.zeros(2, dtype=torch.int32, device="cuda")
-    with pytest.raises(RuntimeError):
-        dec.verify(kv, i32([1, 2]), i32([3, 4]), 0, out)   # needs a bf16 batched handle
+    out = torch.zeros(5, dtype=torch.int32, device="cuda")
+    with pytest.raises(RuntimeError):       # blocks of 5 and more need the batched step
+        dec.verify(kv, i32([1, 2, 3, 4, 5]), i32([3, 4, 5, 6, 7]), 0, out)
+    dec.close()
+
+
+def test_int8_verify_block_equals_single_steps():
+    """A block of 4 tokens verified on an int8 handle (persistent kernel)
+    equals 4 teacher-forced single steps of the oracle's int8 model."""
+    s = synth.TINY
+    n0, k = 30, 4
+    m, caches, dec, kv = _setup_int8(s, 320, 1, 64, [n0], "bf16", 0.0, max_batch=4)
+    toks = [int(t) for t in synth.tokens(s.vocab, k, seed=321)]
+    out = torch.full((k,), -7, dtype=torch.int32, device="cuda")
+    logits = torch.empty((k, s.vocab), dtype=torch.float32, device="cuda")
+    dec.verify(kv, i32(toks), i32(range(n0, n0 + k)), 0, out, logits)
+    assert dec.check() == 0
+    ids, lg = out.cpu().tolist(), logits.cpu().numpy()
+    for i in range(k):
+        r = m.step(caches[0], toks[i], n0 + i)
+        assert_close(lg[i], r.logits, f"int8 verify row {i} logits")
+        assert_id(ids[i], r, f"int8 verify row {i}")
+        _check_kv_row(kv, caches[0], 0, n0 + i, f"int8 verify row {i}")
     dec.close()
 
 

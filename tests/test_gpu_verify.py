@@ -53,12 +53,15 @@ def _verify(dec, kv, toks, p0, seq):
 
 
 @pytest.mark.parametrize("kind", ["bf16", "fp8"])
-def test_verify_block_equals_single_steps(kind):
-    """A block of 9 tokens of sequence 1 (of 3 in the cache) equals 9
+@pytest.mark.parametrize("k", [1, 2, 3, 4, 9])
+def test_verify_block_equals_single_steps(kind, k):
+    """A block of k tokens of sequence 1 (of 3 in the cache) equals k
     teacher-forced single steps of the oracle: logits, ids, appended rows;
-    the other sequences' rows are untouched."""
+    the other sequences' rows are untouched.  Blocks of up to 4 run on the
+    persistent kernel (the prefix read once for the whole block), larger
+    ones on the batched step."""
     s = synth.TINY
-    n0, k, seq = 40, 9, 1
+    n0, seq = 40, 1
     m, dec, kv, kv_host, sc_host = _setup(s, 80, 3, 64, [30, n0, 50], kind)
     cache = oracle_cache(kv_host, sc_host, seq)
     toks = [int(t) for t in synth.tokens(s.vocab, k, seed=81)]
@@ -119,14 +122,64 @@ def test_speculative_decode_commits_the_greedy_sequence():
     dec.close()
 
 
-def test_verify_needs_a_batched_handle():
+def test_verify_block_limits():
+    """A handle of max_batch 4 verifies blocks of up to 4 (persistent kernel),
+    not 5; a block whose positions are not consecutive is reported on the
+    device and leaves the cache unchanged."""
     s = synth.TINY
     w = to_device(synth.model_weights(s, seed=93))
     dec = Decoder(s, w, max_batch=4)
     kv = dec.kv_cache(1, 32)
-    out = torch.zeros(2, dtype=torch.int32, device="cuda")
+    out = torch.zeros(5, dtype=torch.int32, device="cuda")
     with pytest.raises(RuntimeError):
-        dec.verify(kv, i32([1, 2]), i32([3, 4]), 0, out)
+        dec.verify(kv, i32([1, 2, 3, 4, 5]), i32([3, 4, 5, 6, 7]), 0, out)
+    before = kv.buf.clone()
+    dec.verify(kv, i32([1, 2]), i32([3, 5]), 0, out[:2])
+    assert dec.check() == capi.DEC_DEV_BAD_POSITION
+    assert out[:2].cpu().tolist() == [-1, -1]
+    assert torch.equal(before, kv.buf)
+    dec.verify(kv, i32([1, 2]), i32([3, 4]), 0, out[:2])
+    assert dec.check() == 0
+    dec.close()
+
+
+@pytest.mark.parametrize("blk", [2, 4])
+def test_speculative_small_blocks_commit_the_greedy_sequence(blk):
+    """Speculation with blocks of 2 and 4 (the persistent kernel verifies
+    them): the committed tokens equal the oracle's greedy sequence."""
+    s = synth.TINY
+    n0, total = 24, 24
+    m, dec, kv, kv_host, _ = _setup(s, 96, 1, 96, [n0], max_batch=4)
+    ref_cache = oracle_cache(kv_host, None, 0)
+    t0 = int(synth.tokens(s.vocab, 1, seed=97)[0])
+    ref, margins, tok = [], [], t0
+    for i in range(total + blk):
+        r = m.step(ref_cache, tok, n0 + i)
+        ref.append(r.token)
+        margins.append(r.margin)
+        tok = r.token
+    rng = np.random.default_rng(98)
+    committed, cur, p = [], t0, n0
+    while len(committed) < total:
+        c = len(committed)
+        draft = list(ref[c:c + blk - 1])
+        if rng.random() < 0.5:
+            j = int(rng.integers(0, len(draft)))
+            draft[j] = (draft[j] + 1 + int(rng.integers(0, s.vocab - 1))) % s.vocab
+        ids, _ = _verify(dec, kv, [cur] + draft, p, 0)
+        emitted = capi.dec_accept_greedy([cur] + draft, ids)
+        for e in emitted:
+            i = len(committed)
+            if i >= total:
+                break
+            if e != ref[i]:
+                assert margins[i] < NEAR_TIE, f"token {i}: {e} != {ref[i]}"
+                dec.close()
+                return
+            committed.append(e)
+        p += len(emitted)
+        cur = emitted[-1]
+    assert committed == ref[:total]
     dec.close()
 
 
@@ -137,10 +190,12 @@ def big06():
     return s, w, to_device(w)
 
 
-def test_0p6b_verify_block_of_16(big06):
-    """0.6B shape, context 795, a 16-token block: sampled rows vs the oracle."""
+@pytest.mark.parametrize("k", [4, 16])
+def test_0p6b_verify_block(big06, k):
+    """0.6B shape, context 795, blocks of 4 (persistent kernel) and 16
+    (batched step): sampled rows vs the oracle."""
     s, w, wd = big06
-    n0, k = 795, 16
+    n0 = 795
     kv_host, _ = synth.kv_prefill(s, 1, 816, [n0], seed=94)
     dec = Decoder(s, wd, max_batch=64)
     kv = dec.kv_cache(1, 816)
@@ -151,7 +206,7 @@ def test_0p6b_verify_block_of_16(big06):
     ids, logits = _verify(dec, kv, toks, n0, 0)
     for i in range(k):
         r = m.step(cache, toks[i], n0 + i)
-        if i in (0, 7, 15):
+        if i in (0, k // 2, k - 1):
             assert_close(logits[i], r.logits, f"row {i} logits")
             _check_kv_row(kv, cache, 0, n0 + i, f"row {i}")
         assert_id(ids[i], r, f"row {i}")
