@@ -677,6 +677,19 @@ struct AttnArgs2 {
   int chunk_rows, chunks;
 };
 
+// (d0, d1) += (a0, a1) * (b0, b1) as one packed fp32x2 instruction.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0,
+                                     float b1) {
+  asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\t"
+      "mov.b64 pb, {%4, %5};\n\t"
+      "mov.b64 pd, {%0, %1};\n\t"
+      "fma.rn.f32x2 pd, pa, pb, pd;\n\t"
+      "mov.b64 {%0, %1}, pd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // Elements [i*HALF, i*HALF + HALF) (i = 0, 1) of this lane's two spans of a
 // K or V row as fp32: bf16 values, or E4M3 code values (the caller applies
 // the row scale once per row).
@@ -801,59 +814,97 @@ __global__ void __launch_bounds__(kAttThreads, 4) attn_kernel(const AttnArgs2 a)
     }
     const uint8_t* tb = ring + (t % kAttStages) * kTile;
     const float* tsc = reinterpret_cast<const float*>(tb + 2 * kHalf);
-    // kAttWarps x 4 rows per pass; every lane takes part in the shuffles,
-    // rows past nr are masked out of the softmax
+    // the tile's two passes of kAttWarps x 4 rows at once: this octet takes
+    // rows r1 and r1 + kAttWarps * 4, scores both against every query head,
+    // then folds both into its online softmax with one rescale, which it
+    // skips when the running maximum did not move.  Dot products and the
+    // value accumulation use packed fp32 pairs.  Every lane takes part in the
+    // shuffles; rows past nr are masked out of the softmax.
+    {
+      static_assert(kAttTileRows == 2 * kAttWarps * 4, "two rows per octet per tile");
+      const int r1 = warp * 4 + oct, r2 = r1 + kAttWarps * 4;
+      const bool ok1 = r1 < nr, ok2 = r2 < nr;  // ok2 implies ok1
+      const uint8_t* krow1 = tb + static_cast<size_t>(ok1 ? r1 : 0) * RB;
+      const uint8_t* krow2 = tb + static_cast<size_t>(ok2 ? r2 : 0) * RB;
+      float s1[REP], s2[REP];
+      {
+        float e1[REP], o1[REP], e2[REP], o2[REP];
 #pragma unroll
-    for (int pass = 0; pass < kAttTileRows / (kAttWarps * 4); ++pass) {
-      const int r = (pass * kAttWarps + warp) * 4 + oct;
-      const bool valid = r < nr;
-      const int rr = valid ? r : 0;
-      const uint8_t* krow = tb + static_cast<size_t>(rr) * RB;
-      const uint8_t* vrow = krow + kHalf;
-      const float ks = FP8 ? tsc[rr] : 1.f;
-      float s[REP];
+        for (int h = 0; h < REP; ++h) e1[h] = o1[h] = e2[h] = o2[h] = 0.f;
 #pragma unroll
-      for (int h = 0; h < REP; ++h) s[h] = 0.f;
+        for (int i = 0; i < 2; ++i) {
+          float kx1[HALF], kx2[HALF];
+          load_span<D, FP8>(krow1, o, i, kx1);
+          load_span<D, FP8>(krow2, o, i, kx2);
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        float kx[HALF];
-        load_span<D, FP8>(krow, o, i, kx);
+          for (int h = 0; h < REP; ++h)
 #pragma unroll
-        for (int h = 0; h < REP; ++h)
+            for (int e = 0; e < HALF; e += 2) {
+              fma2(e1[h], o1[h], qv[h][i][e], qv[h][i][e + 1], kx1[e], kx1[e + 1]);
+              fma2(e2[h], o2[h], qv[h][i][e], qv[h][i][e + 1], kx2[e], kx2[e + 1]);
+            }
+        }
 #pragma unroll
-          for (int e = 0; e < HALF; ++e) s[h] = fmaf(qv[h][i][e], kx[e], s[h]);
+        for (int h = 0; h < REP; ++h) {
+          s1[h] = e1[h] + o1[h];
+          s2[h] = e2[h] + o2[h];
+        }
       }
 #pragma unroll
       for (int sh = 4; sh > 0; sh >>= 1)
 #pragma unroll
-        for (int h = 0; h < REP; ++h) s[h] += __shfl_xor_sync(0xffffffffu, s[h], sh);
-      if (FP8) {
-#pragma unroll
-        for (int h = 0; h < REP; ++h) s[h] *= ks;  // q . (code x scale) = scale x (q . code)
-      }
-      if (valid) {
-        float al[REP], p[REP];
+        for (int h = 0; h < REP; ++h) {
+          s1[h] += __shfl_xor_sync(0xffffffffu, s1[h], sh);
+          s2[h] += __shfl_xor_sync(0xffffffffu, s2[h], sh);
+        }
+      if (FP8) {  // q . (code x scale) = scale x (q . code)
+        const float ks1 = tsc[ok1 ? r1 : 0], ks2 = tsc[ok2 ? r2 : 0];
 #pragma unroll
         for (int h = 0; h < REP; ++h) {
-          const float mn = fmaxf(m[h], s[h]);
-          al[h] = exp2f(m[h] - mn);
-          p[h] = exp2f(s[h] - mn);
-          ls[h] = ls[h] * al[h] + p[h];
-          m[h] = mn;
+          s1[h] *= ks1;
+          s2[h] *= ks2;
         }
-        if (FP8) {
-          const float vs = tsc[kAttTileRows + rr];
+      }
+      if (ok1) {
+        float p1[REP], p2[REP];
 #pragma unroll
-          for (int h = 0; h < REP; ++h) p[h] *= vs;  // p (code x scale) = (p scale) code
+        for (int h = 0; h < REP; ++h) {
+          const float x2 = ok2 ? s2[h] : -INFINITY;
+          const float mn = fmaxf(m[h], fmaxf(s1[h], x2));
+          const float al = exp2f(m[h] - mn);
+          p1[h] = exp2f(s1[h] - mn);
+          p2[h] = exp2f(x2 - mn);
+          ls[h] = ls[h] * al + (p1[h] + p2[h]);
+          m[h] = mn;
+          if (al != 1.f) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+              for (int e = 0; e < HALF; ++e) acc[h][i][e] *= al;
+          }
         }
+        if (FP8) {  // p (code x scale) = (p scale) code
+          const float vs1 = tsc[kAttTileRows + r1], vs2 = tsc[kAttTileRows + (ok2 ? r2 : r1)];
+#pragma unroll
+          for (int h = 0; h < REP; ++h) {
+            p1[h] *= vs1;
+            p2[h] *= vs2;
+          }
+        }
+        const uint8_t* vrow1 = krow1 + kHalf;
+        const uint8_t* vrow2 = (ok2 ? krow2 : krow1) + kHalf;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-          float vx[HALF];
-          load_span<D, FP8>(vrow, o, i, vx);
+          float vx1[HALF], vx2[HALF];
+          load_span<D, FP8>(vrow1, o, i, vx1);
+          load_span<D, FP8>(vrow2, o, i, vx2);
 #pragma unroll
           for (int h = 0; h < REP; ++h)
 #pragma unroll
-            for (int e = 0; e < HALF; ++e) acc[h][i][e] = fmaf(acc[h][i][e], al[h], p[h] * vx[e]);
+            for (int e = 0; e < HALF; e += 2) {
+              fma2(acc[h][i][e], acc[h][i][e + 1], p1[h], p1[h], vx1[e], vx1[e + 1]);
+              fma2(acc[h][i][e], acc[h][i][e + 1], p2[h], p2[h], vx2[e], vx2[e + 1]);
+            }
         }
       }
     }
