@@ -9,16 +9,20 @@ Bottleneck Analysis", 01 Method & setup: 795 prompt tokens -> 130 generated;
 795 + (i mod 130), so any number of timed steps keeps that context mix.
 Weights and cache are seeded synthetic random-init data.
 
-One step = one dec_step launch (the whole hot path).  Prints one JSON line.
-The line also carries a "bs64" object: the same decoder serving 64
-sequences at once (contexts drawn in [200, 420], a 128-step window; the
-Baseten Qwen3-ASR article, "KV cache quantization": many concurrent
-30-second windows), in tokens/s, through the batched tensor-core step; a
-"verify" object (block verification, "Can CTC make Qwen3-ASR faster?", 11
-Phase A); an "int8" object (the batch-1 workload with weight-only int8
-projections and lm_head, faster-qwen-asr GB10 record, "cuda_graph_int8");
-and an "attention" object (isolated decode attention over a length x batch
-grid).  `--impl reference` times the CPU oracle on a bounded sample instead.
+One step = one dec_step launch (the whole hot path); the timed steps rotate
+over three live handles (the step time depends slightly on where a handle's
+workspace lands).  Prints one JSON line.  The line also carries, after the
+headline keys: an "attention" object (isolated decode attention over a
+length x batch grid); a "verify" object (block verification, "Can CTC make
+Qwen3-ASR faster?", 11 Phase A); an "int8" object (the batch-1 workload with
+weight-only int8 projections and lm_head, faster-qwen-asr GB10 record,
+"cuda_graph_int8"); a "bs64" object (the same decoder serving 64 sequences
+at once, contexts drawn in [200, 420], a 128-step window; the Baseten
+Qwen3-ASR article, "KV cache quantization"), in tokens/s, through the
+batched tensor-core step; a "cfg5" object (the 1.7B-shaped decoder at batch
+1 and 64, bf16 and E4M3 caches); and a "generate" object (dec_generate: the
+130-token window in one launch).  `--impl reference` times the CPU oracle on
+a bounded sample instead.
 """
 from __future__ import annotations
 
@@ -164,6 +168,8 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sel)}
 
 
+HANDLES = 3       # live handles the batch-1 timed steps rotate over
+
 BS64 = 64
 BS64_LO, BS64_HI, BS64_WINDOW = 200, 420, 128
 BS64_STEPS = 64
@@ -266,7 +272,6 @@ def run_verify(s, wd, dev, seed):
 
 
 INT8_STEPS = 260
-INT8_HANDLES = 3
 
 
 def run_int8(s, wd, kv_host, tok0, dev, seed):
@@ -274,41 +279,44 @@ def run_int8(s, wd, kv_host, tok0, dev, seed):
     text decoder + lm_head): the same batch-1 workload (context 795, the
     130-step window, self-feeding) with every projection and lm_head
     quantised per row by dec_quantize_int8.  Device time per step over
-    INT8_STEPS steps after 5 warm-ups, on INT8_HANDLES live handles (the
-    step time depends by a few per cent on where a handle's workspace lands
-    in memory): the median handle is the value, all are listed.  Bytes: int8
-    weights + row scales, the KV rows and the embedding row."""
+    INT8_STEPS steps after 5 warm-ups, the steps rotating over HANDLES live
+    handles exactly as the bf16 line does.  Bytes: int8 weights + row scales,
+    the KV rows and the embedding row."""
     import torch
     from decoder_greedy_decode_b200 import capi, roofline
     from decoder_greedy_decode_b200.decoder import Decoder, quantize_int8
     w8 = quantize_int8(wd)
-    decs = [Decoder(s, w8, max_batch=1) for _ in range(INT8_HANDLES)]
+    decs = [Decoder(s, w8, max_batch=1) for _ in range(HANDLES)]
     kv = decs[0].kv_cache(1, 928)
     stream = torch.cuda.current_stream(dev)
     pos = torch.tensor([N0 + (i % WINDOW) for i in range(INT8_STEPS)], dtype=torch.int32,
                        device=dev)
-    per_handle = []
+    kv.values.copy_(kv_host.to(dev))
+    tok = torch.tensor([tok0], dtype=torch.int32, device=dev)
+
+    def launch(i):
+        capi.dec_step(decs[i % HANDLES].h, 1, tok, pos.data_ptr() + 4 * i, kv.kv, tok, None,
+                      stream)
+
+    for i in range(5):
+        launch(i)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(INT8_STEPS + 1)]
+    torch.cuda.synchronize(dev)
+    evs[0].record(stream)
+    for i in range(INT8_STEPS):
+        launch(i)
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
     for dec in decs:
-        kv.values.copy_(kv_host.to(dev))
-        tok = torch.tensor([tok0], dtype=torch.int32, device=dev)
-        for i in range(5):
-            capi.dec_step(dec.h, 1, tok, pos.data_ptr() + 4 * i, kv.kv, tok, None, stream)
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(INT8_STEPS + 1)]
-        torch.cuda.synchronize(dev)
-        evs[0].record(stream)
-        for i in range(INT8_STEPS):
-            capi.dec_step(dec.h, 1, tok, pos.data_ptr() + 4 * i, kv.kv, tok, None, stream)
-            evs[i + 1].record(stream)
-        torch.cuda.synchronize(dev)
         st = dec.check()
         if st != 0:
             raise RuntimeError(f"int8 device status {st}")
-        per_handle.append(statistics.fmean(evs[i].elapsed_time(evs[i + 1])
-                                           for i in range(INT8_STEPS)) * 1e3)
+    per = [evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(INT8_STEPS)]
+    per_handle = [statistics.fmean(per[h::HANDLES]) for h in range(HANDLES)]
     for dec in decs:
         dec.close()
     del w8
-    us = statistics.median(per_handle)
+    us = statistics.fmean(per)
     nbytes = statistics.fmean(roofline.step_bytes(s, [N0 + (i % WINDOW)], weights="int8")
                               for i in range(WINDOW))
     peak, kind = peaks()
@@ -580,7 +588,11 @@ def run_ours(args):
     kv_host, _ = synth.kv_prefill(s, B, 928, [N0], seed=args.seed + 1)
     tok0 = int(synth.tokens(s.vocab, 1, seed=args.seed + 2)[0])
     wd = to_device(w, dev)
-    dec = Decoder(s, wd, max_batch=B)
+    # The step time depends by a few per cent on where a handle's workspace
+    # lands in memory; the timed steps rotate over HANDLES live handles (step
+    # i on handle i mod HANDLES) so that the value averages the placements.
+    decs = [Decoder(s, wd, max_batch=B) for _ in range(HANDLES)]
+    dec = decs[0]
     kv = dec.kv_cache(B, 928)
     kv.values.copy_(kv_host.to(dev))
     stream = torch.cuda.current_stream(dev)
@@ -593,14 +605,16 @@ def run_ours(args):
 
     def launch(i):
         # self-feeding: out_ids aliases token_ids; positions from the host's schedule
-        capi.dec_step(dec.h, B, tok, pos_all.data_ptr() + esz * i, kv.kv, tok, None, stream)
+        capi.dec_step(decs[i % HANDLES].h, B, tok, pos_all.data_ptr() + esz * i, kv.kv, tok,
+                      None, stream)
 
     for i in range(W):
         launch(i)
     torch.cuda.synchronize(dev)
-    st = dec.check()
-    if st != 0:
-        raise RuntimeError(f"device status {st}: {capi.error_string(st)}")
+    for d in decs:
+        st = d.check()
+        if st != 0:
+            raise RuntimeError(f"device status {st}: {capi.error_string(st)}")
 
     sampler = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
     time.sleep(0.3)
@@ -619,7 +633,13 @@ def run_ours(args):
         dist.barrier()
     per = [evs[i].elapsed_time(evs[i + 1]) for i in range(K)]     # ms, one launch each
     total_ms = evs[0].elapsed_time(evs[K])
+    per_handle = [statistics.fmean(per[h::HANDLES]) * 1e3 for h in range(min(HANDLES, K))]
     clocks = ClockSampler.summarize(sampler.stop(), t_wall0, t_wall1) if sampler else None
+    for d in decs[1:]:
+        st = d.check()
+        if st != 0:
+            raise RuntimeError(f"device status {st}: {capi.error_string(st)}")
+        d.close()
     st = dec.check()
     if st != 0:
         raise RuntimeError(f"device status {st}: {capi.error_string(st)}")
@@ -685,7 +705,8 @@ def run_ours(args):
                          "algorithmic_bytes_per_launch": bytes_mean,
                          "mean_launch_us": mean_launch_ms * 1e3,
                          "median_launch_us": statistics.median(per) * 1e3,
-                         "best_launch_us": min(per) * 1e3},
+                         "best_launch_us": min(per) * 1e3,
+                         "mean_launch_us_per_handle": [round(v, 1) for v in per_handle]},
             "e2e": {"value": e2e_ms * 1e3 / (KE * B * ws), "unit": UNIT,
                     "h2d_bytes_per_step": 8 * B, "d2h_bytes_per_step": 4 * B,
                     "steps": KE, "api": "dec_step_host"},
