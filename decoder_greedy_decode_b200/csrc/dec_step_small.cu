@@ -702,100 +702,93 @@ struct Cta {
     for (int st = 0; !dead && !stop; ++st) {
     for (int l = 0; l < a.L && !dead; ++l) {
       const LayerPtrs& lw = slw[l];
-      // ---- QKV rows [q0, q1) of [Wq; Wk; Wv]
-      for (int r = q0; r < q1 && !dead; r += rpt_h) {
-        const int nr = min(rpt_h, q1 - r);
-        uint8_t* dst = acquire(static_cast<uint32_t>(nr) * H * e);
-        if (!dst) break;
-        if (r == q0) DEC_PSTAMP(kStampsPerLayer * l + StPQ);
-        int rr = r, left = nr;
-        while (left > 0) {
-          const uint16_t* base;
-          int lo, cnt;
-          if (rr < HqD) {
-            base = lw.w[1]; lo = rr; cnt = min(left, HqD - rr);
-          } else if (rr < HqD + HkvD) {
-            base = lw.w[2]; lo = rr - HqD; cnt = min(left, HqD + HkvD - rr);
-          } else {
-            base = lw.w[3]; lo = rr - HqD - HkvD; cnt = left;
+      // The layer's tiles in consumption order: the four projection stages
+      // (one copy of this code serves them all), the attention tiles before
+      // o_proj.  s = 0: QKV rows [q0, q1) of [Wq; Wk; Wv]; 1: o_proj rows
+      // [h0, h1), K = Hq*D; 2: gate/up rows [f0, f1), a tile is nr gate rows
+      // then nr up rows; 3: down rows [h0, h1), K = F.
+#pragma unroll 1
+      for (int s = 0; s < 4 && !dead; ++s) {
+        if (s == 1) {
+          // A later step's attention rows depend on the ids of the step
+          // before (a sequence that emitted the end token keeps its
+          // position): wait for them once the first layer's QKV rows are on
+          // their way.
+          if (l == 0 && st > 0) {
+            if (!next_step(*pplan, tok_flag(st - 1))) dead = true;
+            if (dead || pplan->bad || pplan->all_done) {
+              stop = true;
+              break;
+            }
           }
-          rows_to(dst, base, lo, cnt, H);
-          dst += static_cast<size_t>(cnt) * rstride(H);
-          rr += cnt;
-          left -= cnt;
+          // attention: cached rows [j0, min(j1, p_b)) of every item of this CTA
+          for (int it = cta; it < pl->n_items && !dead; it += nc) {
+            int b, g, ci;
+            item(it, b, g, ci);
+            const int j0 = ci * pl->crow;
+            const int jc = min(j0 + pl->crow, pl->pos[b]);  // (verify: b = 0, the prefix end)
+            if (a.vseq >= 0) b = a.vseq;                     // the cache sequence
+            for (int j = j0; j < jc && !dead; j += art) {
+              const int nr = min(art, jc - j);
+              if constexpr (!FP8) {
+                const uint32_t rb = static_cast<uint32_t>(nr) * D * 2;
+                uint8_t* dst = acquire(2 * rb);
+                if (!dst) break;
+                if (j == j0) DEC_PSTAMP(kStampsPerLayer * l + StPA);
+                const uint16_t* kvb = reinterpret_cast<const uint16_t*>(a.kv);
+                bulk_g2s(dst, kvb + kv_row(l, 0, b, g, j) * D, rb, fb, pol);
+                bulk_g2s(dst + rb, kvb + kv_row(l, 1, b, g, j) * D, rb, fb, pol);
+              } else {
+                const uint32_t rb = static_cast<uint32_t>(nr) * D;
+                const uint32_t sb = static_cast<uint32_t>((nr + 3) & ~3) * 4;
+                uint8_t* dst = acquire(2 * rb + 2 * sb);
+                if (!dst) break;
+                bulk_g2s(dst, a.kv + kv_row(l, 0, b, g, j) * D, rb, fb, pol);
+                bulk_g2s(dst + rb, a.kv + kv_row(l, 1, b, g, j) * D, rb, fb, pol);
+                bulk_g2s(dst + 2 * rb, a.kv_scales + kv_row(l, 0, b, g, j), sb, fb, pol);
+                bulk_g2s(dst + 2 * rb + sb, a.kv_scales + kv_row(l, 1, b, g, j), sb, fb,
+                         pol);
+              }
+              advance();
+            }
+          }
         }
-        advance();
-      }
-      // A later step's attention rows depend on the ids of the step before
-      // (a sequence that emitted the end token keeps its position): wait for
-      // them once the first layer's QKV rows are on their way.
-      if (l == 0 && st > 0) {
-        if (!next_step(*pplan, tok_flag(st - 1))) dead = true;
-        if (dead || pplan->bad || pplan->all_done) {
-          stop = true;
-          break;
-        }
-      }
-      // ---- attention: cached rows [j0, min(j1, p_b)) of every item of this CTA
-      for (int it = cta; it < pl->n_items && !dead; it += nc) {
-        int b, g, ci;
-        item(it, b, g, ci);
-        const int j0 = ci * pl->crow;
-        const int jc = min(j0 + pl->crow, pl->pos[b]);  // (verify: b = 0, the prefix end)
-        if (a.vseq >= 0) b = a.vseq;                     // the cache sequence
-        for (int j = j0; j < jc && !dead; j += art) {
-          const int nr = min(art, jc - j);
-          if constexpr (!FP8) {
-            const uint32_t rb = static_cast<uint32_t>(nr) * D * 2;
-            uint8_t* dst = acquire(2 * rb);
-            if (!dst) break;
-            if (j == j0) DEC_PSTAMP(kStampsPerLayer * l + StPA);
-            const uint16_t* kvb = reinterpret_cast<const uint16_t*>(a.kv);
-            bulk_g2s(dst, kvb + kv_row(l, 0, b, g, j) * D, rb, fb, pol);
-            bulk_g2s(dst + rb, kvb + kv_row(l, 1, b, g, j) * D, rb, fb, pol);
+        const int lo = s == 0 ? q0 : s == 2 ? f0 : h0;
+        const int hi = s == 0 ? q1 : s == 2 ? f1 : h1;
+        const int rpt = s == 0 ? rpt_h : s == 1 ? rpt_o : s == 2 ? rpt_u : rpt_d;
+        const int K = s == 1 ? HqD : s == 3 ? a.F : H;
+        const uint32_t mats = s == 2 ? 2u : 1u;
+        for (int r = lo; r < hi && !dead; r += rpt) {
+          const int nr = min(rpt, hi - r);
+          uint8_t* dst = acquire(mats * static_cast<uint32_t>(nr) * K * e);
+          if (!dst) break;
+          if (r == lo)
+            DEC_PSTAMP(kStampsPerLayer * l + (s == 0 ? StPQ : s == 1 ? StPO : s == 2 ? StPU : StPD));
+          if (s == 0) {
+            int rr = r, left = nr;
+            while (left > 0) {
+              const uint16_t* base;
+              int r0, cnt;
+              if (rr < HqD) {
+                base = lw.w[1]; r0 = rr; cnt = min(left, HqD - rr);
+              } else if (rr < HqD + HkvD) {
+                base = lw.w[2]; r0 = rr - HqD; cnt = min(left, HqD + HkvD - rr);
+              } else {
+                base = lw.w[3]; r0 = rr - HqD - HkvD; cnt = left;
+              }
+              rows_to(dst, base, r0, cnt, H);
+              dst += static_cast<size_t>(cnt) * rstride(H);
+              rr += cnt;
+              left -= cnt;
+            }
           } else {
-            const uint32_t rb = static_cast<uint32_t>(nr) * D;
-            const uint32_t sb = static_cast<uint32_t>((nr + 3) & ~3) * 4;
-            uint8_t* dst = acquire(2 * rb + 2 * sb);
-            if (!dst) break;
-            bulk_g2s(dst, a.kv + kv_row(l, 0, b, g, j) * D, rb, fb, pol);
-            bulk_g2s(dst + rb, a.kv + kv_row(l, 1, b, g, j) * D, rb, fb, pol);
-            bulk_g2s(dst + 2 * rb, a.kv_scales + kv_row(l, 0, b, g, j), sb, fb, pol);
-            bulk_g2s(dst + 2 * rb + sb, a.kv_scales + kv_row(l, 1, b, g, j), sb, fb,
-                     pol);
+            rows_to(dst, s == 1 ? lw.w[6] : s == 2 ? lw.w[8] : lw.w[10], r, nr, K);
+            if (s == 2) rows_to(dst + static_cast<size_t>(nr) * rstride(H), lw.w[9], r, nr, H);
           }
           advance();
         }
       }
-      // ---- o_proj rows [h0, h1), K = Hq*D
-      for (int r = h0; r < h1 && !dead; r += rpt_o) {
-        const int nr = min(rpt_o, h1 - r);
-        uint8_t* dst = acquire(static_cast<uint32_t>(nr) * HqD * e);
-        if (!dst) break;
-        if (r == h0) DEC_PSTAMP(kStampsPerLayer * l + StPO);
-        rows_to(dst, lw.w[6], r, nr, HqD);
-        advance();
-      }
-      // ---- gate / up rows [f0, f1): a tile is nr gate rows then nr up rows
-      for (int r = f0; r < f1 && !dead; r += rpt_u) {
-        const int nr = min(rpt_u, f1 - r);
-        const uint32_t rb = static_cast<uint32_t>(nr) * H * e;
-        uint8_t* dst = acquire(2 * rb);
-        if (!dst) break;
-        if (r == f0) DEC_PSTAMP(kStampsPerLayer * l + StPU);
-        rows_to(dst, lw.w[8], r, nr, H);
-        rows_to(dst + static_cast<size_t>(nr) * rstride(H), lw.w[9], r, nr, H);
-        advance();
-      }
-      // ---- down rows [h0, h1), K = F
-      for (int r = h0; r < h1 && !dead; r += rpt_d) {
-        const int nr = min(rpt_d, h1 - r);
-        uint8_t* dst = acquire(static_cast<uint32_t>(nr) * a.F * e);
-        if (!dst) break;
-        if (r == h0) DEC_PSTAMP(kStampsPerLayer * l + StPD);
-        rows_to(dst, lw.w[10], r, nr, a.F);
-        advance();
-      }
+      if (stop) break;
     }
     if (stop) break;
     // ---- lm_head rows [v0, v1)
@@ -1791,17 +1784,23 @@ struct Cta {
       const LayerPtrs& lw = slw[l];
       const uint32_t f = flag(l);
       // QKV (the layer-0 input is the embedding row)
-      kstage(SQ, l, l == 0 ? nullptr : a.x_out, flag(l - 1), lw.w[0], H, q1 - q0, rpt_h, false,
-             true);
-      DEC_STAMP(kStampsPerLayer * l + StQkv);
-      attention(l);
-      DEC_STAMP(kStampsPerLayer * l + StAtt);
-      kstage(SO, l, a.x_o, f, nullptr, HqD, h1 - h0, rpt_o, false, false);
-      DEC_STAMP(kStampsPerLayer * l + StO);
-      kstage(SU, l, a.x_mid, f, lw.w[7], H, f1 - f0, rpt_u, true, true);
-      DEC_STAMP(kStampsPerLayer * l + StU);
-      kstage(SD, l, a.x_u, f, nullptr, F, h1 - h0, rpt_d, false, false);
-      DEC_STAMP(kStampsPerLayer * l + StD);
+      // the four projection stages share one copy of the stage code
+#pragma unroll 1
+      for (int st = 0; st < 4; ++st) {
+        if (st == 1) {
+          attention(l);
+          DEC_STAMP(kStampsPerLayer * l + StAtt);
+        }
+        const int sc = st == 0 ? SQ : st == 1 ? SO : st == 2 ? SU : SD;
+        const uint64_t* src = st == 0 ? (l == 0 ? nullptr : a.x_out)
+                              : st == 1 ? a.x_o : st == 2 ? a.x_mid : a.x_u;
+        const uint16_t* gn = st == 0 ? lw.w[0] : st == 2 ? lw.w[7] : nullptr;
+        const int K = st == 1 ? HqD : st == 3 ? F : H;
+        const int nrows = st == 0 ? q1 - q0 : st == 2 ? f1 - f0 : h1 - h0;
+        const int rpt = st == 0 ? rpt_h : st == 1 ? rpt_o : st == 2 ? rpt_u : rpt_d;
+        kstage(sc, l, src, st == 0 ? flag(l - 1) : f, gn, K, nrows, rpt, st == 2, (st & 1) == 0);
+        DEC_STAMP(kStampsPerLayer * l + (st == 0 ? StQkv : st == 1 ? StO : st == 2 ? StU : StD));
+      }
     }
     // final norm + lm_head: the whole input in act, the norm factor applied
     // to every logit
