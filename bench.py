@@ -168,6 +168,63 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sel)}
 
 
+class NvmlSampler:
+    """SM clock and throttle reasons read through NVML every millisecond on a
+    background thread (the batch-1 timed region lasts ~16 ms, too short for
+    nvidia-smi's sampling period); same summary as ClockSampler."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
+
+    def __init__(self, dev):
+        import threading
+        import pynvml
+        import torch
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(dev)
+        self.h = pynvml.nvmlDeviceGetHandleByPciBusId(
+            f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0")
+        self.get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.rows, self.stop_flag = [], threading.Event()
+        self.t = threading.Thread(target=self._loop, daemon=True)
+        self.t.start()
+
+    def _loop(self):
+        nv = self.nv
+        while not self.stop_flag.is_set():
+            try:
+                self.rows.append((time.time(), float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)),
+                                  int(self.get_reasons(self.h))))
+            except Exception:
+                pass
+            time.sleep(0.001)
+
+    def stop(self):
+        self.stop_flag.set()
+        self.t.join(timeout=5)
+        return self.rows
+
+    def summarize(self, rows, t0: float, t1: float):
+        sel = [r for r in rows if t0 <= r[0] <= t1]
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "nvml, 1 ms"}
+        reasons = sorted({n for _, _, m in sel for n, bit in self.REASONS if m & bit})
+        return {"sm_mhz": statistics.median(r[1] for r in sel), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sel), "source": "nvml, 1 ms"}
+
+
+def clock_sampler(dev):
+    """NVML sampler when the bindings load, else nvidia-smi's."""
+    try:
+        return NvmlSampler(dev)
+    except Exception:
+        return ClockSampler(dev.index if dev.index is not None else 0)
+
+
 HANDLES = 3       # live handles the batch-1 timed steps rotate over
 
 BS64 = 64
@@ -223,7 +280,8 @@ def run_bs64(s, wd, dev, ws, seed):
             "launches_per_step": 1 + 5 * s.n_layers + 2}
 
 
-VERIFY_BLOCKS = (1, 2, 4, 8, 16, 32)
+VERIFY_BLOCKS = (1, 2, 3, 4, 8, 16, 32)
+VERIFY_FULL = 130  # the whole 130-token output window, in blocks of at most 64
 
 
 def run_verify(s, wd, dev, seed):
@@ -232,13 +290,15 @@ def run_verify(s, wd, dev, seed):
     795, a block of k tokens per dec_verify call; device time per call (median
     of 20 after 3 warm-ups) and per committed token if the whole block is
     accepted.  Bytes: the weights, the sequence's cache rows once, the block's
-    embedding rows."""
+    embedding rows.  "full_output": the whole 130-token window verified by
+    consecutive calls of at most 64 tokens (the batched step's limit), each
+    block attending to the ones before it."""
     import torch
     from decoder_greedy_decode_b200 import roofline
     from decoder_greedy_decode_b200.decoder import Decoder
     kmax = max(VERIFY_BLOCKS)
-    dec = Decoder(s, wd, max_batch=kmax)
-    max_ctx = (N0 + kmax + 15) // 16 * 16
+    dec = Decoder(s, wd, max_batch=64)
+    max_ctx = (N0 + max(kmax, VERIFY_FULL) + 15) // 16 * 16
     kv = dec.kv_cache(1, max_ctx)
     kv.values.normal_(generator=torch.Generator(device=dev).manual_seed(seed + 30))
     stream = torch.cuda.current_stream(dev)
@@ -262,13 +322,36 @@ def run_verify(s, wd, dev, seed):
         nbytes = (roofline.weight_bytes(s) + (N0 + k) * roofline.kv_bytes_per_token(s)
                   + k * s.hidden * 2)
         cells.append((k, round(us, 1), round(us / k, 1), round(nbytes / (us * 1e-6) / 1e9, 1)))
+    # the whole output window: blocks of <= 64 tokens, one after the other
+    toks = torch.randint(0, s.vocab, (VERIFY_FULL,), dtype=torch.int32, device=dev)
+    pos = torch.arange(N0, N0 + VERIFY_FULL, dtype=torch.int32, device=dev)
+    out = torch.empty(VERIFY_FULL, dtype=torch.int32, device=dev)
+    blocks = [(i, min(64, VERIFY_FULL - i)) for i in range(0, VERIFY_FULL, 64)]
+
+    def full():
+        for i, n in blocks:
+            dec.verify(kv, toks[i:i + n], pos[i:i + n], 0, out[i:i + n], None, stream)
+    for _ in range(3):
+        full()
+    evs = []
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        full()
+        e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    full_us = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs) * 1e3
     st = dec.check()
     dec.close()
     if st != 0:
         raise RuntimeError(f"verify device status {st}")
     return {"workload": "0.6b, one sequence, context 795, blocks of k tokens",
             "k": [c[0] for c in cells], "us_per_call": [c[1] for c in cells],
-            "us_per_token_full_accept": [c[2] for c in cells], "GB/s": [c[3] for c in cells]}
+            "us_per_token_full_accept": [c[2] for c in cells], "GB/s": [c[3] for c in cells],
+            "full_output": {"tokens": VERIFY_FULL, "calls": len(blocks),
+                            "us": round(full_us, 1),
+                            "us_per_token": round(full_us / VERIFY_FULL, 1)}}
 
 
 INT8_STEPS = 260
@@ -616,7 +699,7 @@ def run_ours(args):
         if st != 0:
             raise RuntimeError(f"device status {st}: {capi.error_string(st)}")
 
-    sampler = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
+    sampler = clock_sampler(dev) if rank == 0 else None
     time.sleep(0.3)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
     if ws > 1:
@@ -634,7 +717,7 @@ def run_ours(args):
     per = [evs[i].elapsed_time(evs[i + 1]) for i in range(K)]     # ms, one launch each
     total_ms = evs[0].elapsed_time(evs[K])
     per_handle = [statistics.fmean(per[h::HANDLES]) * 1e3 for h in range(min(HANDLES, K))]
-    clocks = ClockSampler.summarize(sampler.stop(), t_wall0, t_wall1) if sampler else None
+    clocks = sampler.summarize(sampler.stop(), t_wall0, t_wall1) if sampler else None
     for d in decs[1:]:
         st = d.check()
         if st != 0:

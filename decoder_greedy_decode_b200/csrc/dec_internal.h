@@ -17,6 +17,7 @@ constexpr int kMinLargeSlots = 3;
 constexpr int kMaxBatchSmall = 4;                   // batch handled by the GEMV step kernel
 constexpr int kMaxRep = 4;                          // query heads per KV head (step kernel)
 constexpr int kMaxVerifyHeads = 8;                  // query heads per KV head of a block the step kernel verifies
+constexpr int kVerifyPersistent = 1;  // verification blocks the persistent kernel takes when a batched step exists
 constexpr int kLayerPtrs = 11;
 constexpr int kMaxBatch = 64;                       // batched step: the N of the tensor-core tiles
 constexpr int kProfStampsPerLayer = 32;             // profiling builds: timestamps per layer and CTA

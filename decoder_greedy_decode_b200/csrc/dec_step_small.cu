@@ -80,8 +80,11 @@ enum {
   // SM cycles warp 0 spent waiting for ring tiles in each stage
   StWQ, StWA, StWO, StWU, StWD,
   // SM cycles of warp 0's GEMV of each stage (waits included)
-  StCQ, StCO, StCU, StCD
+  StCQ, StCO, StCU, StCD,
+  // attention: partial state published (other chunks) / chunks gathered (chunk 0)
+  StAttPub, StAttCmb
 };
+static_assert(StAttCmb < kStampsPerLayer, "profiling stamps of a layer");
 enum { StLmStart = 0, StLmGath, StLmDone, StEnd, StBegin };
 #ifdef DEC_PROFILE
 #define DEC_STAMP(i)                                                                   \
@@ -1717,6 +1720,7 @@ struct Cta {
           }
         }
       }
+      DEC_STAMP(kStampsPerLayer * l + StAttPub);
       if (combiner) {  // uniform over the CTA: ci is the item's
         const int nc1 = pl->nchunk[ver ? 0 : b] - 1;
         const int win = kStageWords / (hi * (D + 2));
@@ -1748,6 +1752,7 @@ struct Cta {
           }
           csync();  // stg is refilled by the next window
         }
+        DEC_STAMP(kStampsPerLayer * l + StAttCmb);
         if (!ab) {
 #pragma unroll
           for (int i = 0; i < kSlots; ++i) {

@@ -169,7 +169,7 @@ typedef struct dec_weights_int8 {
 /* dec_init for a weight-only int8 model.  Same ownership and errors as
  * dec_init; max_batch must be 1..4 (DEC_ERR_BATCH otherwise): int8 weights
  * run on the single persistent kernel (dec_step, dec_step_host,
- * dec_generate, and dec_verify for blocks of up to 4). */
+ * dec_generate, and dec_verify for the blocks it takes). */
 int dec_init_int8(const dec_shape *shape, const dec_weights_int8 *weights, dec_handle **out);
 
 /* Release the handle and its workspace (synchronises the device first). */
@@ -262,10 +262,13 @@ int dec_generate(dec_handle *h, int batch, int n_steps, const int32_t *token_ids
 
 /* Verify a block of k consecutive tokens of ONE cached sequence in a single
  * step ("Can CTC make Qwen3-ASR faster?", §11 Phase A steps 2-3: one target
- * forward over the whole draft block; §03: greedy verification).  Blocks of
- * k <= 4 (with k * n_q_heads / n_kv_heads <= 8) run as one launch of the
- * persistent kernel, which reads the committed prefix of the sequence once
- * for the whole block; larger blocks run the batched step.
+ * forward over the whole draft block; §03: greedy verification).  A block
+ * of one token runs as one launch of the persistent kernel; so do blocks of
+ * 2 to 4 (with k * n_q_heads / n_kv_heads <= 8) on a handle without a
+ * batched step (max_batch <= 4, and every int8 handle), the committed prefix
+ * of the sequence read once for the whole block.  Other blocks run the
+ * batched step, as fast or faster than the persistent kernel from 2 tokens
+ * on.
  *   token_ids  int32 [k] (device)  t_0 = the last committed token, then the
  *                                  draft tokens t_1 .. t_{k-1}
  *   positions  int32 [k] (device)  p0 + i: row i is written to cache row

@@ -53,16 +53,18 @@ def _verify(dec, kv, toks, p0, seq):
 
 
 @pytest.mark.parametrize("kind", ["bf16", "fp8"])
-@pytest.mark.parametrize("k", [1, 2, 3, 4, 9])
-def test_verify_block_equals_single_steps(kind, k):
+@pytest.mark.parametrize("k,max_batch", [(1, 16), (2, 16), (3, 16), (4, 16), (9, 16),
+                                         (2, 4), (3, 4), (4, 4)])
+def test_verify_block_equals_single_steps(kind, k, max_batch):
     """A block of k tokens of sequence 1 (of 3 in the cache) equals k
     teacher-forced single steps of the oracle: logits, ids, appended rows;
-    the other sequences' rows are untouched.  Blocks of up to 4 run on the
-    persistent kernel (the prefix read once for the whole block), larger
-    ones on the batched step."""
+    the other sequences' rows are untouched.  One-token blocks run on the
+    persistent kernel, and so do blocks of 2 to 4 on a handle without a
+    batched step (max_batch 4; the prefix read once for the whole block);
+    the others run on the batched step."""
     s = synth.TINY
     n0, seq = 40, 1
-    m, dec, kv, kv_host, sc_host = _setup(s, 80, 3, 64, [30, n0, 50], kind)
+    m, dec, kv, kv_host, sc_host = _setup(s, 80, 3, 64, [30, n0, 50], kind, max_batch=max_batch)
     cache = oracle_cache(kv_host, sc_host, seq)
     toks = [int(t) for t in synth.tokens(s.vocab, k, seed=81)]
     before = kv.buf.clone()
@@ -190,14 +192,15 @@ def big06():
     return s, w, to_device(w)
 
 
-@pytest.mark.parametrize("k", [4, 16])
-def test_0p6b_verify_block(big06, k):
-    """0.6B shape, context 795, blocks of 4 (persistent kernel) and 16
-    (batched step): sampled rows vs the oracle."""
+@pytest.mark.parametrize("k,max_batch", [(4, 4), (4, 64), (16, 64)])
+def test_0p6b_verify_block(big06, k, max_batch):
+    """0.6B shape, context 795, blocks of 4 (persistent kernel on a handle of
+    max_batch 4, batched step otherwise) and 16 (batched step): sampled rows
+    vs the oracle."""
     s, w, wd = big06
     n0 = 795
     kv_host, _ = synth.kv_prefill(s, 1, 816, [n0], seed=94)
-    dec = Decoder(s, wd, max_batch=64)
+    dec = Decoder(s, wd, max_batch=max_batch)
     kv = dec.kv_cache(1, 816)
     kv.values.copy_(kv_host.cuda())
     m = oracle.Model(oracle_shape(s), oracle_weights(w))
