@@ -16,7 +16,7 @@ headline keys: an "attention" object (isolated decode attention over a
 length x batch grid); a "verify" object (block verification, "Can CTC make
 Qwen3-ASR faster?", 11 Phase A); an "int8" object (the batch-1 workload with
 weight-only int8 projections and lm_head, faster-qwen-asr GB10 record,
-"cuda_graph_int8"); a "bs64" object (the same decoder serving 64 sequences
+"cuda_graph_int8", and the batch-64 workload with them); a "bs64" object (the same decoder serving 64 sequences
 at once, contexts drawn in [200, 420], a 128-step window; the Baseten
 Qwen3-ASR article, "KV cache quantization"), in tokens/s, through the
 batched tensor-core step; a "cfg5" object (the 1.7B-shaped decoder at batch
@@ -232,16 +232,18 @@ BS64_LO, BS64_HI, BS64_WINDOW = 200, 420, 128
 BS64_STEPS = 64
 
 
-def run_bs64(s, wd, dev, ws, seed):
+def run_bs64(s, wd, dev, ws, seed, w8=False):
     """Batch 64, ragged contexts U[200, 420], self-feeding over a 128-step
     window: device time of BS64_STEPS steps (max over ranks); tokens/s for
-    all ranks, and the step's algorithmic bytes over that time."""
+    all ranks, and the step's algorithmic bytes over that time.  w8: the
+    same with weight-only int8 projections and lm_head (dec_quantize_int8 of
+    the same weights)."""
     import torch
     import torch.distributed as dist
     from decoder_greedy_decode_b200 import roofline, synth
-    from decoder_greedy_decode_b200.decoder import Decoder
+    from decoder_greedy_decode_b200.decoder import Decoder, quantize_int8
     max_ctx = (BS64_HI + BS64_WINDOW + 15) // 16 * 16
-    dec = Decoder(s, wd, max_batch=BS64)
+    dec = Decoder(s, quantize_int8(wd) if w8 else wd, max_batch=BS64)
     kv = dec.kv_cache(BS64, max_ctx)
     g = torch.Generator(device=dev).manual_seed(seed + 10)
     kv.values.normal_(generator=g)
@@ -268,13 +270,16 @@ def run_bs64(s, wd, dev, ws, seed):
     if st != 0:
         raise RuntimeError(f"bs64 device status {st}")
     step_ms = ms / BS64_STEPS
-    nbytes = statistics.fmean(roofline.step_bytes(s, [n + (i % BS64_WINDOW) for n in lengths])
+    wk = "int8" if w8 else "bf16"
+    nbytes = statistics.fmean(roofline.step_bytes(s, [n + (i % BS64_WINDOW) for n in lengths],
+                                                  weights=wk)
                               for i in range(BS64_STEPS))
     peak, kind = peaks()
     achieved = nbytes / (step_ms * 1e-3) / 1e9
     return {"value": round(replica_throughput(BS64, step_ms, ws), 1), "unit": "tokens/s",
             "ms_per_step": round(step_ms, 4), "steps": BS64_STEPS,
-            "workload": "0.6b, batch 64, contexts U[200,420], bf16 KV",
+            "workload": "0.6b, batch 64, contexts U[200,420], bf16 KV, "
+                        + ("int8" if w8 else "bf16") + " weights",
             "roofline": {"achieved": round(achieved, 1), "peak": peak,
                          "frac": round(achieved / peak, 4)},
             "launches_per_step": 1 + 5 * s.n_layers + 2}
@@ -750,8 +755,13 @@ def run_ours(args):
 
     # ---- the other configurations (rank 0 prints their summaries)
     bs64 = run_bs64(s, wd, dev, ws, args.seed)
+    bs64_w8 = run_bs64(s, wd, dev, ws, args.seed, w8=True)
     verify = run_verify(s, wd, dev, args.seed) if rank == 0 else None
     int8 = run_int8(s, wd, kv_host, tok0, dev, args.seed) if rank == 0 else None
+    if int8 is not None:
+        int8["bs64"] = {"tokens_per_s": bs64_w8["value"], "ms_per_step": bs64_w8["ms_per_step"],
+                        "frac": bs64_w8["roofline"]["frac"],
+                        "workload": "0.6b, batch 64, contexts U[200,420], int8 weights"}
     generate = run_generate(s, wd, kv_host, tok0, dev) if rank == 0 else None
     kernel_config = dec.config()
     dec.close()

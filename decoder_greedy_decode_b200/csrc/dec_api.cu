@@ -109,7 +109,6 @@ extern "C" int dec_init_int8(const dec_shape* shape, const dec_weights_int8* w,
   *out = nullptr;
   int rc = check_shape(shape);
   if (rc) return rc;
-  if (shape->max_batch > kMaxBatchSmall) return DEC_ERR_BATCH;
   if (!w->embed || !w->lm_head || !w->lm_head_scale || !w->final_norm || !w->layers ||
       !w->scales)
     return DEC_ERR_NULL;
@@ -240,8 +239,9 @@ static int init_handle(const dec_shape* shape, const InitWeights& w, dec_handle*
   h->layers_dev = reinterpret_cast<LayerPtrs*>(h->ws + layers_off);
   if (e == cudaSuccess)
     e = cudaMemcpy(h->layers_dev, lp.data(), sizeof(LayerPtrs) * L, cudaMemcpyHostToDevice);
+  std::vector<LayerScales> ls;
   if (w.w8) {
-    std::vector<LayerScales> ls(L);
+    ls.resize(L);
     for (int l = 0; l < L; ++l)
       for (int j = 0; j < DEC_LW_COUNT; ++j)
         ls[l].s[j] = is_projection(j) ? w.scales[l * DEC_LW_COUNT + j] : nullptr;
@@ -259,7 +259,9 @@ static int init_handle(const dec_shape* shape, const InitWeights& w, dec_handle*
     const BtShape bs{L, H, Hq, Hkv, D, F, shape->vocab, shape->rms_eps};
     cudaError_t ce = cudaSuccess;
     rc = bt_plan_create(bs, h->embed, h->lm_head, h->final_norm, lp.data(),
-                        reinterpret_cast<const float*>(h->ws + wl.inv_freq), h->sms, &h->bt, &ce);
+                        reinterpret_cast<const float*>(h->ws + wl.inv_freq), h->sms, &h->bt, &ce,
+                        w.w8 ? static_cast<const float*>(w.lm_scale) : nullptr,
+                        w.w8 ? ls.data() : nullptr);
     if (rc) {
       cudaFree(h->ws);
       delete h;

@@ -143,9 +143,12 @@ struct BtShape {
 };
 struct BtPlan;  // tensor maps, launch configuration and scratch (dec_step_batched.cu)
 // Returns 0, or a DEC_ERR_* code (DEC_ERR_CUDA with *cerr set).
-int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_head,
+// int8 handles pass the lm_head row scales and every layer's projection row
+// scales (host array of device pointers); bf16 handles pass null for both.
+int bt_plan_create(const BtShape& s, const uint16_t* embed, const void* lm_head,
                    const uint16_t* final_norm, const LayerPtrs* layers_host,
-                   const float* inv_freq_dev, int sms, BtPlan** out, cudaError_t* cerr);
+                   const float* inv_freq_dev, int sms, BtPlan** out, cudaError_t* cerr,
+                   const float* lm_scale, const LayerScales* scales_host);
 void bt_plan_destroy(BtPlan* p);
 struct BtIO {
   int B;

@@ -171,6 +171,23 @@ __device__ __forceinline__ uint16_t f_to_bf16(float f) {
   asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(f));
   return r;
 }
+// prmt.b32 (generic mode) of x with zero: result byte n is byte (s_n & 7),
+// or that byte's sign bit replicated when s_n & 8 (s_n = nibble n of s)
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t x, uint32_t s) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(x), "r"(s));
+  return r;
+}
+// two fp32 -> two bf16 in one word (lo = a in the low half), RNE
+__device__ __forceinline__ uint32_t f2_to_bf16x2(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+// two bf16 values in one 32-bit word (lo in the low half)
+__device__ __forceinline__ uint32_t pack_bf16x2(uint16_t lo, uint16_t hi) {
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
 // two fp32 -> two E4M3 codes (lo = a, hi = b), RNE, saturating to +-448
 __device__ __forceinline__ uint16_t f2_to_e4m3x2(float a, float b) {
   uint16_t r;

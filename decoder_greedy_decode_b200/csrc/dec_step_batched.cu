@@ -69,6 +69,16 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, kTileN);
 constexpr int kTStride = kTileM + 4;              // accumulator tile in smem: T[b][row]
 constexpr int kWOffset = 40 * 1024;               // reduced rows of this CTA's sequences
 constexpr size_t kGemmSmem = 1024 + kGemmStages * kStageBytes + 256;
+// int8 weights: the codes of a weight tile land (TMA, no swizzle: row r at
+// byte 64 r) in the upper half of the stage's bf16 weight tile; the CTA's
+// epilogue warps, idle during the main loop, read them all into registers,
+// then widen them into the whole bf16 tile.  The shared memory stays that of
+// the bf16 GEMM, so two GEMM CTAs still fit an SM and a GEMM's prologue
+// overlaps its predecessor (programmatic dependent launch).
+constexpr int kA8Bytes = kTileM * kChunkK;        // 8 KB
+constexpr int kA8Offset = kABytes - kA8Bytes;     // codes inside the weight tile
+constexpr int kConvThreads = 128;                 // warps 4..7
+constexpr int kConvBarrier = 1;                   // their named barrier
 constexpr int kMaxSplits = 16;                    // cluster size (16: non-portable, allowed per kernel)
 constexpr int kMaxAttnChunks = 32;
 constexpr int kAttWarps = 4;
@@ -169,6 +179,7 @@ struct GemmArgs {
   int* status;
   unsigned long long timeout_ns;
   unsigned long long* prof;  // profiling builds: [4 modes][kProfCtas][16] timestamps, else null
+  const float* wsc[3];       // int8 weights: fp32 row scales of each matrix (kSwiGLU: gate, up)
 };
 
 // Phase timestamps of one GEMM CTA (profiling builds only).
@@ -185,7 +196,7 @@ struct GemmArgs {
   } while (0)
 #endif
 
-template <int MODE>
+template <int MODE, bool W8>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap w0,
                                                             const __grid_constant__ CUtensorMap w1,
                                                             const __grid_constant__ CUtensorMap w2,
@@ -200,7 +211,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + kGemmStages * kStageBytes);
   uint64_t* empty = full + kGemmStages;
   uint64_t* done = empty + kGemmStages;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* afull = done + 1;         // W8: the int8 codes of stage s landed
+  uint64_t* conv = afull + kGemmStages;  // W8: stage s's bf16 weight tile written
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(conv + kGemmStages);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) BT_STAMP(0);
@@ -229,6 +242,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     for (int s = 0; s < kGemmStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      if constexpr (W8) {
+        mbar_init(&afull[s], 1);
+        mbar_init(&conv[s], kConvThreads / 32);
+      }
     }
     mbar_init(done, 1);
     fence_mbar_init();
@@ -242,9 +259,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   }
   const uint32_t tmem = *tslot;
   // per-row constants of the epilogue (weights: no earlier kernel writes them)
-  float row_gain = 1.f, row_invf = 0.f;
+  float row_gain = 1.f, row_invf = 0.f, row_scale = 1.f;
   {
     const int r = tile * kTileM + (warp & 3) * 32 + lane;
+    if constexpr (W8) {
+      // the int8 row scale of accumulator row (warp & 3) * 32 + lane
+      const int m = (warp & 3) * 32 + lane;
+      if constexpr (MODE == kSwiGLU) {
+        const int fr = tile * (kTileM / 2) + (m & (kTileM / 2 - 1));
+        row_scale = fr < mrows ? (m < kTileM / 2 ? g.wsc[0] : g.wsc[1])[fr] : 0.f;
+      } else {
+        const float* sc = mat == 0 ? g.wsc[0] : (mat == 1 ? g.wsc[1] : g.wsc[2]);
+        row_scale = r < mrows ? sc[r] : 0.f;
+      }
+    }
     if constexpr (MODE == kQKV) {
       const int d = r % g.D;
       if (mat < 2) row_gain = bf16_to_f((mat == 0 ? g.gain : g.gain2)[d]);
@@ -262,23 +290,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       tma_prefetch_map(&xm);
       const uint64_t pw = policy_evict_first();
       const uint64_t px = policy_evict_last();
+      // bf16 weights: the tile into the stage, counted by full[s]; int8: the
+      // codes into the staging area, counted by afull[s]
       auto load_a = [&](int i, int s) {
-        const uint32_t st = smem_u32(sm + s * kStageBytes);
         const int x = (c0 + i) * kChunkK;
-        if constexpr (MODE == kSwiGLU) {
-          tma_load_2d(st, &w0, x, tile * (kTileM / 2), smem_u32(&full[s]), pw);
-          tma_load_2d(st + kHalfA, &w1, x, tile * (kTileM / 2), smem_u32(&full[s]), pw);
+        uint32_t st, bar;
+        if constexpr (W8) {
+          st = smem_u32(sm + s * kStageBytes + kA8Offset);
+          bar = smem_u32(&afull[s]);
+          mbar_arrive_expect_tx(&afull[s], kA8Bytes);
         } else {
-          tma_load_2d(st, wm, x, tile * kTileM, smem_u32(&full[s]), pw);
+          st = smem_u32(sm + s * kStageBytes);
+          bar = smem_u32(&full[s]);
+        }
+        constexpr uint32_t half = W8 ? kA8Bytes / 2 : kHalfA;
+        if constexpr (MODE == kSwiGLU) {
+          tma_load_2d(st, &w0, x, tile * (kTileM / 2), bar, pw);
+          tma_load_2d(st + half, &w1, x, tile * (kTileM / 2), bar, pw);
+        } else {
+          tma_load_2d(st, wm, x, tile * kTileM, bar, pw);
         }
       };
+      constexpr uint32_t kFullBytes = W8 ? kBBytes : kStageBytes;
       auto load_b = [&](int i, int s) {
         const uint32_t st = smem_u32(sm + s * kStageBytes);
         tma_load_2d(st + kABytes, &xm, (c0 + i) * kChunkK, 0, smem_u32(&full[s]), px);
       };
       const int pre = nch < kGemmStages ? nch : kGemmStages;
       for (int i = 0; i < pre; ++i) {
-        mbar_arrive_expect_tx(&full[i], kStageBytes);
+        mbar_arrive_expect_tx(&full[i], kFullBytes);
         load_a(i, i);
       }
       BT_STAMP(2);
@@ -289,7 +329,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       for (int i = pre; i < nch; ++i) {
         const int s = i % kGemmStages;
         if (!bt_wait(&empty[s], ((i / kGemmStages) - 1) & 1, g.timeout_ns, g.status)) break;
-        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        mbar_arrive_expect_tx(&full[s], kFullBytes);
         load_a(i, s);
         load_b(i, s);
         ++issued;
@@ -298,6 +338,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       for (int s = 0; s < kGemmStages && s < issued; ++s) {
         const int last = issued - 1 - ((issued - 1 - s) % kGemmStages);
         bt_wait(&full[s], (last / kGemmStages) & 1, g.timeout_ns, g.status, false);
+        if constexpr (W8) bt_wait(&afull[s], (last / kGemmStages) & 1, g.timeout_ns, g.status, false);
       }
     }
     __syncwarp();
@@ -307,6 +348,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       for (int i = 0; i < nch; ++i) {
         const int s = i % kGemmStages;
         if (!bt_wait(&full[s], (i / kGemmStages) & 1, g.timeout_ns, g.status)) break;
+        if constexpr (W8)
+          if (!bt_wait(&conv[s], (i / kGemmStages) & 1, g.timeout_ns, g.status)) break;
         if (i == 0) BT_STAMP(4);
         tc_fence_after();
         const uint32_t a_addr = smem_u32(sm + s * kStageBytes);
@@ -323,7 +366,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       tc_commit(smem_u32(done));
     }
     __syncwarp();
-  } else if (tid >= 64 && tid < 64 + kTileN) {
+  } else if (W8 && warp >= 4) {
+    // ---- int8 weights: widen each stage's codes into the bf16 operand tile
+    // (128-byte swizzle: row r at byte 128 r of its 8-row atom, 16-byte chunk
+    // j at chunk position j ^ (r mod 8)).  A code is sign-extended by a byte
+    // permute, converted to fp32 and packed to bf16 two at a time (|c| <= 127:
+    // exact in both).
+    const int ct = tid - 128;
+    constexpr int kItems = kA8Bytes / 8 / kConvThreads;  // 8 codes each
+    for (int i = 0; i < nch; ++i) {
+      const int s = i % kGemmStages;
+      // every converter waits; the barrier below makes the outcome uniform
+      const bool ok = bt_wait(&afull[s], (i / kGemmStages) & 1, g.timeout_ns, g.status);
+      uint8_t* dst = sm + s * kStageBytes;
+      const uint8_t* src = dst + kA8Offset;
+      uint2 c8s[kItems];
+#pragma unroll
+      for (int t = 0; t < kItems; ++t)
+        c8s[t] = ok ? *reinterpret_cast<const uint2*>(src + (t * kConvThreads + ct) * 8)
+                    : make_uint2(0u, 0u);
+      // every code is read before the tile is rewritten; a wait that gave up
+      // anywhere stops all converters together
+      if (named_sync_or(kConvBarrier, kConvThreads, !ok)) break;
+#pragma unroll
+      for (int t = 0; t < kItems; ++t) {
+        const int it = t * kConvThreads + ct;  // 8 codes: row it / 8, chunk it % 8
+        const int r = it >> 3, j = it & 7;
+        const uint2 c8 = c8s[t];
+        uint32_t w[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t x = h == 0 ? c8.x : c8.y;
+          // selector 0x8880 + 0x1111 e: byte e, then its sign bit replicated
+          float f[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            f[e] = static_cast<float>(static_cast<int>(prmt_b32(x, 0x8880u + 0x1111u * e)));
+          w[2 * h] = f2_to_bf16x2(f[0], f[1]);
+          w[2 * h + 1] = f2_to_bf16x2(f[2], f[3]);
+        }
+        *reinterpret_cast<uint4*>(dst + (r >> 3) * 1024 + (r & 7) * 128 + ((j ^ (r & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&conv[s]);
+    }
+  }
+  if (tid >= 64 && tid < 64 + kTileN) {
     // idle during the main loop: the epilogue's per-sequence inputs
     pdl_wait();
     const int b = tid - 64;
@@ -343,6 +433,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   tc_ld16(tl, v);
   tc_ld16(tl + 16, v + 16);
   tc_wait_ld();
+  if constexpr (W8) {
+#pragma unroll
+    for (int c = 0; c < kHalfN; ++c) v[c] *= row_scale;
+  }
   const int m = quad * 32 + lane;
   if (tid == 0) BT_STAMP(7);
   pdl_wait();  // everything below reads or writes what earlier kernels use
@@ -1054,6 +1148,7 @@ struct GemmPlan {
 struct BtPlan {
   BtShape s;
   int sms = 0;
+  bool w8 = false;  // int8 projections and lm_head (codes + fp32 row scales)
   int n_ssp = 0;
   const uint16_t* embed = nullptr;
   const uint16_t* final_norm = nullptr;
@@ -1076,14 +1171,17 @@ struct BtPlan {
 
 namespace {
 
+// bf16 [rows][cols] (128-byte swizzle, the MMA's operand layout), or int8
+// codes (i8: no swizzle, row r of a box at byte 64 r; widened by the CTA)
 bool encode_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
-                uint32_t box_rows) {
+                uint32_t box_rows, bool i8 = false) {
   const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint64_t strides[1] = {cols * (i8 ? 1 : 2)};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(kChunkK), box_rows};
   const cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return enc(m, i8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             i8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1098,9 +1196,10 @@ int pick_splits(int tiles, int k_chunks, int sms) {
 
 // n_mat matrices stacked along their rows; box_rows = 128 (one matrix per
 // tile) or 64 (gate/up pairs: 64 rows of each per tile).
-bool make_gemm(EncodeTiledFn enc, GemmPlan& gp, int n_mat, const uint16_t* const* w,
+// w8: the matrices are int8 codes with fp32 row scales sc[i]
+bool make_gemm(EncodeTiledFn enc, GemmPlan& gp, int n_mat, const void* const* w,
                const int* rows, int K, uint32_t box_rows, const CUtensorMap* xmap, int sms,
-               bool one_split) {
+               bool one_split, bool w8 = false, const float* const* sc = nullptr) {
   GemmArgs& g = gp.args;
   g = GemmArgs{};
   g.n_mat = box_rows == kTileM ? n_mat : 1;
@@ -1110,9 +1209,11 @@ bool make_gemm(EncodeTiledFn enc, GemmPlan& gp, int n_mat, const uint16_t* const
       g.rows[i] = rows[i];
       g.tiles[i] = (rows[i] + static_cast<int>(box_rows) - 1) / static_cast<int>(box_rows);
       if (box_rows == kTileM || i == 0) tiles += g.tiles[i];
-      if (!encode_map(enc, &gp.w[i], w[i], K, rows[i], box_rows)) return false;
+      if (!encode_map(enc, &gp.w[i], w[i], K, rows[i], box_rows, w8)) return false;
+      g.wsc[i] = w8 ? sc[i] : nullptr;
     } else {
       gp.w[i] = gp.w[0];
+      g.wsc[i] = g.wsc[0];
     }
   }
   g.k_chunks = (K + kChunkK - 1) / kChunkK;
@@ -1123,9 +1224,32 @@ bool make_gemm(EncodeTiledFn enc, GemmPlan& gp, int n_mat, const uint16_t* const
 }
 
 template <int MODE>
-cudaError_t launch_gemm(const GemmPlan& gp, const GemmArgs& g, cudaStream_t st) {
-  return launch_pdl(gemm_kernel<MODE>, gp.grid, dim3(kGemmThreads), kGemmSmem, st,
+cudaError_t launch_gemm(const GemmPlan& gp, const GemmArgs& g, bool w8, cudaStream_t st) {
+  if (w8)
+    return launch_pdl(gemm_kernel<MODE, true>, gp.grid, dim3(kGemmThreads), kGemmSmem, st,
+                      static_cast<unsigned>(g.splits), gp.w[0], gp.w[1], gp.w[2], *gp.x, g);
+  return launch_pdl(gemm_kernel<MODE, false>, gp.grid, dim3(kGemmThreads), kGemmSmem, st,
                     static_cast<unsigned>(g.splits), gp.w[0], gp.w[1], gp.w[2], *gp.x, g);
+}
+
+template <int MODE, bool W8>
+cudaError_t gemm_attrs() {
+  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<MODE, W8>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kGemmSmem));
+  if (e == cudaSuccess && MODE != kLm)
+    e = cudaFuncSetAttribute(gemm_kernel<MODE, W8>,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+template <bool W8>
+cudaError_t all_gemm_attrs() {
+  cudaError_t e = gemm_attrs<kQKV, W8>();
+  if (e == cudaSuccess) e = gemm_attrs<kResid, W8>();
+  if (e == cudaSuccess) e = gemm_attrs<kSwiGLU, W8>();
+  if (e == cudaSuccess) e = gemm_attrs<kLm, W8>();
+  return e;
 }
 
 template <int D, int REP>
@@ -1173,10 +1297,12 @@ cudaError_t attn_attrs_for(int rep) {
 
 }  // namespace
 
-int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_head,
+int bt_plan_create(const BtShape& s, const uint16_t* embed, const void* lm_head,
                    const uint16_t* final_norm, const LayerPtrs* layers_host,
-                   const float* inv_freq_dev, int sms, BtPlan** out, cudaError_t* cerr) {
+                   const float* inv_freq_dev, int sms, BtPlan** out, cudaError_t* cerr,
+                   const float* lm_scale, const LayerScales* scales_host) {
   *out = nullptr;
+  const bool w8 = scales_host != nullptr;
   *cerr = cudaSuccess;
   const int HqD = s.Hq * s.D, HkvD = s.Hkv * s.D;
   // tiles of 128 q / k / v rows hold whole heads; gate/up tiles pair 64 rows
@@ -1194,6 +1320,7 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_h
   if (!p) return DEC_ERR_ARG;
   p->s = s;
   p->sms = sms;
+  p->w8 = w8;
   p->n_ssp = (s.H + kTileM - 1) / kTileM;
   p->embed = embed;
   p->final_norm = final_norm;
@@ -1252,34 +1379,32 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const uint16_t* lm_h
   p->down.resize(s.L);
   for (int l = 0; ok && l < s.L; ++l) {
     const LayerPtrs& lp = p->layers[l];
-    const uint16_t* wqkv[3] = {lp.w[DEC_LW_Q], lp.w[DEC_LW_K], lp.w[DEC_LW_V]};
+    const float* const* ls = w8 ? scales_host[l].s : nullptr;
+    auto sc = [&](int j) { return ls ? ls[j] : nullptr; };
+    const void* wqkv[3] = {lp.w[DEC_LW_Q], lp.w[DEC_LW_K], lp.w[DEC_LW_V]};
+    const float* sqkv[3] = {sc(DEC_LW_Q), sc(DEC_LW_K), sc(DEC_LW_V)};
     const int rqkv[3] = {HqD, HkvD, HkvD};
-    const uint16_t* wo[1] = {lp.w[DEC_LW_O]};
+    const void* wo[1] = {lp.w[DEC_LW_O]};
+    const float* so[1] = {sc(DEC_LW_O)};
     const int ro[1] = {s.H};
-    const uint16_t* wgu[2] = {lp.w[DEC_LW_GATE], lp.w[DEC_LW_UP]};
+    const void* wgu[2] = {lp.w[DEC_LW_GATE], lp.w[DEC_LW_UP]};
+    const float* sgu[2] = {sc(DEC_LW_GATE), sc(DEC_LW_UP)};
     const int rgu[2] = {s.F, s.F};
-    const uint16_t* wd[1] = {lp.w[DEC_LW_DOWN]};
-    ok = make_gemm(enc, p->qkv[l], 3, wqkv, rqkv, s.H, kTileM, &p->map_h, sms, false) &&
-         make_gemm(enc, p->o[l], 1, wo, ro, HqD, kTileM, &p->map_o, sms, false) &&
-         make_gemm(enc, p->gu[l], 2, wgu, rgu, s.H, kTileM / 2, &p->map_h, sms, false) &&
-         make_gemm(enc, p->down[l], 1, wd, ro, s.F, kTileM, &p->map_u, sms, false);
+    const void* wd[1] = {lp.w[DEC_LW_DOWN]};
+    const float* sd[1] = {sc(DEC_LW_DOWN)};
+    ok = make_gemm(enc, p->qkv[l], 3, wqkv, rqkv, s.H, kTileM, &p->map_h, sms, false, w8, sqkv) &&
+         make_gemm(enc, p->o[l], 1, wo, ro, HqD, kTileM, &p->map_o, sms, false, w8, so) &&
+         make_gemm(enc, p->gu[l], 2, wgu, rgu, s.H, kTileM / 2, &p->map_h, sms, false, w8, sgu) &&
+         make_gemm(enc, p->down[l], 1, wd, ro, s.F, kTileM, &p->map_u, sms, false, w8, sd);
   }
   if (ok) {
-    const uint16_t* wl[1] = {lm_head};
+    const void* wl[1] = {lm_head};
+    const float* sl[1] = {lm_scale};
     const int rl[1] = {s.V};
-    ok = make_gemm(enc, p->lm, 1, wl, rl, s.H, kTileM, &p->map_h, sms, true);
+    ok = make_gemm(enc, p->lm, 1, wl, rl, s.H, kTileM, &p->map_h, sms, true, w8, sl);
   }
   // kernel attributes, once
-  const int smem = static_cast<int>(kGemmSmem);
-  const cudaFuncAttribute dyn = cudaFuncAttributeMaxDynamicSharedMemorySize;
-  const cudaFuncAttribute npc = cudaFuncAttributeNonPortableClusterSizeAllowed;
-  if (ok) e = cudaFuncSetAttribute(gemm_kernel<kQKV>, dyn, smem);
-  if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kResid>, dyn, smem);
-  if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kSwiGLU>, dyn, smem);
-  if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kLm>, dyn, smem);
-  if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kQKV>, npc, 1);
-  if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kResid>, npc, 1);
-  if (ok && e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<kSwiGLU>, npc, 1);
+  if (ok) e = w8 ? all_gemm_attrs<true>() : all_gemm_attrs<false>();
   const int rep = s.Hq / s.Hkv;
   if (ok && e == cudaSuccess) e = s.D == 128 ? attn_attrs_for<128>(rep) : attn_attrs_for<64>(rep);
   if (!ok || e != cudaSuccess) {
@@ -1337,6 +1462,7 @@ cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
     }
     g.k_chunks = gp.args.k_chunks;
     g.splits = gp.args.splits;
+    for (int i = 0; i < 3; ++i) g.wsc[i] = gp.args.wsc[i];
     return g;
   };
 
@@ -1394,7 +1520,7 @@ cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
     g.layer = l;
     g.gain = lp.w[DEC_LW_Q_NORM];
     g.gain2 = lp.w[DEC_LW_K_NORM];
-    if ((e = launch_gemm<kQKV>(p->qkv[l], g, st)) != cudaSuccess) return e;
+    if ((e = launch_gemm<kQKV>(p->qkv[l], g, p->w8, st)) != cudaSuccess) return e;
     at.l = l;
     e = s.D == 128 ? launch_attn<128>(at, rep, io.kv_fp8 != 0, st)
                    : launch_attn<64>(at, rep, io.kv_fp8 != 0, st);
@@ -1403,19 +1529,19 @@ cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
     g.gain = lp.w[DEC_LW_POST_NORM];
     g.act = p->act_h;
     g.hidden = nullptr;
-    if ((e = launch_gemm<kResid>(p->o[l], g, st)) != cudaSuccess) return e;
+    if ((e = launch_gemm<kResid>(p->o[l], g, p->w8, st)) != cudaSuccess) return e;
     g = args_of(p->gu[l]);
     g.act = p->act_u;
-    if ((e = launch_gemm<kSwiGLU>(p->gu[l], g, st)) != cudaSuccess) return e;
+    if ((e = launch_gemm<kSwiGLU>(p->gu[l], g, p->w8, st)) != cudaSuccess) return e;
     g = args_of(p->down[l]);
     g.gain = l + 1 < s.L ? p->layers[l + 1].w[DEC_LW_IN_NORM] : p->final_norm;
     g.act = p->act_h;
     g.hidden = io.hidden ? io.hidden + static_cast<size_t>(l + 1) * io.B * s.H : nullptr;
-    if ((e = launch_gemm<kResid>(p->down[l], g, st)) != cudaSuccess) return e;
+    if ((e = launch_gemm<kResid>(p->down[l], g, p->w8, st)) != cudaSuccess) return e;
   }
   GemmArgs g = args_of(p->lm);
   g.logits = io.logits;
-  if ((e = launch_gemm<kLm>(p->lm, g, st)) != cudaSuccess) return e;
+  if ((e = launch_gemm<kLm>(p->lm, g, p->w8, st)) != cudaSuccess) return e;
   return launch_pdl(finish_kernel, dim3(1), dim3(kTileN), 0, st, 1u, sa);
 }
 

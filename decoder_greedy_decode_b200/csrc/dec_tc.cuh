@@ -98,6 +98,13 @@ __device__ __forceinline__ void tc_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Order this thread's generic-proxy shared-memory writes (an operand tile
+// written by threads, not by TMA) before later async-proxy reads of it (the
+// tensor core's MMA operand loads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ------------------------------------------------------------ TMA
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;
@@ -108,8 +115,9 @@ __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
 }
 // Tile (x = column, y = row) of a 2-D tensor map into shared memory,
-// completing on `mbar` (transaction bytes = the box size).  x * 2 bytes is
-// always a multiple of 128 here (x is a multiple of 64 bf16 columns).
+// completing on `mbar` (transaction bytes = the box size).  x is always a
+// multiple of 64 columns here (128 bytes of bf16, 64 bytes of int8), so the
+// start of every copied row is 16-byte aligned.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst_smem, const CUtensorMap* m, int x, int y,
                                             uint32_t mbar_smem, uint64_t policy) {
   asm volatile(

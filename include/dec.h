@@ -166,10 +166,14 @@ typedef struct dec_weights_int8 {
   const float *const *scales;
 } dec_weights_int8;
 
-/* dec_init for a weight-only int8 model.  Same ownership and errors as
- * dec_init; max_batch must be 1..4 (DEC_ERR_BATCH otherwise): int8 weights
- * run on the single persistent kernel (dec_step, dec_step_host,
- * dec_generate, and dec_verify for the blocks it takes). */
+/* dec_init for a weight-only int8 model.  Same ownership, errors and
+ * max_batch range (1..64) as dec_init.  Batches of 1..4 run on the single
+ * persistent kernel (int8 rows in its ring, CUDA-core dot products); batches
+ * of 5..64 on the batched step, whose tensor-core GEMMs stage each int8
+ * weight tile by TMA and widen it to a bf16 operand tile in shared memory
+ * (codes up to 127 are exact in bf16), with the row scale applied to the
+ * fp32 accumulator.  dec_step, dec_step_host, dec_generate and dec_verify
+ * work as with bf16 weights. */
 int dec_init_int8(const dec_shape *shape, const dec_weights_int8 *weights, dec_handle **out);
 
 /* Release the handle and its workspace (synchronises the device first). */

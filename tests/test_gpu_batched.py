@@ -14,7 +14,7 @@ import torch
 import oracle
 from conftest import oracle_cache, oracle_shape, oracle_weights
 from decoder_greedy_decode_b200 import capi, synth
-from decoder_greedy_decode_b200.decoder import Decoder, to_device
+from decoder_greedy_decode_b200.decoder import Decoder, quantize_int8, to_device
 from gpu_util import assert_close, assert_id, i32
 from test_gpu_step import _check_kv_row, _check_only_rows_changed, _gpu_step, _run_teacher_forced
 
@@ -204,9 +204,12 @@ def _seq_cache(vals, sc):
     return oracle.Cache("fp8", np.ascontiguousarray(vals.numpy()), np.ascontiguousarray(sc.numpy()))
 
 
-def _full_size(s, w, wd, batch, lengths, max_ctx, kind, sampled, steps, seed):
-    m = oracle.Model(oracle_shape(s), oracle_weights(w))
-    dec = Decoder(s, wd, batch)
+def _full_size(s, w, wd, batch, lengths, max_ctx, kind, sampled, steps, seed, w8=False):
+    """w8: an int8 handle (dec_quantize_int8 of wd) against the oracle's int8
+    model of the same weights."""
+    ow = oracle_weights(w)
+    m = oracle.Model(oracle_shape(s), oracle.quantize_weights_int8(ow) if w8 else ow)
+    dec = Decoder(s, quantize_int8(wd) if w8 else wd, batch)
     kv = dec.kv_cache(batch, max_ctx, kind)
     host = _fill_batch(s, kv, lengths, seed, kind, sampled)
     caches = {b: _seq_cache(*host[b]) for b in sampled}

@@ -116,10 +116,16 @@ def _step(dec, kv, toks, poss):
 
 
 @pytest.mark.parametrize("batch,kind,gain_std", [(1, "bf16", 0.0), (2, "fp8", 0.1),
-                                                 (3, "bf16", 0.1), (4, "bf16", 0.0)])
+                                                 (3, "bf16", 0.1), (4, "bf16", 0.0),
+                                                 (5, "bf16", 0.1), (16, "fp8", 0.0),
+                                                 (64, "bf16", 0.0)])
 def test_tiny_int8_teacher_forced(batch, kind, gain_std):
+    """Batches of 1-4 run on the persistent kernel, 5-64 on the batched
+    step (int8 codes widened to bf16 operand tiles, row scales in the
+    epilogue)."""
     s = synth.TINY
-    lengths = [17, 1, 40, 63][:batch]
+    lengths = [17, 1, 40, 63][:batch] if batch <= 4 else \
+        [(13 * b + 5) % 76 for b in range(batch)]
     m, caches, dec, kv = _setup_int8(s, 300 + batch, batch, 80, lengths, kind, gain_std)
     toks = [int(t) for t in synth.tokens(s.vocab, batch, seed=400 + batch)]
     for t in range(4):
@@ -143,7 +149,7 @@ def test_int8_handle_limits():
     s = synth.TINY
     w8 = quantize_int8(to_device(synth.model_weights(s, seed=310)))
     with pytest.raises(capi.DecError):
-        Decoder(s, w8, max_batch=5)          # int8 runs on the persistent kernel only
+        Decoder(s, w8, max_batch=65)         # the batched step takes up to 64
     dec = Decoder(s, w8, max_batch=4)
     kv = dec.kv_cache(1, 32)
     out = torch.zeros(5, dtype=torch.int32, device="cuda")
@@ -169,6 +175,26 @@ def test_int8_verify_block_equals_single_steps():
         assert_close(lg[i], r.logits, f"int8 verify row {i} logits")
         assert_id(ids[i], r, f"int8 verify row {i}")
         _check_kv_row(kv, caches[0], 0, n0 + i, f"int8 verify row {i}")
+    dec.close()
+
+
+def test_int8_verify_block_on_the_batched_step():
+    """A block of 9 tokens on an int8 handle of max_batch 16 (the batched
+    step) equals 9 teacher-forced single steps of the oracle's int8 model."""
+    s = synth.TINY
+    n0, k = 30, 9
+    m, caches, dec, kv = _setup_int8(s, 322, 1, 64, [n0], "bf16", 0.0, max_batch=16)
+    toks = [int(t) for t in synth.tokens(s.vocab, k, seed=323)]
+    out = torch.full((k,), -7, dtype=torch.int32, device="cuda")
+    logits = torch.empty((k, s.vocab), dtype=torch.float32, device="cuda")
+    dec.verify(kv, i32(toks), i32(range(n0, n0 + k)), 0, out, logits)
+    assert dec.check() == 0
+    ids, lg = out.cpu().tolist(), logits.cpu().numpy()
+    for i in range(k):
+        r = m.step(caches[0], toks[i], n0 + i)
+        assert_close(lg[i], r.logits, f"int8 batched verify row {i} logits")
+        assert_id(ids[i], r, f"int8 batched verify row {i}")
+        _check_kv_row(kv, caches[0], 0, n0 + i, f"int8 batched verify row {i}")
     dec.close()
 
 
@@ -238,3 +264,15 @@ def test_0p6b_int8_bs1_ctx795(big06_int8):
         _check_kv_row(kv, cache, 0, p, tag)
         tok = r.token
     dec.close()
+
+
+def test_0p6b_int8_bs64_every_sequence_one_step():
+    """The 0.6B shape with int8 weights, 64 sequences, contexts U[200, 420]
+    (the batched step): every sequence of the batch against the oracle's
+    int8 model for one step."""
+    from test_gpu_batched import _full_size
+    s = synth.QWEN3_0_6B
+    w = synth.model_weights(s, seed=2)
+    wd = to_device(w)
+    lengths = synth.ragged_lengths(200, 420, 64, seed=76)
+    _full_size(s, w, wd, 64, lengths, 432, "bf16", list(range(64)), steps=1, seed=77, w8=True)
