@@ -75,6 +75,9 @@ def lib() -> ctypes.CDLL:
         L.or_int8_quantize_rows.argtypes = [P, I, I, P, P]
         L.or_int8_quantize_rows.restype = None
         L.or_gemv_i8.argtypes, L.or_gemv_i8.restype = [P, P, P, I, I, P], None
+        L.or_fp8w_quantize_rows.argtypes = [P, I, I, P, P]
+        L.or_fp8w_quantize_rows.restype = None
+        L.or_gemv_f8.argtypes, L.or_gemv_f8.restype = [P, P, P, I, I, P], None
         L.or_step.argtypes = [P, P, P, P, P, P, I, P, P, I, P, P, P, I, I, I, P, P, P, P, P]
         L.or_step.restype = I
         L.or_set_threads.argtypes, L.or_set_threads.restype = [I], None
@@ -138,6 +141,17 @@ def int8_quantize_rows(W_bits) -> tuple:
     return codes.reshape(W.shape), scales.reshape(W.shape[:-1])
 
 
+def fp8w_quantize_rows(W_bits) -> tuple:
+    """Per-row E4M3 codes and fp32 scales of a bf16 matrix [rows, cols]
+    (reading in dec_oracle.c, or_fp8w_quantize_rows)."""
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    W2 = W.reshape(-1, W.shape[-1])
+    codes = np.zeros(W2.shape, dtype=np.uint8)
+    scales = np.zeros(W2.shape[0], dtype=np.float32)
+    lib().or_fp8w_quantize_rows(_p(W2), W2.shape[0], W2.shape[1], _p(codes), _p(scales))
+    return codes.reshape(W.shape), scales.reshape(W.shape[:-1])
+
+
 # ---------------------------------------------------------- building blocks
 def rmsnorm(x, g_bits, eps: float) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float64)
@@ -161,6 +175,15 @@ def gemv_i8(codes, scales, x) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float64)
     y = np.zeros(C.shape[0], dtype=np.float64)
     lib().or_gemv_i8(_p(C), _p(sc), _p(x), C.shape[0], C.shape[1], _p(y))
+    return y
+
+
+def gemv_f8(codes, scales, x) -> np.ndarray:
+    C = np.ascontiguousarray(codes, dtype=np.uint8)
+    sc = np.ascontiguousarray(scales, dtype=np.float32)
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.zeros(C.shape[0], dtype=np.float64)
+    lib().or_gemv_f8(_p(C), _p(sc), _p(x), C.shape[0], C.shape[1], _p(y))
     return y
 
 
@@ -226,9 +249,9 @@ PROJ_KEYS = ("q", "k", "v", "o", "gate", "up", "down")
 class Weights:
     """bf16 bits (np.uint16) of every tensor; layer tensors keyed by LAYER_KEYS.
 
-    kind "int8": the PROJ_KEYS tensors of every layer and lm_head are int8
-    codes, with fp32 row scales in `scales` (per layer, keyed by PROJ_KEYS)
-    and `lm_scale`; the embedding and the norm gains stay bf16."""
+    kind "int8" / "fp8": the PROJ_KEYS tensors of every layer and lm_head are
+    int8 / E4M3 codes, with fp32 row scales in `scales` (per layer, keyed by
+    PROJ_KEYS) and `lm_scale`; the embedding and the norm gains stay bf16."""
     embed: np.ndarray
     lm_head: np.ndarray
     final_norm: np.ndarray
@@ -238,20 +261,30 @@ class Weights:
     scales: Optional[List[Dict[str, np.ndarray]]] = None
 
 
-def quantize_weights_int8(w: Weights) -> Weights:
-    """The int8 weight-only model of a bf16 one: every projection and lm_head
-    quantised per row (int8_quantize_rows)."""
+def _quantize_weights(w: Weights, rows_fn, kind: str) -> Weights:
     assert w.kind == "bf16"
     layers, scales = [], []
     for lw in w.layers:
         nl, ns = dict(lw), {}
         for key in PROJ_KEYS:
-            nl[key], ns[key] = int8_quantize_rows(lw[key])
+            nl[key], ns[key] = rows_fn(lw[key])
         layers.append(nl)
         scales.append(ns)
-    lm, lms = int8_quantize_rows(w.lm_head)
+    lm, lms = rows_fn(w.lm_head)
     return Weights(embed=w.embed, lm_head=lm, final_norm=w.final_norm, layers=layers,
-                   kind="int8", lm_scale=lms, scales=scales)
+                   kind=kind, lm_scale=lms, scales=scales)
+
+
+def quantize_weights_int8(w: Weights) -> Weights:
+    """The int8 weight-only model of a bf16 one: every projection and lm_head
+    quantised per row (int8_quantize_rows)."""
+    return _quantize_weights(w, int8_quantize_rows, "int8")
+
+
+def quantize_weights_fp8(w: Weights) -> Weights:
+    """The E4M3 weight-only model of a bf16 one: every projection and lm_head
+    quantised per row (fp8w_quantize_rows)."""
+    return _quantize_weights(w, fp8w_quantize_rows, "fp8")
 
 
 @dataclass
@@ -285,15 +318,16 @@ class Model:
         self.w = w
         self._keep = []
         L = shape.n_layers
-        i8 = w.kind == "int8"
-        if w.kind not in ("bf16", "int8"):
+        i8 = w.kind in ("int8", "fp8")   # 8-bit codes with row scales
+        if w.kind not in ("bf16", "int8", "fp8"):
             raise ValueError(w.kind)
+        cdt = np.int8 if w.kind == "int8" else np.uint8
         ptrs = (ctypes.c_void_p * (L * len(LAYER_KEYS)))()
         sptrs = (ctypes.c_void_p * (L * len(LAYER_KEYS)))()
         for l, lw in enumerate(w.layers):
             for j, key in enumerate(LAYER_KEYS):
                 proj = i8 and key in PROJ_KEYS
-                a = np.ascontiguousarray(lw[key], dtype=np.int8 if proj else np.uint16)
+                a = np.ascontiguousarray(lw[key], dtype=cdt if proj else np.uint16)
                 self._keep.append(a)
                 ptrs[l * len(LAYER_KEYS) + j] = a.ctypes.data
                 if proj:
@@ -303,9 +337,9 @@ class Model:
                     sptrs[l * len(LAYER_KEYS) + j] = sc.ctypes.data
         self._ptrs = ptrs
         self._sptrs = sptrs
-        self._wkind = 1 if i8 else 0
+        self._wkind = {"bf16": 0, "int8": 1, "fp8": 2}[w.kind]
         self._emb = np.ascontiguousarray(w.embed, dtype=np.uint16)
-        self._lm = np.ascontiguousarray(w.lm_head, dtype=np.int8 if i8 else np.uint16)
+        self._lm = np.ascontiguousarray(w.lm_head, dtype=cdt if i8 else np.uint16)
         self._lms = np.ascontiguousarray(w.lm_scale, dtype=np.float32) if i8 else None
         self._fn = np.ascontiguousarray(w.final_norm, dtype=np.uint16)
         s = shape

@@ -171,6 +171,28 @@ void or_int8_quantize_rows(const uint16_t *W, int rows, int cols, int8_t *codes,
     scales[r] = or_int8_quantize_row(W + (size_t)r * cols, cols, codes + (size_t)r * cols);
 }
 
+/* Per-row E4M3 weight-only quantisation of a row-major bf16 W[rows, cols]
+ * ("Qwen3-ASR -- Latency & Bottleneck Analysis", 08 Optimization roadmap:
+ * an fp8 lm_head; the same weight-only scheme for the projections).
+ * Reading (the page names the format only): each row is quantised by the
+ * per-row E4M3 quantiser of the KV rows (or_e4m3_quantize_row) applied to
+ * the fp32 values of the bf16 weights: scale = max(amax, 2^-126) / 448 in
+ * fp32, code_i = E4M3_rne_satfinite(fp32(w_i) / scale).  The weight the step
+ * multiplies is e4m3(code) * scale. */
+void or_fp8w_quantize_rows(const uint16_t *W, int rows, int cols, uint8_t *codes,
+                           float *scales) {
+#pragma omp parallel
+  {
+    float *row = (float *)malloc(sizeof(float) * (size_t)cols);
+#pragma omp for schedule(static)
+    for (int r = 0; r < rows; ++r) {
+      for (int c = 0; c < cols; ++c) row[c] = (float)or_bf16_to_double(W[(size_t)r * cols + c]);
+      scales[r] = or_e4m3_quantize_row(row, cols, codes + (size_t)r * cols);
+    }
+    free(row);
+  }
+}
+
 /* ------------------------------------------------------------------ */
 /* Building blocks                                                     */
 /* ------------------------------------------------------------------ */
@@ -213,12 +235,28 @@ void or_gemv_i8(const int8_t *C, const float *s, const double *x, int rows, int 
   }
 }
 
-/* A projection in either weight format: wkind 0 -> bf16 W, 1 -> int8 codes
- * with row scales s. */
+/* y = W x for E4M3 codes C[rows, cols] with one fp32 scale per row: the
+ * weight is e4m3_decode(code) * scale in double; double dot products in
+ * ascending column order, as or_gemv. */
+void or_gemv_f8(const uint8_t *C, const float *s, const double *x, int rows, int cols,
+                double *y) {
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < rows; ++r) {
+    const uint8_t *c = C + (size_t)r * cols;
+    const double sr = (double)s[r];
+    double acc = 0.0;
+    for (int j = 0; j < cols; ++j) acc += (or_e4m3_decode(c[j]) * sr) * x[j];
+    y[r] = acc;
+  }
+}
+
+/* A projection in any weight format: wkind 0 -> bf16 W, 1 -> int8 codes,
+ * 2 -> E4M3 codes, the last two with row scales s. */
 static void project(int wkind, const void *W, const float *s, const double *x, int rows,
                     int cols, double *y) {
   if (wkind == 0) or_gemv((const uint16_t *)W, x, rows, cols, y);
-  else or_gemv_i8((const int8_t *)W, s, x, rows, cols, y);
+  else if (wkind == 1) or_gemv_i8((const int8_t *)W, s, x, rows, cols, y);
+  else or_gemv_f8((const uint8_t *)W, s, x, rows, cols, y);
 }
 
 /* Rotary embedding of one head vector at position p ("MRoPE, fp32" in
@@ -332,9 +370,9 @@ enum { W_IN_NORM, W_Q, W_K, W_V, W_Q_NORM, W_K_NORM, W_O, W_POST_NORM,
  *    h = rmsnorm(x, g_post);  x += Wd (silu(Wg h) * (Wu h))
  *  logits = W_lm rmsnorm(x, g_final);  token' = argmax(logits)
  *
- * Weights: wkind 0 -> every tensor bf16 bits; wkind 1 -> the seven
+ * Weights: wkind 0 -> every tensor bf16 bits; wkind 1 / 2 -> the seven
  * projections of every layer (q, k, v, o, gate, up, down) and lm_head are
- * int8 codes with fp32 row scales (lsc[l * W_N + idx], lm_scale), the
+ * int8 / E4M3 codes with fp32 row scales (lsc[l * W_N + idx], lm_scale), the
  * embedding and the norm gains stay bf16.
  * KV cache of this sequence: kind 0 -> bf16 bits kv16[L][2][Hkv][max_ctx][D];
  * kind 1 -> codes kv8[L][2][Hkv][max_ctx][D] and scales kvs[L][2][Hkv][max_ctx].
