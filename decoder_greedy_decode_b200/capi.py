@@ -28,7 +28,7 @@ EXPORTS = (
     "dec_error_string", "dec_last_cuda_error", "dec_get_config",
     "dec_attention_workspace_bytes", "dec_attention", "dec_kv_quantize_e4m3",
     "dec_attention_noalloc", "dec_verify", "dec_accept_greedy", "dec_generate",
-    "dec_init_int8", "dec_quantize_int8",
+    "dec_init_int8", "dec_quantize_int8", "dec_init_fp8w", "dec_quantize_fp8w",
 )
 #: the projections an int8 handle holds as int8 codes + row scales
 PROJ_KEYS = ("q", "k", "v", "o", "gate", "up", "down")
@@ -102,6 +102,9 @@ def lib() -> ctypes.CDLL:
             "dec_init_int8": ([ctypes.POINTER(dec_shape), ctypes.POINTER(dec_weights_int8),
                                ctypes.POINTER(P)], I),
             "dec_quantize_int8": ([P, I, I, P, P, P], I),
+            "dec_init_fp8w": ([ctypes.POINTER(dec_shape), ctypes.POINTER(dec_weights_int8),
+                               ctypes.POINTER(P)], I),
+            "dec_quantize_fp8w": ([P, I, I, P, P, P], I),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -144,7 +147,10 @@ def dec_init(shape: dec_shape, embed, lm_head, final_norm, layer_ptrs: Sequence[
 
 
 def dec_init_int8(shape: dec_shape, embed, lm_head, lm_head_scale, final_norm,
-                  layer_ptrs: Sequence[int], scale_ptrs: Sequence[Optional[int]]) -> int:
+                  layer_ptrs: Sequence[int], scale_ptrs: Sequence[Optional[int]],
+                  entry: str = "dec_init_int8") -> int:
+    """dec_init_int8, or with entry="dec_init_fp8w" the same call for E4M3
+    codes."""
     arr = (ctypes.c_void_p * len(layer_ptrs))(*[int(p) for p in layer_ptrs])
     sarr = (ctypes.c_void_p * len(scale_ptrs))(*[None if p is None else int(p)
                                                  for p in scale_ptrs])
@@ -152,14 +158,24 @@ def dec_init_int8(shape: dec_shape, embed, lm_head, lm_head_scale, final_norm,
                          ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)),
                          ctypes.cast(sarr, ctypes.POINTER(ctypes.c_void_p)))
     h = ctypes.c_void_p()
-    _ok(lib().dec_init_int8(ctypes.byref(shape), ctypes.byref(w), ctypes.byref(h)),
-        "dec_init_int8")
+    _ok(getattr(lib(), entry)(ctypes.byref(shape), ctypes.byref(w), ctypes.byref(h)), entry)
     return h.value
+
+
+def dec_init_fp8w(shape: dec_shape, embed, lm_head, lm_head_scale, final_norm,
+                  layer_ptrs: Sequence[int], scale_ptrs: Sequence[Optional[int]]) -> int:
+    return dec_init_int8(shape, embed, lm_head, lm_head_scale, final_norm, layer_ptrs,
+                         scale_ptrs, entry="dec_init_fp8w")
 
 
 def dec_quantize_int8(w, rows: int, cols: int, codes, scales, stream=None) -> None:
     _ok(lib().dec_quantize_int8(_ptr(w), rows, cols, _ptr(codes), _ptr(scales),
                                 _stream(stream)), "dec_quantize_int8")
+
+
+def dec_quantize_fp8w(w, rows: int, cols: int, codes, scales, stream=None) -> None:
+    _ok(lib().dec_quantize_fp8w(_ptr(w), rows, cols, _ptr(codes), _ptr(scales),
+                                _stream(stream)), "dec_quantize_fp8w")
 
 
 def dec_free(h: int) -> None:

@@ -37,7 +37,7 @@ struct dec_handle {
   const uint16_t* lm_head = nullptr;
   const uint16_t* final_norm = nullptr;
   LayerPtrs* layers_dev = nullptr;
-  int w8 = 0;                         // weight-only int8 handle
+  int w8 = 0;                         // weight-only 8-bit handle: 1 int8, 2 E4M3 codes
   const float* lm_scale = nullptr;    // int8: lm_head row scales
   LayerScales* scales_dev = nullptr;  // int8: projection row scales
   int wsc_n = 0;
@@ -103,8 +103,22 @@ extern "C" int dec_init(const dec_shape* shape, const dec_weights* w, dec_handle
   return init_handle(shape, iw, out);
 }
 
+static int init_8bit(const dec_shape* shape, const dec_weights_int8* w, int fmt,
+                     dec_handle** out);
+
 extern "C" int dec_init_int8(const dec_shape* shape, const dec_weights_int8* w,
                              dec_handle** out) {
+  return init_8bit(shape, w, 1, out);
+}
+
+extern "C" int dec_init_fp8w(const dec_shape* shape, const dec_weights_int8* w,
+                             dec_handle** out) {
+  return init_8bit(shape, w, 2, out);
+}
+
+// fmt 1: int8 codes, 2: E4M3 codes (both with fp32 row scales)
+static int init_8bit(const dec_shape* shape, const dec_weights_int8* w, int fmt,
+                     dec_handle** out) {
   if (!shape || !w || !out) return DEC_ERR_NULL;
   *out = nullptr;
   int rc = check_shape(shape);
@@ -125,7 +139,7 @@ extern "C" int dec_init_int8(const dec_shape* shape, const dec_weights_int8* w,
     }
   }
   const InitWeights iw{w->embed, w->lm_head, w->final_norm, w->layers,
-                       1, w->lm_head_scale, w->scales};
+                       fmt, w->lm_head_scale, w->scales};
   return init_handle(shape, iw, out);
 }
 
@@ -174,7 +188,7 @@ static int init_handle(const dec_shape* shape, const InitWeights& w, dec_handle*
     }
     h->smem[b] = step_smem_bytes(h->nslot[b], h->slot_bytes[b], b, H, F, HqD, D, rep, h->wsc_n,
                                  h->prow);
-    e = step_set_smem(b, D, w.w8 != 0, h->smem[b]);
+    e = step_set_smem(b, D, w.w8, h->smem[b]);
     if (e != cudaSuccess) {
       delete h;
       return cuda_fail(e);
@@ -261,7 +275,7 @@ static int init_handle(const dec_shape* shape, const InitWeights& w, dec_handle*
     rc = bt_plan_create(bs, h->embed, h->lm_head, h->final_norm, lp.data(),
                         reinterpret_cast<const float*>(h->ws + wl.inv_freq), h->sms, &h->bt, &ce,
                         w.w8 ? static_cast<const float*>(w.lm_scale) : nullptr,
-                        w.w8 ? ls.data() : nullptr);
+                        w.w8 ? ls.data() : nullptr, w.w8);
     if (rc) {
       cudaFree(h->ws);
       delete h;
@@ -680,6 +694,18 @@ extern "C" int dec_quantize_int8(const void* w, int rows, int cols, int8_t* code
   if (!aligned(w, 16) || !aligned(codes, 8) || !aligned(scales, 4)) return DEC_ERR_ALIGN;
   if (rows == 0) return DEC_OK;
   cudaError_t e = launch_quantize_int8(static_cast<const uint16_t*>(w), rows, cols, codes, scales,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return DEC_OK;
+}
+
+extern "C" int dec_quantize_fp8w(const void* w, int rows, int cols, uint8_t* codes,
+                                 float* scales, void* stream) {
+  if (!w || !codes || !scales) return DEC_ERR_NULL;
+  if (rows < 0 || cols < 8 || cols % 8) return DEC_ERR_ARG;
+  if (!aligned(w, 16) || !aligned(codes, 8) || !aligned(scales, 4)) return DEC_ERR_ALIGN;
+  if (rows == 0) return DEC_OK;
+  cudaError_t e = launch_quantize_fp8w(static_cast<const uint16_t*>(w), rows, cols, codes, scales,
                                        static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return DEC_OK;

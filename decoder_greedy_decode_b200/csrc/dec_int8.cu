@@ -62,7 +62,54 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
   }
 }
 
+// Per-row E4M3 weight-only quantisation ("Qwen3-ASR -- Latency & Bottleneck
+// Analysis", 08 Optimization roadmap: an fp8 lm_head): the per-row E4M3
+// quantiser of the KV rows applied to the fp32 values of a bf16 weight row,
+// scale = max(amax, 2^-126) / 448 (IEEE fp32 division), code = E4M3(w /
+// scale) (IEEE fp32 division, round to nearest even, saturating).  The
+// weight the step multiplies is e4m3(code) * scale.
+__device__ __forceinline__ uint32_t e4m3_pair(float a, float b, float scale) {
+  return f2_to_e4m3x2(__fdiv_rn(a, scale), __fdiv_rn(b, scale));
+}
+
+__global__ void __launch_bounds__(kQuantWarps * 32)
+    quantize_fp8_kernel(const uint16_t* __restrict__ w, int rows, int cols,
+                        uint8_t* __restrict__ codes, float* __restrict__ scales) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kQuantWarps + warp;
+  if (r >= rows) return;
+  const uint4* src = reinterpret_cast<const uint4*>(w + static_cast<size_t>(r) * cols);
+  const int nv = cols >> 3;
+  float amax = 0.f;
+  for (int v = lane; v < nv; v += 32) {
+    const uint4 q = src[v];
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16lo(q.x)), fabsf(bf16hi(q.x))),
+                             fmaxf(fabsf(bf16lo(q.y)), fabsf(bf16hi(q.y)))));
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16lo(q.z)), fabsf(bf16hi(q.z))),
+                             fmaxf(fabsf(bf16lo(q.w)), fabsf(bf16hi(q.w)))));
+  }
+  amax = fmaxf(warp_max(amax), 1.17549435e-38f);  // 2^-126
+  const float scale = __fdiv_rn(amax, 448.0f);
+  if (lane == 0) scales[r] = scale;
+  uint2* dst = reinterpret_cast<uint2*>(codes + static_cast<size_t>(r) * cols);
+  for (int v = lane; v < nv; v += 32) {
+    const uint4 q = src[v];
+    const uint32_t lo = e4m3_pair(bf16lo(q.x), bf16hi(q.x), scale) |
+                        (e4m3_pair(bf16lo(q.y), bf16hi(q.y), scale) << 16);
+    const uint32_t hi = e4m3_pair(bf16lo(q.z), bf16hi(q.z), scale) |
+                        (e4m3_pair(bf16lo(q.w), bf16hi(q.w), scale) << 16);
+    dst[v] = make_uint2(lo, hi);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_fp8w(const uint16_t* w, int rows, int cols, uint8_t* codes,
+                                 float* scales, cudaStream_t s) {
+  const int grid = (rows + kQuantWarps - 1) / kQuantWarps;
+  quantize_fp8_kernel<<<grid, kQuantWarps * 32, 0, s>>>(w, rows, cols, codes, scales);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quantize_int8(const uint16_t* w, int rows, int cols, int8_t* codes,
                                  float* scales, cudaStream_t s) {

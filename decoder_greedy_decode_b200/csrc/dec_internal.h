@@ -104,11 +104,13 @@ void step_ring(int B, int H, int F, int HqD, int D, int rep, int wsc_n, int prow
 // counted separately).
 int step_part_rows(int H, int F, int nqkv, int ctas);
 // Dynamic shared-memory limit of the step kernels a handle launches.
-cudaError_t step_set_smem(int B, int D, bool w8, size_t smem);
+cudaError_t step_set_smem(int B, int D, int w8, size_t smem);
 // Shared-memory row-scale slots an int8 step needs: the most rows one CTA
 // computes in any stage (gate and up rows counted twice).
 int step_wsc_slots(int H, int F, int nqkv, int V, int ctas);
 cudaError_t launch_quantize_int8(const uint16_t* w, int rows, int cols, int8_t* codes,
+                                 float* scales, cudaStream_t s);
+cudaError_t launch_quantize_fp8w(const uint16_t* w, int rows, int cols, uint8_t* codes,
                                  float* scales, cudaStream_t s);
 cudaError_t launch_step_small(const StepArgs& a, int ctas, size_t smem, cudaStream_t s);
 
@@ -143,12 +145,13 @@ struct BtShape {
 };
 struct BtPlan;  // tensor maps, launch configuration and scratch (dec_step_batched.cu)
 // Returns 0, or a DEC_ERR_* code (DEC_ERR_CUDA with *cerr set).
-// int8 handles pass the lm_head row scales and every layer's projection row
-// scales (host array of device pointers); bf16 handles pass null for both.
+// 8-bit handles (w8 1: int8, 2: E4M3 codes) pass the lm_head row scales and
+// every layer's projection row scales (host array of device pointers); bf16
+// handles pass null for both and w8 = 0.
 int bt_plan_create(const BtShape& s, const uint16_t* embed, const void* lm_head,
                    const uint16_t* final_norm, const LayerPtrs* layers_host,
                    const float* inv_freq_dev, int sms, BtPlan** out, cudaError_t* cerr,
-                   const float* lm_scale, const LayerScales* scales_host);
+                   const float* lm_scale, const LayerScales* scales_host, int w8);
 void bt_plan_destroy(BtPlan* p);
 struct BtIO {
   int B;

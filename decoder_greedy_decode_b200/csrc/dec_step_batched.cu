@@ -196,7 +196,7 @@ struct GemmArgs {
   } while (0)
 #endif
 
-template <int MODE, bool W8>
+template <int MODE, int W8>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap w0,
                                                             const __grid_constant__ CUtensorMap w1,
                                                             const __grid_constant__ CUtensorMap w2,
@@ -367,11 +367,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
     __syncwarp();
   } else if (W8 && warp >= 4) {
-    // ---- int8 weights: widen each stage's codes into the bf16 operand tile
+    // ---- 8-bit weights: widen each stage's codes into the bf16 operand tile
     // (128-byte swizzle: row r at byte 128 r of its 8-row atom, 16-byte chunk
-    // j at chunk position j ^ (r mod 8)).  A code is sign-extended by a byte
-    // permute, converted to fp32 and packed to bf16 two at a time (|c| <= 127:
-    // exact in both).
+    // j at chunk position j ^ (r mod 8)).  An int8 code is sign-extended by a
+    // byte permute and converted to fp32 (|c| <= 127: exact in bf16); E4M3
+    // codes go through the hardware e4m3x2 -> f16x2 conversion; both are
+    // packed to bf16 two at a time.
     const int ct = tid - 128;
     constexpr int kItems = kA8Bytes / 8 / kConvThreads;  // 8 codes each
     for (int i = 0; i < nch; ++i) {
@@ -397,11 +398,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const uint32_t x = h == 0 ? c8.x : c8.y;
-          // selector 0x8880 + 0x1111 e: byte e, then its sign bit replicated
           float f[4];
+          if constexpr (W8 == 2) {
+            // E4M3: every finite value is exact in bf16
+            const float2 a = e4m3x2_to_f2(static_cast<uint16_t>(x & 0xFFFFu));
+            const float2 b = e4m3x2_to_f2(static_cast<uint16_t>(x >> 16));
+            f[0] = a.x;
+            f[1] = a.y;
+            f[2] = b.x;
+            f[3] = b.y;
+          } else {
+            // selector 0x8880 + 0x1111 e: byte e, then its sign bit replicated
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            f[e] = static_cast<float>(static_cast<int>(prmt_b32(x, 0x8880u + 0x1111u * e)));
+            for (int e = 0; e < 4; ++e)
+              f[e] = static_cast<float>(static_cast<int>(prmt_b32(x, 0x8880u + 0x1111u * e)));
+          }
           w[2 * h] = f2_to_bf16x2(f[0], f[1]);
           w[2 * h + 1] = f2_to_bf16x2(f[2], f[3]);
         }
@@ -1148,7 +1159,7 @@ struct GemmPlan {
 struct BtPlan {
   BtShape s;
   int sms = 0;
-  bool w8 = false;  // int8 projections and lm_head (codes + fp32 row scales)
+  int w8 = 0;  // 1 / 2: int8 / E4M3 projections and lm_head (codes + fp32 row scales)
   int n_ssp = 0;
   const uint16_t* embed = nullptr;
   const uint16_t* final_norm = nullptr;
@@ -1224,15 +1235,18 @@ bool make_gemm(EncodeTiledFn enc, GemmPlan& gp, int n_mat, const void* const* w,
 }
 
 template <int MODE>
-cudaError_t launch_gemm(const GemmPlan& gp, const GemmArgs& g, bool w8, cudaStream_t st) {
-  if (w8)
-    return launch_pdl(gemm_kernel<MODE, true>, gp.grid, dim3(kGemmThreads), kGemmSmem, st,
+cudaError_t launch_gemm(const GemmPlan& gp, const GemmArgs& g, int w8, cudaStream_t st) {
+  if (w8 == 1)
+    return launch_pdl(gemm_kernel<MODE, 1>, gp.grid, dim3(kGemmThreads), kGemmSmem, st,
                       static_cast<unsigned>(g.splits), gp.w[0], gp.w[1], gp.w[2], *gp.x, g);
-  return launch_pdl(gemm_kernel<MODE, false>, gp.grid, dim3(kGemmThreads), kGemmSmem, st,
+  if (w8 == 2)
+    return launch_pdl(gemm_kernel<MODE, 2>, gp.grid, dim3(kGemmThreads), kGemmSmem, st,
+                      static_cast<unsigned>(g.splits), gp.w[0], gp.w[1], gp.w[2], *gp.x, g);
+  return launch_pdl(gemm_kernel<MODE, 0>, gp.grid, dim3(kGemmThreads), kGemmSmem, st,
                     static_cast<unsigned>(g.splits), gp.w[0], gp.w[1], gp.w[2], *gp.x, g);
 }
 
-template <int MODE, bool W8>
+template <int MODE, int W8>
 cudaError_t gemm_attrs() {
   cudaError_t e = cudaFuncSetAttribute(gemm_kernel<MODE, W8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1243,7 +1257,7 @@ cudaError_t gemm_attrs() {
   return e;
 }
 
-template <bool W8>
+template <int W8>
 cudaError_t all_gemm_attrs() {
   cudaError_t e = gemm_attrs<kQKV, W8>();
   if (e == cudaSuccess) e = gemm_attrs<kResid, W8>();
@@ -1300,9 +1314,9 @@ cudaError_t attn_attrs_for(int rep) {
 int bt_plan_create(const BtShape& s, const uint16_t* embed, const void* lm_head,
                    const uint16_t* final_norm, const LayerPtrs* layers_host,
                    const float* inv_freq_dev, int sms, BtPlan** out, cudaError_t* cerr,
-                   const float* lm_scale, const LayerScales* scales_host) {
+                   const float* lm_scale, const LayerScales* scales_host, int w8) {
   *out = nullptr;
-  const bool w8 = scales_host != nullptr;
+  if ((w8 != 0) != (scales_host != nullptr)) return DEC_ERR_ARG;
   *cerr = cudaSuccess;
   const int HqD = s.Hq * s.D, HkvD = s.Hkv * s.D;
   // tiles of 128 q / k / v rows hold whole heads; gate/up tiles pair 64 rows
@@ -1379,7 +1393,7 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const void* lm_head,
   p->down.resize(s.L);
   for (int l = 0; ok && l < s.L; ++l) {
     const LayerPtrs& lp = p->layers[l];
-    const float* const* ls = w8 ? scales_host[l].s : nullptr;
+    const float* const* ls = w8 ? scales_host[l].s : nullptr;  // row scales of 8-bit codes
     auto sc = [&](int j) { return ls ? ls[j] : nullptr; };
     const void* wqkv[3] = {lp.w[DEC_LW_Q], lp.w[DEC_LW_K], lp.w[DEC_LW_V]};
     const float* sqkv[3] = {sc(DEC_LW_Q), sc(DEC_LW_K), sc(DEC_LW_V)};
@@ -1404,7 +1418,7 @@ int bt_plan_create(const BtShape& s, const uint16_t* embed, const void* lm_head,
     ok = make_gemm(enc, p->lm, 1, wl, rl, s.H, kTileM, &p->map_h, sms, true, w8, sl);
   }
   // kernel attributes, once
-  if (ok) e = w8 ? all_gemm_attrs<true>() : all_gemm_attrs<false>();
+  if (ok) e = w8 == 1 ? all_gemm_attrs<1>() : (w8 == 2 ? all_gemm_attrs<2>() : all_gemm_attrs<0>());
   const int rep = s.Hq / s.Hkv;
   if (ok && e == cudaSuccess) e = s.D == 128 ? attn_attrs_for<128>(rep) : attn_attrs_for<64>(rep);
   if (!ok || e != cudaSuccess) {

@@ -265,8 +265,42 @@ __device__ __forceinline__ float dot8_i8(uint32_t w0, uint32_t w1, const float* 
   return s;
 }
 
-// int8 rows (K bytes): the sums of code * x; the caller applies the row scale.
-template <int R, int B>
+// The four 8-bit weight codes of a word as floats (exact): W8 = 1 signed
+// int8 codes, W8 = 2 E4M3 codes (two hardware e4m3x2 -> f16x2 conversions).
+template <int W8>
+__device__ __forceinline__ void codes4(uint32_t w, float (&f)[4]) {
+  if constexpr (W8 == 2) {
+    const float2 a = e4m3x2_to_f2(static_cast<uint16_t>(w & 0xFFFFu));
+    const float2 b = e4m3x2_to_f2(static_cast<uint16_t>(w >> 16));
+    f[0] = a.x;
+    f[1] = a.y;
+    f[2] = b.x;
+    f[3] = b.y;
+  } else {
+    const uint32_t u = w ^ 0x80808080u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) f[e] = i8_at(u, static_cast<uint32_t>(e));
+  }
+}
+template <int W8>
+__device__ __forceinline__ float dot8_w8(uint32_t w0, uint32_t w1, const float* x) {
+  if constexpr (W8 == 1) return dot8_i8(w0, w1, x);
+  float a[4], b[4];
+  codes4<W8>(w0, a);
+  codes4<W8>(w1, b);
+  float s = a[0] * x[0];
+  s = fmaf(a[1], x[1], s);
+  s = fmaf(a[2], x[2], s);
+  s = fmaf(a[3], x[3], s);
+  s = fmaf(b[0], x[4], s);
+  s = fmaf(b[1], x[5], s);
+  s = fmaf(b[2], x[6], s);
+  return fmaf(b[3], x[7], s);
+}
+
+// 8-bit rows (K bytes, int8 or E4M3 codes): the sums of code * x; the caller
+// applies the row scale.
+template <int R, int B, int W8>
 __device__ __noinline__ GroupSums<R, B> group_dot_i8(const uint32_t* rows, uint32_t act,
                                                      int act_stride, int nblk, int lane) {
   float acc[R][B], acc2[R][B];
@@ -294,7 +328,7 @@ __device__ __noinline__ GroupSums<R, B> group_dot_i8(const uint32_t* rows, uint3
                    : "=f"(x[4]), "=f"(x[5]), "=f"(x[6]), "=f"(x[7]) : "r"(xa + 512));
 #pragma unroll
       for (int i = 0; i < R; ++i) {
-        const float d = dot8_i8(w[i][0], w[i][1], x);
+        const float d = dot8_w8<W8>(w[i][0], w[i][1], x);
         if (odd) acc2[i][b] += d;
         else acc[i][b] += d;
       }
@@ -382,7 +416,7 @@ struct KSums {
   float s[R / 4][B];
 };
 
-template <int R, int B, bool W8>
+template <int R, int B, int W8>
 __device__ __forceinline__ KSums<R, B> kdot(const uint32_t (&rows)[R], uint32_t act,
                                             int act_stride, int blk0, int nb, int lane) {
   float acc[R][B];
@@ -414,9 +448,7 @@ __device__ __forceinline__ KSums<R, B> kdot(const uint32_t (&rows)[R], uint32_t 
     for (int i = 0; i < R; ++i) {
       float wf[4];
       if constexpr (W8) {
-        const uint32_t u = w[i][0] ^ 0x80808080u;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) wf[e] = i8_at(u, e);
+        codes4<W8>(w[i][0], wf);
       } else {
         wf[0] = bf16lo(w[i][0]);
         wf[1] = bf16hi(w[i][0]);
@@ -469,8 +501,9 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
 }
 
 // The per-launch state of one CTA.  FP8: the cache holds E4M3 codes + scales.
-// W8: the projections and lm_head are int8 codes with fp32 row scales.
-template <int B, int D, bool FP8, bool W8>
+// W8: 0 bf16 weights; 1 / 2: the projections and lm_head are int8 / E4M3
+// codes with fp32 row scales.
+template <int B, int D, bool FP8, int W8>
 struct Cta {
   static constexpr int DL = D / 32;  // attention dims per lane (warp-wide vectors)
   static constexpr int DQ = D / 8;   // attention dims per lane (lane octets)
@@ -1359,7 +1392,7 @@ struct Cta {
             rows[i] = smem_u32(tb) + static_cast<uint32_t>(j < nr ? j : 0) * row_bytes;
           }
           const GroupSums<R, B> gs4 =
-              W8 ? group_dot_i8<R, B>(rows, smem_u32(act), kmax, K >> 8, lane)
+              W8 ? group_dot_i8<R, B, (W8 ? W8 : 1)>(rows, smem_u32(act), kmax, K >> 8, lane)
                  : group_dot<R, B>(rows, smem_u32(act), kmax, K >> 8, lane);
           const int ri = R == 4 ? (lane >> 3) : (R == 2 ? (lane >> 4) : 0);
           const bool leader = R == 4 ? ((lane & 7) == 0) : (R == 2 ? ((lane & 15) == 0) : lane == 0);
@@ -1924,7 +1957,7 @@ struct Cta {
   }
 };
 
-template <int B, int D, bool FP8, bool W8>
+template <int B, int D, bool FP8, int W8>
 __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a, int kmax) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Cta<B, D, FP8, W8> c(a, smem, kmax);
@@ -1989,7 +2022,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const StepArgs a,
   }
 }
 
-template <int B, int D, bool FP8, bool W8>
+template <int B, int D, bool FP8, int W8>
 cudaError_t launch_bd(const StepArgs& a, int ctas, size_t smem, int kmax,
                       cudaStream_t s) {
   auto k = step_kernel<B, D, FP8, W8>;
@@ -1999,7 +2032,7 @@ cudaError_t launch_bd(const StepArgs& a, int ctas, size_t smem, int kmax,
                                      dim3(kStepThreads), params, smem, s);
 }
 
-template <int B, int D, bool FP8, bool W8>
+template <int B, int D, bool FP8, int W8>
 cudaError_t attr_bd(size_t smem) {
   return cudaFuncSetAttribute(step_kernel<B, D, FP8, W8>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -2063,17 +2096,23 @@ int step_part_rows(int H, int F, int nqkv, int ctas) {
 
 // Sets the dynamic shared-memory limit of the kernel instantiations a
 // handle launches (once, when the handle is created).
-cudaError_t step_set_smem(int B, int D, bool w8, size_t smem) {
+cudaError_t step_set_smem(int B, int D, int w8, size_t smem) {
   cudaError_t e = cudaErrorInvalidValue;
+#define DEC_ATTR_W(BB, DD, WW)                                                  \
+  {                                                                             \
+    e = attr_bd<BB, DD, false, WW>(smem);                                       \
+    if (e == cudaSuccess) e = attr_bd<BB, DD, true, WW>(smem);                  \
+  }
 #define DEC_ATTR(BB, DD)                                                        \
   if (B == BB && D == DD) {                                                     \
-    e = w8 ? attr_bd<BB, DD, false, true>(smem) : attr_bd<BB, DD, false, false>(smem); \
-    if (e == cudaSuccess)                                                       \
-      e = w8 ? attr_bd<BB, DD, true, true>(smem) : attr_bd<BB, DD, true, false>(smem); \
+    if (w8 == 1) DEC_ATTR_W(BB, DD, 1)                                          \
+    else if (w8 == 2) DEC_ATTR_W(BB, DD, 2)                                     \
+    else DEC_ATTR_W(BB, DD, 0)                                                  \
   }
   DEC_ATTR(1, 128) DEC_ATTR(2, 128) DEC_ATTR(3, 128) DEC_ATTR(4, 128)
   DEC_ATTR(1, 64) DEC_ATTR(2, 64) DEC_ATTR(3, 64) DEC_ATTR(4, 64)
 #undef DEC_ATTR
+#undef DEC_ATTR_W
   return e;
 }
 
@@ -2081,15 +2120,19 @@ cudaError_t launch_step_small(const StepArgs& a, int ctas, size_t smem, cudaStre
   const int HqD = a.Hq * a.D;
   const int kmax = kmax_of(a.H, a.F, HqD);
   const bool f8 = a.kv_fp8 != 0;
+#define DEC_CASE_W(BB, DD, WW)                                                      \
+  return f8 ? launch_bd<BB, DD, true, WW>(a, ctas, smem, kmax, s)                    \
+            : launch_bd<BB, DD, false, WW>(a, ctas, smem, kmax, s);
 #define DEC_CASE(BB, DD)                                                            \
-  if (a.B == BB && a.D == DD)                                                       \
-    return f8 ? (a.w8 ? launch_bd<BB, DD, true, true>(a, ctas, smem, kmax, s)        \
-                      : launch_bd<BB, DD, true, false>(a, ctas, smem, kmax, s))      \
-              : (a.w8 ? launch_bd<BB, DD, false, true>(a, ctas, smem, kmax, s)       \
-                      : launch_bd<BB, DD, false, false>(a, ctas, smem, kmax, s));
+  if (a.B == BB && a.D == DD) {                                                     \
+    if (a.w8 == 1) DEC_CASE_W(BB, DD, 1)                                            \
+    if (a.w8 == 2) DEC_CASE_W(BB, DD, 2)                                            \
+    DEC_CASE_W(BB, DD, 0)                                                           \
+  }
   DEC_CASE(1, 128) DEC_CASE(2, 128) DEC_CASE(3, 128) DEC_CASE(4, 128)
   DEC_CASE(1, 64) DEC_CASE(2, 64) DEC_CASE(3, 64) DEC_CASE(4, 64)
 #undef DEC_CASE
+#undef DEC_CASE_W
   return cudaErrorInvalidValue;
 }
 

@@ -23,15 +23,20 @@ def to_device(w: Dict[str, object], device: str = "cuda") -> Dict[str, object]:
             "layers": [{k: t.to(device) for k, t in lw.items()} for lw in w["layers"]]}
 
 
-def quantize_int8(w: Dict[str, object]) -> Dict[str, object]:
-    """Weight-only int8 copy of device weights (to_device(...) layout): every
+def quantize_int8(w: Dict[str, object], kind: str = "int8") -> Dict[str, object]:
+    """Weight-only 8-bit copy of device weights (to_device(...) layout): every
     projection and lm_head quantised per output row by dec_quantize_int8
-    (codes int8 + fp32 row scales); embedding and norm gains shared."""
+    (kind "int8": int8 codes) or dec_quantize_fp8w (kind "fp8": E4M3 codes),
+    with fp32 row scales; embedding and norm gains shared."""
     def q(t):
         rows, cols = t.shape
-        codes = torch.empty((rows, cols), dtype=torch.int8, device=t.device)
+        codes = torch.empty((rows, cols), dtype=torch.int8 if kind == "int8" else torch.uint8,
+                            device=t.device)
         scales = torch.empty(rows, dtype=torch.float32, device=t.device)
-        capi.dec_quantize_int8(t, rows, cols, codes, scales)
+        if kind == "int8":
+            capi.dec_quantize_int8(t, rows, cols, codes, scales)
+        else:
+            capi.dec_quantize_fp8w(t, rows, cols, codes, scales)
         return codes, scales
 
     layers, scales = [], []
@@ -42,8 +47,13 @@ def quantize_int8(w: Dict[str, object]) -> Dict[str, object]:
         layers.append(nl)
         scales.append(ns)
     lm, lms = q(w["lm_head"])
-    return {"kind": "int8", "embed": w["embed"], "lm_head": lm, "lm_head_scale": lms,
+    return {"kind": kind, "embed": w["embed"], "lm_head": lm, "lm_head_scale": lms,
             "final_norm": w["final_norm"], "layers": layers, "scales": scales}
+
+
+def quantize_fp8w(w: Dict[str, object]) -> Dict[str, object]:
+    """Weight-only E4M3 copy of device weights (quantize_int8 with E4M3 codes)."""
+    return quantize_int8(w, kind="fp8")
 
 
 class KVCache:
@@ -85,12 +95,13 @@ class Decoder:
                             shape.rope_theta, max_batch)
         ptrs = [weights["layers"][l][k].data_ptr() for l in range(shape.n_layers)
                 for k in capi.LW_ORDER]
-        if weights.get("kind") == "int8":
+        if weights.get("kind") in ("int8", "fp8"):
             sptrs = [weights["scales"][l][k].data_ptr() if k in capi.PROJ_KEYS else None
                      for l in range(shape.n_layers) for k in capi.LW_ORDER]
             self.h = capi.dec_init_int8(cs, weights["embed"], weights["lm_head"],
                                         weights["lm_head_scale"], weights["final_norm"], ptrs,
-                                        sptrs)
+                                        sptrs, entry="dec_init_int8" if weights["kind"] == "int8"
+                                        else "dec_init_fp8w")
         else:
             self.h = capi.dec_init(cs, weights["embed"], weights["lm_head"],
                                    weights["final_norm"], ptrs)

@@ -6,9 +6,9 @@ quick timing.
 
 Weights have the 0.6B (default) or 1.7B widths with --layers layers; every
 sequence's cache holds N(0,1) rows up to a context drawn in [lo, hi]; the
-steps feed their own ids back.  --weights int8 quantises every projection and
-lm_head per row (dec_quantize_int8) and runs the weight-only int8 step
-(batch 1..4).  Prints the device time per step of the --steps steps that
+steps feed their own ids back.  --weights int8 / fp8 quantises every projection
+and lm_head per row (dec_quantize_int8 / dec_quantize_fp8w) and runs the
+weight-only 8-bit step.  Prints the device time per step of the --steps steps that
 follow --warmup untimed ones."""
 from __future__ import annotations
 
@@ -29,15 +29,15 @@ def main() -> None:
     p.add_argument("--steps", type=int, default=2)
     p.add_argument("--warmup", type=int, default=0)
     p.add_argument("--kv", choices=["bf16", "fp8"], default="bf16")
-    p.add_argument("--weights", choices=["bf16", "int8"], default="bf16")
+    p.add_argument("--weights", choices=["bf16", "int8", "fp8"], default="bf16")
     a = p.parse_args()
     base = synth.QWEN3_0_6B if a.shape == "0.6b" else synth.QWEN3_1_7B
     s = synth.ModelShape(a.layers, base.hidden, base.n_q_heads, base.n_kv_heads, base.head_dim,
                          base.ffn, base.vocab)
     lo, hi = (int(x) for x in a.ctx.split(","))
     w = to_device(synth.model_weights(s, seed=2))
-    if a.weights == "int8":
-        w = quantize_int8(w)
+    if a.weights in ("int8", "fp8"):
+        w = quantize_int8(w, kind=a.weights)
     dec = Decoder(s, w, max_batch=a.batch)
     max_ctx = (hi + a.warmup + a.steps + 15) // 16 * 16
     kv = dec.kv_cache(a.batch, max_ctx, a.kv)

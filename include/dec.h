@@ -176,6 +176,15 @@ typedef struct dec_weights_int8 {
  * work as with bf16 weights. */
 int dec_init_int8(const dec_shape *shape, const dec_weights_int8 *weights, dec_handle **out);
 
+/* Weight-only E4M3 model ("Qwen3-ASR -- Latency & Bottleneck Analysis", 08
+ * Optimization roadmap: an fp8 lm_head; the same scheme for the
+ * projections).  The same dec_weights_int8 layout, with OCP E4M3 codes in
+ * place of the int8 codes of the projections and lm_head (dec_quantize_fp8w
+ * makes them from bf16); the weight the step multiplies is e4m3(code) *
+ * scale.  Same ownership, errors, max_batch range and paths as
+ * dec_init_int8. */
+int dec_init_fp8w(const dec_shape *shape, const dec_weights_int8 *weights, dec_handle **out);
+
 /* Release the handle and its workspace (synchronises the device first). */
 void dec_free(dec_handle *h);
 
@@ -412,6 +421,17 @@ int dec_attention_noalloc(int batch, int n_q_heads, int n_kv_heads, int head_dim
  * w 16-byte, codes 8-byte and scales 4-byte aligned (DEC_ERR_ALIGN).
  * Asynchronous on `stream`. */
 int dec_quantize_int8(const void *w, int rows, int cols, int8_t *codes, float *scales,
+                      void *stream);
+
+/* Quantise a bf16 weight matrix w [rows, cols] (row-major, device) to OCP
+ * E4M3 codes [rows, cols] and one fp32 scale per row (device), the format
+ * dec_init_fp8w reads: the per-row quantiser of the FP8 cache rows applied
+ * to the weight row, scale = max(amax, 2^-126)/448 and code =
+ * RNE-satfinite(w/scale), both divisions in IEEE fp32 ("Latency & Bottleneck
+ * Analysis", 08 Optimization roadmap: fp8 lm_head).  cols must be a multiple
+ * of 8 (DEC_ERR_ARG); w 16-byte, codes 8-byte and scales 4-byte aligned
+ * (DEC_ERR_ALIGN).  Asynchronous on `stream`. */
+int dec_quantize_fp8w(const void *w, int rows, int cols, uint8_t *codes, float *scales,
                       void *stream);
 
 /* ------------------------------------------------------------------ */

@@ -77,34 +77,37 @@ def _int8_weights(L, aligned=True, null_scale_at=None, norm_scale_null=True):
     return w, (arr, sarr)
 
 
-def test_int8_init_checks_on_host():
-    """dec_init_int8: shape first, then max_batch <= 4, NULL pointers (a
-    projection's scale array is required, a norm slot's is not), alignment."""
-    L = capi.lib()
+@pytest.mark.parametrize("entry", ["dec_init_int8", "dec_init_fp8w"])
+def test_8bit_init_checks_on_host(entry):
+    """dec_init_int8 / dec_init_fp8w: shape first, then max_batch <= 64, NULL
+    pointers (a projection's scale array is required, a norm slot's is not),
+    alignment."""
+    init = getattr(capi.lib(), entry)
     h = ctypes.c_void_p()
     ok_shape = capi.dec_shape(2, 256, 4, 2, 64, 768, 4096, 1e-6, 1e6, 1)
     w, keep = _int8_weights(2)
     bad = capi.dec_shape(2, 200, 4, 2, 64, 768, 4096, 1e-6, 1e6, 1)
-    assert L.dec_init_int8(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(h)) == -2
-    big = capi.dec_shape(2, 256, 4, 2, 64, 768, 4096, 1e-6, 1e6, 5)
-    assert L.dec_init_int8(ctypes.byref(big), ctypes.byref(w), ctypes.byref(h)) == -3
+    assert init(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(h)) == -2
+    big = capi.dec_shape(2, 256, 4, 2, 64, 768, 4096, 1e-6, 1e6, 65)
+    assert init(ctypes.byref(big), ctypes.byref(w), ctypes.byref(h)) == -3
     q_of_layer1 = len(capi.LW_ORDER) + capi.LW_ORDER.index("q")
     w2, keep2 = _int8_weights(2, null_scale_at=q_of_layer1)
-    assert L.dec_init_int8(ctypes.byref(ok_shape), ctypes.byref(w2), ctypes.byref(h)) == -1
+    assert init(ctypes.byref(ok_shape), ctypes.byref(w2), ctypes.byref(h)) == -1
     w3, keep3 = _int8_weights(2, aligned=False)
-    assert L.dec_init_int8(ctypes.byref(ok_shape), ctypes.byref(w3), ctypes.byref(h)) == -6
+    assert init(ctypes.byref(ok_shape), ctypes.byref(w3), ctypes.byref(h)) == -6
     w4 = capi.dec_weights_int8(1 << 28, 1 << 29, None, 1 << 27, w.layers, w.scales)
-    assert L.dec_init_int8(ctypes.byref(ok_shape), ctypes.byref(w4), ctypes.byref(h)) == -1
+    assert init(ctypes.byref(ok_shape), ctypes.byref(w4), ctypes.byref(h)) == -1
     w5 = capi.dec_weights_int8(1 << 28, 1 << 29, (1 << 30) + 2, 1 << 27, w.layers, w.scales)
-    assert L.dec_init_int8(ctypes.byref(ok_shape), ctypes.byref(w5), ctypes.byref(h)) == -6
+    assert init(ctypes.byref(ok_shape), ctypes.byref(w5), ctypes.byref(h)) == -6
     assert not h.value
 
 
-def test_int8_quantizer_checks_on_host():
-    L = capi.lib()
-    assert L.dec_quantize_int8(None, 4, 16, 1 << 20, 1 << 21, None) == -1
-    assert L.dec_quantize_int8(1 << 20, 4, 20, 1 << 21, 1 << 22, None) == -9    # cols % 8
-    assert L.dec_quantize_int8(1 << 20, -1, 16, 1 << 21, 1 << 22, None) == -9
-    assert L.dec_quantize_int8((1 << 20) + 8, 4, 16, 1 << 21, 1 << 22, None) == -6  # w 16 B
-    assert L.dec_quantize_int8(1 << 20, 4, 16, (1 << 21) + 4, 1 << 22, None) == -6  # codes 8 B
-    assert L.dec_quantize_int8(1 << 20, 0, 16, 1 << 21, 1 << 22, None) == 0      # no rows: no-op
+@pytest.mark.parametrize("entry", ["dec_quantize_int8", "dec_quantize_fp8w"])
+def test_8bit_quantizer_checks_on_host(entry):
+    q = getattr(capi.lib(), entry)
+    assert q(None, 4, 16, 1 << 20, 1 << 21, None) == -1
+    assert q(1 << 20, 4, 20, 1 << 21, 1 << 22, None) == -9    # cols % 8
+    assert q(1 << 20, -1, 16, 1 << 21, 1 << 22, None) == -9
+    assert q((1 << 20) + 8, 4, 16, 1 << 21, 1 << 22, None) == -6  # w 16 B
+    assert q(1 << 20, 4, 16, (1 << 21) + 4, 1 << 22, None) == -6  # codes 8 B
+    assert q(1 << 20, 0, 16, 1 << 21, 1 << 22, None) == 0      # no rows: no-op

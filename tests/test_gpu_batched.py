@@ -205,11 +205,17 @@ def _seq_cache(vals, sc):
 
 
 def _full_size(s, w, wd, batch, lengths, max_ctx, kind, sampled, steps, seed, w8=False):
-    """w8: an int8 handle (dec_quantize_int8 of wd) against the oracle's int8
-    model of the same weights."""
+    """w8: an 8-bit handle (True or "int8": dec_quantize_int8 of wd; "fp8":
+    dec_quantize_fp8w) against the oracle's model of the same codes."""
     ow = oracle_weights(w)
-    m = oracle.Model(oracle_shape(s), oracle.quantize_weights_int8(ow) if w8 else ow)
-    dec = Decoder(s, quantize_int8(wd) if w8 else wd, batch)
+    wk = "int8" if w8 is True else w8
+    if wk:
+        m = oracle.Model(oracle_shape(s), oracle.quantize_weights_int8(ow) if wk == "int8"
+                         else oracle.quantize_weights_fp8(ow))
+        dec = Decoder(s, quantize_int8(wd, kind=wk), batch)
+    else:
+        m = oracle.Model(oracle_shape(s), ow)
+        dec = Decoder(s, wd, batch)
     kv = dec.kv_cache(batch, max_ctx, kind)
     host = _fill_batch(s, kv, lengths, seed, kind, sampled)
     caches = {b: _seq_cache(*host[b]) for b in sampled}
