@@ -16,7 +16,8 @@ headline keys: an "attention" object (isolated decode attention over a
 length x batch grid); a "verify" object (block verification, "Can CTC make
 Qwen3-ASR faster?", 11 Phase A); an "int8" object (the batch-1 workload with
 weight-only int8 projections and lm_head, faster-qwen-asr GB10 record,
-"cuda_graph_int8", and the batch-64 workload with them); a "bs64" object (the same decoder serving 64 sequences
+"cuda_graph_int8", and the batch-64 workload with them); an "fp8w" object
+(the same with weight-only E4M3 codes); a "bs64" object (the same decoder serving 64 sequences
 at once, contexts drawn in [200, 420], a 128-step window; the Baseten
 Qwen3-ASR article, "KV cache quantization"), in tokens/s, through the
 batched tensor-core step; a "cfg5" object (the 1.7B-shaped decoder at batch
@@ -235,15 +236,14 @@ BS64_STEPS = 64
 def run_bs64(s, wd, dev, ws, seed, w8=False):
     """Batch 64, ragged contexts U[200, 420], self-feeding over a 128-step
     window: device time of BS64_STEPS steps (max over ranks); tokens/s for
-    all ranks, and the step's algorithmic bytes over that time.  w8: the
-    same with weight-only int8 projections and lm_head (dec_quantize_int8 of
-    the same weights)."""
+    all ranks, and the step's algorithmic bytes over that time.  w8 "int8" /
+    "fp8": the same with weight-only 8-bit projections and lm_head."""
     import torch
     import torch.distributed as dist
     from decoder_greedy_decode_b200 import roofline, synth
     from decoder_greedy_decode_b200.decoder import Decoder, quantize_int8
     max_ctx = (BS64_HI + BS64_WINDOW + 15) // 16 * 16
-    dec = Decoder(s, quantize_int8(wd) if w8 else wd, max_batch=BS64)
+    dec = Decoder(s, quantize_int8(wd, kind=w8) if w8 else wd, max_batch=BS64)
     kv = dec.kv_cache(BS64, max_ctx)
     g = torch.Generator(device=dev).manual_seed(seed + 10)
     kv.values.normal_(generator=g)
@@ -270,7 +270,7 @@ def run_bs64(s, wd, dev, ws, seed, w8=False):
     if st != 0:
         raise RuntimeError(f"bs64 device status {st}")
     step_ms = ms / BS64_STEPS
-    wk = "int8" if w8 else "bf16"
+    wk = w8 if w8 else "bf16"
     nbytes = statistics.fmean(roofline.step_bytes(s, [n + (i % BS64_WINDOW) for n in lengths],
                                                   weights=wk)
                               for i in range(BS64_STEPS))
@@ -278,8 +278,7 @@ def run_bs64(s, wd, dev, ws, seed, w8=False):
     achieved = nbytes / (step_ms * 1e-3) / 1e9
     return {"value": round(replica_throughput(BS64, step_ms, ws), 1), "unit": "tokens/s",
             "ms_per_step": round(step_ms, 4), "steps": BS64_STEPS,
-            "workload": "0.6b, batch 64, contexts U[200,420], bf16 KV, "
-                        + ("int8" if w8 else "bf16") + " weights",
+            "workload": f"0.6b, batch 64, contexts U[200,420], bf16 KV, {wk} weights",
             "roofline": {"achieved": round(achieved, 1), "peak": peak,
                          "frac": round(achieved / peak, 4)},
             "launches_per_step": 1 + 5 * s.n_layers + 2}
@@ -362,18 +361,19 @@ def run_verify(s, wd, dev, seed):
 INT8_STEPS = 260
 
 
-def run_int8(s, wd, kv_host, tok0, dev, seed):
+def run_int8(s, wd, kv_host, tok0, dev, seed, kind="int8"):
     """Weight-only int8 (faster-qwen-asr GB10 record, "cuda_graph_int8": int8
-    text decoder + lm_head): the same batch-1 workload (context 795, the
-    130-step window, self-feeding) with every projection and lm_head
-    quantised per row by dec_quantize_int8.  Device time per step over
-    INT8_STEPS steps after 5 warm-ups, the steps rotating over HANDLES live
-    handles exactly as the bf16 line does.  Bytes: int8 weights + row scales,
-    the KV rows and the embedding row."""
+    text decoder + lm_head), or with kind "fp8" weight-only E4M3 ("Latency &
+    Bottleneck Analysis", 08 Optimization roadmap): the same batch-1 workload
+    (context 795, the 130-step window, self-feeding) with every projection
+    and lm_head quantised per row (dec_quantize_int8 / dec_quantize_fp8w).
+    Device time per step over INT8_STEPS steps after 5 warm-ups, the steps
+    rotating over HANDLES live handles exactly as the bf16 line does.  Bytes:
+    8-bit weights + row scales, the KV rows and the embedding row."""
     import torch
     from decoder_greedy_decode_b200 import capi, roofline
     from decoder_greedy_decode_b200.decoder import Decoder, quantize_int8
-    w8 = quantize_int8(wd)
+    w8 = quantize_int8(wd, kind=kind)
     decs = [Decoder(s, w8, max_batch=1) for _ in range(HANDLES)]
     kv = decs[0].kv_cache(1, 928)
     stream = torch.cuda.current_stream(dev)
@@ -398,23 +398,23 @@ def run_int8(s, wd, kv_host, tok0, dev, seed):
     for dec in decs:
         st = dec.check()
         if st != 0:
-            raise RuntimeError(f"int8 device status {st}")
+            raise RuntimeError(f"{kind} device status {st}")
     per = [evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(INT8_STEPS)]
     per_handle = [statistics.fmean(per[h::HANDLES]) for h in range(HANDLES)]
     for dec in decs:
         dec.close()
     del w8
     us = statistics.fmean(per)
-    nbytes = statistics.fmean(roofline.step_bytes(s, [N0 + (i % WINDOW)], weights="int8")
+    nbytes = statistics.fmean(roofline.step_bytes(s, [N0 + (i % WINDOW)], weights=kind)
                               for i in range(WINDOW))
-    peak, kind = peaks()
+    peak, _ = peaks()
     achieved = nbytes / (us * 1e-6) / 1e9
     return {"value": round(us, 1), "unit": "us/token",
-            "workload": "0.6b, batch 1, ctx 795 window, int8 projections + lm_head",
+            "workload": f"0.6b, batch 1, ctx 795 window, {kind} projections + lm_head",
             "us_per_handle": [round(v, 1) for v in per_handle],
             "roofline": {"achieved": round(achieved, 1), "peak": peak,
                          "frac": round(achieved / peak, 4),
-                         "traffic": ncu_traffic("step_kernel_int8_0p6b_bs1_ctx795")}}
+                         "traffic": ncu_traffic(f"step_kernel_{kind}_0p6b_bs1_ctx795")}}
 
 
 ATT_LENGTHS = (128, 795, 4096, 16384, 32768)
@@ -755,13 +755,16 @@ def run_ours(args):
 
     # ---- the other configurations (rank 0 prints their summaries)
     bs64 = run_bs64(s, wd, dev, ws, args.seed)
-    bs64_w8 = run_bs64(s, wd, dev, ws, args.seed, w8=True)
+    bs64_w8 = {k: run_bs64(s, wd, dev, ws, args.seed, w8=k) for k in ("int8", "fp8")}
     verify = run_verify(s, wd, dev, args.seed) if rank == 0 else None
     int8 = run_int8(s, wd, kv_host, tok0, dev, args.seed) if rank == 0 else None
-    if int8 is not None:
-        int8["bs64"] = {"tokens_per_s": bs64_w8["value"], "ms_per_step": bs64_w8["ms_per_step"],
-                        "frac": bs64_w8["roofline"]["frac"],
-                        "workload": "0.6b, batch 64, contexts U[200,420], int8 weights"}
+    fp8w = run_int8(s, wd, kv_host, tok0, dev, args.seed, kind="fp8") if rank == 0 else None
+    for k, o in (("int8", int8), ("fp8", fp8w)):
+        if o is not None:
+            b = bs64_w8[k]
+            o["bs64"] = {"tokens_per_s": b["value"], "ms_per_step": b["ms_per_step"],
+                         "frac": b["roofline"]["frac"],
+                         "workload": f"0.6b, batch 64, contexts U[200,420], {k} weights"}
     generate = run_generate(s, wd, kv_host, tok0, dev) if rank == 0 else None
     kernel_config = dec.config()
     dec.close()
@@ -808,6 +811,7 @@ def run_ours(args):
             "attention": attention,
             "verify": verify,
             "int8": int8,
+            "fp8w": fp8w,
             "bs64": bs64,
             "cfg5": cfg5,
             "generate": generate,

@@ -41,11 +41,11 @@ def projection_rows(s) -> int:
 def weight_bytes(s, weights: str = "bf16") -> int:
     """Every weight the step reads once: layers + lm_head + final norm.
 
-    weights "int8": the projections and lm_head as int8 codes (1 byte each)
-    plus one fp32 scale per output row; norm gains stay bf16."""
+    weights "int8" / "fp8": the projections and lm_head as 8-bit codes (1
+    byte each) plus one fp32 scale per output row; norm gains stay bf16."""
     if weights == "bf16":
         return (s.n_layers * layer_weight_params(s) + s.vocab * s.hidden + s.hidden) * BF16
-    assert weights == "int8"
+    assert weights in ("int8", "fp8")
     norms = 2 * s.hidden + 2 * s.head_dim
     proj = layer_weight_params(s) - norms
     per_layer = proj + 4 * projection_rows(s) + norms * BF16
