@@ -571,34 +571,41 @@ GEN_STEPS = 130
 def run_generate(s, wd, kv_host, tok0, dev):
     """dec_generate on the batch-1 workload: the 130-token window from
     position 795 in one call (ids fed back and positions advanced on the
-    device); device time per generated token over 3 calls after one warm-up
-    call."""
+    device); device time per generated token, the median of 2 calls after a
+    warm-up call on each of HANDLES live handles, averaged over the handles
+    (as the batch-1 line averages the workspace placements)."""
     import torch
     from decoder_greedy_decode_b200.decoder import Decoder
-    dec = Decoder(s, wd, max_batch=1)
-    kv = dec.kv_cache(1, 928)
     stream = torch.cuda.current_stream(dev)
     out = torch.empty((GEN_STEPS, 1), dtype=torch.int32, device=dev)
-    times = []
-    for rep in range(4):
-        kv.values.copy_(kv_host.to(dev))
-        tok = torch.tensor([tok0], dtype=torch.int32, device=dev)
-        pos = torch.tensor([N0], dtype=torch.int32, device=dev)
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        dec.generate(kv, tok, pos, out, -1, stream)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        if rep > 0:
-            times.append(e0.elapsed_time(e1))
-    st = dec.check()
-    dec.close()
-    if st != 0:
-        raise RuntimeError(f"generate device status {st}")
-    ms = statistics.median(times)
+    decs = [Decoder(s, wd, max_batch=1) for _ in range(HANDLES)]
+    per_handle = []
+    for dec in decs:
+        kv = dec.kv_cache(1, 928)
+        times = []
+        for rep in range(3):
+            kv.values.copy_(kv_host.to(dev))
+            tok = torch.tensor([tok0], dtype=torch.int32, device=dev)
+            pos = torch.tensor([N0], dtype=torch.int32, device=dev)
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dec.generate(kv, tok, pos, out, -1, stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if rep > 0:
+                times.append(e0.elapsed_time(e1))
+        st = dec.check()
+        if st != 0:
+            raise RuntimeError(f"generate device status {st}")
+        per_handle.append(statistics.median(times))
+        del kv
+    for dec in decs:
+        dec.close()
+    ms = statistics.fmean(per_handle)
     return {"us_per_token": round(ms * 1e3 / GEN_STEPS, 1), "steps_per_call": GEN_STEPS,
-            "ms_per_call": round(ms, 3)}
+            "ms_per_call": round(ms, 3),
+            "us_per_token_per_handle": [round(t * 1e3 / GEN_STEPS, 1) for t in per_handle]}
 
 
 def cpu_baseline(s, w, kv_host, tok0, budget_s=20.0):
