@@ -143,6 +143,72 @@ static int init_8bit(const dec_shape* shape, const dec_weights_int8* w, int fmt,
   return init_handle(shape, iw, out);
 }
 
+static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* pos,
+                   const dec_kv* kv, int32_t* out_ids, float* logits, float* hidden,
+                   cudaStream_t stream, int n_steps = 1, int eos = -1,
+                   int32_t* gen_pos = nullptr, const int* retired = nullptr, int vseq = -1);
+
+// The persistent step's time depends by a few per cent on where its
+// workspace (above all the tagged exchange words, which every CTA polls)
+// lands in device memory, and a placement keeps its time.  So a handle sets
+// up kWsCandidates workspaces, times a few batch-1 steps on each over a
+// small scratch cache (zero rows, token 0, position 0), keeps the fastest
+// and frees the others.  h is bound to its first (filled) workspace on
+// entry; on any failure the first one stays.
+constexpr int kWsCandidates = 6;
+template <class Fill, class Bind>
+static cudaError_t pick_workspace(dec_handle* h, Fill&& fill, Bind&& bind) {
+  uint8_t* cand[kWsCandidates] = {h->ws};
+  float ms[kWsCandidates];
+  void* scratch = nullptr;
+  cudaStream_t st = nullptr;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  const size_t kvb = dec_kv_bytes(h, 1, 16, DEC_KV_BF16);
+  cudaError_t e = cudaMalloc(&scratch, kvb + 256);
+  if (e == cudaSuccess) e = cudaMemset(scratch, 0, kvb + 256);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreate(&e0);
+  if (e == cudaSuccess) e = cudaEventCreate(&e1);
+  int n = 0;
+  bool ok = e == cudaSuccess;
+  for (int c = 0; ok && c < kWsCandidates; ++c) {
+    if (c > 0) {
+      ok = cudaMalloc(&cand[c], h->wl.total) == cudaSuccess;
+      if (!ok) cand[c] = nullptr;
+      ok = ok && fill(cand[c]) == cudaSuccess;
+      if (!ok) break;
+    }
+    bind(cand[c]);
+    n = c + 1;
+    int32_t* io = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + kvb);  // tok, pos, out
+    const dec_kv kv{scratch, kvb, 1, 16, DEC_KV_BF16};
+    for (int i = 0; ok && i < 6; ++i) {  // 2 untimed, 4 timed steps
+      if (i == 2) ok = cudaEventRecord(e0, st) == cudaSuccess;
+      ok = ok && do_step(h, 1, io, io + 1, &kv, io + 2, nullptr, nullptr, st) == DEC_OK;
+    }
+    ok = ok && cudaEventRecord(e1, st) == cudaSuccess && cudaStreamSynchronize(st) == cudaSuccess;
+    int status = 1;
+    ok = ok && cudaMemcpy(&status, cand[c] + h->wl.status, sizeof(int),
+                          cudaMemcpyDeviceToHost) == cudaSuccess && status == 0;
+    ok = ok && cudaEventElapsedTime(&ms[c], e0, e1) == cudaSuccess;
+  }
+  int best = 0;
+  if (ok) {
+    for (int c = 1; c < n; ++c)
+      if (ms[c] < ms[best]) best = c;
+  } else {
+    e = fill(cand[0]);  // a calibration step failed: keep the first, as new
+  }
+  bind(cand[best]);
+  for (int c = 0; c < kWsCandidates; ++c)
+    if (c != best && cand[c]) cudaFree(cand[c]);
+  if (e0) cudaEventDestroy(e0);
+  if (e1) cudaEventDestroy(e1);
+  if (st) cudaStreamDestroy(st);
+  cudaFree(scratch);
+  return e;
+}
+
 static int init_handle(const dec_shape* shape, const InitWeights& w, dec_handle** out) {
   int rc = DEC_OK;
   const int L = shape->n_layers;
@@ -232,38 +298,50 @@ static int init_handle(const dec_shape* shape, const InitWeights& w, dec_handle*
   size_t scales_off = w.w8 ? take(sizeof(LayerScales) * L) : 0;
   size_t logits_off = take(sizeof(float) * static_cast<size_t>(Bfull) * shape->vocab);
   wl.total = o;
-  e = cudaMalloc(&h->ws, wl.total);
-  if (e != cudaSuccess) {
-    delete h;
-    return cuda_fail(e);
-  }
-  e = cudaMemset(h->ws, 0, wl.total);
-  // rotary inverse frequencies theta^(-2i/D), rounded once to fp32
-  std::vector<float> inv(D / 2);
+  // host copies of the tables every workspace holds
+  std::vector<float> inv(D / 2);  // rotary inverse frequencies theta^(-2i/D), rounded once to fp32
   for (int i = 0; i < D / 2; ++i)
     inv[i] = static_cast<float>(1.0 / pow(static_cast<double>(shape->rope_theta),
                                           (2.0 * i) / static_cast<double>(D)));
-  if (e == cudaSuccess)
-    e = cudaMemcpy(h->ws + wl.inv_freq, inv.data(), sizeof(float) * inv.size(),
-                   cudaMemcpyHostToDevice);
   std::vector<LayerPtrs> lp(L);
   for (int l = 0; l < L; ++l)
     for (int j = 0; j < DEC_LW_COUNT; ++j)
       lp[l].w[j] = static_cast<const uint16_t*>(w.layers[l * DEC_LW_COUNT + j]);
-  h->layers_dev = reinterpret_cast<LayerPtrs*>(h->ws + layers_off);
-  if (e == cudaSuccess)
-    e = cudaMemcpy(h->layers_dev, lp.data(), sizeof(LayerPtrs) * L, cudaMemcpyHostToDevice);
   std::vector<LayerScales> ls;
   if (w.w8) {
     ls.resize(L);
     for (int l = 0; l < L; ++l)
       for (int j = 0; j < DEC_LW_COUNT; ++j)
         ls[l].s[j] = is_projection(j) ? w.scales[l * DEC_LW_COUNT + j] : nullptr;
-    h->scales_dev = reinterpret_cast<LayerScales*>(h->ws + scales_off);
-    if (e == cudaSuccess)
-      e = cudaMemcpy(h->scales_dev, ls.data(), sizeof(LayerScales) * L, cudaMemcpyHostToDevice);
   }
-  h->logits_dev = reinterpret_cast<float*>(h->ws + logits_off);
+  auto fill = [&](uint8_t* ws) {
+    cudaError_t r = cudaMemset(ws, 0, wl.total);
+    if (r == cudaSuccess)
+      r = cudaMemcpy(ws + wl.inv_freq, inv.data(), sizeof(float) * inv.size(),
+                     cudaMemcpyHostToDevice);
+    if (r == cudaSuccess)
+      r = cudaMemcpy(ws + layers_off, lp.data(), sizeof(LayerPtrs) * L, cudaMemcpyHostToDevice);
+    if (r == cudaSuccess && w.w8)
+      r = cudaMemcpy(ws + scales_off, ls.data(), sizeof(LayerScales) * L, cudaMemcpyHostToDevice);
+    return r;
+  };
+  auto bind = [&](uint8_t* ws) {
+    h->ws = ws;
+    h->layers_dev = reinterpret_cast<LayerPtrs*>(ws + layers_off);
+    h->scales_dev = w.w8 ? reinterpret_cast<LayerScales*>(ws + scales_off) : nullptr;
+    h->logits_dev = reinterpret_cast<float*>(ws + logits_off);
+  };
+  uint8_t* ws0 = nullptr;
+  e = cudaMalloc(&ws0, wl.total);
+  if (e != cudaSuccess) {
+    delete h;
+    return cuda_fail(e);
+  }
+  e = fill(ws0);
+  if (e == cudaSuccess) {
+    bind(ws0);
+    e = pick_workspace(h, fill, bind);
+  }
   if (e != cudaSuccess) {
     cudaFree(h->ws);
     delete h;
@@ -336,8 +414,8 @@ extern "C" int dec_kv_alloc(dec_handle* h, int batch, int max_ctx, int dtype, vo
 // steps itself, feeding the ids back and advancing gen_pos (== pos) in place.
 static int do_step(dec_handle* h, int batch, const int32_t* tok, const int32_t* pos,
                    const dec_kv* kv, int32_t* out_ids, float* logits, float* hidden,
-                   cudaStream_t stream, int n_steps = 1, int eos = -1,
-                   int32_t* gen_pos = nullptr, const int* retired = nullptr, int vseq = -1) {
+                   cudaStream_t stream, int n_steps, int eos, int32_t* gen_pos,
+                   const int* retired, int vseq) {
   if (!h || !kv || !tok || !pos || !out_ids || !kv->base) return DEC_ERR_NULL;
   if (batch < 1 || batch > h->shape.max_batch || (vseq < 0 && batch > kv->batch))
     return DEC_ERR_BATCH;

@@ -139,8 +139,13 @@ typedef struct dec_handle dec_handle;
  * the weight pointer table (not the weights: they stay caller-owned and must
  * stay alive and unchanged), allocates the workspace (activation exchange
  * buffers, attention partials, counters; a few MB) and picks the kernel
- * configuration.  Synchronous.  Returns DEC_ERR_SHAPE for unsupported shapes
- * and DEC_ERR_DEVICE if the device is not compute capability 10.0. */
+ * configuration.  The step time depends by a few per cent on where the
+ * workspace lands in device memory, so dec_init times a few batch-1 steps
+ * (on a scratch cache of zeros) in each of several candidate workspaces and
+ * keeps the fastest: it runs the weights it is given, which must therefore
+ * be valid device memory already.  Synchronous.  Returns DEC_ERR_SHAPE for
+ * unsupported shapes and DEC_ERR_DEVICE if the device is not compute
+ * capability 10.0. */
 int dec_init(const dec_shape *shape, const dec_weights *weights, dec_handle **out);
 
 /* Weight-only int8 model (faster-qwen-asr GB10 benchmark record,
