@@ -81,6 +81,7 @@ constexpr int kConvThreads = 128;                 // warps 4..7
 constexpr int kConvBarrier = 1;                   // their named barrier
 constexpr int kMaxSplits = 16;                    // cluster size (16: non-portable, allowed per kernel)
 constexpr int kMaxAttnChunks = 32;
+constexpr int kAttMinSplitRows = 1024;            // shortest chunk of a multi-wave split
 constexpr int kAttWarps = 4;
 constexpr int kAttThreads = kAttWarps * 32;
 constexpr int kAttStages = 3;
@@ -1484,6 +1485,14 @@ cudaError_t bt_step(BtPlan* p, const BtIO& io, cudaStream_t st) {
   // (sequence, KV head) pairs, i.e. one chunk per pair once there are enough
   // pairs; at most kMaxAttnChunks chunks per pair
   int per_pair = (4 * p->sms) / (io.B * s.Hkv);
+  // Long contexts: up to three waves, in chunks of at least kAttMinSplitRows
+  // rows, so that the longest sequence of a ragged batch does not alone set
+  // the kernel's length (1.7B shape, batch 64, contexts U[2048, 4064]:
+  // attention -8 % with E4M3 rows, -4.5 % with bf16); below that the extra
+  // merges cost more than the balance saves (0.6B, contexts U[200, 420]: +11 %).
+  const int waves3 = (3 * 4 * p->sms) / (io.B * s.Hkv);
+  const int by_len = io.max_ctx / kAttMinSplitRows;
+  if (waves3 > per_pair) per_pair = max(per_pair, min(waves3, by_len));
   if (per_pair < 1) per_pair = 1;
   if (per_pair > kMaxAttnChunks) per_pair = kMaxAttnChunks;
   int cr = (io.max_ctx + per_pair - 1) / per_pair;
