@@ -1715,10 +1715,11 @@ struct Cta {
       constexpr int kSlots = (8 * D + kCT - 1) / kCT;
       const bool combiner = (ci == 0);
       const int pc = a.part_chunks;
-      // partial state of chunk c for item head h
-      auto pstate = [&](int h, int c) {
-        return a.part + ((static_cast<size_t>(hrow(h, b)) * a.Hq + hq(h, g)) * pc + c) * (D + 2);
-      };
+      // partial state of chunk c for item head h: the item's states are one
+      // contiguous range [chunk][head][D + 2], so that the combiner's window
+      // of chunks is a plain address range
+      uint64_t* const pbase = a.part + (static_cast<size_t>(b) * a.Hkv + g) * pc * hi * (D + 2);
+      auto pstate = [&](int h, int c) { return pbase + (static_cast<size_t>(c) * hi + h) * (D + 2); };
       float RM[kSlots], RL[kSlots], RA[kSlots];
 #pragma unroll
       for (int i = 0; i < kSlots; ++i) {
@@ -1756,10 +1757,8 @@ struct Cta {
         const int win = kStageWords / (hi * (D + 2));
         for (int c0 = 1; c0 <= nc1; c0 += win) {
           const int nw = min(win, nc1 - c0 + 1);
-          gather(nw * hi * (D + 2), f, [=](int w) {
-            const int sg = w / (D + 2), off = w % (D + 2);
-            return pstate(sg % hi, c0 + sg / hi) + off;
-          });
+          const uint64_t* const wsrc = pstate(0, c0);  // chunks c0 .. c0 + nw - 1, every head
+          gather(nw * hi * (D + 2), f, [=](int w) { return wsrc + w; });
           if (!ab) {
 #pragma unroll
             for (int i = 0; i < kSlots; ++i) {
