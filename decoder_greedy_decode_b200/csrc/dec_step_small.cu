@@ -1023,6 +1023,17 @@ struct Cta {
   // With `planes` (bf16 weights) the values go to act as two bf16 planes per
   // sequence instead, hi = bf16(x) and lo = bf16(x - hi) (row 2b + plane,
   // rstride(K) bytes apart): the operands of the tensor-core projections.
+  // Unit u of a warp's input units: batch 1 in block order (u = j), larger
+  // batches block-major (u = j * B + b, compile-time divisors).
+  __device__ __forceinline__ void unit_of(int u, int nbw, int& b, int& blk) const {
+    if constexpr (B == 1) {
+      b = u / nbw;
+      blk = warp + (u % nbw) * kCW;
+    } else {
+      b = u % B;
+      blk = warp + (u / B) * kCW;
+    }
+  }
   __device__ void warp_input(const uint64_t* src, int K, uint32_t f, const uint16_t* g,
                              float (&ss)[B], bool planes) {
 #pragma unroll
@@ -1043,12 +1054,16 @@ struct Cta {
       const int nu = min(per, units - u0);
       if (src)
         warp_gather(ws, nu * kBlk, f, [=](int i) {
-          const int u = u0 + i / kBlk, b = u / nbw, blk = warp + (u % nbw) * kCW;
+          const int u = u0 + i / kBlk;
+          int b, blk;
+          unit_of(u, nbw, b, blk);
           return src + static_cast<size_t>(b) * K + blk * kBlk + (i % kBlk);
         });
       if (ab) continue;
       for (int uu = 0; uu < nu; ++uu) {
-        const int u = u0 + uu, b = u / nbw, blk = warp + (u % nbw) * kCW;
+        const int u = u0 + uu;
+        int b, blk;
+        unit_of(u, nbw, b, blk);
         const int k = blk * kBlk + lane * 4;
         float v[4];
         if (src) {
@@ -1068,7 +1083,7 @@ struct Cta {
         for (int bb = 0; bb < B; ++bb)
           if (bb == b) ss[bb] += q;
         if (g) {
-          const int j = u % nbw;
+          const int j = B == 1 ? u % nbw : u / B;
           uint2 gs = gv[0];
 #pragma unroll
           for (int jj = 1; jj < kMaxGainBlk; ++jj)
