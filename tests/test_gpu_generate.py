@@ -185,3 +185,79 @@ def test_generate_rejects_bad_arguments():
     with pytest.raises(RuntimeError):
         capi.dec_generate(dec.h, 2, 2, i32(toks), i32([10]), kv.kv, out)
     dec.close()
+
+
+def _follows_oracle(m, caches, toks, n0s, got, n):
+    """The ids of each sequence are the oracle's greedy ids for the first n
+    steps, up to the first permitted near-tie."""
+    for b, cache in enumerate(caches):
+        tok = toks[b]
+        for i in range(n):
+            r = m.step(cache, tok, n0s[b] + i)
+            if got[i][b] != r.token:
+                assert r.margin < NEAR_TIE, f"seq {b} step {i}"
+                break
+            tok = r.token
+
+
+@pytest.mark.parametrize("batch,max_batch", [(3, 4), (6, 8)])
+def test_generate_fp8_cache_equals_step_loop(batch, max_batch):
+    """An E4M3 cache (one fp32 scale per row): batch 3 runs on the persistent
+    kernel, batch 6 on the batched step.  The loop equals dec_step calls bit
+    for bit and follows the oracle's E4M3-cache model."""
+    s = synth.TINY
+    n0s = [15 + 9 * b for b in range(batch)]
+    w = synth.model_weights(s, seed=160 + batch)
+    codes, scales = synth.kv_prefill(s, batch, 96, n0s, seed=161 + batch, kind="fp8")
+    dec = Decoder(s, to_device(w), max_batch=max_batch)
+    toks = [int(t) for t in synth.tokens(s.vocab, batch, seed=162 + batch)]
+
+    def cache():
+        kv = dec.kv_cache(batch, 96, "fp8")
+        kv.codes.copy_(codes.cuda())
+        kv.scales.copy_(scales.cuda())
+        return kv
+
+    n = 10
+    kv_a = cache()
+    out = torch.empty((n, batch), dtype=torch.int32, device="cuda")
+    pos = i32(n0s)
+    dec.generate(kv_a, i32(toks), pos, out)
+    assert dec.check() == 0
+    kv_b = cache()
+    ref, ref_pos = _step_loop(dec, kv_b, toks, n0s, n)
+    assert out.cpu().tolist() == ref
+    assert pos.cpu().tolist() == ref_pos == [p + n for p in n0s]
+    assert torch.equal(kv_a.buf, kv_b.buf)
+    m = oracle.Model(oracle_shape(s), oracle_weights(w))
+    _follows_oracle(m, [oracle_cache(codes, scales, b) for b in range(batch)], toks, n0s, ref, n)
+    dec.close()
+
+
+def test_0p6b_bs1_generate_130_steps_in_one_launch():
+    """The one-launch loop as the benchmark runs it: 0.6B shape, batch 1, 795
+    prefilled rows, the 130-token window ("Qwen3-ASR -- Latency & Bottleneck
+    Analysis", 01 Method & setup) in one dec_generate call.  It equals 130
+    dec_step calls bit for bit (ids, final position, every cache row), and its
+    first 8 ids are the oracle's greedy ids (up to a permitted near-tie)."""
+    s = synth.QWEN3_0_6B
+    w = synth.model_weights(s, seed=2)
+    dec = Decoder(s, to_device(w), 1)
+    kv_host, _ = synth.kv_prefill(s, 1, 928, [795], seed=3)
+    tok0 = int(synth.tokens(s.vocab, 1, seed=4)[0])
+    n = 130
+    kv_a = _cache(dec, 1, 928, kv_host)
+    out = torch.full((n, 1), -7, dtype=torch.int32, device="cuda")
+    pos = i32([795])
+    dec.generate(kv_a, i32([tok0]), pos, out)
+    assert dec.check() == 0
+    got = out.cpu().tolist()
+    kv_b = _cache(dec, 1, 928, kv_host)
+    ref, ref_pos = _step_loop(dec, kv_b, [tok0], [795], n)
+    assert got == ref
+    assert pos.cpu().tolist() == ref_pos == [795 + n]
+    assert torch.equal(kv_a.buf, kv_b.buf)
+    del kv_a, kv_b
+    m = oracle.Model(oracle_shape(s), oracle_weights(w))
+    _follows_oracle(m, [oracle_cache(kv_host, None, 0)], [tok0], [795], got, 8)
+    dec.close()
