@@ -16,7 +16,7 @@ import oracle
 from conftest import oracle_cache, oracle_shape, oracle_weights
 from decoder_greedy_decode_b200 import capi, synth
 from decoder_greedy_decode_b200.decoder import Decoder, quantize_fp8w, to_device
-from gpu_util import assert_close, assert_id, i32
+from gpu_util import NEAR_TIE, assert_close, assert_id, i32
 from test_gpu_step import _check_kv_row, _check_only_rows_changed
 
 pytestmark = pytest.mark.gpu
@@ -177,3 +177,39 @@ def test_0p6b_fp8w_bs64_every_sequence_one_step():
     wd = to_device(w)
     lengths = synth.ragged_lengths(200, 420, 64, seed=78)
     _full_size(s, w, wd, 64, lengths, 432, "bf16", list(range(64)), steps=1, seed=79, w8="fp8")
+
+
+@pytest.mark.parametrize("batch,max_batch", [(2, 2), (6, 8)])
+def test_fp8w_generate_equals_steps(batch, max_batch):
+    """dec_generate on an E4M3-weight handle (batch 2 on the persistent
+    kernel, batch 6 on the batched step) equals step-by-step decoding bit for
+    bit, and its ids are the oracle's E4M3 model's greedy ids (up to a
+    permitted near-tie)."""
+    s = synth.TINY
+    n0s = [12 + 8 * b for b in range(batch)]
+    m, caches, dec, kv = _setup(s, 540 + batch, batch, 64, n0s, max_batch=max_batch)
+    kv2 = dec.kv_cache(batch, 64)
+    kv2.buf.copy_(kv.buf)
+    toks = [int(t) for t in synth.tokens(s.vocab, batch, seed=541 + batch)]
+    n = 6
+    out = torch.empty((n, batch), dtype=torch.int32, device="cuda")
+    pos = i32(n0s)
+    dec.generate(kv, i32(toks), pos, out)
+    assert dec.check() == 0
+    ref, tok, p = [], i32(toks), list(n0s)
+    for _ in range(n):
+        o = torch.empty(batch, dtype=torch.int32, device="cuda")
+        dec.step(kv2, tok, i32(p), o)
+        ref.append(o.cpu().tolist())
+        tok, p = o, [x + 1 for x in p]
+    assert out.cpu().tolist() == ref and pos.cpu().tolist() == p
+    assert torch.equal(kv.buf, kv2.buf)
+    for b in range(batch):
+        t = toks[b]
+        for i in range(n):
+            r = m.step(caches[b], t, n0s[b] + i)
+            if ref[i][b] != r.token:
+                assert r.margin < NEAR_TIE, f"seq {b} step {i}"
+                break
+            t = r.token
+    dec.close()
