@@ -52,6 +52,17 @@ def test_null_arguments():
     assert L.dec_kv_quantize_e4m3(None, 1, 128, None, None, None) == -1
 
 
+def test_attention_rejects_no_query_heads():
+    """n_q_heads < 1 is a shape error in both attention entry points, decided on
+    the host before any CUDA call (the pointers are fake and never read)."""
+    L = capi.lib()
+    p = 1 << 20
+    for hq in (0, -8):
+        assert L.dec_attention_workspace_bytes(1, hq, 8, 128, 64) == 0
+        assert L.dec_attention(1, hq, 8, 128, p, p, p, 64, p, p, p, 1 << 20, None, None) == -2
+        assert L.dec_attention_noalloc(1, hq, 8, 128, p, p, p, 64, p, p, None, None) == -2
+
+
 def test_error_strings():
     assert capi.error_string(0) == "ok"
     assert "NULL" in capi.error_string(-1)
